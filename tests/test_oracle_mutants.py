@@ -1,0 +1,108 @@
+"""Planted mistakes in the oracle must be caught by its pins (no GPU).
+
+Each mutant is the oracle with one plausible error planted in it, on the CPU.
+If the pin suite in oracle_checks.py lets any of them through, the pins are
+too weak to trust the oracle they vouch for.
+"""
+import math
+import types
+
+import numpy as np
+import pytest
+
+import oracle
+from tests import oracle_checks as oc
+
+
+def _mutant(**overrides):
+    m = types.SimpleNamespace(
+        retained_count=oracle.retained_count,
+        column_scores_sq=oracle.column_scores_sq,
+        topk_indices=oracle.topk_indices,
+        reduced_product=oracle.reduced_product,
+    )
+    for k, v in overrides.items():
+        setattr(m, k, v)
+    return m
+
+
+def _topk_ties_high(s2, k):
+    order = sorted(range(len(s2)), key=lambda j: (-s2[j], -j))
+    return np.array(sorted(order[:k]), dtype=np.int32)
+
+
+def _topk_smallest(s2, k):
+    order = sorted(range(len(s2)), key=lambda j: (s2[j], j))
+    return np.array(sorted(order[:k]), dtype=np.int32)
+
+
+def _topk_unsorted(s2, k):
+    order = sorted(range(len(s2)), key=lambda j: (-s2[j], j))
+    return np.array(order[:k], dtype=np.int32)
+
+
+def _scores_l1(A):
+    return np.abs(oracle.as_f64(A)).sum(axis=0)
+
+
+def _scores_rows(A):
+    A = oracle.as_f64(A)
+    s = (A ** 2).sum(axis=1)
+    return np.resize(s, A.shape[1])
+
+
+def _product_drops_last(A, B, I, rows=None):
+    return oracle.reduced_product(A, B, np.asarray(I)[:-1] if len(I) > 1 else I, rows)
+
+
+def _product_shifted_rows(A, B, I, rows=None):
+    A = oracle.as_f64(A)
+    B = oracle.as_f64(B)
+    d = B.shape[0]
+    Bs = np.ascontiguousarray(np.roll(B, -1, axis=0)) if d > 1 else B * 2
+    return oracle.reduced_product(A, Bs, I, rows)
+
+
+def _product_wrong_sign(A, B, I, rows=None):
+    Y = oracle.reduced_product(A, B, I, rows)
+    I = np.asarray(I)
+    if len(I):
+        A = oracle.as_f64(A)
+        B = oracle.as_f64(B)
+        j = int(I[0])
+        Y = Y - 2.0 * np.outer(A[:, j] if rows is None else A[rows, j], B[j])
+    return Y
+
+
+def _count_floor(rho, d):
+    return max(1, int(math.floor(rho * d)))
+
+
+def _count_no_snap(rho, d):
+    return min(d, max(1, int(math.ceil(rho * d))))
+
+
+MUTANTS = {
+    "ties_to_higher_index": _mutant(topk_indices=_topk_ties_high),
+    "keeps_smallest": _mutant(topk_indices=_topk_smallest),
+    "index_set_not_sorted": _mutant(topk_indices=_topk_unsorted),
+    "l1_scores": _mutant(column_scores_sq=_scores_l1),
+    "row_norms_not_column_norms": _mutant(column_scores_sq=_scores_rows),
+    "product_drops_an_index": _mutant(reduced_product=_product_drops_last),
+    "product_off_by_one_row": _mutant(reduced_product=_product_shifted_rows),
+    "product_sign_error": _mutant(reduced_product=_product_wrong_sign),
+    "k_floor_not_ceil": _mutant(retained_count=_count_floor),
+    "k_no_rounding_snap": _mutant(retained_count=_count_no_snap),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name):
+    impl = MUTANTS[name]
+    caught = []
+    for check in oc.ALL_CHECKS:
+        try:
+            check(impl)
+        except (AssertionError, ValueError, IndexError):
+            caught.append(check.__name__)
+    assert caught, f"no pin catches the planted mistake '{name}'"

@@ -1,0 +1,175 @@
+/*
+ * rmm.h -- C ABI of librmm, Reduced Matrix Multiplication (RMM) on NVIDIA B200
+ * (sm_100a).
+ *
+ * Method: "Reduced Matrix Multiplication: Input-Adaptive Matrix-Product
+ * Reduction for LLM Inference" (arXiv 2608.13426), "the RMM paper" below.
+ * For Y = A B with A in R^{n x d} (activations) and B in R^{d x m}, RMM
+ *   1. scores every contraction index j by s_j = ||A[:, j]||_2        (§3.2)
+ *   2. keeps I = TopK({s_j}, k), k = ceil(rho d), rho in (0, 1]         (§3.2)
+ *   3. returns A[:, I] B[I, :]                                         (§3.2)
+ * and has per-head forms for attention (§3.3): QK^T with features chosen
+ * per query head from Q's column norms (grouped-query attention gathers the
+ * same features of the shared K head), scaled by alpha (the paper uses
+ * 1/sqrt(d_h)) and optionally causally masked; and PV with token positions
+ * chosen per head from the column norms of P.
+ *
+ * Readings where the paper is silent (fixed by this library):
+ *   - ties between equal scores keep the lower index;
+ *   - I is returned in ascending order, int32;
+ *   - k = ceil(rho d), except that a product rho*d within 1e-9 d of an
+ *     integer counts as that integer; k is clamped to [1, d];
+ *   - the causal mask writes -inf where key index > query index;
+ *   - scores are accumulated in fp32 from the stored values; the product
+ *     accumulates in fp32 (bf16 inputs) or tf32 (fp32 inputs) and is stored
+ *     in the input dtype.
+ *
+ * Memory: every pointer passed to a compute call is DEVICE memory on the
+ * current CUDA device, owned by the caller, and must be 16-byte aligned (the
+ * workspace 256-byte aligned).  The library never allocates device memory.
+ * A plan is host memory owned by the caller through create/destroy.
+ *
+ * Execution: compute calls only enqueue kernels on `stream` (a cudaStream_t
+ * passed as void*; NULL = the legacy default stream) and return without
+ * synchronising.  Argument errors are detected on the host before anything
+ * is enqueued; outputs are then untouched.  A kernel that gives up on an
+ * internal wait (bounded at about two seconds) records it in the workspace;
+ * rmm_workspace_status() reports it.  One plan and one workspace may be used
+ * by one stream at a time.  Nothing is thrown across this ABI.
+ */
+#ifndef RMM_H_
+#define RMM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RMM_API __attribute__((visibility("default")))
+#else
+#define RMM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum rmm_status {
+    RMM_OK = 0,
+    RMM_ERR_INVALID_ARG = 1,  /* a NULL, misaligned, out-of-range or inconsistent argument */
+    RMM_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels implement (e.g. d too large) */
+    RMM_ERR_WORKSPACE = 3,    /* workspace missing, too small or misaligned */
+    RMM_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed (launch, attribute, encode) */
+    RMM_ERR_TIMEOUT = 5       /* a kernel gave up on an internal wait (see rmm_workspace_status) */
+} rmm_status;
+
+typedef enum rmm_dtype {
+    RMM_BF16 = 0, /* bfloat16 storage, fp32 accumulation (tcgen05 kind::f16) */
+    RMM_F32 = 1   /* fp32 storage, tf32 products with fp32 accumulation (tcgen05 kind::tf32) */
+} rmm_dtype;
+
+typedef enum rmm_mode {
+    /* Y[h] = RMM(A[h], B[g]): A n x d (lda), B d x m (ldb, row j = contraction
+       index j), Y n x m (ldy).  The RMM paper §3.2, §3.3 "MLP and linear
+       projections". */
+    RMM_LINEAR = 0,
+    /* S[h] = alpha * Q[h][:, I_h] K[g][:, I_h]^T (+ causal mask): A = Q[h] is
+       n x d with d = d_h (lda), B = K[g] is m x d (ldb; m = number of keys,
+       the contraction axis is contiguous), Y = S[h] is n x m.  I_h is chosen
+       from Q[h]'s column norms.  The RMM paper §3.3 "Attention". */
+    RMM_QK = 1,
+    /* O[h] = P[h][:, T_h] V[g][T_h, :]: A = P[h] is n x d with d = number of
+       key tokens (lda), B = V[g] is d x m (ldb; m = d_v), Y = O[h] is n x m.
+       T_h is chosen from P[h]'s column norms.  The RMM paper §3.3, last
+       sentence of "Attention"; Appendix D.1 Eq. (2). */
+    RMM_PV = 2
+} rmm_mode;
+
+/* Causal mask on the QK output: S[i][c] = -inf for c > i. */
+#define RMM_FLAG_CAUSAL 1u
+/* rmm_matmul*: take I from the caller (I_inout, [heads][k], ascending,
+   distinct, each in [0, d)) instead of computing it; no scores are formed. */
+#define RMM_FLAG_USE_GIVEN_INDICES 2u
+
+/* One problem shape.  All sizes and strides count ELEMENTS.  Heads: query
+   head h (0 <= h < heads) reads A, I and Y at offset h * stride_{a,y} and B at
+   offset g * stride_b with g = h / (heads / kv_heads) (grouped-query sharing;
+   kv_heads = heads means one B per head, kv_heads = 1 one shared B). */
+typedef struct rmm_problem {
+    int32_t mode;      /* rmm_mode */
+    int32_t dtype;     /* rmm_dtype of A, B and Y */
+    int64_t n;         /* rows of A and Y (tokens / queries), >= 0 */
+    int64_t d;         /* contraction size, >= 1, multiple of 8 (bf16) or 4 (fp32) */
+    int64_t m;         /* columns of Y, >= 0, multiple of 8 (bf16) or 4 (fp32) */
+    int64_t lda, ldb, ldy; /* row strides; multiples of 16 bytes; lda >= d, ldy >= m,
+                              ldb >= m (LINEAR, PV) or >= d (QK) */
+    int64_t heads;     /* >= 1 */
+    int64_t kv_heads;  /* >= 1, divides heads */
+    int64_t stride_a, stride_b, stride_y; /* per-head strides (multiples of 16 bytes);
+                                             ignored when the count of that operand is 1 */
+    double rho;        /* retention ratio in (0, 1]; used when k == 0 */
+    int64_t k;         /* 0: k = ceil(rho d) (see readings above); else 1 <= k <= d */
+    float alpha;       /* output scale applied in fp32 before rounding; QK: 1/sqrt(d_h) */
+    uint32_t flags;    /* RMM_FLAG_* */
+} rmm_problem;
+
+typedef struct rmm_plan rmm_plan;
+
+/* Fill *p with defaults for a single-head LINEAR problem (alpha 1, rho 1,
+   dense row-major strides lda = d, ldb = m, ldy = m). */
+RMM_API void rmm_problem_init(rmm_problem* p, int32_t mode, int32_t dtype, int64_t n, int64_t d,
+                      int64_t m);
+
+/* Validate *p, fix k and the kernel choices, and report the workspace the
+   compute calls need (bytes, may be 0 only for n == 0 or m == 0 problems).
+   Reads the current CUDA device's SM count.  On error *plan is set to NULL. */
+RMM_API rmm_status rmm_plan_create(rmm_plan** plan, const rmm_problem* p, size_t* workspace_bytes);
+
+/* Release a plan (NULL is allowed). */
+RMM_API rmm_status rmm_plan_destroy(rmm_plan* plan);
+
+/* The number of retained indices k of a plan (-1 for NULL). */
+RMM_API int64_t rmm_plan_k(const rmm_plan* plan);
+
+/* Workspace size of a plan in bytes (0 for NULL). */
+RMM_API size_t rmm_plan_workspace_size(const rmm_plan* plan);
+
+/* Selection only (§3.2 scores + TopK): for every head write I[h][0..k) in
+   ascending order and, when s2 != NULL, s2[h][0..d) = fp32 sum_i A[h][i][j]^2.
+   A: as in the plan.  I: device int32 [heads][k].  s2: device fp32 [heads][d]
+   or NULL. */
+RMM_API rmm_status rmm_select(const rmm_plan* plan, const void* A, int32_t* I, float* s2,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Full op for a plan with heads == 1: Y = A[:, I] B[I, :] (LINEAR, PV) or
+   alpha * A[:, I] B[:, I]^T with the optional causal mask (QK).
+   I_inout: NULL, or device int32 [k] that receives I (or supplies it with
+   RMM_FLAG_USE_GIVEN_INDICES).  Y must not overlap A, B or the workspace. */
+RMM_API rmm_status rmm_matmul(const rmm_plan* plan, const void* A, const void* B, void* Y,
+                      int32_t* I_inout, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Same as rmm_matmul for any number of heads; I_inout is [heads][k]. */
+RMM_API rmm_status rmm_matmul_batched(const rmm_plan* plan, const void* A, const void* B, void* Y,
+                              int32_t* I_inout, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/* Zero the workspace's error word (its first 256 bytes) on `stream`.  Call
+   once after allocating a workspace, before the first compute call. */
+RMM_API rmm_status rmm_workspace_init(const rmm_plan* plan, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/* Synchronise `stream` and read the workspace's error word: RMM_OK, or
+   RMM_ERR_TIMEOUT if a kernel gave up on a wait since the last check (the
+   word is then cleared), or RMM_ERR_CUDA if the stream reports an error. */
+RMM_API rmm_status rmm_workspace_status(const rmm_plan* plan, void* workspace, void* stream);
+
+/* Static string naming a status code. */
+RMM_API const char* rmm_status_string(rmm_status s);
+
+/* Library version, "major.minor.patch". */
+RMM_API const char* rmm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RMM_H_ */

@@ -1,0 +1,361 @@
+"""Python binding of librmm: Reduced Matrix Multiplication on B200 (sm_100a).
+
+Argument marshalling only.  Every step of the op (column scores, TopK,
+staging, the tensor-core product) runs in the CUDA kernels of librmm.so behind
+the C ABI of include/rmm.h; PyTorch supplies device memory and streams.  There
+is no CPU fallback: importing this package fails when librmm.so is missing,
+and every call raises RmmError on a non-OK status.
+
+Method: "Reduced Matrix Multiplication: Input-Adaptive Matrix-Product
+Reduction for LLM Inference" (arXiv 2608.13426), §3.2-§3.3.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+__all__ = [
+    "RMM_OK", "RMM_ERR_INVALID_ARG", "RMM_ERR_UNSUPPORTED", "RMM_ERR_WORKSPACE", "RMM_ERR_CUDA",
+    "RMM_ERR_TIMEOUT", "RMM_BF16", "RMM_F32", "RMM_LINEAR", "RMM_QK", "RMM_PV", "RMM_FLAG_CAUSAL",
+    "RMM_FLAG_USE_GIVEN_INDICES", "RmmError", "rmm_problem", "Plan", "lib", "library_path",
+    "rmm_problem_init", "rmm_plan_create", "rmm_select", "rmm_matmul", "rmm_matmul_batched",
+    "rmm_workspace_init", "rmm_workspace_status", "rmm_status_string", "rmm_version",
+    "EXPORTED_SYMBOLS", "select", "matmul", "qk", "pv", "workspace_for", "check_workspaces",
+]
+
+RMM_OK, RMM_ERR_INVALID_ARG, RMM_ERR_UNSUPPORTED, RMM_ERR_WORKSPACE, RMM_ERR_CUDA, RMM_ERR_TIMEOUT = range(6)
+RMM_BF16, RMM_F32 = 0, 1
+RMM_LINEAR, RMM_QK, RMM_PV = 0, 1, 2
+RMM_FLAG_CAUSAL = 1
+RMM_FLAG_USE_GIVEN_INDICES = 2
+
+EXPORTED_SYMBOLS = (
+    "rmm_problem_init", "rmm_plan_create", "rmm_plan_destroy", "rmm_plan_k", "rmm_plan_workspace_size",
+    "rmm_select", "rmm_matmul", "rmm_matmul_batched", "rmm_workspace_init", "rmm_workspace_status",
+    "rmm_status_string", "rmm_version",
+)
+
+library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librmm.so")
+
+
+class RmmError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_status_name(status)}")
+
+
+class rmm_problem(ctypes.Structure):
+    _fields_ = [
+        ("mode", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("n", ctypes.c_int64), ("d", ctypes.c_int64), ("m", ctypes.c_int64),
+        ("lda", ctypes.c_int64), ("ldb", ctypes.c_int64), ("ldy", ctypes.c_int64),
+        ("heads", ctypes.c_int64), ("kv_heads", ctypes.c_int64),
+        ("stride_a", ctypes.c_int64), ("stride_b", ctypes.c_int64), ("stride_y", ctypes.c_int64),
+        ("rho", ctypes.c_double), ("k", ctypes.c_int64), ("alpha", ctypes.c_float),
+        ("flags", ctypes.c_uint32),
+    ]
+
+
+def _load_library():
+    from . import build as _build
+    if _build.stale():
+        try:
+            _build.build()
+        except Exception as exc:  # no compiler, no sources: there is no other path
+            raise ImportError(f"librmm.so is missing or stale and could not be built ({exc}); "
+                              "this package has no CPU fallback") from exc
+    if not os.path.exists(library_path):
+        raise ImportError("librmm.so is not built; this package has no CPU fallback")
+    L = ctypes.CDLL(library_path)
+    vp, sz, i64, st = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64, ctypes.c_int
+    pp = ctypes.POINTER(rmm_problem)
+    L.rmm_problem_init.restype = None
+    L.rmm_problem_init.argtypes = [pp, ctypes.c_int32, ctypes.c_int32, i64, i64, i64]
+    L.rmm_plan_create.restype = st
+    L.rmm_plan_create.argtypes = [ctypes.POINTER(vp), pp, ctypes.POINTER(sz)]
+    L.rmm_plan_destroy.restype = st
+    L.rmm_plan_destroy.argtypes = [vp]
+    L.rmm_plan_k.restype = i64
+    L.rmm_plan_k.argtypes = [vp]
+    L.rmm_plan_workspace_size.restype = sz
+    L.rmm_plan_workspace_size.argtypes = [vp]
+    L.rmm_select.restype = st
+    L.rmm_select.argtypes = [vp, vp, vp, vp, vp, sz, vp]
+    L.rmm_matmul.restype = st
+    L.rmm_matmul.argtypes = [vp, vp, vp, vp, vp, vp, sz, vp]
+    L.rmm_matmul_batched.restype = st
+    L.rmm_matmul_batched.argtypes = [vp, vp, vp, vp, vp, vp, sz, vp]
+    L.rmm_workspace_init.restype = st
+    L.rmm_workspace_init.argtypes = [vp, vp, sz, vp]
+    L.rmm_workspace_status.restype = st
+    L.rmm_workspace_status.argtypes = [vp, vp, vp]
+    L.rmm_status_string.restype = ctypes.c_char_p
+    L.rmm_status_string.argtypes = [st]
+    L.rmm_version.restype = ctypes.c_char_p
+    L.rmm_version.argtypes = []
+    return L
+
+
+lib = _load_library()
+
+
+def _status_name(s: int) -> str:
+    return lib.rmm_status_string(int(s)).decode()
+
+
+def rmm_status_string(s: int) -> str:
+    return _status_name(s)
+
+
+def rmm_version() -> str:
+    return lib.rmm_version().decode()
+
+
+def _check(status: int, what: str):
+    if status != RMM_OK:
+        raise RmmError(status, what)
+
+
+def rmm_problem_init(mode: int, dtype: int, n: int, d: int, m: int) -> rmm_problem:
+    p = rmm_problem()
+    lib.rmm_problem_init(ctypes.byref(p), mode, dtype, n, d, m)
+    return p
+
+
+class Plan:
+    """Owns an rmm_plan (host memory) created from an rmm_problem."""
+
+    def __init__(self, problem: rmm_problem):
+        self.problem = problem
+        h = ctypes.c_void_p()
+        ws = ctypes.c_size_t()
+        _check(lib.rmm_plan_create(ctypes.byref(h), ctypes.byref(problem), ctypes.byref(ws)),
+               "rmm_plan_create")
+        self.handle = h
+        self.workspace_bytes = int(ws.value)
+        self.k = int(lib.rmm_plan_k(h))
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        L = globals().get("lib")
+        if h is not None and h.value and L is not None:  # lib is gone at interpreter exit
+            L.rmm_plan_destroy(h)
+            self.handle = None
+
+
+def rmm_plan_create(problem: rmm_problem) -> Plan:
+    return Plan(problem)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ws(workspace):
+    if workspace is None:
+        return None, 0
+    return ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size()
+
+
+def rmm_workspace_init(plan: Plan, workspace, stream=None):
+    wp, wb = _ws(workspace)
+    _check(lib.rmm_workspace_init(plan.handle, wp, wb, _stream(stream)), "rmm_workspace_init")
+
+
+def rmm_workspace_status(plan: Plan, workspace, stream=None) -> int:
+    return int(lib.rmm_workspace_status(plan.handle, _ptr(workspace), _stream(stream)))
+
+
+def rmm_select(plan: Plan, A, I, s2=None, workspace=None, stream=None):
+    wp, wb = _ws(workspace)
+    _check(lib.rmm_select(plan.handle, _ptr(A), _ptr(I), _ptr(s2), wp, wb, _stream(stream)), "rmm_select")
+
+
+def rmm_matmul(plan: Plan, A, B, Y, I=None, workspace=None, stream=None):
+    wp, wb = _ws(workspace)
+    _check(lib.rmm_matmul(plan.handle, _ptr(A), _ptr(B), _ptr(Y), _ptr(I), wp, wb, _stream(stream)),
+           "rmm_matmul")
+
+
+def rmm_matmul_batched(plan: Plan, A, B, Y, I=None, workspace=None, stream=None):
+    wp, wb = _ws(workspace)
+    _check(lib.rmm_matmul_batched(plan.handle, _ptr(A), _ptr(B), _ptr(Y), _ptr(I), wp, wb,
+                                  _stream(stream)), "rmm_matmul_batched")
+
+
+# ----------------------------------------------------------------------------
+# Convenience layer over torch tensors (still marshalling only).
+# ----------------------------------------------------------------------------
+_cache_lock = threading.Lock()
+_plans: dict = {}
+_workspaces: dict = {}
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return RMM_BF16
+    if t.dtype == torch.float32:
+        return RMM_F32
+    raise TypeError(f"RMM supports bfloat16 and float32 tensors, not {t.dtype}")
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("RMM tensors must live on a CUDA device (there is no CPU path)")
+
+
+def _row_stride(t) -> int:
+    if t.numel() == 0:
+        return t.shape[-1]
+    if t.stride(-1) != 1:
+        raise ValueError("the last dimension must be contiguous")
+    return t.stride(-2) if t.dim() >= 2 and t.shape[-2] > 1 else t.shape[-1]
+
+
+def _plan_for(p: rmm_problem) -> Plan:
+    key = tuple(getattr(p, f) for f, _ in rmm_problem._fields_)
+    import torch
+    key = key + (torch.cuda.current_device(),)
+    with _cache_lock:
+        plan = _plans.get(key)
+        if plan is None:
+            plan = Plan(p)
+            _plans[key] = plan
+    return plan
+
+
+def workspace_for(plan: Plan, device=None, stream=None):
+    """A zero-initialised workspace for a plan, cached per (plan, device, stream)."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    s = torch.cuda.current_stream(dev) if stream is None else stream
+    key = (id(plan), dev.index, s.cuda_stream)
+    with _cache_lock:
+        ws = _workspaces.get(key)
+    if ws is None or ws.numel() < plan.workspace_bytes:
+        ws = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device=dev)
+        rmm_workspace_init(plan, ws, s)
+        with _cache_lock:
+            _workspaces[key] = ws
+    return ws
+
+
+def check_workspaces():
+    """Synchronise and read the error word of every workspace this module
+    allocated; raise RmmError(RMM_ERR_TIMEOUT) if a kernel gave up on a wait."""
+    with _cache_lock:
+        items = list(_workspaces.items())
+        plans = {id(p): p for p in _plans.values()}
+    for (pid, _dev, _s), ws in items:
+        plan = plans.get(pid)
+        if plan is not None:
+            _check(rmm_workspace_status(plan, ws), "kernel wait")
+
+
+def _k_fields(p: rmm_problem, rho, k):
+    if k is not None:
+        p.k = int(k)
+    elif rho is not None:
+        p.rho = float(rho)
+    else:
+        raise ValueError("give rho or k")
+
+
+def select(A, rho=None, k=None, return_scores=False):
+    """I (and optionally fp32 s^2) for activations A [n, d] or [heads, n, d]."""
+    import torch
+    _require_cuda(A)
+    heads = A.shape[0] if A.dim() == 3 else 1
+    n, d = A.shape[-2], A.shape[-1]
+    p = rmm_problem_init(RMM_LINEAR, _dtype_code(A), n, d, 8)
+    p.lda = _row_stride(A)
+    p.heads = heads
+    p.kv_heads = 1
+    p.stride_a = A.stride(0) if A.dim() == 3 else 0
+    _k_fields(p, rho, k)
+    plan = _plan_for(p)
+    I = torch.empty((heads, plan.k) if A.dim() == 3 else (plan.k,), dtype=torch.int32, device=A.device)
+    s2 = torch.empty((heads, d) if A.dim() == 3 else (d,), dtype=torch.float32, device=A.device) \
+        if return_scores else None
+    rmm_select(plan, A, I, s2, workspace_for(plan))
+    return (I, s2) if return_scores else I
+
+
+def matmul(A, B, rho=None, k=None, indices=None, return_indices=False, out=None):
+    """RMM_rho(A, B) = A[:, I] B[I, :] for A [n, d], B [d, m] (§3.2)."""
+    import torch
+    _require_cuda(A, B, out, indices)
+    n, d = A.shape
+    m = B.shape[1]
+    if B.shape[0] != d or B.dtype != A.dtype:
+        raise ValueError("A is n x d and B is d x m with the same dtype")
+    p = rmm_problem_init(RMM_LINEAR, _dtype_code(A), n, d, m)
+    p.lda, p.ldb = _row_stride(A), _row_stride(B)
+    if indices is not None:
+        p.k = indices.numel()
+        p.flags |= RMM_FLAG_USE_GIVEN_INDICES
+    else:
+        _k_fields(p, rho, k)
+    Y = torch.empty((n, m), dtype=A.dtype, device=A.device) if out is None else out
+    p.ldy = _row_stride(Y)
+    plan = _plan_for(p)
+    I = indices
+    if I is None and return_indices:
+        I = torch.empty(plan.k, dtype=torch.int32, device=A.device)
+    rmm_matmul(plan, A, B, Y, I, workspace_for(plan))
+    return (Y, I) if return_indices else Y
+
+
+def qk(Q, K, rho, alpha=None, causal=True, return_indices=False):
+    """Reduced attention scores S[h] = alpha Q[h][:, I_h] K[g][:, I_h]^T (+ causal
+    mask) for Q [H, n, d_h] and K [H_kv, m, d_h] (§3.3 "Attention")."""
+    import torch
+    _require_cuda(Q, K)
+    H, n, dh = Q.shape
+    Hkv, m, _ = K.shape
+    p = rmm_problem_init(RMM_QK, _dtype_code(Q), n, dh, m)
+    p.lda, p.ldb = _row_stride(Q), _row_stride(K)
+    p.heads, p.kv_heads = H, Hkv
+    p.stride_a, p.stride_b = Q.stride(0), K.stride(0)
+    p.alpha = 1.0 / math.sqrt(dh) if alpha is None else float(alpha)
+    p.flags = RMM_FLAG_CAUSAL if causal else 0
+    _k_fields(p, rho, None)
+    S = torch.empty((H, n, m), dtype=Q.dtype, device=Q.device)
+    p.ldy, p.stride_y = m, n * m
+    plan = _plan_for(p)
+    I = torch.empty((H, plan.k), dtype=torch.int32, device=Q.device) if return_indices else None
+    rmm_matmul_batched(plan, Q, K, S, I, workspace_for(plan))
+    return (S, I) if return_indices else S
+
+
+def pv(P, V, rho, return_indices=False):
+    """Token-reduced value product O[h] = P[h][:, T_h] V[g][T_h, :] for
+    P [H, n, n_k] and V [H_kv, n_k, d_v] (§3.3 "Attention", last sentence)."""
+    import torch
+    _require_cuda(P, V)
+    H, n, nk = P.shape
+    Hkv, _, dv = V.shape
+    p = rmm_problem_init(RMM_PV, _dtype_code(P), n, nk, dv)
+    p.lda, p.ldb = _row_stride(P), _row_stride(V)
+    p.heads, p.kv_heads = H, Hkv
+    p.stride_a, p.stride_b = P.stride(0), V.stride(0)
+    _k_fields(p, rho, None)
+    O = torch.empty((H, n, dv), dtype=P.dtype, device=P.device)
+    p.ldy, p.stride_y = dv, n * dv
+    plan = _plan_for(p)
+    T = torch.empty((H, plan.k), dtype=torch.int32, device=P.device) if return_indices else None
+    rmm_matmul_batched(plan, P, V, O, T, workspace_for(plan))
+    return (O, T) if return_indices else O

@@ -1,0 +1,459 @@
+// rmm_api.cu -- the C ABI of librmm (declared in include/rmm.h): problem
+// validation, plans, workspace layout, tensor-map encoding and the launch
+// sequence of Reduced Matrix Multiplication ("Reduced Matrix Multiplication:
+// Input-Adaptive Matrix-Product Reduction for LLM Inference", §3.2-§3.3).
+//
+// Launch sequence of one call (all on the caller's stream, no host sync):
+//   select : normselect (small inputs)  |  colnorm -> topk      -> I
+//            identity fill when k == d (TopK of every index is all of them)
+//   stage  : pack A[:, I] (and K[:, I] in QK mode) when k < d or I is given
+//   product: gather_gemm (tcgen05, TMEM accumulators)
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "../../include/rmm.h"
+#include "rmm_internal.h"
+
+struct rmm_plan {
+    rmm_problem p;
+    int64_t k;
+    int64_t ldp;        // row stride of the packed operands (k rounded up to 8)
+    int es;             // element size
+    int group;          // heads / kv_heads
+    bool need_select;   // scores + TopK on each call
+    bool fused_select;  // one-kernel selection
+    int nsplit;
+    int64_t rows_per_split;
+    int bn;
+    int num_sms;
+    size_t off_err, off_partials, off_I, off_apack, off_bpack, ws_bytes;
+};
+
+namespace {
+
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+constexpr size_t kFusedSelectBytes = size_t(1) << 20;  // per head
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// k = ceil(rho d) with near-integer products snapped (see include/rmm.h).
+int64_t retained_count(double rho, int64_t d) {
+    const double x = rho * static_cast<double>(d);
+    const double r = std::nearbyint(x);
+    int64_t k = (std::fabs(x - r) <= 1e-9 * static_cast<double>(d)) ? static_cast<int64_t>(r)
+                                                                      : static_cast<int64_t>(std::ceil(x));
+    if (k < 1) k = 1;
+    if (k > d) k = d;
+    return k;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 3-D K-major map {K extent, rows, heads} with a {box_k, box_rows, 1} box,
+// 128-byte swizzle and zero fill outside the extents.
+bool encode_kmajor_map(CUtensorMap* map, int es, const void* base, int64_t kext, int64_t rows,
+                       int64_t heads, int64_t ld, int64_t stride_h, uint32_t box_k, uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const uint64_t row_bytes = static_cast<uint64_t>(ld) * es;
+    uint64_t head_bytes = static_cast<uint64_t>(stride_h) * es;
+    if (heads <= 1 || head_bytes == 0) head_bytes = row_bytes * static_cast<uint64_t>(rows > 0 ? rows : 1);
+    head_bytes = (head_bytes + 15) & ~uint64_t(15);
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(kext), static_cast<cuuint64_t>(rows > 0 ? rows : 1),
+                          static_cast<cuuint64_t>(heads)};
+    cuuint64_t strides[2] = {row_bytes, head_bytes};
+    cuuint32_t box[3] = {box_k, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = enc(map, es == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                           const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+rmm_status validate_problem(const rmm_problem* p) {
+    if (!p) return RMM_ERR_INVALID_ARG;
+    if (p->mode < RMM_LINEAR || p->mode > RMM_PV) return RMM_ERR_INVALID_ARG;
+    if (p->dtype != RMM_BF16 && p->dtype != RMM_F32) return RMM_ERR_INVALID_ARG;
+    const int es = p->dtype == RMM_F32 ? 4 : 2;
+    const int vec = 16 / es;
+    if (p->n < 0 || p->m < 0 || p->d < 1) return RMM_ERR_INVALID_ARG;
+    if (p->n > kMaxDim || p->m > kMaxDim || p->d > kMaxDim) return RMM_ERR_UNSUPPORTED;
+    if (p->d % vec != 0 || p->m % vec != 0) return RMM_ERR_INVALID_ARG;
+    if (p->heads < 1 || p->kv_heads < 1 || p->heads % p->kv_heads != 0) return RMM_ERR_INVALID_ARG;
+    if (p->heads > 65535) return RMM_ERR_UNSUPPORTED;
+    if (p->lda < p->d || p->lda % vec != 0) return RMM_ERR_INVALID_ARG;
+    if (p->ldy < p->m || p->ldy % vec != 0) return RMM_ERR_INVALID_ARG;
+    const int64_t b_cols = p->mode == RMM_QK ? p->d : p->m;
+    if (p->ldb < b_cols || p->ldb % vec != 0) return RMM_ERR_INVALID_ARG;
+    if (p->heads > 1) {
+        if (p->stride_a < 0 || p->stride_a % vec != 0) return RMM_ERR_INVALID_ARG;
+        if (p->stride_y % vec != 0 || (p->n > 0 && p->stride_y < p->n * p->ldy)) return RMM_ERR_INVALID_ARG;
+    }
+    if (p->kv_heads > 1 && (p->stride_b < 0 || p->stride_b % vec != 0)) return RMM_ERR_INVALID_ARG;
+    if (p->k == 0) {
+        if (!(p->rho > 0.0) || p->rho > 1.0) return RMM_ERR_INVALID_ARG;
+    } else if (p->k < 0 || p->k > p->d) {
+        return RMM_ERR_INVALID_ARG;
+    }
+    if (p->flags & ~(RMM_FLAG_CAUSAL | RMM_FLAG_USE_GIVEN_INDICES)) return RMM_ERR_INVALID_ARG;
+    if ((p->flags & RMM_FLAG_CAUSAL) && p->mode != RMM_QK) return RMM_ERR_INVALID_ARG;
+    if (!std::isfinite(p->alpha)) return RMM_ERR_INVALID_ARG;
+    return RMM_OK;
+}
+
+rmm_status check_workspace(const rmm_plan* plan, void* ws, size_t ws_bytes) {
+    if (ws_bytes < plan->ws_bytes) return RMM_ERR_WORKSPACE;
+    if (plan->ws_bytes > 0 && (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)) return RMM_ERR_WORKSPACE;
+    return RMM_OK;
+}
+
+template <typename T>
+T* ws_at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+rmm_status run_select(const rmm_plan* plan, const void* A, int32_t* I, float* s2, void* ws,
+                      cudaStream_t stream) {
+    const rmm_problem& p = plan->p;
+    rmm::SelectArgs a{};
+    a.A = A;
+    a.dtype = p.dtype;
+    a.n = p.n;
+    a.d = p.d;
+    a.lda = p.lda;
+    a.stride_a = p.stride_a;
+    a.heads = static_cast<int>(p.heads);
+    a.k = plan->k;
+    a.I = I;
+    a.s2 = s2;
+    cudaError_t e;
+    if (plan->fused_select) {
+        e = rmm::launch_normselect(a, stream);
+    } else {
+        a.partials = ws_at<float>(ws, plan->off_partials);
+        a.nsplit = plan->nsplit;
+        a.rows_per_split = plan->rows_per_split;
+        e = rmm::launch_colnorm(a, stream);
+        if (e == cudaSuccess) e = rmm::launch_topk(a, stream);
+    }
+    return e == cudaSuccess ? RMM_OK : RMM_ERR_CUDA;
+}
+
+rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* Y, int32_t* I_inout,
+                      void* ws, size_t ws_bytes, void* stream_v) {
+    if (!plan) return RMM_ERR_INVALID_ARG;
+    const rmm_problem& p = plan->p;
+    const bool given = (p.flags & RMM_FLAG_USE_GIVEN_INDICES) != 0;
+    const bool empty = p.n == 0 || p.m == 0;  // nothing to read or write but I
+    if (!empty && (!A || !B || !Y)) return RMM_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(Y)) return RMM_ERR_INVALID_ARG;
+    if (I_inout && (reinterpret_cast<uintptr_t>(I_inout) & 3u)) return RMM_ERR_INVALID_ARG;
+    if (given && !I_inout) return RMM_ERR_INVALID_ARG;
+    rmm_status st = check_workspace(plan, ws, ws_bytes);
+    if (st != RMM_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    const int es = plan->es;
+    const int64_t k = plan->k;
+
+    // ---- index set
+    int32_t* I = I_inout ? I_inout : ws_at<int32_t>(ws, plan->off_I);
+    const bool identity = !given && k == p.d;
+    if (!given) {
+        if (identity) {
+            if (I_inout && rmm::launch_identity(I_inout, k, static_cast<int>(p.heads), stream) != cudaSuccess)
+                return RMM_ERR_CUDA;
+        } else {
+            st = run_select(plan, A, I, nullptr, ws, stream);
+            if (st != RMM_OK) return st;
+        }
+    }
+    if (p.n == 0 || p.m == 0) return RMM_OK;
+
+    // ---- stage the gathered A columns (and K columns in QK mode)
+    rmm::GemmParams gp;
+    std::memset(&gp, 0, sizeof(gp));
+    const uint32_t box_k = static_cast<uint32_t>(128 / es);
+    if (!identity) {
+        rmm::PackArgs pa{};
+        pa.src = A;
+        pa.dtype = p.dtype;
+        pa.rows = p.n;
+        pa.d = p.d;
+        pa.ld_src = p.lda;
+        pa.stride_src = p.stride_a;
+        pa.group = 1;
+        pa.I = I;
+        pa.I_stride = k;
+        pa.k = k;
+        pa.dst = ws_at<void>(ws, plan->off_apack);
+        pa.ld_dst = plan->ldp;
+        pa.stride_dst = p.n * plan->ldp;
+        pa.heads = static_cast<int>(p.heads);
+        if (rmm::launch_pack(pa, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        if (!encode_kmajor_map(&gp.map_a, es, pa.dst, k, p.n, p.heads, plan->ldp, p.n * plan->ldp, box_k, 128))
+            return RMM_ERR_CUDA;
+    } else {
+        if (!encode_kmajor_map(&gp.map_a, es, A, p.d, p.n, p.heads, p.lda, p.stride_a, box_k, 128))
+            return RMM_ERR_CUDA;
+    }
+
+    rmm::GemmLaunch gl;
+    gl.dtype = p.dtype;
+    gl.bn = plan->bn;
+    gl.num_sms = plan->num_sms;
+    gp.Y = Y;
+    gp.ldy = p.ldy;
+    gp.stride_y = p.stride_y;
+    gp.n = static_cast<int32_t>(p.n);
+    gp.m = static_cast<int32_t>(p.m);
+    gp.k = static_cast<int32_t>(k);
+    gp.d = static_cast<int32_t>(p.d);
+    gp.heads = static_cast<int32_t>(p.heads);
+    gp.group = plan->group;
+    gp.m_tiles = static_cast<int32_t>((p.n + 127) / 128);
+    gp.n_tiles = static_cast<int32_t>((p.m + plan->bn - 1) / plan->bn);
+    gp.alpha = p.alpha;
+    gp.causal = (p.flags & RMM_FLAG_CAUSAL) ? 1 : 0;
+    gp.err = ws_at<int>(ws, plan->off_err);
+    gp.b_head_div = 1;
+
+    if (p.mode == RMM_QK) {
+        gl.b_gather = false;
+        if (!identity) {
+            rmm::PackArgs pb{};
+            pb.src = B;
+            pb.dtype = p.dtype;
+            pb.rows = p.m;
+            pb.d = p.d;
+            pb.ld_src = p.ldb;
+            pb.stride_src = p.stride_b;
+            pb.group = plan->group;
+            pb.I = I;
+            pb.I_stride = k;
+            pb.k = k;
+            pb.dst = ws_at<void>(ws, plan->off_bpack);
+            pb.ld_dst = plan->ldp;
+            pb.stride_dst = p.m * plan->ldp;
+            pb.heads = static_cast<int>(p.heads);
+            if (rmm::launch_pack(pb, stream) != cudaSuccess) return RMM_ERR_CUDA;
+            if (!encode_kmajor_map(&gp.map_b, es, pb.dst, k, p.m, p.heads, plan->ldp, p.m * plan->ldp, box_k,
+                                   static_cast<uint32_t>(plan->bn)))
+                return RMM_ERR_CUDA;
+        } else {
+            if (!encode_kmajor_map(&gp.map_b, es, B, p.d, p.m, p.kv_heads, p.ldb, p.stride_b, box_k,
+                                   static_cast<uint32_t>(plan->bn)))
+                return RMM_ERR_CUDA;
+            gp.b_head_div = plan->group;
+        }
+    } else if (p.dtype == RMM_F32) {
+        // tf32 operands are staged K-major: B[I, :] is written transposed (m x k).
+        gl.b_gather = false;
+        rmm::PackArgs pb{};
+        pb.src = B;
+        pb.dtype = p.dtype;
+        pb.rows = p.m;
+        pb.d = p.d;
+        pb.ld_src = p.ldb;
+        pb.stride_src = p.stride_b;
+        pb.group = plan->group;
+        pb.I = identity ? nullptr : I;
+        pb.I_stride = k;
+        pb.k = k;
+        pb.dst = ws_at<void>(ws, plan->off_bpack);
+        pb.ld_dst = plan->ldp;
+        pb.stride_dst = p.m * plan->ldp;
+        pb.heads = static_cast<int>(p.heads);
+        if (rmm::launch_pack_rows_transposed(pb, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        if (!encode_kmajor_map(&gp.map_b, es, pb.dst, k, p.m, p.heads, plan->ldp, p.m * plan->ldp, box_k,
+                               static_cast<uint32_t>(plan->bn)))
+            return RMM_ERR_CUDA;
+    } else {
+        gl.b_gather = true;
+        gp.B = B;
+        gp.ldb = p.ldb;
+        gp.stride_b = p.stride_b;
+        gp.I = identity ? nullptr : I;
+        gp.I_stride = k;
+    }
+    return rmm::launch_gemm(gp, gl, stream) == cudaSuccess ? RMM_OK : RMM_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+void rmm_problem_init(rmm_problem* p, int32_t mode, int32_t dtype, int64_t n, int64_t d, int64_t m) {
+    if (!p) return;
+    std::memset(p, 0, sizeof(*p));
+    p->mode = mode;
+    p->dtype = dtype;
+    p->n = n;
+    p->d = d;
+    p->m = m;
+    p->lda = d;
+    p->ldb = mode == RMM_QK ? d : m;
+    p->ldy = m;
+    p->heads = 1;
+    p->kv_heads = 1;
+    p->rho = 1.0;
+    p->alpha = 1.0f;
+}
+
+rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspace_bytes) {
+    if (!out) return RMM_ERR_INVALID_ARG;
+    *out = nullptr;
+    rmm_status st = validate_problem(p);
+    if (st != RMM_OK) return st;
+    rmm_plan* plan = new (std::nothrow) rmm_plan;
+    if (!plan) return RMM_ERR_UNSUPPORTED;
+    std::memset(plan, 0, sizeof(*plan));
+    plan->p = *p;
+    plan->es = p->dtype == RMM_F32 ? 4 : 2;
+    plan->k = p->k > 0 ? p->k : retained_count(p->rho, p->d);
+    plan->ldp = (plan->k + 7) / 8 * 8;
+    plan->group = static_cast<int>(p->heads / p->kv_heads);
+    const bool given = (p->flags & RMM_FLAG_USE_GIVEN_INDICES) != 0;
+    plan->need_select = !given && plan->k < p->d;
+    plan->bn = p->m <= 128 ? 128 : 256;
+
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+        cudaGetLastError();
+        delete plan;
+        return RMM_ERR_CUDA;
+    }
+    plan->num_sms = sms;
+
+    // Selection kernels need every score of a head in shared memory.
+    const bool select_possible = p->d <= rmm::kMaxSelectD;
+    if (plan->need_select && !select_possible) {
+        delete plan;
+        return RMM_ERR_UNSUPPORTED;
+    }
+    const size_t head_bytes = static_cast<size_t>(p->n) * p->d * plan->es;
+    plan->fused_select = head_bytes <= kFusedSelectBytes && rmm::normselect_smem_bytes(p->d, p->dtype) <= 200 * 1024;
+    const int vec = 16 / plan->es;
+    const int64_t colblocks = (p->d + 32 * vec - 1) / (32 * vec);
+    const int64_t target = 4LL * sms;
+    int64_t nsplit = (target + colblocks * p->heads - 1) / (colblocks * p->heads);
+    const int64_t max_split = (p->n + 31) / 32;
+    if (nsplit > max_split) nsplit = max_split;
+    if (nsplit < 1) nsplit = 1;
+    int64_t rps = (p->n + nsplit - 1) / nsplit;
+    if (rps < 1) rps = 1;
+    nsplit = p->n > 0 ? (p->n + rps - 1) / rps : 1;
+    plan->nsplit = static_cast<int>(nsplit);
+    plan->rows_per_split = rps;
+
+    size_t off = 0;
+    plan->off_err = off;
+    off += 256;
+    plan->off_partials = off;
+    if (select_possible && !plan->fused_select)
+        off += align256(static_cast<size_t>(p->heads) * nsplit * p->d * sizeof(float));
+    plan->off_I = off;
+    off += align256(static_cast<size_t>(p->heads) * plan->k * sizeof(int32_t));
+    plan->off_apack = off;
+    off += align256(static_cast<size_t>(p->heads) * p->n * plan->ldp * plan->es);
+    plan->off_bpack = off;
+    if (p->mode == RMM_QK || p->dtype == RMM_F32)
+        off += align256(static_cast<size_t>(p->heads) * p->m * plan->ldp * plan->es);
+    plan->ws_bytes = off;
+    if (workspace_bytes) *workspace_bytes = plan->ws_bytes;
+    *out = plan;
+    return RMM_OK;
+}
+
+rmm_status rmm_plan_destroy(rmm_plan* plan) {
+    delete plan;
+    return RMM_OK;
+}
+
+int64_t rmm_plan_k(const rmm_plan* plan) { return plan ? plan->k : -1; }
+
+size_t rmm_plan_workspace_size(const rmm_plan* plan) { return plan ? plan->ws_bytes : 0; }
+
+rmm_status rmm_select(const rmm_plan* plan, const void* A, int32_t* I, float* s2, void* ws, size_t ws_bytes,
+                      void* stream) {
+    if (!plan || !A || !I) return RMM_ERR_INVALID_ARG;
+    if (!aligned16(A) || (reinterpret_cast<uintptr_t>(I) & 3u) || (s2 && (reinterpret_cast<uintptr_t>(s2) & 3u)))
+        return RMM_ERR_INVALID_ARG;
+    if (plan->p.d > rmm::kMaxSelectD) return RMM_ERR_UNSUPPORTED;
+    rmm_status st = check_workspace(plan, ws, ws_bytes);
+    if (st != RMM_OK) return st;
+    return run_select(plan, A, I, s2, ws, static_cast<cudaStream_t>(stream));
+}
+
+rmm_status rmm_matmul(const rmm_plan* plan, const void* A, const void* B, void* Y, int32_t* I_inout, void* ws,
+                      size_t ws_bytes, void* stream) {
+    if (!plan) return RMM_ERR_INVALID_ARG;
+    if (plan->p.heads != 1) return RMM_ERR_INVALID_ARG;
+    return run_matmul(plan, A, B, Y, I_inout, ws, ws_bytes, stream);
+}
+
+rmm_status rmm_matmul_batched(const rmm_plan* plan, const void* A, const void* B, void* Y, int32_t* I_inout,
+                              void* ws, size_t ws_bytes, void* stream) {
+    return run_matmul(plan, A, B, Y, I_inout, ws, ws_bytes, stream);
+}
+
+rmm_status rmm_workspace_init(const rmm_plan* plan, void* ws, size_t ws_bytes, void* stream) {
+    if (!plan) return RMM_ERR_INVALID_ARG;
+    rmm_status st = check_workspace(plan, ws, ws_bytes);
+    if (st != RMM_OK) return st;
+    if (cudaMemsetAsync(ws_at<int>(ws, plan->off_err), 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return RMM_ERR_CUDA;
+    return RMM_OK;
+}
+
+rmm_status rmm_workspace_status(const rmm_plan* plan, void* ws, void* stream) {
+    if (!plan || !ws) return RMM_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return RMM_ERR_CUDA;
+    int word = 0;
+    int* dev_word = ws_at<int>(ws, plan->off_err);
+    if (cudaMemcpy(&word, dev_word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return RMM_ERR_CUDA;
+    if (word != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(dev_word, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return RMM_ERR_CUDA;
+        return RMM_ERR_TIMEOUT;
+    }
+    return RMM_OK;
+}
+
+const char* rmm_status_string(rmm_status s) {
+    switch (s) {
+        case RMM_OK: return "RMM_OK";
+        case RMM_ERR_INVALID_ARG: return "RMM_ERR_INVALID_ARG";
+        case RMM_ERR_UNSUPPORTED: return "RMM_ERR_UNSUPPORTED";
+        case RMM_ERR_WORKSPACE: return "RMM_ERR_WORKSPACE";
+        case RMM_ERR_CUDA: return "RMM_ERR_CUDA";
+        case RMM_ERR_TIMEOUT: return "RMM_ERR_TIMEOUT";
+    }
+    return "RMM_ERR_UNKNOWN";
+}
+
+const char* rmm_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,89 @@
+// rmm_internal.h -- launchers shared between the C-ABI layer (rmm_api.cu) and
+// the kernels.  Not part of the public ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace rmm {
+
+// ---------------------------------------------------------------- selection
+struct SelectArgs {
+    const void* A;       // [heads][n][lda]
+    int dtype;           // RMM_BF16 / RMM_F32
+    int64_t n, d, lda, stride_a;
+    int heads;
+    int64_t k;
+    int32_t* I;          // [heads][k] out, ascending
+    float* s2;           // [heads][d] out or nullptr
+    // two-stage path only
+    float* partials;     // [heads][nsplit][d]
+    int nsplit;
+    int64_t rows_per_split;
+};
+
+// Column sums of squares in fp32, one partial per row split.
+cudaError_t launch_colnorm(const SelectArgs& a, cudaStream_t s);
+// Sum the partials in split order, radix-select the k largest, emit I.
+cudaError_t launch_topk(const SelectArgs& a, cudaStream_t s);
+// Scores and selection in one CTA per head (small inputs).
+cudaError_t launch_normselect(const SelectArgs& a, cudaStream_t s);
+// I[h][j] = j for j < k (k == d: every index kept).
+cudaError_t launch_identity(int32_t* I, int64_t k, int heads, cudaStream_t s);
+
+constexpr int64_t kMaxSelectD = 49152;  // keys staged in shared memory (192 KiB)
+size_t topk_smem_bytes(int64_t d);
+size_t normselect_smem_bytes(int64_t d, int dtype);
+
+// ---------------------------------------------------------------- pack
+// dst[h][r][t] = src[h / group][r][I[h][t]] for t < k, 0 for k <= t < ld_dst.
+struct PackArgs {
+    const void* src;
+    int dtype;
+    int64_t rows, d, ld_src, stride_src;
+    int group;
+    const int32_t* I;
+    int64_t I_stride, k;
+    void* dst;
+    int64_t ld_dst, stride_dst;
+    int heads;
+};
+cudaError_t launch_pack(const PackArgs& a, cudaStream_t s);
+// dst[h][c][t] = src[h / group][I[h][t]][c]: gathered rows written K-major
+// (rows = number of source columns c; I == nullptr means I[t] = t).
+cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- GEMM
+// A operand: TMA tile loads from a 3-D map {K extent, rows, heads}, K-major.
+// B operand: either gathered rows of a d x m row-major matrix (LINEAR, PV;
+// MN-major in shared memory) or TMA tiles of an m x K row-major matrix
+// (QK; K-major).
+struct __align__(64) GemmParams {
+    CUtensorMap map_a;
+    CUtensorMap map_b;          // TMA-B mode only
+    const void* B;              // gather mode: base of B
+    int64_t ldb, stride_b;      // gather mode
+    const int32_t* I;           // gather mode: [heads][k] row indices, nullptr = identity
+    int64_t I_stride;
+    void* Y;
+    int64_t ldy, stride_y;
+    int32_t n, m, k, d;
+    int32_t heads, group;       // B head = h / group (gather mode)
+    int32_t b_head_div;         // TMA-B mode: B head coordinate = h / b_head_div
+    int32_t m_tiles, n_tiles;
+    float alpha;
+    int32_t causal;
+    int* err;
+};
+
+struct GemmLaunch {
+    int dtype;
+    bool b_gather;
+    int bn;           // 128 or 256
+    int num_sms;
+};
+cudaError_t launch_gemm(const GemmParams& p, const GemmLaunch& l, cudaStream_t s);
+size_t gemm_smem_bytes(int dtype, int bn);
+
+}  // namespace rmm

@@ -1,0 +1,124 @@
+// rmm_pack.cu -- staging of the gathered operand columns A[:, I] of Reduced
+// Matrix Multiplication ("Reduced Matrix Multiplication: Input-Adaptive
+// Matrix-Product Reduction for LLM Inference", §3.2: the product runs over the
+// retained slice A[:, I] only).  A row-major operand keeps the contraction
+// axis contiguous, so its retained columns are element-granular and cannot be
+// fetched by tensor-memory-access tiles; this pass compacts them into a dense
+// K-major buffer (rows x roundup(k, 8)) that the tensor-core GEMM then reads
+// with TMA.  Used for A in every mode and for K in the QK mode.
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "rmm_internal.h"
+
+namespace rmm {
+namespace {
+
+constexpr int kPackThreads = 256;
+constexpr int kPackRows = 16;  // rows per CTA; the 8 indices of a thread are reused across them
+
+// grid (ceil(ld_dst / (8*256)), ceil(rows / 16), heads).  Thread t owns output
+// columns [8t, 8t+8) of its CTA's slice; it loads their 8 source indices once
+// and writes 16-byte (bf16) or 2 x 16-byte (fp32) rows of the packed buffer.
+template <typename T>
+__global__ void __launch_bounds__(kPackThreads) pack_kernel(
+    const T* __restrict__ src, int64_t rows, int64_t d, int64_t ld_src, int64_t stride_src, int group,
+    const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
+    int64_t stride_dst) {
+    const int h = blockIdx.z;
+    const int64_t t0 = ((int64_t)blockIdx.x * kPackThreads + threadIdx.x) * 8;
+    if (t0 >= ld_dst) return;
+    int32_t idx[8];
+    bool live[8];
+    const int32_t* Ih = I + (int64_t)h * I_stride;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+        live[v] = t0 + v < k;
+        int32_t j = live[v] ? __ldg(Ih + t0 + v) : 0;
+        idx[v] = min(max(j, 0), (int32_t)(d - 1));  // keep every load in bounds
+    }
+    const T* sh = src + (int64_t)(h / group) * stride_src;
+    T* dh = dst + (int64_t)h * stride_dst;
+    const int64_t r_beg = (int64_t)blockIdx.y * kPackRows;
+    const int64_t r_end = min(rows, r_beg + kPackRows);
+    for (int64_t r = r_beg; r < r_end; ++r) {
+        const T* s = sh + r * ld_src;
+        T vals[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) vals[v] = live[v] ? s[idx[v]] : T(0.f);
+        T* o = dh + r * ld_dst + t0;
+        if constexpr (sizeof(T) == 2) {
+            *reinterpret_cast<uint4*>(o) = *reinterpret_cast<const uint4*>(vals);
+        } else {
+            reinterpret_cast<uint4*>(o)[0] = reinterpret_cast<const uint4*>(vals)[0];
+            reinterpret_cast<uint4*>(o)[1] = reinterpret_cast<const uint4*>(vals)[1];
+        }
+    }
+}
+
+// Transposing variant for fp32 operands: dst[h][c][t] = src[h / group][I[h][t]][c]
+// (t < k; 0 for k <= t < ld_dst), i.e. the gathered rows B[I, :] of a row-major
+// d x m matrix written K-major (m x ld_dst).  32 x 32 tiles through shared memory.
+template <typename T>
+__global__ void __launch_bounds__(256) pack_rows_transposed_kernel(
+    const T* __restrict__ src, int64_t d, int64_t cols, int64_t ld_src, int64_t stride_src, int group,
+    const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
+    int64_t stride_dst) {
+    __shared__ T tile[32][33];
+    const int h = blockIdx.z;
+    const int64_t t0 = (int64_t)blockIdx.x * 32, c0 = (int64_t)blockIdx.y * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+    const T* sh = src + (int64_t)(h / group) * stride_src;
+    const int32_t* Ih = I ? I + (int64_t)h * I_stride : nullptr;
+    for (int r = ty; r < 32; r += 8) {
+        const int64_t t = t0 + r, c = c0 + tx;
+        T v = T(0.f);
+        if (t < k && c < cols) {
+            int64_t j = Ih ? (int64_t)__ldg(Ih + t) : t;
+            j = j < 0 ? 0 : (j >= d ? d - 1 : j);
+            v = sh[j * ld_src + c];
+        }
+        tile[r][tx] = v;
+    }
+    __syncthreads();
+    T* dh = dst + (int64_t)h * stride_dst;
+    for (int r = ty; r < 32; r += 8) {
+        const int64_t c = c0 + r, t = t0 + tx;
+        if (c < cols && t < ld_dst) dh[c * ld_dst + t] = tile[tx][r];
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s) {
+    // a.rows = columns of the source (m), a.d = rows of the source, a.I may be null (identity)
+    dim3 grid((unsigned)((a.ld_dst + 31) / 32), (unsigned)((a.rows + 31) / 32), (unsigned)a.heads);
+    if (grid.y == 0) return cudaSuccess;
+    if (a.dtype == 1)
+        pack_rows_transposed_kernel<float><<<grid, 256, 0, s>>>(
+            (const float*)a.src, a.d, a.rows, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k,
+            (float*)a.dst, a.ld_dst, a.stride_dst);
+    else
+        pack_rows_transposed_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+            (const __nv_bfloat16*)a.src, a.d, a.rows, a.ld_src, a.stride_src, a.group, a.I, a.I_stride,
+            a.k, (__nv_bfloat16*)a.dst, a.ld_dst, a.stride_dst);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack(const PackArgs& a, cudaStream_t s) {
+    dim3 grid((unsigned)((a.ld_dst + 8 * kPackThreads - 1) / (8 * kPackThreads)),
+              (unsigned)((a.rows + kPackRows - 1) / kPackRows), (unsigned)a.heads);
+    if (grid.y == 0) return cudaSuccess;
+    if (a.dtype == 1)
+        pack_kernel<float><<<grid, kPackThreads, 0, s>>>(
+            (const float*)a.src, a.rows, a.d, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k,
+            (float*)a.dst, a.ld_dst, a.stride_dst);
+    else
+        pack_kernel<__nv_bfloat16><<<grid, kPackThreads, 0, s>>>(
+            (const __nv_bfloat16*)a.src, a.rows, a.d, a.ld_src, a.stride_src, a.group, a.I,
+            a.I_stride, a.k, (__nv_bfloat16*)a.dst, a.ld_dst, a.stride_dst);
+    return cudaGetLastError();
+}
+
+}  // namespace rmm

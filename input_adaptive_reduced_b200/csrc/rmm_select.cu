@@ -1,0 +1,391 @@
+// rmm_select.cu -- activation-aware index selection of Reduced Matrix
+// Multiplication: column scores s_j = ||A[:, j]||_2 and I = TopK(s, k)
+// ("Reduced Matrix Multiplication: Input-Adaptive Matrix-Product Reduction for
+// LLM Inference", §3.2 "Activation-aware dimension selection"; the same rule
+// per attention head in §3.3).
+//
+// Scores are kept squared (ordering by s^2 equals ordering by s) in fp32.
+// Every column is summed in the same fixed order regardless of its position,
+// so equal columns give bit-equal scores and the result does not depend on
+// the launch.  Selection compares the fp32 bit patterns (monotone for
+// non-negative values) with a 4-pass radix select; among equal scores the
+// lower index is kept, and I is written in ascending order.
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "rmm_internal.h"
+
+namespace rmm {
+namespace {
+
+template <typename T>
+struct Vec16;
+template <>
+struct Vec16<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ static void load(const __nv_bfloat16* p, float (&x)[8]) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(w[i] << 16);
+            x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+};
+template <>
+struct Vec16<float> {
+    static constexpr int N = 4;
+    __device__ static void load(const float* p, float (&x)[4]) {
+        const float4 u = __ldg(reinterpret_cast<const float4*>(p));
+        x[0] = u.x;
+        x[1] = u.y;
+        x[2] = u.z;
+        x[3] = u.w;
+    }
+};
+
+// ------------------------------------------------------------------ colnorm
+// grid (ceil(d / (32*V)), nsplit, heads), 256 threads.  Warp w of split s sums
+// rows r0+w, r0+w+8, ... of its 32*V columns in increasing row order; the 8
+// warp partials are added in warp order; splits are added in split order by
+// the TopK kernel.
+template <typename T>
+__global__ void __launch_bounds__(256) colnorm_kernel(const T* __restrict__ A, int64_t n, int64_t d,
+                                                      int64_t lda, int64_t stride_a,
+                                                      int64_t rows_per_split, int nsplit,
+                                                      float* __restrict__ partials) {
+    constexpr int V = Vec16<T>::N;
+    constexpr int COLS = 32 * V;
+    __shared__ float red[8][COLS];
+    const int h = blockIdx.z, split = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t col = (int64_t)blockIdx.x * COLS + lane * V;
+    const int64_t r0 = (int64_t)split * rows_per_split;
+    const int64_t r1 = min(n, r0 + rows_per_split);
+    float acc[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) acc[v] = 0.f;
+    if (col < d) {
+        const T* base = A + (int64_t)h * stride_a + col;
+        int64_t r = r0 + warp;
+        for (; r + 24 < r1; r += 32) {
+            float x0[V], x1[V], x2[V], x3[V];
+            Vec16<T>::load(base + r * lda, x0);
+            Vec16<T>::load(base + (r + 8) * lda, x1);
+            Vec16<T>::load(base + (r + 16) * lda, x2);
+            Vec16<T>::load(base + (r + 24) * lda, x3);
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                acc[v] = fmaf(x0[v], x0[v], acc[v]);
+                acc[v] = fmaf(x1[v], x1[v], acc[v]);
+                acc[v] = fmaf(x2[v], x2[v], acc[v]);
+                acc[v] = fmaf(x3[v], x3[v], acc[v]);
+            }
+        }
+        for (; r < r1; r += 8) {
+            float x0[V];
+            Vec16<T>::load(base + r * lda, x0);
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[v] = fmaf(x0[v], x0[v], acc[v]);
+        }
+    }
+#pragma unroll
+    for (int v = 0; v < V; ++v) red[warp][lane * V + v] = acc[v];
+    __syncthreads();
+    for (int c = threadIdx.x; c < COLS; c += 256) {
+        float s = red[0][c];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) s += red[w][c];
+        const int64_t gcol = (int64_t)blockIdx.x * COLS + c;
+        if (gcol < d) partials[((int64_t)h * nsplit + split) * d + gcol] = s;
+    }
+}
+
+// ------------------------------------------------------------------ TopK core
+// Works on keys[0..d) in shared memory (fp32 bit patterns of s^2 >= 0) with a
+// 1024-thread block.  Writes the k selected indices, ascending, to out[].
+struct TopkShared {
+    uint32_t hist[256];
+    uint32_t prefix;
+    uint32_t remaining;
+    uint32_t warp_gt[32];
+    uint32_t warp_eq[32];
+    uint32_t eq_before[32];
+    uint32_t sel_before[32];
+};
+
+__device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k, int32_t* out,
+                                      TopkShared& sh) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t prefix = 0, mask = 0, remaining = (uint32_t)k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        if (tid < 256) sh.hist[tid] = 0;
+        __syncthreads();
+        for (int64_t base = 0; base < d; base += 1024) {
+            const int64_t j = base + tid;
+            int bin = -1;
+            if (j < d) {
+                const uint32_t key = keys[j];
+                if ((key & mask) == prefix) bin = (int)((key >> shift) & 255u);
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, bin);
+            if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], (uint32_t)__popc(peers));
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // lane l owns bins 255-8l down to 248-8l (descending order)
+            uint32_t c[8], tot = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                c[i] = sh.hist[255 - 8 * lane - i];
+                tot += c[i];
+            }
+            uint32_t incl = tot;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            const uint32_t excl = incl - tot;
+            if (excl < remaining && remaining <= incl) {
+                uint32_t above = excl;
+                for (int i = 0; i < 8; ++i) {
+                    if (above + c[i] >= remaining) {
+                        const uint32_t b = 255u - 8u * lane - i;
+                        sh.prefix = prefix | (b << shift);
+                        sh.remaining = remaining - above;
+                        break;
+                    }
+                    above += c[i];
+                }
+            }
+        }
+        __syncthreads();
+        prefix = sh.prefix;
+        remaining = sh.remaining;
+        mask |= 255u << shift;
+        __syncthreads();
+    }
+    const uint32_t T = prefix;      // the k-th largest key
+    const uint32_t r = remaining;   // how many keys equal to T are kept (lowest indices)
+
+    // Each warp owns a contiguous segment; count, scan over warps, then emit.
+    const int64_t seg = ((d + 31) / 32 + 31) / 32 * 32;
+    const int64_t beg = (int64_t)warp * seg;
+    const int64_t end = min(d, beg + seg);
+    uint32_t gt = 0, eq = 0;
+    for (int64_t j0 = beg; j0 < end; j0 += 32) {
+        const int64_t j = j0 + lane;
+        const uint32_t key = j < end ? keys[j] : 0u;
+        gt += __popc(__ballot_sync(0xffffffffu, j < end && key > T));
+        eq += __popc(__ballot_sync(0xffffffffu, j < end && key == T));
+    }
+    if (lane == 0) {
+        sh.warp_gt[warp] = gt;
+        sh.warp_eq[warp] = eq;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t e = sh.warp_eq[lane], g = sh.warp_gt[lane];
+        uint32_t incl = e;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        const uint32_t eb = incl - e;
+        const uint32_t take_eq = eb >= r ? 0u : min(e, r - eb);
+        const uint32_t sel = g + take_eq;
+        uint32_t sincl = sel;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, sincl, off);
+            if (lane >= off) sincl += y;
+        }
+        sh.eq_before[lane] = eb;
+        sh.sel_before[lane] = sincl - sel;
+    }
+    __syncthreads();
+    uint32_t eq_run = sh.eq_before[warp], sel_run = sh.sel_before[warp];
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int64_t j0 = beg; j0 < end; j0 += 32) {
+        const int64_t j = j0 + lane;
+        const uint32_t key = j < end ? keys[j] : 0u;
+        const bool is_gt = j < end && key > T;
+        const bool is_eq = j < end && key == T;
+        const unsigned em = __ballot_sync(0xffffffffu, is_eq);
+        const uint32_t rank = eq_run + __popc(em & lt_mask);
+        const bool sel = is_gt || (is_eq && rank < r);
+        const unsigned sm = __ballot_sync(0xffffffffu, sel);
+        const uint32_t pos = sel_run + __popc(sm & lt_mask);
+        if (sel && pos < (uint32_t)k) out[pos] = (int32_t)j;
+        eq_run += __popc(em);
+        sel_run += __popc(sm);
+    }
+}
+
+// ------------------------------------------------------------------ TopK
+// One 1024-thread CTA per head: sum the split partials in split order, then
+// select.
+__global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ partials, int nsplit,
+                                                    int64_t d, int64_t k, int32_t* __restrict__ I,
+                                                    float* __restrict__ s2) {
+    extern __shared__ uint32_t keys[];
+    __shared__ TopkShared sh;
+    const int h = blockIdx.x;
+    const float* p = partials + (int64_t)h * nsplit * d;
+    for (int64_t j = threadIdx.x; j < d; j += 1024) {
+        float s = p[j];
+        for (int sp = 1; sp < nsplit; ++sp) s += p[(int64_t)sp * d + j];
+        keys[j] = __float_as_uint(s);
+        if (s2) s2[(int64_t)h * d + j] = s;
+    }
+    __syncthreads();
+    radix_select_and_emit(keys, d, k, I + (int64_t)h * k, sh);
+}
+
+// ------------------------------------------------------------------ fused
+// One 1024-thread CTA per head.  Threads form RG row groups x (1024/RG)
+// column lanes; lane c of group g sums rows g, g+RG, ... of its 16-byte
+// column vectors; the RG partials are added in group order.
+template <typename T>
+__global__ void __launch_bounds__(1024) normselect_kernel(const T* __restrict__ A, int64_t n,
+                                                          int64_t d, int64_t lda, int64_t stride_a,
+                                                          int rg, int64_t k, int32_t* __restrict__ I,
+                                                          float* __restrict__ s2) {
+    constexpr int V = Vec16<T>::N;
+    extern __shared__ uint32_t smem[];
+    uint32_t* keys = smem;                                        // d
+    float* red = reinterpret_cast<float*>(smem + ((d + 3) & ~3ll)); // rg x d when rg > 1
+    __shared__ TopkShared sh;
+    const int h = blockIdx.x;
+    const int tpr = 1024 / rg;
+    const int g = threadIdx.x / tpr, tl = threadIdx.x % tpr;
+    const T* Ah = A + (int64_t)h * stride_a;
+    const int64_t dv = d / V;
+    for (int64_t cv = tl; cv < dv; cv += tpr) {
+        float acc[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = 0.f;
+        int64_t r = g;
+        for (; r + 3 * rg < n; r += 4 * rg) {
+            float x0[V], x1[V], x2[V], x3[V];
+            Vec16<T>::load(Ah + r * lda + cv * V, x0);
+            Vec16<T>::load(Ah + (r + rg) * lda + cv * V, x1);
+            Vec16<T>::load(Ah + (r + 2 * rg) * lda + cv * V, x2);
+            Vec16<T>::load(Ah + (r + 3 * rg) * lda + cv * V, x3);
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                acc[v] = fmaf(x0[v], x0[v], acc[v]);
+                acc[v] = fmaf(x1[v], x1[v], acc[v]);
+                acc[v] = fmaf(x2[v], x2[v], acc[v]);
+                acc[v] = fmaf(x3[v], x3[v], acc[v]);
+            }
+        }
+        for (; r < n; r += rg) {
+            float x0[V];
+            Vec16<T>::load(Ah + r * lda + cv * V, x0);
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[v] = fmaf(x0[v], x0[v], acc[v]);
+        }
+        if (rg == 1) {
+#pragma unroll
+            for (int v = 0; v < V; ++v) keys[cv * V + v] = __float_as_uint(acc[v]);
+        } else {
+#pragma unroll
+            for (int v = 0; v < V; ++v) red[(int64_t)g * d + cv * V + v] = acc[v];
+        }
+    }
+    __syncthreads();
+    if (rg > 1) {
+        for (int64_t j = threadIdx.x; j < d; j += 1024) {
+            float s = red[j];
+            for (int gg = 1; gg < rg; ++gg) s += red[(int64_t)gg * d + j];
+            keys[j] = __float_as_uint(s);
+        }
+        __syncthreads();
+    }
+    if (s2) {
+        for (int64_t j = threadIdx.x; j < d; j += 1024) s2[(int64_t)h * d + j] = __uint_as_float(keys[j]);
+    }
+    radix_select_and_emit(keys, d, k, I + (int64_t)h * k, sh);
+}
+
+__global__ void identity_kernel(int32_t* __restrict__ I, int64_t k, int heads) {
+    const int64_t total = k * heads;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x)
+        I[i] = (int32_t)(i % k);
+}
+
+int normselect_row_groups(int64_t d, int dtype) {
+    const int64_t dv = d / (dtype == 1 ? 4 : 8);
+    int rg = 1;
+    while (rg * 2 * dv <= 1024 && rg < 1024) rg *= 2;
+    return rg;
+}
+
+}  // namespace
+
+size_t topk_smem_bytes(int64_t d) { return (size_t)d * 4; }
+
+size_t normselect_smem_bytes(int64_t d, int dtype) {
+    const int rg = normselect_row_groups(d, dtype);
+    size_t bytes = (size_t)((d + 3) & ~3ll) * 4;
+    if (rg > 1) bytes += (size_t)rg * d * 4;
+    return bytes;
+}
+
+cudaError_t launch_colnorm(const SelectArgs& a, cudaStream_t s) {
+    const int V = a.dtype == 1 ? 4 : 8;
+    dim3 grid((unsigned)((a.d + 32 * V - 1) / (32 * V)), (unsigned)a.nsplit, (unsigned)a.heads);
+    if (a.dtype == 1)
+        colnorm_kernel<float><<<grid, 256, 0, s>>>((const float*)a.A, a.n, a.d, a.lda, a.stride_a,
+                                                   a.rows_per_split, a.nsplit, a.partials);
+    else
+        colnorm_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)a.A, a.n, a.d,
+                                                           a.lda, a.stride_a, a.rows_per_split,
+                                                           a.nsplit, a.partials);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const SelectArgs& a, cudaStream_t s) {
+    const size_t smem = topk_smem_bytes(a.d);
+    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    topk_kernel<<<a.heads, 1024, smem, s>>>(a.partials, a.nsplit, a.d, a.k, a.I, a.s2);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_normselect(const SelectArgs& a, cudaStream_t s) {
+    const int rg = normselect_row_groups(a.d, a.dtype);
+    const size_t smem = normselect_smem_bytes(a.d, a.dtype);
+    cudaError_t e;
+    if (a.dtype == 1) {
+        e = cudaFuncSetAttribute(normselect_kernel<float>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        normselect_kernel<float><<<a.heads, 1024, smem, s>>>((const float*)a.A, a.n, a.d, a.lda,
+                                                             a.stride_a, rg, a.k, a.I, a.s2);
+    } else {
+        e = cudaFuncSetAttribute(normselect_kernel<__nv_bfloat16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        normselect_kernel<__nv_bfloat16><<<a.heads, 1024, smem, s>>>(
+            (const __nv_bfloat16*)a.A, a.n, a.d, a.lda, a.stride_a, rg, a.k, a.I, a.s2);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_identity(int32_t* I, int64_t k, int heads, cudaStream_t s) {
+    const int64_t total = k * heads;
+    const int64_t want = (total + 255) / 256;
+    const int blocks = (int)(want < 1024 ? (want > 0 ? want : 1) : 1024);
+    identity_kernel<<<blocks, 256, 0, s>>>(I, k, heads);
+    return cudaGetLastError();
+}
+
+}  // namespace rmm

@@ -1,0 +1,94 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports exactly
+the entry points include/rmm.h declares, and rejects bad problems on the host
+before touching a device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import input_adaptive_reduced_b200 as rmm
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "rmm.h")).read()
+    return sorted(set(re.findall(r"RMM_API\s+[\w\s\*]+?\b(rmm_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names():
+    assert _declared() == sorted(rmm.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.check_output(["nm", "-D", "--defined-only", rmm.library_path], text=True)
+    exported = sorted(l.split()[-1] for l in out.splitlines() if l.split()[-1].startswith("rmm_"))
+    assert exported == _declared()
+    for name in _declared():
+        assert getattr(rmm.lib, name) is not None
+
+
+def test_no_cuda_runtime_symbols_leak():
+    out = subprocess.check_output(["nm", "-D", "--defined-only", rmm.library_path], text=True)
+    assert not [l for l in out.splitlines() if " cuda" in l]
+
+
+def test_status_strings_and_version():
+    assert rmm.rmm_status_string(rmm.RMM_OK) == "RMM_OK"
+    assert rmm.rmm_status_string(rmm.RMM_ERR_TIMEOUT) == "RMM_ERR_TIMEOUT"
+    assert rmm.rmm_status_string(99) == "RMM_ERR_UNKNOWN"
+    assert re.fullmatch(r"\d+\.\d+\.\d+", rmm.rmm_version())
+
+
+def test_problem_init_defaults():
+    p = rmm.rmm_problem_init(rmm.RMM_QK, rmm.RMM_BF16, 10, 128, 40)
+    assert (p.lda, p.ldb, p.ldy, p.heads, p.kv_heads, p.rho, p.alpha) == (128, 128, 40, 1, 1, 1.0, 1.0)
+    p = rmm.rmm_problem_init(rmm.RMM_LINEAR, rmm.RMM_BF16, 10, 64, 40)
+    assert p.ldb == 40
+
+
+def _status(p):
+    h = ctypes.c_void_p()
+    ws = ctypes.c_size_t()
+    s = rmm.lib.rmm_plan_create(ctypes.byref(h), ctypes.byref(p), ctypes.byref(ws))
+    if h.value:
+        rmm.lib.rmm_plan_destroy(h)
+    return s
+
+
+def _base():
+    p = rmm.rmm_problem_init(rmm.RMM_LINEAR, rmm.RMM_BF16, 64, 256, 256)
+    p.rho = 0.5
+    return p
+
+
+@pytest.mark.parametrize("field,value", [
+    ("mode", 7), ("dtype", 5), ("n", -1), ("d", 0), ("d", 250), ("m", 12), ("lda", 200),
+    ("lda", 260), ("ldy", 100), ("ldb", 100), ("heads", 0), ("kv_heads", 3), ("rho", 0.0),
+    ("rho", 1.5), ("k", 300), ("k", -2), ("flags", 8), ("flags", 1),
+])
+def test_invalid_problems_are_rejected_on_the_host(field, value):
+    p = _base()
+    setattr(p, field, value)
+    assert _status(p) == rmm.RMM_ERR_INVALID_ARG
+
+
+def test_valid_problem_reaches_the_device_query():
+    # Validation passes, so the next step asks the CUDA runtime for the SM count:
+    # OK on a GPU machine, RMM_ERR_CUDA where there is no device.
+    import torch
+    want = rmm.RMM_OK if torch.cuda.is_available() else rmm.RMM_ERR_CUDA
+    assert _status(_base()) == want
+
+
+def test_null_arguments():
+    assert rmm.lib.rmm_plan_create(None, None, None) == rmm.RMM_ERR_INVALID_ARG
+    h = ctypes.c_void_p()
+    assert rmm.lib.rmm_plan_create(ctypes.byref(h), None, None) == rmm.RMM_ERR_INVALID_ARG
+    assert rmm.lib.rmm_plan_destroy(None) == rmm.RMM_OK
+    assert rmm.lib.rmm_plan_k(None) == -1
+    assert rmm.lib.rmm_plan_workspace_size(None) == 0
+    assert rmm.lib.rmm_matmul(None, None, None, None, None, None, 0, None) == rmm.RMM_ERR_INVALID_ARG
+    assert rmm.lib.rmm_select(None, None, None, None, None, 0, None) == rmm.RMM_ERR_INVALID_ARG

@@ -1,0 +1,214 @@
+"""GPU parity of the CUDA path (through the C ABI) against the CPU oracle on
+oracle-scale inputs: several tiles and ragged tails, every mode, the
+tie-break, given index sets, empty and degenerate shapes.
+
+Inputs come from workloads/ with the oracle-measured score gap of
+tests/gap.py, so that fp32 (GPU) and fp64 (oracle) scores order the
+boundary the same way."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests import gap
+from tests.parity import assert_indices_equal, assert_product_close, np64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rmm(cuda_device):
+    import input_adaptive_reduced_b200 as r
+    return r
+
+
+def _linear_case(rmm, A, B, rho, rows=None):
+    dev = torch.device("cuda")
+    Ag, Bg = A.to(dev), B.to(dev)
+    Y, I = rmm.matmul(Ag, Bg, rho=rho, return_indices=True)
+    torch.cuda.synchronize()
+    I_ref, _ = oracle.select(A, rho=rho)
+    assert_indices_equal(I, I_ref)
+    A64, B64 = oracle.as_f64(A), oracle.as_f64(B)
+    r = slice(None) if rows is None else rows
+    Y_ref = oracle.reduced_product(A64, B64, I_ref, rows)
+    assert_product_close(Y[r] if rows is None else Y[rows], Y_ref,
+                         np.abs(A64[r][:, I_ref]), np.abs(B64[I_ref, :]))
+    return Y, I
+
+
+@pytest.mark.parametrize("rho", [0.25, 0.5, 1.0])
+@pytest.mark.parametrize("seed", [1, 2])
+def test_linear_fp32_tiny(rmm, rho, seed):
+    """64 x 256 x 256 fp32 (tf32 tensor cores), all sorted scores >= 1e-3 apart."""
+    A, B = W.linear_small(seed)
+    g = gap.all_gaps_gain(oracle.column_scores_sq(A))
+    A, B = W.linear_small(seed, col_gain=g)
+    assert gap.min_adjacent_gap(oracle.column_scores_sq(A)) >= 1e-3
+    _linear_case(rmm, A, B, rho)
+
+
+@pytest.mark.parametrize("direction", ["copy_up", "copy_down"])
+@pytest.mark.parametrize("rho", [0.25, 0.5])
+def test_exact_tie_lower_index_wins(rmm, rho, direction):
+    """Duplicated columns straddling the k-th rank: equal scores, lower index kept."""
+    A, B = W.linear_small(5)
+    A, B = W.linear_small(5, col_gain=gap.all_gaps_gain(oracle.column_scores_sq(A)))
+    s2 = oracle.column_scores_sq(A)
+    order = gap.descending_order(s2)
+    k = oracle.retained_count(rho, A.shape[1])
+    src = int(order[k - 1])  # the last kept column
+    dropped = order[k:].tolist()
+    # copy it over a dropped column above it (src stays kept) or below it (the copy wins)
+    cands = [j for j in dropped if (j > src if direction == "copy_up" else j < src)]
+    if not cands:
+        pytest.skip("no dropped column on that side of the boundary column")
+    dst = cands[0]
+    A2 = W.duplicate_columns(A, [(src, dst)])
+    s2b = oracle.column_scores_sq(A2)
+    assert s2b[src] == s2b[dst]
+    Y, I = _linear_case(rmm, A2, B, rho)
+    lo, hi = min(src, dst), max(src, dst)
+    got = set(I.cpu().tolist())
+    assert lo in got and hi not in got
+
+
+LINEAR_SHAPES = [
+    ("up", 200, 4096, 520),
+    ("down", 136, 14336, 264),
+    ("up", 1, 8192, 264),
+    ("up", 16, 8192, 776),
+    ("down", 130, 136, 24),
+]
+
+
+@pytest.mark.parametrize("kind,n,d,m", LINEAR_SHAPES)
+def test_linear_bf16(rmm, kind, n, d, m):
+    rhos = [0.5, 0.7, 0.8, 1.0]
+    ks = [oracle.retained_count(r, d) for r in rhos]
+    gen = W.mlp_up if kind == "up" else W.mlp_down
+    (A, B), _ = gap.enforce_boundary_gaps(lambda g: gen(11, n=n, d=d, m=m, col_gain=g),
+                                          lambda x: gap.scores_2d(x[0]), ks)
+    for rho in rhos:
+        _linear_case(rmm, A, B, rho)
+
+
+def test_select_scores_and_indices(rmm):
+    A, _ = W.mlp_up(3, n=300, d=4096, m=8)
+    Ag = A.cuda()
+    for rho in (0.5, 0.8):
+        I, s2 = rmm.select(Ag, rho=rho, return_scores=True)
+        torch.cuda.synchronize()
+        s2_ref = oracle.column_scores_sq(A)
+        rel = np.abs(np64(s2) - s2_ref) / np.maximum(s2_ref, 1e-30)
+        assert rel.max() <= 300 * 2.0 ** -24 + 1e-7
+        # the index set is the TopK of the GPU's own scores (ties to the lower index)
+        mine = oracle.topk_indices(np64(s2), I.numel())
+        assert np.array_equal(I.cpu().numpy(), mine)
+
+
+def test_given_indices(rmm):
+    A, B = W.mlp_up(4, n=150, d=1024, m=264)
+    rng = np.random.default_rng(0)
+    I = np.sort(rng.choice(1024, size=333, replace=False)).astype(np.int32)
+    Y = rmm.matmul(A.cuda(), B.cuda(), indices=torch.from_numpy(I).cuda())
+    torch.cuda.synchronize()
+    A64, B64 = oracle.as_f64(A), oracle.as_f64(B)
+    assert_product_close(Y, oracle.reduced_product(A64, B64, I), np.abs(A64[:, I]), np.abs(B64[I]))
+
+
+def test_dense_identity_and_indices_out(rmm):
+    A, B = W.mlp_down(6, n=140, d=512, m=136)
+    Y, I = rmm.matmul(A.cuda(), B.cuda(), rho=1.0, return_indices=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(I.cpu().numpy(), np.arange(512))
+    A64, B64 = oracle.as_f64(A), oracle.as_f64(B)
+    assert_product_close(Y, A64 @ B64, np.abs(A64), np.abs(B64))
+
+
+def test_single_index_and_empty(rmm):
+    A, B = W.mlp_up(8, n=40, d=256, m=72)
+    Y, I = rmm.matmul(A.cuda(), B.cuda(), k=1, return_indices=True)
+    torch.cuda.synchronize()
+    I_ref, _ = oracle.select(A, k=1)
+    assert_indices_equal(I, I_ref)
+    A64, B64 = oracle.as_f64(A), oracle.as_f64(B)
+    assert_product_close(Y, oracle.reduced_product(A64, B64, I_ref), np.abs(A64[:, I_ref]),
+                         np.abs(B64[I_ref]))
+    Y0 = rmm.matmul(torch.empty((0, 256), dtype=torch.bfloat16, device="cuda"), B.cuda(), rho=0.5)
+    assert Y0.shape == (0, 72)
+    Ym = rmm.matmul(A.cuda(), torch.empty((256, 0), dtype=torch.bfloat16, device="cuda"), rho=0.5)
+    assert Ym.shape == (40, 0)
+
+
+def test_deterministic(rmm):
+    A, B = W.mlp_up(9, n=260, d=4096, m=520)
+    Ag, Bg = A.cuda(), B.cuda()
+    Y1, I1 = rmm.matmul(Ag, Bg, rho=0.7, return_indices=True)
+    Y2, I2 = rmm.matmul(Ag, Bg, rho=0.7, return_indices=True)
+    torch.cuda.synchronize()
+    assert torch.equal(I1, I2) and torch.equal(Y1, Y2)
+
+
+def _qk_check(rmm, Q, K, rho, causal):
+    H, n, dh = Q.shape
+    alpha = 1.0 / math.sqrt(dh)
+    S, I = rmm.qk(Q.cuda(), K.cuda(), rho=rho, alpha=alpha, causal=causal, return_indices=True)
+    torch.cuda.synchronize()
+    S_ref, I_ref = oracle.rmm_qk(Q, K, rho=rho, alpha=alpha, causal=causal)
+    assert_indices_equal(I, I_ref)
+    Q64, K64 = oracle.as_f64(Q), oracle.as_f64(K)
+    mask = np.triu(np.ones((n, K.shape[1]), dtype=bool), 1) if causal else None
+    for h in range(H):
+        g = oracle.kv_head_of(h, H, K.shape[0])
+        assert_product_close(S[h], S_ref[h], np.abs(Q64[h][:, I_ref[h]]), np.abs(K64[g][:, I_ref[h]]).T,
+                             alpha=alpha, mask=mask)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("rho", [0.5, 0.8, 1.0])
+def test_attention_qk(rmm, rho, causal):
+    H, Hkv, n, dh = 4, 2, 200, 128
+    ks = [oracle.retained_count(r, dh) for r in (0.5, 0.8)]
+    (Q, K), _ = gap.enforce_boundary_gaps(
+        lambda g: W.attn_qk(21, n=n, heads=H, kv_heads=Hkv, head_dim=dh, col_gain=g),
+        lambda x: gap.scores_per_head(x[0]), ks)
+    _qk_check(rmm, Q, K, rho, causal)
+
+
+@pytest.mark.parametrize("rho", [0.5, 0.8, 1.0])
+def test_attention_pv(rmm, rho):
+    H, Hkv, n, dv = 4, 2, 264, 128
+    ks = [oracle.retained_count(r, n) for r in (0.5, 0.8)]
+    (P, V), _ = gap.enforce_boundary_gaps(
+        lambda g: W.attn_pv(31, n=n, heads=H, kv_heads=Hkv, v_dim=dv, col_gain=g),
+        lambda x: gap.scores_per_head(x[0]), ks)
+    O, T = rmm.pv(P.cuda(), V.cuda(), rho=rho, return_indices=True)
+    torch.cuda.synchronize()
+    O_ref, T_ref = oracle.rmm_pv(P, V, rho=rho)
+    assert_indices_equal(T, T_ref)
+    P64, V64 = oracle.as_f64(P), oracle.as_f64(V)
+    for h in range(H):
+        g = oracle.kv_head_of(h, H, Hkv)
+        assert_product_close(O[h], O_ref[h], np.abs(P64[h][:, T_ref[h]]), np.abs(V64[g][T_ref[h]]))
+
+
+def test_workspace_status_clean(rmm):
+    A, B = W.mlp_up(12, n=64, d=512, m=64)
+    Ag, Bg = A.cuda(), B.cuda()
+    p = rmm.rmm_problem_init(rmm.RMM_LINEAR, rmm.RMM_BF16, 64, 512, 64)
+    p.rho = 0.5
+    plan = rmm.Plan(p)
+    ws = rmm.workspace_for(plan)
+    Y = torch.empty((64, 64), dtype=torch.bfloat16, device="cuda")
+    rmm.rmm_matmul(plan, Ag, Bg, Y, None, ws)
+    assert rmm.rmm_workspace_status(plan, ws) == rmm.RMM_OK
+    with pytest.raises(rmm.RmmError) as e:
+        rmm.rmm_matmul(plan, Ag, Bg, Y, None, ws[: plan.workspace_bytes - 1])
+    assert e.value.status == rmm.RMM_ERR_WORKSPACE
+    with pytest.raises(rmm.RmmError) as e:
+        rmm.rmm_matmul(plan, Ag[:, 1:], Bg, Y, None, ws)  # 2-byte offset: misaligned
+    assert e.value.status == rmm.RMM_ERR_INVALID_ARG

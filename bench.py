@@ -1,0 +1,437 @@
+"""Benchmark of Reduced Matrix Multiplication (RMM) on B200.
+
+One step = one pass of the whole RMM hot path (column scores, TopK, staging of
+A[:, I], the gathered tensor-core product) over the Llama-3.1-8B-shaped MLP
+workload at n = 4096 tokens, rho = 0.8, bf16: the up/gate-projection shape
+(A 4096 x 4096, B 4096 x 14336) and the down-projection shape
+(A 4096 x 14336, B 14336 x 4096), each with its own index set.
+
+Metric: useful TFLOP/s = sum of 2 n ceil(rho d) m over the step / step time,
+with the same kernels at rho = 1 (identity index set) and cuBLAS dense
+matmul reported beside it.  Inputs (149 MB and 234 MB per op) exceed the
+126 MB L2, so no flush runs between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rmm|reference]
+N > 1 runs one independent replica per GPU (weak scaling, no collective on the
+data path; a barrier and a max over ranks bracket the timing).
+`--impl reference` times the CPU oracle (a deliberately slow fp64 program) on
+a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "RMM op latency and useful TFLOP/s (2·n·⌈ρd⌉·m) vs ρ=1, % of bf16 peak"
+WORKLOAD = "llama3.1-8b-mlp-linear-rmm"
+SHAPES = {"up": (4096, 14336), "down": (14336, 4096)}
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gather_gemm_llama8b_mlp_n4096.md")
+GEMM_SOURCE = os.path.join(ROOT, "input_adaptive_reduced_b200", "csrc", "rmm_gemm.cu")
+
+
+def retained(rho: float, d: int) -> int:
+    x = rho * d
+    r = round(x)
+    k = r if abs(x - r) <= 1e-9 * d else math.ceil(x)
+    return max(1, min(d, int(k)))
+
+
+def useful_flops(n: int, rho: float) -> float:
+    return float(sum(2.0 * n * retained(rho, d) * m for d, m in SHAPES.values()))
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            pk = json.load(f)
+        return pk["bf16_tflops"], pk.get("bf16_tflops_sustained"), pk["hbm_gbs"], "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def load_traffic():
+    """Per-launch DRAM bytes of the product kernel from the committed ncu summary,
+    only if the kernel source has not changed since the counters were taken."""
+    try:
+        text = open(TRAFFIC_FILE).read()
+        want = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text).group(1)
+        have = hashlib.sha256(open(GEMM_SOURCE, "rb").read()).hexdigest()
+        if want != have:
+            return None
+        return float(re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text).group(1))
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sms, maxs, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sms.append(float(parts[0]))
+                maxs.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        loaded = [s for s, p in zip(sms, power) if p > 250.0] or sms
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(maxs) if maxs else None,
+                "reasons": sorted(reasons), "samples": len(sms),
+                "power_w_max": max(power) if power else None}
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(inputs64, rho: float, rows: int):
+    """Time the oracle on full selection of both ops plus `rows` output rows of
+    each product.  Returns (seconds, useful flops done)."""
+    import oracle
+    t0 = time.perf_counter()
+    flops = 0.0
+    for name, (A64, B64) in inputs64.items():
+        d, m = SHAPES[name]
+        I, _ = oracle.select(A64, rho=rho)
+        oracle.reduced_product(A64, B64, I, rows=list(range(rows)))
+        flops += 2.0 * rows * len(I) * m
+    return time.perf_counter() - t0, flops
+
+
+def cpu_inputs(n_rows: int, seed: int):
+    import workloads as W
+    import oracle
+    out = {}
+    for name, gen in (("up", W.mlp_up), ("down", W.mlp_down)):
+        A, B = gen(seed, n=n_rows)
+        out[name] = (oracle.as_f64(A), oracle.as_f64(B))
+    return out
+
+
+def cores_used() -> int:
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n and n.isdigit() else (os.cpu_count() or 1)
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    n, rho = args.n, args.rho
+    inputs64 = cpu_inputs(n, seed=1)
+    # size the per-step sample so that warmup + steps stay within ~3 minutes
+    t1, _ = oracle_sample(inputs64, rho, rows=1)
+    t5, _ = oracle_sample(inputs64, rho, rows=5)
+    per_row = max((t5 - t1) / 4.0, 1e-4)
+    budget = 180.0 / max(1, args.steps + args.warmup)
+    rows = int(max(1, min(64, (budget - t1) / per_row)))
+    for _ in range(args.warmup):
+        oracle_sample(inputs64, rho, rows)
+    total_t, total_f = 0.0, 0.0
+    for _ in range(args.steps):
+        t, f = oracle_sample(inputs64, rho, rows)
+        total_t += t
+        total_f += f
+    value = total_f / total_t / 1e12
+    ms = total_t / args.steps * 1e3
+    sample = (f"full selection (scores + TopK) of both ops and {rows} of {n} output rows of each "
+              f"reduced product per step, fp64, OpenMP over rows")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "n": n, "rho": rho, "shapes": SHAPES, "sample_rows": rows},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- RMM arm
+def run_rmm(args):
+    import torch
+    import torch.distributed as dist
+    import input_adaptive_reduced_b200 as rmm
+    import workloads as W
+
+    rank, world, local = dist_env()
+    if args.gpus != world:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}; using WORLD_SIZE", file=sys.stderr)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the RMM kernels have no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    n, rho = args.n, args.rho
+    stream = torch.cuda.current_stream(dev)
+    ops = {}
+    for name, gen in (("up", W.mlp_up), ("down", W.mlp_down)):
+        d, m = SHAPES[name]
+        A, B = gen(1000 * rank + 1, n=n, device=dev)
+        entry = {"A": A, "B": B, "d": d, "m": m}
+        for tag, r in (("rmm", rho), ("dense", 1.0)):
+            p = rmm.rmm_problem_init(rmm.RMM_LINEAR, rmm.RMM_BF16, n, d, m)
+            p.rho = r
+            plan = rmm.Plan(p)
+            ws = rmm.workspace_for(plan, dev, stream)
+            entry[tag] = {"plan": plan, "ws": ws, "k": plan.k,
+                          "Y": torch.empty((n, m), dtype=torch.bfloat16, device=dev)}
+        ops[name] = entry
+
+    def run_op(e, tag):
+        c = e[tag]
+        rmm.rmm_matmul(c["plan"], e["A"], e["B"], c["Y"], None, c["ws"], stream)
+
+    def step(tag="rmm"):
+        for e in ops.values():
+            run_op(e, tag)
+
+    # warm-up
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+
+    # product-kernel events, one pair per op per timed step
+    n_ev = args.steps * len(ops)
+    ev_start = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    ev_stop = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    for e in ev_start + ev_stop:
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    i_ev = 0
+    for _ in range(args.steps):
+        for e in ops.values():
+            c = e["rmm"]
+            c["plan"].set_product_events(ev_start[i_ev], ev_stop[i_ev])
+            run_op(e, "rmm")
+            i_ev += 1
+    t_stop.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    for e in ops.values():
+        e["rmm"]["plan"].set_product_events(None, None)
+    rmm.check_workspaces()
+
+    ms_total = t_start.elapsed_time(t_stop)
+    if world > 1:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    flops_step = useful_flops(n, rho)
+    value = flops_step * world / (ms_step * 1e-3) / 1e12
+
+    # product kernel (dominant kernel): algorithmic flops per launch / event time
+    gemm_ms = [s.elapsed_time(t) for s, t in zip(ev_start, ev_stop)]
+    per_op = list(ops.values())
+    gemm_flops = [2.0 * n * per_op[i % len(per_op)]["rmm"]["k"] * per_op[i % len(per_op)]["m"]
+                  for i in range(len(gemm_ms))]
+    achieved = sum(gemm_flops) / (sum(gemm_ms) * 1e-3) / 1e12
+    peak_burst, peak_sust, hbm, peak_src = load_peaks()
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s",
+                "frac": achieved / peak_burst, "traffic": load_traffic(),
+                "peak_kind": f"{peak_src} cuBLAS bf16 burst",
+                "frac_of_sustained": (achieved / peak_sust) if peak_sust else None,
+                "kernel": "gather_gemm_kernel<bf16, kBGather (tile::gather4 B rows), BN=256>",
+                "avg_launch_us": sum(gemm_ms) / len(gemm_ms) * 1e3}
+
+    # per-op latency at rho and at rho = 1 (same kernels, identity I) and cuBLAS dense
+    def op_latency(fn, iters=20):
+        for _ in range(3):
+            fn()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(iters):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / iters
+
+    points = {}
+    for name, e in ops.items():
+        d, m = e["d"], e["m"]
+        t_r = op_latency(lambda: run_op(e, "rmm"))
+        t_1 = op_latency(lambda: run_op(e, "dense"))
+        t_cb = op_latency(lambda: torch.matmul(e["A"], e["B"]))
+        k = e["rmm"]["k"]
+        points[name] = {"n": n, "d": d, "m": m, "k": k, "ms": t_r,
+                        "useful_tflops": 2.0 * n * k * m / (t_r * 1e-3) / 1e12,
+                        "ms_rho1": t_1, "tflops_rho1": 2.0 * n * d * m / (t_1 * 1e-3) / 1e12,
+                        "ms_cublas_dense": t_cb, "speedup_vs_rho1": t_1 / t_r,
+                        "kernel_launches": e["rmm"]["plan"].kernel_launches}
+
+    # end to end through the public API with host buffers (pinned), copies timed
+    e2e = None
+    if not args.no_e2e:
+        host = {}
+        h2d = d2h = 0
+        for name, e in ops.items():
+            hA = e["A"].cpu().pin_memory()
+            hB = e["B"].cpu().pin_memory()
+            hY = torch.empty_like(e["rmm"]["Y"], device="cpu").pin_memory()
+            dA = torch.empty_like(e["A"])
+            dB = torch.empty_like(e["B"])
+            host[name] = (hA, hB, hY, dA, dB)
+            h2d += hA.numel() * hA.element_size() + hB.numel() * hB.element_size()
+            d2h += hY.numel() * hY.element_size()
+
+        def e2e_step():
+            for name, e in ops.items():
+                hA, hB, hY, dA, dB = host[name]
+                dA.copy_(hA, non_blocking=True)
+                dB.copy_(hB, non_blocking=True)
+                c = e["rmm"]
+                rmm.rmm_matmul(c["plan"], dA, dB, c["Y"], None, c["ws"], stream)
+                hY.copy_(c["Y"], non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        e2e_steps = max(3, min(args.steps, 20))
+        barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = a.elapsed_time(b) / e2e_steps
+        if world > 1:
+            t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": flops_step * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+               "path": "pinned host A, B -> device, rmm_matmul (C ABI), Y -> pinned host"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        rows = args.cpu_rows
+        inputs64 = cpu_inputs(n, seed=1)
+        t, f = oracle_sample(inputs64, rho, rows)
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle",
+               "sample": f"full selection of both ops and {rows} of {n} output rows of each product, "
+                         f"fp64 C with OpenMP over rows; {t:.1f} s"}
+
+    launches = sum(e["rmm"]["plan"].kernel_launches for e in ops.values()) * args.steps
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Llama-3.1-8B-shaped activations and N(0,0.02) weights)",
+            "config": {"workload": WORKLOAD, "n": n, "rho": rho, "shapes": SHAPES,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (149 MB and 234 MB per op); no flush"},
+            "roofline": roofline, "points": points, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["rmm", "reference"], default="rmm")
+    ap.add_argument("--n", type=int, default=4096)
+    ap.add_argument("--rho", type=float, default=0.8)
+    ap.add_argument("--cpu-rows", type=int, default=64)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_rmm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -152,7 +152,8 @@ RMM_API rmm_status rmm_matmul_batched(const rmm_plan* plan, const void* A, const
                               int32_t* I_inout, void* workspace, size_t workspace_bytes,
                               void* stream);
 
-/* Zero the workspace's error word (its first 256 bytes) on `stream`.  Call
+/* Zero the workspace's header (its error word and the score pass's
+   completion counters, which the kernels return to zero) on `stream`.  Call
    once after allocating a workspace, before the first compute call. */
 RMM_API rmm_status rmm_workspace_init(const rmm_plan* plan, void* workspace, size_t workspace_bytes,
                               void* stream);
@@ -161,6 +162,18 @@ RMM_API rmm_status rmm_workspace_init(const rmm_plan* plan, void* workspace, siz
    RMM_ERR_TIMEOUT if a kernel gave up on a wait since the last check (the
    word is then cleared), or RMM_ERR_CUDA if the stream reports an error. */
 RMM_API rmm_status rmm_workspace_status(const rmm_plan* plan, void* workspace, void* stream);
+
+/* Tracing hook.  When both are non-NULL, every later rmm_matmul* call with
+   this plan records `start` immediately before and `stop` immediately after
+   the launch of its reduced-product kernel, on the call's stream, so that
+   cudaEventElapsedTime isolates that kernel (the RMM paper §6.3 times the
+   whole operation, norms + TopK + product; this separates the last step).
+   The events are cudaEvent_t passed as void*, created by the caller; NULL
+   clears the hook.  Not thread-safe with concurrent calls on the plan. */
+RMM_API rmm_status rmm_plan_set_product_events(rmm_plan* plan, void* start, void* stop);
+
+/* Number of kernels one rmm_matmul* call of this plan launches (-1 for NULL). */
+RMM_API int32_t rmm_plan_kernel_launches(const rmm_plan* plan);
 
 /* Static string naming a status code. */
 RMM_API const char* rmm_status_string(rmm_status s);

@@ -23,6 +23,7 @@ __all__ = [
     "rmm_problem_init", "rmm_plan_create", "rmm_select", "rmm_matmul", "rmm_matmul_batched",
     "rmm_workspace_init", "rmm_workspace_status", "rmm_status_string", "rmm_version",
     "EXPORTED_SYMBOLS", "select", "matmul", "qk", "pv", "workspace_for", "check_workspaces",
+    "rmm_plan_set_product_events", "rmm_plan_kernel_launches",
 ]
 
 RMM_OK, RMM_ERR_INVALID_ARG, RMM_ERR_UNSUPPORTED, RMM_ERR_WORKSPACE, RMM_ERR_CUDA, RMM_ERR_TIMEOUT = range(6)
@@ -34,7 +35,7 @@ RMM_FLAG_USE_GIVEN_INDICES = 2
 EXPORTED_SYMBOLS = (
     "rmm_problem_init", "rmm_plan_create", "rmm_plan_destroy", "rmm_plan_k", "rmm_plan_workspace_size",
     "rmm_select", "rmm_matmul", "rmm_matmul_batched", "rmm_workspace_init", "rmm_workspace_status",
-    "rmm_status_string", "rmm_version",
+    "rmm_status_string", "rmm_version", "rmm_plan_set_product_events", "rmm_plan_kernel_launches",
 )
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librmm.so")
@@ -91,6 +92,10 @@ def _load_library():
     L.rmm_workspace_init.argtypes = [vp, vp, sz, vp]
     L.rmm_workspace_status.restype = st
     L.rmm_workspace_status.argtypes = [vp, vp, vp]
+    L.rmm_plan_set_product_events.restype = st
+    L.rmm_plan_set_product_events.argtypes = [vp, vp, vp]
+    L.rmm_plan_kernel_launches.restype = ctypes.c_int32
+    L.rmm_plan_kernel_launches.argtypes = [vp]
     L.rmm_status_string.restype = ctypes.c_char_p
     L.rmm_status_string.argtypes = [st]
     L.rmm_version.restype = ctypes.c_char_p
@@ -136,6 +141,19 @@ class Plan:
         self.handle = h
         self.workspace_bytes = int(ws.value)
         self.k = int(lib.rmm_plan_k(h))
+        self.kernel_launches = int(lib.rmm_plan_kernel_launches(h))
+
+    def set_product_events(self, start=None, stop=None):
+        """Bracket the reduced-product kernel of later calls with torch.cuda.Event
+        objects (created with enable_timing=True); None clears the hook."""
+        def raw(e):
+            if e is None:
+                return None
+            if not e.cuda_event:
+                e.record()  # torch creates the event lazily on its first record
+            return ctypes.c_void_p(e.cuda_event)
+        _check(lib.rmm_plan_set_product_events(self.handle, raw(start), raw(stop)),
+               "rmm_plan_set_product_events")
 
     def __del__(self):
         h = getattr(self, "handle", None)
@@ -147,6 +165,14 @@ class Plan:
 
 def rmm_plan_create(problem: rmm_problem) -> Plan:
     return Plan(problem)
+
+
+def rmm_plan_set_product_events(plan: Plan, start=None, stop=None):
+    plan.set_product_events(start, stop)
+
+
+def rmm_plan_kernel_launches(plan: Plan) -> int:
+    return int(lib.rmm_plan_kernel_launches(plan.handle))
 
 
 def _ptr(t):

@@ -32,8 +32,11 @@ struct rmm_plan {
     int nsplit;
     int64_t rows_per_split;
     int bn;
+    bool pack_b;        // bf16 LINEAR/PV with k < d: stage B[I, :] contiguously
     int num_sms;
-    size_t off_err, off_partials, off_I, off_apack, off_bpack, ws_bytes;
+    size_t off_err, off_counters, off_partials, off_scores, off_I, off_apack, off_bpack, ws_bytes;
+    size_t header_bytes;  // zeroed by rmm_workspace_init: error word + colnorm counters
+    cudaEvent_t product_start, product_stop;  // tracing hook, may be null
 };
 
 namespace {
@@ -91,6 +94,22 @@ bool encode_kmajor_map(CUtensorMap* map, int es, const void* base, int64_t kext,
     return r == CUDA_SUCCESS;
 }
 
+// 2-D row-major map {m columns, rows} of an MN-major B operand with a
+// {64, box_rows} box (128 bytes of columns), 128-byte swizzle, zero fill.
+bool encode_rows_map(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int64_t ld,
+                     uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 rmm_status validate_problem(const rmm_problem* p) {
     if (!p) return RMM_ERR_INVALID_ARG;
     if (p->mode < RMM_LINEAR || p->mode > RMM_PV) return RMM_ERR_INVALID_ARG;
@@ -111,6 +130,13 @@ rmm_status validate_problem(const rmm_problem* p) {
         if (p->stride_y % vec != 0 || (p->n > 0 && p->stride_y < p->n * p->ldy)) return RMM_ERR_INVALID_ARG;
     }
     if (p->kv_heads > 1 && (p->stride_b < 0 || p->stride_b % vec != 0)) return RMM_ERR_INVALID_ARG;
+    // bf16 row gathers address every B head through one 2-D map: heads must sit
+    // a whole number of rows apart.
+    if (p->kv_heads > 1 && p->mode != RMM_QK && p->dtype == RMM_BF16 && p->stride_b % p->ldb != 0)
+        return RMM_ERR_INVALID_ARG;
+    if (p->kv_heads > 1 && p->mode != RMM_QK && p->dtype == RMM_BF16 &&
+        ((p->kv_heads - 1) * (p->stride_b / p->ldb) + p->d) > kMaxDim - 1)
+        return RMM_ERR_UNSUPPORTED;
     if (p->k == 0) {
         if (!(p->rho > 0.0) || p->rho > 1.0) return RMM_ERR_INVALID_ARG;
     } else if (p->k < 0 || p->k > p->d) {
@@ -152,6 +178,8 @@ rmm_status run_select(const rmm_plan* plan, const void* A, int32_t* I, float* s2
         e = rmm::launch_normselect(a, stream);
     } else {
         a.partials = ws_at<float>(ws, plan->off_partials);
+        a.counters = ws_at<unsigned>(ws, plan->off_counters);
+        a.scores = s2 ? s2 : ws_at<float>(ws, plan->off_scores);
         a.nsplit = plan->nsplit;
         a.rows_per_split = plan->rows_per_split;
         e = rmm::launch_colnorm(a, stream);
@@ -239,7 +267,7 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
     gp.b_head_div = 1;
 
     if (p.mode == RMM_QK) {
-        gl.b_gather = false;
+        gl.b_mode = rmm::kBKMajor;
         if (!identity) {
             rmm::PackArgs pb{};
             pb.src = B;
@@ -268,7 +296,7 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         }
     } else if (p.dtype == RMM_F32) {
         // tf32 operands are staged K-major: B[I, :] is written transposed (m x k).
-        gl.b_gather = false;
+        gl.b_mode = rmm::kBKMajor;
         rmm::PackArgs pb{};
         pb.src = B;
         pb.dtype = p.dtype;
@@ -288,15 +316,64 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         if (!encode_kmajor_map(&gp.map_b, es, pb.dst, k, p.m, p.heads, plan->ldp, p.m * plan->ldp, box_k,
                                static_cast<uint32_t>(plan->bn)))
             return RMM_ERR_CUDA;
+    } else if (!identity && plan->pack_b) {
+        // The retained rows B[I, :] are copied into a contiguous k x m buffer per
+        // head (a streaming copy at HBM rate), which the product then reads with
+        // plain TMA row tiles.
+        rmm::PackArgs pb{};
+        pb.src = B;
+        pb.dtype = p.dtype;
+        pb.rows = p.m;
+        pb.d = p.d;
+        pb.ld_src = p.ldb;
+        pb.stride_src = p.stride_b;
+        pb.group = plan->group;
+        pb.I = I;
+        pb.I_stride = k;
+        pb.k = k;
+        pb.dst = ws_at<void>(ws, plan->off_bpack);
+        pb.ld_dst = p.m;
+        pb.stride_dst = k * p.m;
+        pb.heads = static_cast<int>(p.heads);
+        if (rmm::launch_pack_rows(pb, plan->num_sms, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        gl.b_mode = rmm::kBRows;
+        gp.group = 1;
+        gp.b_head_rows = static_cast<int32_t>(k);
+        gp.b_rows_total = static_cast<int32_t>(k * p.heads);
+        if (!encode_rows_map(&gp.map_b, pb.dst, p.m, k * p.heads, p.m, 64u)) return RMM_ERR_CUDA;
     } else {
-        gl.b_gather = true;
-        gp.B = B;
-        gp.ldb = p.ldb;
-        gp.stride_b = p.stride_b;
+        // Plain row tiles only where rows past d are out of the map (one B head)
+        // or never reached (d a whole number of K blocks); otherwise rows are
+        // fetched four at a time through the index set with tile::gather4.
+        const bool row_tiles = identity && (p.kv_heads == 1 || p.d % 64 == 0);
+        gl.b_mode = row_tiles ? rmm::kBRows : rmm::kBGather;
+        const int64_t head_rows = p.kv_heads > 1 ? p.stride_b / p.ldb : p.d;
+        const int64_t rows_total = (p.kv_heads - 1) * head_rows + p.d;
+        gp.b_head_rows = static_cast<int32_t>(head_rows);
+        gp.b_rows_total = static_cast<int32_t>(rows_total);
         gp.I = identity ? nullptr : I;
         gp.I_stride = k;
+        if (!encode_rows_map(&gp.map_b, B, p.m, rows_total, p.ldb, row_tiles ? 64u : 1u)) return RMM_ERR_CUDA;
     }
-    return rmm::launch_gemm(gp, gl, stream) == cudaSuccess ? RMM_OK : RMM_ERR_CUDA;
+    const bool traced = plan->product_start && plan->product_stop;
+    if (traced && cudaEventRecord(plan->product_start, stream) != cudaSuccess) return RMM_ERR_CUDA;
+    if (rmm::launch_gemm(gp, gl, stream) != cudaSuccess) return RMM_ERR_CUDA;
+    if (traced && cudaEventRecord(plan->product_stop, stream) != cudaSuccess) return RMM_ERR_CUDA;
+    return RMM_OK;
+}
+
+int32_t launches_per_call(const rmm_plan* plan) {
+    const rmm_problem& p = plan->p;
+    const bool given = (p.flags & RMM_FLAG_USE_GIVEN_INDICES) != 0;
+    const bool identity = !given && plan->k == p.d;
+    int32_t n = 0;
+    if (!given && !identity) n += plan->fused_select ? 1 : 2;
+    if (p.n == 0 || p.m == 0) return n;
+    if (!identity) n += 1;                                   // pack A[:, I]
+    if (p.mode == RMM_QK && !identity) n += 1;               // pack K[:, I]
+    if (p.mode != RMM_QK && p.dtype == RMM_F32) n += 1;      // B[I, :] transposed for tf32
+    if (!identity && plan->pack_b) n += 1;                   // B[I, :] rows, contiguous
+    return n + 1;                                            // the product
 }
 
 }  // namespace
@@ -336,6 +413,7 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     const bool given = (p->flags & RMM_FLAG_USE_GIVEN_INDICES) != 0;
     plan->need_select = !given && plan->k < p->d;
     plan->bn = p->m <= 128 ? 128 : 256;
+    plan->pack_b = p->mode != RMM_QK && p->dtype == RMM_BF16 && (plan->k < p->d || given);
 
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -353,16 +431,20 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
         return RMM_ERR_UNSUPPORTED;
     }
     const size_t head_bytes = static_cast<size_t>(p->n) * p->d * plan->es;
-    plan->fused_select = head_bytes <= kFusedSelectBytes && rmm::normselect_smem_bytes(p->d, p->dtype) <= 200 * 1024;
+    plan->fused_select = head_bytes <= kFusedSelectBytes && rmm::normselect_smem_bytes(p->d, p->dtype) <= 190 * 1024;
+    // Row splits for the score pass: enough CTAs to keep HBM busy (about two
+    // per SM), at most kMaxSplitRows partials per column, at least 64 rows each.
     const int vec = 16 / plan->es;
     const int64_t colblocks = (p->d + 32 * vec - 1) / (32 * vec);
-    const int64_t target = 4LL * sms;
+    const int64_t target = 2LL * sms;
     int64_t nsplit = (target + colblocks * p->heads - 1) / (colblocks * p->heads);
-    const int64_t max_split = (p->n + 31) / 32;
+    const int64_t max_split = (p->n + 63) / 64;
     if (nsplit > max_split) nsplit = max_split;
+    if (nsplit > rmm::kMaxSplitRows) nsplit = rmm::kMaxSplitRows;
     if (nsplit < 1) nsplit = 1;
     int64_t rps = (p->n + nsplit - 1) / nsplit;
-    if (rps < 1) rps = 1;
+    rps = (rps + 7) / 8 * 8;
+    if (rps < 8) rps = 8;
     nsplit = p->n > 0 ? (p->n + rps - 1) / rps : 1;
     plan->nsplit = static_cast<int>(nsplit);
     plan->rows_per_split = rps;
@@ -370,9 +452,16 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     size_t off = 0;
     plan->off_err = off;
     off += 256;
+    plan->off_counters = off;
+    off += align256(static_cast<size_t>(p->heads) * colblocks * sizeof(unsigned));
+    plan->header_bytes = off;
     plan->off_partials = off;
-    if (select_possible && !plan->fused_select)
+    plan->off_scores = off;
+    if (select_possible && !plan->fused_select) {
         off += align256(static_cast<size_t>(p->heads) * nsplit * p->d * sizeof(float));
+        plan->off_scores = off;
+        off += align256(static_cast<size_t>(p->heads) * p->d * sizeof(float));
+    }
     plan->off_I = off;
     off += align256(static_cast<size_t>(p->heads) * plan->k * sizeof(int32_t));
     plan->off_apack = off;
@@ -380,6 +469,8 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     plan->off_bpack = off;
     if (p->mode == RMM_QK || p->dtype == RMM_F32)
         off += align256(static_cast<size_t>(p->heads) * p->m * plan->ldp * plan->es);
+    else if (plan->pack_b || given)
+        off += align256(static_cast<size_t>(p->heads) * plan->k * p->m * plan->es);
     plan->ws_bytes = off;
     if (workspace_bytes) *workspace_bytes = plan->ws_bytes;
     *out = plan;
@@ -422,7 +513,7 @@ rmm_status rmm_workspace_init(const rmm_plan* plan, void* ws, size_t ws_bytes, v
     if (!plan) return RMM_ERR_INVALID_ARG;
     rmm_status st = check_workspace(plan, ws, ws_bytes);
     if (st != RMM_OK) return st;
-    if (cudaMemsetAsync(ws_at<int>(ws, plan->off_err), 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (cudaMemsetAsync(ws, 0, plan->header_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return RMM_ERR_CUDA;
     return RMM_OK;
 }
@@ -441,6 +532,16 @@ rmm_status rmm_workspace_status(const rmm_plan* plan, void* ws, void* stream) {
     }
     return RMM_OK;
 }
+
+rmm_status rmm_plan_set_product_events(rmm_plan* plan, void* start, void* stop) {
+    if (!plan) return RMM_ERR_INVALID_ARG;
+    if ((start == nullptr) != (stop == nullptr)) return RMM_ERR_INVALID_ARG;
+    plan->product_start = static_cast<cudaEvent_t>(start);
+    plan->product_stop = static_cast<cudaEvent_t>(stop);
+    return RMM_OK;
+}
+
+int32_t rmm_plan_kernel_launches(const rmm_plan* plan) { return plan ? launches_per_call(plan) : -1; }
 
 const char* rmm_status_string(rmm_status s) {
     switch (s) {

@@ -3,19 +3,27 @@
 // Input-Adaptive Matrix-Product Reduction for LLM Inference", §3.2; per-head
 // attention forms in §3.3; cost O(n k m) in §3.4 and Appendix D.1 Eq. (1)-(4)).
 //
-// Design (sm_100a, one CTA per SM, persistent over 128 x BN output tiles):
-//   warps 0-3  producer: the A tile (packed A[:, I], K-major) arrives by TMA;
-//              B is either gathered row by row through the index set with
-//              16-byte cp.async into the 128-byte-swizzled MN-major layout
-//              (LINEAR / PV: B[I, :] rows are contiguous), or arrives by TMA
-//              as a K-major tile (QK: packed K[:, I]).
-//   warp  8    MMA issuer: one thread issues tcgen05.mma (kind::f16 for bf16,
-//              kind::tf32 for fp32) into a double-buffered fp32 accumulator in
-//              tensor memory and commits stage releases to mbarriers.
-//   warps 4-7  epilogue: tcgen05.ld of the accumulator (one TMEM lane quadrant
-//              per warp), alpha scaling, the causal -inf mask, rounding to the
-//              storage dtype and 16-byte global stores.  Tiles that the causal
-//              mask covers entirely skip the MMA and store -inf directly.
+// Design (sm_100a, one CTA per SM, persistent over 128 x BN output tiles,
+// 192 threads):
+//   warp 0     producer.  One lane issues the TMA tile of the packed operand
+//              A[:, I] (K-major).  B arrives by TMA in one of three ways:
+//                kGather: the retained rows B[I, :] of a row-major d x m
+//                  matrix (I == nullptr: all rows in order), four indexed
+//                  rows per tile::gather4 instruction
+//                  (16 lanes x BN/64 column groups per stage), written in the
+//                  128-byte-swizzled MN-major layout;
+//                kRows: consecutive rows (every index kept), plain tiles in
+//                  the same MN-major layout;
+//                kKMajor: a K-major tile of an m x K matrix (QK mode: the
+//                  packed K[:, I]; fp32 problems: B[I, :] staged transposed).
+//   warp 1     MMA issuer.  One thread issues tcgen05.mma (kind::f16 for bf16,
+//              kind::tf32 for fp32) into a double-buffered fp32 accumulator
+//              in tensor memory and commits stage releases to mbarriers.
+//   warps 2-5  epilogue.  tcgen05.ld of the accumulator (one TMEM lane
+//              quadrant per warp), alpha scaling, the causal -inf mask,
+//              rounding to the storage dtype and 16-byte global stores.
+//              Tiles that the causal mask covers entirely skip the MMA and
+//              store -inf directly.
 // Every wait is bounded (rmm_device.cuh); on expiry the kernel records an
 // error word and returns.
 #include <cstdint>
@@ -28,22 +36,24 @@
 namespace rmm {
 namespace {
 
-constexpr int kThreads = 288;  // 9 warps
+constexpr int kThreads = 192;  // 6 warps
 constexpr int kBM = 128;
 
-template <typename T, int BN>
+template <typename T, int BMODE, int BN>
 struct Cfg {
     static constexpr int ES = sizeof(T);
     static constexpr bool TF32 = (ES == 4);
+    static constexpr bool B_MN = (BMODE != kBKMajor);
     static constexpr int BK = 128 / ES;        // one 128-byte swizzle row of K
     static constexpr int UK = 32 / ES;         // K per tcgen05.mma
     static constexpr int A_BYTES = kBM * 128;  // 128 rows x 128 B
-    static constexpr int B_BYTES = BN * 128;   // BK rows x BN cols (gather) or BN rows x 128 B (TMA)
+    static constexpr int B_BYTES = BN * 128;   // BK rows x BN cols (MN-major) or BN rows x 128 B
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES = (BN == 256) ? 4 : 6;
     static constexpr int TMEM_COLS = 2 * BN;
-    static constexpr int CPR = BN * ES / 16;   // 16-byte chunks per gathered B row
+    static constexpr int GROUP_BYTES = BK * 128;  // one 64-column group of an MN-major B tile
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+    static_assert(!(TF32 && B_MN), "fp32 operands are staged K-major");
 };
 
 struct TileCoord {
@@ -88,9 +98,9 @@ __device__ __forceinline__ void store_chunk(T* yrow, int col0, int m, const floa
     }
 }
 
-template <typename T, bool B_GATHER, int BN>
+template <typename T, int BMODE, int BN>
 __global__ void __launch_bounds__(kThreads, 1) gather_gemm_kernel(const __grid_constant__ GemmParams p) {
-    using C = Cfg<T, BN>;
+    using C = Cfg<T, BMODE, BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
@@ -103,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1) gather_gemm_kernel(const __grid_c
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&full[s], B_GATHER ? 128 + 1 : 1);
+            mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -113,9 +123,9 @@ __global__ void __launch_bounds__(kThreads, 1) gather_gemm_kernel(const __grid_c
         *abort_flag = 0;
         mbar_fence_init();
         tma_prefetch_map(&p.map_a);
-        if (!B_GATHER) tma_prefetch_map(&p.map_b);
+        tma_prefetch_map(&p.map_b);
     }
-    if (warp == 8) {
+    if (warp == 1) {
         tmem_alloc(tmem_holder, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -127,63 +137,65 @@ __global__ void __launch_bounds__(kThreads, 1) gather_gemm_kernel(const __grid_c
     const int total = p.heads * p.m_tiles * p.n_tiles;
     const int num_kb = (p.k + C::BK - 1) / C::BK;
 
-    if (warp < 4) {
+    if (warp == 0) {
         // ------------------------------------------------------------ producer
-        const int tid = threadIdx.x;
-        if (B_GATHER || tid == 0) {
-            uint32_t it = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const TileCoord tc = decode_tile(t, p, BN);
-                if (tc.skip) continue;
-                const T* Bh = nullptr;
-                const int32_t* Ih = nullptr;
-                if constexpr (B_GATHER) {
-                    Bh = static_cast<const T*>(p.B) + (int64_t)(tc.h / p.group) * p.stride_b;
-                    Ih = p.I ? p.I + (int64_t)tc.h * p.I_stride : nullptr;
-                }
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
-                    const int s = it % C::STAGES;
-                    const uint32_t ph = (it / C::STAGES) & 1u;
-                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err, kErrTimeoutProducer)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t* sa = smem + s * C::STAGE_BYTES;
-                    uint8_t* sb = sa + C::A_BYTES;
-                    if (tid == 0) {
-                        mbar_arrive_expect_tx(&full[s], B_GATHER ? C::A_BYTES : C::A_BYTES + C::B_BYTES);
-                        tma_load_3d(sa, &p.map_a, &full[s], kb * C::BK, tc.m0, tc.h);
-                        if constexpr (!B_GATHER)
-                            tma_load_3d(sb, &p.map_b, &full[s], kb * C::BK, tc.n0, tc.h / p.b_head_div);
-                    }
-                    if constexpr (B_GATHER) {
-                        const uint32_t sb_addr = smem_u32(sb);
-#pragma unroll 4
-                        for (int c = tid; c < C::BK * C::CPR; c += 128) {
-                            const int r = c / C::CPR;
-                            const int cc = c % C::CPR;
-                            const int kidx = kb * C::BK + r;
-                            const bool kvalid = kidx < p.k;
-                            int row = kvalid ? (Ih ? __ldg(Ih + kidx) : kidx) : 0;
-                            row = min(max(row, 0), p.d - 1);
-                            const int gcol = tc.n0 + cc * (16 / C::ES);
-                            const bool cvalid = gcol < p.m;
-                            const T* src = Bh + (int64_t)row * p.ldb + (cvalid ? gcol : 0);
-                            const uint32_t dst = sb_addr + (cc >> 3) * (C::BK * 128) + r * 128 +
-                                                 (((cc & 7) ^ (r & 7)) << 4);
-                            cp_async_16(dst, src, (kvalid && cvalid) ? 16u : 0u);
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            const TileCoord tc = decode_tile(t, p, BN);
+            if (tc.skip) continue;
+            const int32_t* Ih = (BMODE == kBGather && p.I) ? p.I + (int64_t)tc.h * p.I_stride : nullptr;
+            const int32_t row_base = (tc.h / p.group) * p.b_head_rows;
+            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                const int s = it % C::STAGES;
+                const uint32_t ph = (it / C::STAGES) & 1u;
+                int32_t rows[4] = {0, 0, 0, 0};
+                if constexpr (BMODE == kBGather) {
+                    if (lane < 16) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int kidx = kb * C::BK + 4 * lane + i;
+                            if (kidx < p.k) {
+                                int32_t j = Ih ? __ldg(Ih + kidx) : kidx;  // no list: every index
+                                j = min(max(j, 0), p.d - 1);
+                                rows[i] = row_base + j;
+                            } else {
+                                rows[i] = p.b_rows_total;  // out of range: reads zeros
+                            }
                         }
-                        cp_async_arrive_noinc(&full[s]);
                     }
+                }
+                if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err, kErrTimeoutProducer)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* sa = smem + s * C::STAGE_BYTES;
+                uint8_t* sb = sa + C::A_BYTES;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
+                    tma_load_3d(sa, &p.map_a, &full[s], kb * C::BK, tc.m0, tc.h);
+                    if constexpr (BMODE == kBKMajor)
+                        tma_load_3d(sb, &p.map_b, &full[s], kb * C::BK, tc.n0, tc.h / p.b_head_div);
+                }
+                __syncwarp();
+                if constexpr (BMODE == kBGather) {
+                    if (lane < 16) {
+#pragma unroll
+                        for (int g = 0; g < BN / 64; ++g)
+                            tma_gather4(sb + g * C::GROUP_BYTES + lane * 4 * 128, &p.map_b, &full[s],
+                                        tc.n0 + 64 * g, rows[0], rows[1], rows[2], rows[3]);
+                    }
+                } else if constexpr (BMODE == kBRows) {
+                    if (lane < BN / 64)
+                        tma_load_2d(sb + lane * C::GROUP_BYTES, &p.map_b, &full[s], tc.n0 + 64 * lane,
+                                    row_base + kb * C::BK);
                 }
             }
-            if constexpr (B_GATHER) cp_async_wait_all();
         }
-    } else if (warp == 8) {
+    } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = umma_idesc(C::TF32, B_GATHER, BN);
+            constexpr uint32_t idesc = umma_idesc(C::TF32, C::B_MN, BN);
             uint32_t it = 0, tcount = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
@@ -202,15 +214,13 @@ __global__ void __launch_bounds__(kThreads, 1) gather_gemm_kernel(const __grid_c
                         break;
                     }
                     tc_fence_after();
-                    fence_proxy_async_smem();
                     const uint32_t a_addr = smem_u32(smem + s * C::STAGE_BYTES);
                     const uint32_t b_addr = a_addr + C::A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < C::BK / C::UK; ++kk) {
                         const uint64_t adesc = sw128_desc(a_addr + kk * 32, 16, 1024);
-                        const uint64_t bdesc = B_GATHER
-                                                   ? sw128_desc(b_addr + kk * C::UK * 128, C::BK * 128, 1024)
-                                                   : sw128_desc(b_addr + kk * 32, 16, 1024);
+                        const uint64_t bdesc = C::B_MN ? sw128_desc(b_addr + kk * C::UK * 128, C::GROUP_BYTES, 1024)
+                                                       : sw128_desc(b_addr + kk * 32, 16, 1024);
                         umma<C::TF32>(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     umma_commit(&empty[s]);
@@ -266,17 +276,17 @@ __global__ void __launch_bounds__(kThreads, 1) gather_gemm_kernel(const __grid_c
     }
 
     __syncthreads();
-    if (warp == 8) {
+    if (warp == 1) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
 }
 
-template <typename T, bool G, int BN>
+template <typename T, int BMODE, int BN>
 cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t s) {
-    using C = Cfg<T, BN>;
-    auto kern = gather_gemm_kernel<T, G, BN>;
+    using C = Cfg<T, BMODE, BN>;
+    auto kern = gather_gemm_kernel<T, BMODE, BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
     if (e != cudaSuccess) return e;
     const int total = p.heads * p.m_tiles * p.n_tiles;
@@ -286,26 +296,28 @@ cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+template <typename T, int BMODE>
+cudaError_t launch_bn(const GemmParams& p, const GemmLaunch& l, cudaStream_t s) {
+    return l.bn == 256 ? launch_one<T, BMODE, 256>(p, l.num_sms, s) : launch_one<T, BMODE, 128>(p, l.num_sms, s);
+}
+
 }  // namespace
 
 size_t gemm_smem_bytes(int dtype, int bn) {
-    if (dtype == 1) return bn == 256 ? Cfg<float, 256>::SMEM : Cfg<float, 128>::SMEM;
-    return bn == 256 ? Cfg<__nv_bfloat16, 256>::SMEM : Cfg<__nv_bfloat16, 128>::SMEM;
+    if (dtype == 1) return bn == 256 ? Cfg<float, kBKMajor, 256>::SMEM : Cfg<float, kBKMajor, 128>::SMEM;
+    return bn == 256 ? Cfg<__nv_bfloat16, kBGather, 256>::SMEM : Cfg<__nv_bfloat16, kBGather, 128>::SMEM;
 }
 
 cudaError_t launch_gemm(const GemmParams& p, const GemmLaunch& l, cudaStream_t s) {
     if (l.dtype == 1) {
-        if (l.b_gather)
-            return l.bn == 256 ? launch_one<float, true, 256>(p, l.num_sms, s)
-                               : launch_one<float, true, 128>(p, l.num_sms, s);
-        return l.bn == 256 ? launch_one<float, false, 256>(p, l.num_sms, s)
-                           : launch_one<float, false, 128>(p, l.num_sms, s);
+        if (l.b_mode != kBKMajor) return cudaErrorInvalidValue;
+        return launch_bn<float, kBKMajor>(p, l, s);
     }
-    if (l.b_gather)
-        return l.bn == 256 ? launch_one<__nv_bfloat16, true, 256>(p, l.num_sms, s)
-                           : launch_one<__nv_bfloat16, true, 128>(p, l.num_sms, s);
-    return l.bn == 256 ? launch_one<__nv_bfloat16, false, 256>(p, l.num_sms, s)
-                       : launch_one<__nv_bfloat16, false, 128>(p, l.num_sms, s);
+    switch (l.b_mode) {
+        case kBGather: return launch_bn<__nv_bfloat16, kBGather>(p, l, s);
+        case kBRows: return launch_bn<__nv_bfloat16, kBRows>(p, l, s);
+        default: return launch_bn<__nv_bfloat16, kBKMajor>(p, l, s);
+    }
 }
 
 }  // namespace rmm

@@ -19,13 +19,17 @@ struct SelectArgs {
     float* s2;           // [heads][d] out or nullptr
     // two-stage path only
     float* partials;     // [heads][nsplit][d]
-    int nsplit;
+    unsigned* counters;  // [heads][column blocks], zero between calls
+    float* scores;       // [heads][d] final fp32 scores (may alias s2)
+    int nsplit;          // 1 .. kMaxSplitRows
     int64_t rows_per_split;
 };
+constexpr int kMaxSplitRows = 16;
 
-// Column sums of squares in fp32, one partial per row split.
+// Column sums of squares in fp32: one partial per row split, then the last
+// CTA of each column block adds the partials in split order into `scores`.
 cudaError_t launch_colnorm(const SelectArgs& a, cudaStream_t s);
-// Sum the partials in split order, radix-select the k largest, emit I.
+// Radix-select the k largest final scores per head, emit I ascending.
 cudaError_t launch_topk(const SelectArgs& a, cudaStream_t s);
 // Scores and selection in one CTA per head (small inputs).
 cudaError_t launch_normselect(const SelectArgs& a, cudaStream_t s);
@@ -53,24 +57,29 @@ cudaError_t launch_pack(const PackArgs& a, cudaStream_t s);
 // dst[h][c][t] = src[h / group][I[h][t]][c]: gathered rows written K-major
 // (rows = number of source columns c; I == nullptr means I[t] = t).
 cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s);
+// dst[h][t][:] = src[h / group][I[h][t]][:] for t < k: the retained rows of a
+// row-major B, contiguous (a.rows = number of columns of B).
+cudaError_t launch_pack_rows(const PackArgs& a, int num_sms, cudaStream_t s);
 
 // ---------------------------------------------------------------- GEMM
+// How the B operand reaches shared memory (see rmm_gemm.cu).
+constexpr int kBKMajor = 0;  // TMA tiles of an m x K row-major matrix (K-major)
+constexpr int kBRows = 1;    // TMA tiles of consecutive rows of a d x m matrix (MN-major)
+constexpr int kBGather = 2;  // tile::gather4 of indexed rows of a d x m matrix (MN-major)
+
 // A operand: TMA tile loads from a 3-D map {K extent, rows, heads}, K-major.
-// B operand: either gathered rows of a d x m row-major matrix (LINEAR, PV;
-// MN-major in shared memory) or TMA tiles of an m x K row-major matrix
-// (QK; K-major).
 struct __align__(64) GemmParams {
     CUtensorMap map_a;
-    CUtensorMap map_b;          // TMA-B mode only
-    const void* B;              // gather mode: base of B
-    int64_t ldb, stride_b;      // gather mode
-    const int32_t* I;           // gather mode: [heads][k] row indices, nullptr = identity
+    CUtensorMap map_b;          // kBKMajor: 3-D {K, m, heads}; kBRows/kBGather: 2-D {m, rows}
+    const int32_t* I;           // kBGather: [heads][I_stride] row indices
     int64_t I_stride;
     void* Y;
     int64_t ldy, stride_y;
     int32_t n, m, k, d;
-    int32_t heads, group;       // B head = h / group (gather mode)
-    int32_t b_head_div;         // TMA-B mode: B head coordinate = h / b_head_div
+    int32_t heads, group;       // MN-major B head = h / group
+    int32_t b_head_rows;        // MN-major B: row offset between consecutive B heads
+    int32_t b_rows_total;       // MN-major B: rows of the 2-D map (an out-of-range row reads zeros)
+    int32_t b_head_div;         // kBKMajor: B head coordinate = h / b_head_div
     int32_t m_tiles, n_tiles;
     float alpha;
     int32_t causal;
@@ -79,7 +88,7 @@ struct __align__(64) GemmParams {
 
 struct GemmLaunch {
     int dtype;
-    bool b_gather;
+    int b_mode;       // kBKMajor / kBRows / kBGather
     int bn;           // 128 or 256
     int num_sms;
 };

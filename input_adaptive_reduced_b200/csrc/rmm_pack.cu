@@ -42,17 +42,27 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(
     T* dh = dst + (int64_t)h * stride_dst;
     const int64_t r_beg = (int64_t)blockIdx.y * kPackRows;
     const int64_t r_end = min(rows, r_beg + kPackRows);
-    for (int64_t r = r_beg; r < r_end; ++r) {
-        const T* s = sh + r * ld_src;
-        T vals[8];
+    // two rows per round: sixteen independent element loads in flight per thread
+    for (int64_t r = r_beg; r < r_end; r += 2) {
+        const bool two = r + 1 < r_end;
+        const T* s0 = sh + r * ld_src;
+        const T* s1 = sh + (two ? r + 1 : r) * ld_src;
+        __align__(16) T vals[2][8];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) vals[v] = live[v] ? s[idx[v]] : T(0.f);
-        T* o = dh + r * ld_dst + t0;
-        if constexpr (sizeof(T) == 2) {
-            *reinterpret_cast<uint4*>(o) = *reinterpret_cast<const uint4*>(vals);
-        } else {
-            reinterpret_cast<uint4*>(o)[0] = reinterpret_cast<const uint4*>(vals)[0];
-            reinterpret_cast<uint4*>(o)[1] = reinterpret_cast<const uint4*>(vals)[1];
+        for (int v = 0; v < 8; ++v) {
+            vals[0][v] = live[v] ? s0[idx[v]] : T(0.f);
+            vals[1][v] = live[v] ? s1[idx[v]] : T(0.f);
+        }
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            if (q == 1 && !two) break;
+            T* o = dh + (r + q) * ld_dst + t0;
+            if constexpr (sizeof(T) == 2) {
+                *reinterpret_cast<uint4*>(o) = *reinterpret_cast<const uint4*>(vals[q]);
+            } else {
+                reinterpret_cast<uint4*>(o)[0] = reinterpret_cast<const uint4*>(vals[q])[0];
+                reinterpret_cast<uint4*>(o)[1] = reinterpret_cast<const uint4*>(vals[q])[1];
+            }
         }
     }
 }
@@ -89,7 +99,66 @@ __global__ void __launch_bounds__(256) pack_rows_transposed_kernel(
     }
 }
 
+// Row gather for bf16 B operands: dst[h][t][:] = src[h / group][I[h][t]][:]
+// for t < k (rows of `cols` elements).  grid (ceil(k / kRowsPerCta), heads);
+// the CTA copies its rows with 16-byte loads and stores, four independent
+// chunks in flight per thread.  The retained rows are contiguous segments of B,
+// so both sides are fully coalesced.
+constexpr int kRowsPerCta = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(256) pack_rows_kernel(
+    const T* __restrict__ src, int64_t d, int64_t cols, int64_t ld_src, int64_t stride_src, int group,
+    const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
+    int64_t stride_dst) {
+    constexpr int V = 16 / sizeof(T);
+    const int h = blockIdx.y;
+    const int cpr = (int)(cols / V);
+    const int64_t t0 = (int64_t)blockIdx.x * kRowsPerCta;
+    const int64_t left = k - t0;
+    const int nrows = left < kRowsPerCta ? (int)left : kRowsPerCta;
+    const int total = nrows * cpr;
+    const T* sh = src + (int64_t)(h / group) * stride_src;
+    T* dh = dst + (int64_t)h * stride_dst;
+    const int32_t* Ih = I + (int64_t)h * I_stride + t0;
+    for (int base = threadIdx.x; base < total; base += 4 * 256) {
+        uint4 v[4];
+        int64_t out[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int idx = base + u * 256;
+            out[u] = -1;
+            if (idx < total) {
+                const int r = idx / cpr;
+                const int c = idx - r * cpr;
+                int64_t j = __ldg(Ih + r);
+                j = j < 0 ? 0 : (j >= d ? d - 1 : j);
+                v[u] = __ldg(reinterpret_cast<const uint4*>(sh + j * ld_src) + c);
+                out[u] = (t0 + r) * ld_dst + (int64_t)c * V;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (out[u] >= 0) *reinterpret_cast<uint4*>(dh + out[u]) = v[u];
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_pack_rows(const PackArgs& a, int num_sms, cudaStream_t s) {
+    (void)num_sms;
+    if (a.k == 0 || a.rows == 0) return cudaSuccess;
+    dim3 grid((unsigned)((a.k + kRowsPerCta - 1) / kRowsPerCta), (unsigned)a.heads);
+    if (a.dtype == 1)
+        pack_rows_kernel<float><<<grid, 256, 0, s>>>((const float*)a.src, a.d, a.rows, a.ld_src, a.stride_src,
+                                                     a.group, a.I, a.I_stride, a.k, (float*)a.dst, a.ld_dst,
+                                                     a.stride_dst);
+    else
+        pack_rows_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+            (const __nv_bfloat16*)a.src, a.d, a.rows, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k,
+            (__nv_bfloat16*)a.dst, a.ld_dst, a.stride_dst);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s) {
     // a.rows = columns of the source (m), a.d = rows of the source, a.I may be null (identity)

@@ -48,17 +48,27 @@ struct Vec16<float> {
 
 // ------------------------------------------------------------------ colnorm
 // grid (ceil(d / (32*V)), nsplit, heads), 256 threads.  Warp w of split s sums
-// rows r0+w, r0+w+8, ... of its 32*V columns in increasing row order; the 8
-// warp partials are added in warp order; splits are added in split order by
-// the TopK kernel.
+// rows r0+w, r0+w+8, ... of its 32*V columns in increasing row order (eight
+// independent 16-byte loads in flight per thread); the 8 warp partials are
+// added in warp order and written as the split's partial.  The last CTA of a
+// column block to finish (device-scope counter) adds the nsplit partials of
+// its columns in split order and writes the final fp32 scores, then resets
+// the counter for the next call.  The order of every sum is fixed and the
+// same for every column.
+constexpr int kMaxSplit = 16;
+
 template <typename T>
 __global__ void __launch_bounds__(256) colnorm_kernel(const T* __restrict__ A, int64_t n, int64_t d,
                                                       int64_t lda, int64_t stride_a,
                                                       int64_t rows_per_split, int nsplit,
-                                                      float* __restrict__ partials) {
+                                                      float* __restrict__ partials,
+                                                      unsigned* __restrict__ counters,
+                                                      float* __restrict__ s2) {
     constexpr int V = Vec16<T>::N;
     constexpr int COLS = 32 * V;
+    constexpr int U = 8;
     __shared__ float red[8][COLS];
+    __shared__ bool last;
     const int h = blockIdx.z, split = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t col = (int64_t)blockIdx.x * COLS + lane * V;
@@ -70,19 +80,14 @@ __global__ void __launch_bounds__(256) colnorm_kernel(const T* __restrict__ A, i
     if (col < d) {
         const T* base = A + (int64_t)h * stride_a + col;
         int64_t r = r0 + warp;
-        for (; r + 24 < r1; r += 32) {
-            float x0[V], x1[V], x2[V], x3[V];
-            Vec16<T>::load(base + r * lda, x0);
-            Vec16<T>::load(base + (r + 8) * lda, x1);
-            Vec16<T>::load(base + (r + 16) * lda, x2);
-            Vec16<T>::load(base + (r + 24) * lda, x3);
+        for (; r + 8 * (U - 1) < r1; r += 8 * U) {
+            float x[U][V];
 #pragma unroll
-            for (int v = 0; v < V; ++v) {
-                acc[v] = fmaf(x0[v], x0[v], acc[v]);
-                acc[v] = fmaf(x1[v], x1[v], acc[v]);
-                acc[v] = fmaf(x2[v], x2[v], acc[v]);
-                acc[v] = fmaf(x3[v], x3[v], acc[v]);
-            }
+            for (int u = 0; u < U; ++u) Vec16<T>::load(base + (r + 8 * u) * lda, x[u]);
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[v] = fmaf(x[u][v], x[u][v], acc[v]);
         }
         for (; r < r1; r += 8) {
             float x0[V];
@@ -95,11 +100,35 @@ __global__ void __launch_bounds__(256) colnorm_kernel(const T* __restrict__ A, i
     for (int v = 0; v < V; ++v) red[warp][lane * V + v] = acc[v];
     __syncthreads();
     for (int c = threadIdx.x; c < COLS; c += 256) {
-        float s = red[0][c];
+        float sum = red[0][c];
 #pragma unroll
-        for (int w = 1; w < 8; ++w) s += red[w][c];
+        for (int w = 1; w < 8; ++w) sum += red[w][c];
         const int64_t gcol = (int64_t)blockIdx.x * COLS + c;
-        if (gcol < d) partials[((int64_t)h * nsplit + split) * d + gcol] = s;
+        if (gcol < d) partials[((int64_t)h * nsplit + split) * d + gcol] = sum;
+    }
+    // last CTA of this column block: fixed-order sum over the splits
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned* ctr = counters + (int64_t)h * gridDim.x + blockIdx.x;
+        last = atomicAdd(ctr, 1u) == (unsigned)(nsplit - 1);
+        if (last) *ctr = 0u;
+    }
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    for (int c = threadIdx.x; c < COLS; c += 256) {
+        const int64_t gcol = (int64_t)blockIdx.x * COLS + c;
+        if (gcol >= d) continue;
+        const float* pc = partials + (int64_t)h * nsplit * d + gcol;
+        float v[kMaxSplit];
+#pragma unroll
+        for (int sp = 0; sp < kMaxSplit; ++sp) v[sp] = sp < nsplit ? __ldcg(pc + (int64_t)sp * d) : 0.f;
+        float sum = v[0];
+#pragma unroll
+        for (int sp = 1; sp < kMaxSplit; ++sp)
+            if (sp < nsplit) sum += v[sp];
+        s2[(int64_t)h * d + gcol] = sum;
     }
 }
 
@@ -107,6 +136,7 @@ __global__ void __launch_bounds__(256) colnorm_kernel(const T* __restrict__ A, i
 // Works on keys[0..d) in shared memory (fp32 bit patterns of s^2 >= 0) with a
 // 1024-thread block.  Writes the k selected indices, ascending, to out[].
 struct TopkShared {
+    uint32_t whist[32][256];  // one private histogram per warp (no inter-warp atomics)
     uint32_t hist[256];
     uint32_t prefix;
     uint32_t remaining;
@@ -121,8 +151,8 @@ __device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t prefix = 0, mask = 0, remaining = (uint32_t)k;
     for (int shift = 24; shift >= 0; shift -= 8) {
-        if (tid < 256) sh.hist[tid] = 0;
-        __syncthreads();
+        for (int b = lane; b < 256; b += 32) sh.whist[warp][b] = 0;
+        __syncwarp();
         for (int64_t base = 0; base < d; base += 1024) {
             const int64_t j = base + tid;
             int bin = -1;
@@ -131,7 +161,15 @@ __device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k
                 if ((key & mask) == prefix) bin = (int)((key >> shift) & 255u);
             }
             const unsigned peers = __match_any_sync(0xffffffffu, bin);
-            if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], (uint32_t)__popc(peers));
+            if (bin >= 0 && lane == __ffs(peers) - 1) sh.whist[warp][bin] += (uint32_t)__popc(peers);
+            __syncwarp();
+        }
+        __syncthreads();
+        if (tid < 256) {
+            uint32_t c = 0;
+#pragma unroll 8
+            for (int w = 0; w < 32; ++w) c += sh.whist[w][tid];
+            sh.hist[tid] = c;
         }
         __syncthreads();
         if (warp == 0) {
@@ -227,21 +265,14 @@ __device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k
 }
 
 // ------------------------------------------------------------------ TopK
-// One 1024-thread CTA per head: sum the split partials in split order, then
-// select.
-__global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ partials, int nsplit,
-                                                    int64_t d, int64_t k, int32_t* __restrict__ I,
-                                                    float* __restrict__ s2) {
+// One 1024-thread CTA per head on the final scores written by colnorm.
+__global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ scores, int64_t d, int64_t k,
+                                                    int32_t* __restrict__ I) {
     extern __shared__ uint32_t keys[];
     __shared__ TopkShared sh;
     const int h = blockIdx.x;
-    const float* p = partials + (int64_t)h * nsplit * d;
-    for (int64_t j = threadIdx.x; j < d; j += 1024) {
-        float s = p[j];
-        for (int sp = 1; sp < nsplit; ++sp) s += p[(int64_t)sp * d + j];
-        keys[j] = __float_as_uint(s);
-        if (s2) s2[(int64_t)h * d + j] = s;
-    }
+    const float* p = scores + (int64_t)h * d;
+    for (int64_t j = threadIdx.x; j < d; j += 1024) keys[j] = __float_as_uint(p[j]);
     __syncthreads();
     radix_select_and_emit(keys, d, k, I + (int64_t)h * k, sh);
 }
@@ -339,15 +370,17 @@ size_t normselect_smem_bytes(int64_t d, int dtype) {
 }
 
 cudaError_t launch_colnorm(const SelectArgs& a, cudaStream_t s) {
+    if (a.nsplit < 1 || a.nsplit > kMaxSplit) return cudaErrorInvalidValue;
     const int V = a.dtype == 1 ? 4 : 8;
     dim3 grid((unsigned)((a.d + 32 * V - 1) / (32 * V)), (unsigned)a.nsplit, (unsigned)a.heads);
     if (a.dtype == 1)
         colnorm_kernel<float><<<grid, 256, 0, s>>>((const float*)a.A, a.n, a.d, a.lda, a.stride_a,
-                                                   a.rows_per_split, a.nsplit, a.partials);
+                                                   a.rows_per_split, a.nsplit, a.partials, a.counters,
+                                                   a.scores);
     else
         colnorm_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)a.A, a.n, a.d,
                                                            a.lda, a.stride_a, a.rows_per_split,
-                                                           a.nsplit, a.partials);
+                                                           a.nsplit, a.partials, a.counters, a.scores);
     return cudaGetLastError();
 }
 
@@ -356,7 +389,7 @@ cudaError_t launch_topk(const SelectArgs& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    topk_kernel<<<a.heads, 1024, smem, s>>>(a.partials, a.nsplit, a.d, a.k, a.I, a.s2);
+    topk_kernel<<<a.heads, 1024, smem, s>>>(a.scores, a.d, a.k, a.I);
     return cudaGetLastError();
 }
 

@@ -1,0 +1,114 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration the
+benchmark times: the index sets are compared in full (every head), the
+products on two seeded rows of every 128-row tile (all rows when n <= 16)
+against the oracle computed row by row."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests import gap
+from tests.parity import assert_indices_equal, assert_product_close, np64, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rmm(cuda_device):
+    import input_adaptive_reduced_b200 as r
+    return r
+
+
+def _linear_full(rmm, gen, n, rhos, seed, **kw):
+    d = gen(seed, n=1, m=8, **kw)[0].shape[1] if "shape" not in kw else W.LLAMA70B_LINEAR[kw["shape"]][0]
+    ks = [oracle.retained_count(r, d) for r in rhos]
+    (A, B), _ = gap.enforce_boundary_gaps(lambda g: gen(seed, n=n, col_gain=g, **kw),
+                                          lambda x: gap.scores_2d(x[0]), ks)
+    Ag, Bg = A.cuda(), B.cuda()
+    A64, B64 = oracle.as_f64(A), oracle.as_f64(B)
+    rows = list(range(n)) if n <= 16 else sample_rows(n, seed)
+    for rho in rhos:
+        Y, I = rmm.matmul(Ag, Bg, rho=rho, return_indices=True)
+        torch.cuda.synchronize()
+        rmm.check_workspaces()
+        I_ref, _ = oracle.select(A64, rho=rho)
+        assert_indices_equal(I, I_ref)
+        Y_ref = oracle.reduced_product(A64, B64, I_ref, rows)
+        assert_product_close(Y[rows], Y_ref, np.abs(A64[rows][:, I_ref]), np.abs(B64[I_ref]))
+
+
+@pytest.mark.parametrize("n", [1024, 4096])
+def test_llama8b_up_gate(rmm, n):
+    _linear_full(rmm, W.mlp_up, n, [0.5, 0.8] if n == 4096 else [0.7], seed=101)
+
+
+@pytest.mark.parametrize("n", [2048, 4096])
+def test_llama8b_down(rmm, n):
+    _linear_full(rmm, W.mlp_down, n, [0.7] if n == 4096 else [0.5, 0.8], seed=102)
+
+
+@pytest.mark.parametrize("shape,n,rhos", [
+    ("up", 1, [0.5, 0.8]), ("up", 16, [0.6, 1.0]), ("down", 16, [0.7]), ("qkv", 16, [0.8]),
+    ("down", 1, [0.6]), ("qkv", 512, [0.5, 0.7]), ("up", 2048, [0.8]),
+])
+def test_llama70b_linear(rmm, shape, n, rhos):
+    _linear_full(rmm, W.linear_70b, n, rhos, seed=103, shape=shape)
+
+
+@pytest.mark.parametrize("n", [1024, 4096])
+def test_attention_qk_full(rmm, n):
+    H, Hkv, dh = 32, 8, 128
+    rhos = [0.5, 0.8]
+    ks = [oracle.retained_count(r, dh) for r in rhos]
+    (Q, K), _ = gap.enforce_boundary_gaps(
+        lambda g: W.attn_qk(104, n=n, col_gain=g), lambda x: gap.scores_per_head(x[0]), ks)
+    Qg, Kg = Q.cuda(), K.cuda()
+    alpha = 1.0 / math.sqrt(dh)
+    Q64, K64 = oracle.as_f64(Q), oracle.as_f64(K)
+    rows = sample_rows(n, 7)
+    heads = [0, 13, 31]
+    for rho in rhos:
+        S, I = rmm.qk(Qg, Kg, rho=rho, alpha=alpha, causal=True, return_indices=True)
+        torch.cuda.synchronize()
+        rmm.check_workspaces()
+        S_ref, I_ref = oracle.rmm_qk(Q64, K64, rho=rho, alpha=alpha, causal=True, heads=heads, rows=rows)
+        assert_indices_equal(I, I_ref)
+        mask = np.arange(n)[None, :] > np.asarray(rows)[:, None]
+        for i, h in enumerate(heads):
+            g = oracle.kv_head_of(h, H, Hkv)
+            assert_product_close(S[h][rows], S_ref[i], np.abs(Q64[h][rows][:, I_ref[h]]),
+                                 np.abs(K64[g][:, I_ref[h]]).T, alpha=alpha, mask=mask)
+        # every masked entry of every head is -inf; no unmasked entry is
+        upper = torch.ones(n, n, dtype=torch.bool, device="cuda").triu_(1)
+        assert bool(torch.isneginf(S[:, upper]).all())
+        assert not bool(torch.isinf(S[:, ~upper]).any())
+
+
+@pytest.mark.parametrize("n", [2048, 4096])
+def test_attention_pv_full(rmm, n):
+    H, Hkv, dv = 32, 8, 128
+    rhos = [0.5, 0.8]
+    ks = [oracle.retained_count(r, n) for r in rhos]
+    dev = torch.device("cuda")
+    (P, V), _ = gap.enforce_boundary_gaps(
+        lambda g: W.attn_pv(105, n=n, col_gain=g, device=dev),
+        lambda x: [oracle.column_scores_sq(x[0][h]) for h in range(H)], ks)
+    rows = sample_rows(n, 9)
+    heads = [0, 17, 31]
+    P64 = {h: oracle.as_f64(P[h]) for h in heads}
+    V64 = oracle.as_f64(V)
+    for rho in rhos:
+        O, T = rmm.pv(P, V, rho=rho, return_indices=True)
+        torch.cuda.synchronize()
+        rmm.check_workspaces()
+        k = oracle.retained_count(rho, n)
+        T_ref = np.stack([oracle.select(P[h], k=k)[0] for h in range(H)])
+        assert_indices_equal(T, T_ref)
+        for h in heads:
+            g = oracle.kv_head_of(h, H, Hkv)
+            O_ref = oracle.reduced_product(P64[h], V64[g], T_ref[h], rows)
+            assert_product_close(O[h][rows], O_ref, np.abs(P64[h][rows][:, T_ref[h]]),
+                                 np.abs(V64[g][T_ref[h]]))

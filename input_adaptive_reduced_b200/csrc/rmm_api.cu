@@ -18,7 +18,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
-#include "../../include/rmm.h"
+#include "rmm.h"
 #include "rmm_internal.h"
 
 struct rmm_plan {

@@ -134,10 +134,12 @@ __global__ void __launch_bounds__(256) colnorm_kernel(const T* __restrict__ A, i
 
 // ------------------------------------------------------------------ TopK core
 // Works on keys[0..d) in shared memory (fp32 bit patterns of s^2 >= 0) with a
-// 1024-thread block.  Writes the k selected indices, ascending, to out[].
+// 1024-thread block.  Three radix passes over bits [31:21], [20:10] and [9:0]
+// find the exact k-th largest key T and how many keys equal to T are kept;
+// then the indices are emitted in ascending order.
 struct TopkShared {
-    uint32_t whist[32][256];  // one private histogram per warp (no inter-warp atomics)
-    uint32_t hist[256];
+    uint32_t hist[2048];
+    uint32_t warp_tot[32];
     uint32_t prefix;
     uint32_t remaining;
     uint32_t warp_gt[32];
@@ -150,60 +152,54 @@ __device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k
                                       TopkShared& sh) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t prefix = 0, mask = 0, remaining = (uint32_t)k;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int b = lane; b < 256; b += 32) sh.whist[warp][b] = 0;
-        __syncwarp();
-        for (int64_t base = 0; base < d; base += 1024) {
-            const int64_t j = base + tid;
-            int bin = -1;
-            if (j < d) {
-                const uint32_t key = keys[j];
-                if ((key & mask) == prefix) bin = (int)((key >> shift) & 255u);
-            }
-            const unsigned peers = __match_any_sync(0xffffffffu, bin);
-            if (bin >= 0 && lane == __ffs(peers) - 1) sh.whist[warp][bin] += (uint32_t)__popc(peers);
-            __syncwarp();
+    const int shifts[3] = {21, 10, 0};
+    const int widths[3] = {11, 11, 10};
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shift = shifts[pass];
+        const int nb = 1 << widths[pass];
+        for (int b = tid; b < nb; b += 1024) sh.hist[b] = 0;
+        __syncthreads();
+        for (int64_t j = tid; j < d; j += 1024) {
+            const uint32_t key = keys[j];
+            if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & (uint32_t)(nb - 1)], 1u);
         }
         __syncthreads();
-        if (tid < 256) {
-            uint32_t c = 0;
-#pragma unroll 8
-            for (int w = 0; w < 32; ++w) c += sh.whist[w][tid];
-            sh.hist[tid] = c;
+        // thread t owns bins nb-1-2t and nb-2-2t: a block scan in descending bin order
+        const int b_hi = nb - 1 - 2 * tid, b_lo = b_hi - 1;
+        const uint32_t c0 = b_hi >= 0 ? sh.hist[b_hi] : 0u;
+        const uint32_t c1 = b_lo >= 0 ? sh.hist[b_lo] : 0u;
+        const uint32_t tot = c0 + c1;
+        uint32_t incl = tot;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
         }
+        if (lane == 31) sh.warp_tot[warp] = incl;
         __syncthreads();
         if (warp == 0) {
-            // lane l owns bins 255-8l down to 248-8l (descending order)
-            uint32_t c[8], tot = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                c[i] = sh.hist[255 - 8 * lane - i];
-                tot += c[i];
-            }
-            uint32_t incl = tot;
+            const uint32_t w = sh.warp_tot[lane];
+            uint32_t wi = w;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += y;
+                const uint32_t y = __shfl_up_sync(0xffffffffu, wi, off);
+                if (lane >= off) wi += y;
             }
-            const uint32_t excl = incl - tot;
-            if (excl < remaining && remaining <= incl) {
-                uint32_t above = excl;
-                for (int i = 0; i < 8; ++i) {
-                    if (above + c[i] >= remaining) {
-                        const uint32_t b = 255u - 8u * lane - i;
-                        sh.prefix = prefix | (b << shift);
-                        sh.remaining = remaining - above;
-                        break;
-                    }
-                    above += c[i];
-                }
-            }
+            sh.warp_tot[lane] = wi - w;  // exclusive prefix of the warp totals
+        }
+        __syncthreads();
+        const uint32_t excl = sh.warp_tot[warp] + incl - tot;
+        if (tot > 0 && excl < remaining && remaining <= excl + tot) {
+            const bool hi = excl + c0 >= remaining;
+            const uint32_t b = (uint32_t)(hi ? b_hi : b_lo);
+            sh.prefix = prefix | (b << shift);
+            sh.remaining = remaining - (hi ? excl : excl + c0);
         }
         __syncthreads();
         prefix = sh.prefix;
         remaining = sh.remaining;
-        mask |= 255u << shift;
+        mask |= (uint32_t)(nb - 1) << shift;
         __syncthreads();
     }
     const uint32_t T = prefix;      // the k-th largest key

@@ -23,7 +23,7 @@ __all__ = [
     "rmm_problem_init", "rmm_plan_create", "rmm_select", "rmm_matmul", "rmm_matmul_batched",
     "rmm_workspace_init", "rmm_workspace_status", "rmm_status_string", "rmm_version",
     "EXPORTED_SYMBOLS", "select", "matmul", "qk", "pv", "workspace_for", "check_workspaces",
-    "rmm_plan_set_product_events", "rmm_plan_kernel_launches",
+    "rmm_plan_set_product_events", "rmm_plan_kernel_launches", "rmm_select_no_alloc",
 ]
 
 RMM_OK, RMM_ERR_INVALID_ARG, RMM_ERR_UNSUPPORTED, RMM_ERR_WORKSPACE, RMM_ERR_CUDA, RMM_ERR_TIMEOUT = range(6)
@@ -36,6 +36,7 @@ EXPORTED_SYMBOLS = (
     "rmm_problem_init", "rmm_plan_create", "rmm_plan_destroy", "rmm_plan_k", "rmm_plan_workspace_size",
     "rmm_select", "rmm_matmul", "rmm_matmul_batched", "rmm_workspace_init", "rmm_workspace_status",
     "rmm_status_string", "rmm_version", "rmm_plan_set_product_events", "rmm_plan_kernel_launches",
+    "rmm_select_no_alloc",
 )
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librmm.so")
@@ -96,6 +97,8 @@ def _load_library():
     L.rmm_plan_set_product_events.argtypes = [vp, vp, vp]
     L.rmm_plan_kernel_launches.restype = ctypes.c_int32
     L.rmm_plan_kernel_launches.argtypes = [vp]
+    L.rmm_select_no_alloc.restype = st
+    L.rmm_select_no_alloc.argtypes = [vp, vp, vp, vp, vp]
     L.rmm_status_string.restype = ctypes.c_char_p
     L.rmm_status_string.argtypes = [st]
     L.rmm_version.restype = ctypes.c_char_p
@@ -206,6 +209,14 @@ def rmm_workspace_status(plan: Plan, workspace, stream=None) -> int:
 def rmm_select(plan: Plan, A, I, s2=None, workspace=None, stream=None):
     wp, wb = _ws(workspace)
     _check(lib.rmm_select(plan.handle, _ptr(A), _ptr(I), _ptr(s2), wp, wb, _stream(stream)), "rmm_select")
+
+
+def rmm_select_no_alloc(plan: Plan, A, I, s2=None, stream=None):
+    """rmm_select without a workspace: scratch lives in a static device array
+    inside librmm (see include/rmm.h for the size limit and the rules on
+    overlapping calls)."""
+    _check(lib.rmm_select_no_alloc(plan.handle, _ptr(A), _ptr(I), _ptr(s2), _stream(stream)),
+           "rmm_select_no_alloc")
 
 
 def rmm_matmul(plan: Plan, A, B, Y, I=None, workspace=None, stream=None):

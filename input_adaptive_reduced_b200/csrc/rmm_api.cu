@@ -21,23 +21,7 @@
 #include "rmm.h"
 #include "rmm_internal.h"
 
-struct rmm_plan {
-    rmm_problem p;
-    int64_t k;
-    int64_t ldp;        // row stride of the packed operands (k rounded up to 8)
-    int es;             // element size
-    int group;          // heads / kv_heads
-    bool need_select;   // scores + TopK on each call
-    bool fused_select;  // one-kernel selection
-    int nsplit;
-    int64_t rows_per_split;
-    int bn;
-    bool pack_b;        // bf16 LINEAR/PV with k < d: stage B[I, :] contiguously
-    int num_sms;
-    size_t off_err, off_counters, off_partials, off_scores, off_I, off_apack, off_bpack, ws_bytes;
-    size_t header_bytes;  // zeroed by rmm_workspace_init: error word + colnorm counters
-    cudaEvent_t product_start, product_stop;  // tracing hook, may be null
-};
+
 
 namespace {
 

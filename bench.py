@@ -137,6 +137,23 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None}
 
 
+def reduce_max(value: float, device=None) -> float:
+    """Max of a per-rank time over all ranks (the replica timing rule); the
+    identity when no process group is initialised."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Useful TFLOP/s of the whole job: every rank's work over the slowest rank's time."""
+    return flops_per_rank_step * world / (ms_per_step * 1e-3) / 1e12
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -293,14 +310,10 @@ def run_rmm(args):
         e["rmm"]["plan"].set_product_events(None, None)
     rmm.check_workspaces()
 
-    ms_total = t_start.elapsed_time(t_stop)
-    if world > 1:
-        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = reduce_max(t_start.elapsed_time(t_stop), dev)
     ms_step = ms_total / args.steps
     flops_step = useful_flops(n, rho)
-    value = flops_step * world / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(flops_step, world, ms_step)
 
     # product kernel (dominant kernel): algorithmic flops per launch / event time
     gemm_ms = [s.elapsed_time(t) for s, t in zip(ev_start, ev_stop)]
@@ -378,12 +391,8 @@ def run_rmm(args):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize(dev)
-        ms_e2e = a.elapsed_time(b) / e2e_steps
-        if world > 1:
-            t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": flops_step * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+        ms_e2e = reduce_max(a.elapsed_time(b) / e2e_steps, dev)
+        e2e = {"value": whole_job_tflops(flops_step, world, ms_e2e), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                "path": "pinned host A, B -> device, rmm_matmul (C ABI), Y -> pinned host"}
 

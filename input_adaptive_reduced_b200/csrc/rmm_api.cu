@@ -231,6 +231,10 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
     }
 
     rmm::GemmLaunch gl;
+    // CTA pairs (256-row tiles) whenever there is more than one 128-row tile of
+    // work; indexed gather4 feeding stays single-CTA.
+    const bool pair_ok = p.n > 128;
+    const uint32_t kmajor_box_rows = static_cast<uint32_t>(pair_ok ? plan->bn / 2 : plan->bn);
     gl.dtype = p.dtype;
     gl.bn = plan->bn;
     gl.num_sms = plan->num_sms;
@@ -243,7 +247,7 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
     gp.d = static_cast<int32_t>(p.d);
     gp.heads = static_cast<int32_t>(p.heads);
     gp.group = plan->group;
-    gp.m_tiles = static_cast<int32_t>((p.n + 127) / 128);
+
     gp.n_tiles = static_cast<int32_t>((p.m + plan->bn - 1) / plan->bn);
     gp.alpha = p.alpha;
     gp.causal = (p.flags & RMM_FLAG_CAUSAL) ? 1 : 0;
@@ -270,11 +274,11 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
             pb.heads = static_cast<int>(p.heads);
             if (rmm::launch_pack(pb, stream) != cudaSuccess) return RMM_ERR_CUDA;
             if (!encode_kmajor_map(&gp.map_b, es, pb.dst, k, p.m, p.heads, plan->ldp, p.m * plan->ldp, box_k,
-                                   static_cast<uint32_t>(plan->bn)))
+                                   kmajor_box_rows))
                 return RMM_ERR_CUDA;
         } else {
             if (!encode_kmajor_map(&gp.map_b, es, B, p.d, p.m, p.kv_heads, p.ldb, p.stride_b, box_k,
-                                   static_cast<uint32_t>(plan->bn)))
+                                   kmajor_box_rows))
                 return RMM_ERR_CUDA;
             gp.b_head_div = plan->group;
         }
@@ -298,7 +302,7 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         pb.heads = static_cast<int>(p.heads);
         if (rmm::launch_pack_rows_transposed(pb, stream) != cudaSuccess) return RMM_ERR_CUDA;
         if (!encode_kmajor_map(&gp.map_b, es, pb.dst, k, p.m, p.heads, plan->ldp, p.m * plan->ldp, box_k,
-                               static_cast<uint32_t>(plan->bn)))
+                               kmajor_box_rows))
             return RMM_ERR_CUDA;
     } else if (!identity && plan->pack_b) {
         // The retained rows B[I, :] are copied into a contiguous k x m buffer per
@@ -339,6 +343,8 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         gp.I_stride = k;
         if (!encode_rows_map(&gp.map_b, B, p.m, rows_total, p.ldb, row_tiles ? 64u : 1u)) return RMM_ERR_CUDA;
     }
+    gl.pair = pair_ok && gl.b_mode != rmm::kBGather;
+    gp.m_tiles = static_cast<int32_t>(gl.pair ? (p.n + 255) / 256 : (p.n + 127) / 128);
     const bool traced = plan->product_start && plan->product_stop;
     if (traced && cudaEventRecord(plan->product_start, stream) != cudaSuccess) return RMM_ERR_CUDA;
     if (rmm::launch_gemm(gp, gl, stream) != cudaSuccess) return RMM_ERR_CUDA;

@@ -283,6 +283,226 @@ __global__ void __launch_bounds__(kThreads, 1) gather_gemm_kernel(const __grid_c
     }
 }
 
+// ----------------------------------------------------------------------------
+// CTA-pair variant (cluster of 2, tcgen05 cta_group::2).  The pair computes a
+// 256 x BN tile: CTA r loads rows [m0 + 128 r, +128) of A and columns
+// [n0 + (BN/2) r, +BN/2) of B into its own shared memory, and both count
+// their TMA bytes on the leader's full barrier.  The leader's MMA thread
+// issues M = 256 MMAs that read both CTAs' operands; each CTA's tensor memory
+// receives its 128 rows x BN accumulator.  Stage releases and accumulator
+// hand-offs are multicast commits to both CTAs; the peer's epilogue releases
+// the accumulator with remote arrivals on the leader's barrier.  Halving B per
+// CTA halves the shared-memory operand traffic of the 1-CTA 128 x BN tile.
+// ----------------------------------------------------------------------------
+template <typename T, int BMODE, int BN>
+struct PairCfg {
+    static constexpr int ES = sizeof(T);
+    static constexpr bool TF32 = (ES == 4);
+    static constexpr bool B_MN = (BMODE != kBKMajor);
+    static constexpr int BK = 128 / ES;
+    static constexpr int UK = 32 / ES;
+    static constexpr int HALF_N = BN / 2;             // B columns held by one CTA
+    static constexpr int A_BYTES = kBM * 128;         // 128 rows x 128 B
+    static constexpr int B_BYTES = HALF_N * 128;      // BK rows x HALF_N (MN) or HALF_N rows x 128 B (K)
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = 6;
+    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int GROUP_BYTES = BK * 128;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+    static_assert(!(TF32 && B_MN), "fp32 operands are staged K-major");
+    static_assert(BMODE != kBGather, "indexed gathers use the single-CTA kernel");
+};
+
+template <typename T, int BMODE, int BN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    pair_gemm_kernel(const __grid_constant__ GemmParams p) {
+    using C = PairCfg<T, BMODE, BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+    uint64_t* empty = full + C::STAGES;
+    uint64_t* tfull = empty + C::STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);   // the leader's expect_tx arrival (+ both CTAs' bytes)
+            mbar_init(&empty[s], 1);  // one multicast commit
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);   // one multicast commit
+            mbar_init(&tempty[a], 8);  // 4 epilogue warps x 2 CTAs (used in the leader)
+        }
+        *abort_flag = 0;
+        mbar_fence_init();
+        tma_prefetch_map(&p.map_a);
+        tma_prefetch_map(&p.map_b);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();  // barriers of both CTAs initialised before any remote arrival
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    const int total = p.heads * p.m_tiles * p.n_tiles;  // 256-row tiles
+    const int num_kb = (p.k + C::BK - 1) / C::BK;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = cluster; t < total && ok; t += nclusters) {
+                const int mt = t % p.m_tiles, rest = t / p.m_tiles;
+                const int nt = rest % p.n_tiles, h = rest / p.n_tiles;
+                const int m0 = mt * 2 * kBM, n0 = nt * BN;
+                if (p.causal && n0 > m0 + 2 * kBM - 1) continue;
+                const int row_base = (h / p.group) * p.b_head_rows;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t ph = (it / C::STAGES) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err, kErrTimeoutProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + s * C::STAGE_BYTES;
+                    uint8_t* sb = sa + C::A_BYTES;
+                    const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::STAGE_BYTES);
+                    tma_load_3d_pair(sa, &p.map_a, bar, kb * C::BK, m0 + (int)rank * kBM, h);
+                    if constexpr (BMODE == kBKMajor) {
+                        tma_load_3d_pair(sb, &p.map_b, bar, kb * C::BK, n0 + (int)rank * C::HALF_N,
+                                         h / p.b_head_div);
+                    } else {
+#pragma unroll
+                        for (int g = 0; g < C::HALF_N / 64; ++g)
+                            tma_load_2d_pair(sb + g * C::GROUP_BYTES, &p.map_b, bar,
+                                             n0 + (int)rank * C::HALF_N + 64 * g, row_base + kb * C::BK);
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader only)
+        if (leader && lane == 0) {
+            constexpr uint32_t idesc = umma_idesc(C::TF32, C::B_MN, BN, 256);
+            uint32_t it = 0, tcount = 0;
+            bool ok = true;
+            for (int t = cluster; t < total && ok; t += nclusters) {
+                const int mt = t % p.m_tiles, rest = t / p.m_tiles;
+                const int nt = rest % p.n_tiles;
+                const int m0 = mt * 2 * kBM, n0 = nt * BN;
+                if (p.causal && n0 > m0 + 2 * kBM - 1) continue;
+                const uint32_t acc = tcount & 1u;
+                const uint32_t aph = (tcount >> 1) & 1u;
+                if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, p.err, kErrTimeoutMma)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * BN;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t ph = (it / C::STAGES) & 1u;
+                    if (!mbar_wait(&full[s], ph, abort_flag, p.err, kErrTimeoutMma)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + s * C::STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + C::A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < C::BK / C::UK; ++kk) {
+                        const uint64_t adesc = sw128_desc(a_addr + kk * 32, 16, 1024);
+                        const uint64_t bdesc = C::B_MN ? sw128_desc(b_addr + kk * C::UK * 128, C::GROUP_BYTES, 1024)
+                                                       : sw128_desc(b_addr + kk * 32, 16, 1024);
+                        umma_pair<C::TF32>(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    umma_commit_pair(&empty[s], 0x3);
+                }
+                if (!ok) break;
+                umma_commit_pair(&tfull[acc], 0x3);
+                ++tcount;
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;
+        const int row_in_tile = (int)rank * kBM + q * 32 + lane;
+        const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
+        const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
+        uint32_t tcount = 0;
+        for (int t = cluster; t < total; t += nclusters) {
+            const int mt = t % p.m_tiles, rest = t / p.m_tiles;
+            const int nt = rest % p.n_tiles, h = rest / p.n_tiles;
+            const int m0 = mt * 2 * kBM, n0 = nt * BN;
+            const int row = m0 + row_in_tile;
+            T* yrow = static_cast<T*>(p.Y) + (int64_t)h * p.stride_y + (int64_t)row * p.ldy;
+            if (p.causal && n0 > m0 + 2 * kBM - 1) {
+                if (row < p.n) {
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = -__int_as_float(0x7f800000);
+                    for (int ch = 0; ch < BN / 32; ++ch) store_chunk<T>(yrow, n0 + ch * 32, p.m, v);
+                }
+                continue;
+            }
+            const uint32_t acc = tcount & 1u;
+            const uint32_t aph = (tcount >> 1) & 1u;
+            if (!mbar_wait(&tfull[acc], aph, abort_flag, p.err, kErrTimeoutEpilogue)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+#pragma unroll 1
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                uint32_t raw[32];
+                tmem_ld_32x32b_x32(taddr + ch * 32, raw);
+                tmem_ld_wait();
+                if (row < p.n) {
+                    const int col0 = n0 + ch * 32;
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float x = __uint_as_float(raw[i]) * p.alpha;
+                        v[i] = (p.causal && col0 + i > row) ? -__int_as_float(0x7f800000) : x;
+                    }
+                    store_chunk<T>(yrow, col0, p.m, v);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+            ++tcount;
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync_all();  // both CTAs done with each other's shared and tensor memory
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+}
+
+template <typename T, int BMODE, int BN>
+cudaError_t launch_pair(const GemmParams& p, int num_sms, cudaStream_t s) {
+    using C = PairCfg<T, BMODE, BN>;
+    auto kern = pair_gemm_kernel<T, BMODE, BN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+    if (e != cudaSuccess) return e;
+    const int total = p.heads * p.m_tiles * p.n_tiles;
+    const int clusters = total < num_sms / 2 ? total : num_sms / 2;
+    if (clusters <= 0) return cudaSuccess;
+    kern<<<2 * clusters, kThreads, C::SMEM, s>>>(p);
+    return cudaGetLastError();
+}
+
 template <typename T, int BMODE, int BN>
 cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t s) {
     using C = Cfg<T, BMODE, BN>;
@@ -303,12 +523,30 @@ cudaError_t launch_bn(const GemmParams& p, const GemmLaunch& l, cudaStream_t s) 
 
 }  // namespace
 
-size_t gemm_smem_bytes(int dtype, int bn) {
+size_t gemm_smem_bytes(int dtype, int bn, bool pair) {
+    if (pair) {
+        if (dtype == 1) return bn == 256 ? PairCfg<float, kBKMajor, 256>::SMEM : PairCfg<float, kBKMajor, 128>::SMEM;
+        return bn == 256 ? PairCfg<__nv_bfloat16, kBRows, 256>::SMEM : PairCfg<__nv_bfloat16, kBRows, 128>::SMEM;
+    }
     if (dtype == 1) return bn == 256 ? Cfg<float, kBKMajor, 256>::SMEM : Cfg<float, kBKMajor, 128>::SMEM;
     return bn == 256 ? Cfg<__nv_bfloat16, kBGather, 256>::SMEM : Cfg<__nv_bfloat16, kBGather, 128>::SMEM;
 }
 
 cudaError_t launch_gemm(const GemmParams& p, const GemmLaunch& l, cudaStream_t s) {
+    if (l.pair) {
+        if (l.dtype == 1) {
+            if (l.b_mode != kBKMajor) return cudaErrorInvalidValue;
+            return l.bn == 256 ? launch_pair<float, kBKMajor, 256>(p, l.num_sms, s)
+                               : launch_pair<float, kBKMajor, 128>(p, l.num_sms, s);
+        }
+        if (l.b_mode == kBRows)
+            return l.bn == 256 ? launch_pair<__nv_bfloat16, kBRows, 256>(p, l.num_sms, s)
+                               : launch_pair<__nv_bfloat16, kBRows, 128>(p, l.num_sms, s);
+        if (l.b_mode == kBKMajor)
+            return l.bn == 256 ? launch_pair<__nv_bfloat16, kBKMajor, 256>(p, l.num_sms, s)
+                               : launch_pair<__nv_bfloat16, kBKMajor, 128>(p, l.num_sms, s);
+        return cudaErrorInvalidValue;
+    }
     if (l.dtype == 1) {
         if (l.b_mode != kBKMajor) return cudaErrorInvalidValue;
         return launch_bn<float, kBKMajor>(p, l, s);

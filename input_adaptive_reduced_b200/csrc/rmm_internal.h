@@ -89,11 +89,13 @@ struct __align__(64) GemmParams {
 struct GemmLaunch {
     int dtype;
     int b_mode;       // kBKMajor / kBRows / kBGather
-    int bn;           // 128 or 256
+    int bn;           // 128 or 256 (the N of one tile)
+    bool pair;        // CTA pairs (cta_group::2): 256-row tiles, m_tiles counts 256-row tiles,
+                      // and a kBKMajor map_b box is bn/2 rows
     int num_sms;
 };
 cudaError_t launch_gemm(const GemmParams& p, const GemmLaunch& l, cudaStream_t s);
-size_t gemm_smem_bytes(int dtype, int bn);
+size_t gemm_smem_bytes(int dtype, int bn, bool pair);
 
 }  // namespace rmm
 

@@ -425,6 +425,103 @@ def run_rmm(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- sweep
+def run_sweep(args):
+    """Latency, useful TFLOP/s and roofline fraction at every point of the five
+    workloads (RMM at each rho, the same kernels at rho = 1, and the dense
+    torch/cuBLAS product), written as JSON lines to --sweep-out."""
+    import torch
+    import input_adaptive_reduced_b200 as rmm
+    import workloads as W
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peak_tf, _, peak_gbs, _ = load_peaks()
+    out = open(args.sweep_out, "w") if args.sweep_out else None
+
+    def lat(fn, iters=20):
+        for _ in range(3):
+            fn()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(iters):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / iters
+
+    def emit(rec):
+        line = json.dumps(rec)
+        print(line, flush=True)
+        if out:
+            out.write(line + "\n")
+            out.flush()
+
+    def linear_points(cfg, name, A, B, rhos):
+        n, d = A.shape
+        m = B.shape[1]
+        t_dense = lat(lambda: torch.matmul(A, B))
+        for rho in rhos:
+            k = retained(rho, d)
+            t = lat(lambda: rmm.matmul(A, B, rho=rho))
+            flops = 2.0 * n * k * m
+            hbm = 2.0 * (n * d + k * m + n * m)  # A once, retained B rows once, Y
+            bound = "tensor" if n >= 512 else "hbm"
+            frac = (flops / (t * 1e-3) / 1e12) / peak_tf if bound == "tensor" else (hbm / (t * 1e-3) / 1e9) / peak_gbs
+            emit({"config": cfg, "op": name, "n": n, "d": d, "m": m, "rho": rho, "k": k, "ms": t,
+                  "useful_tflops": flops / (t * 1e-3) / 1e12, "gbs": hbm / (t * 1e-3) / 1e9,
+                  "bound": bound, "frac": frac, "ms_dense_cublas": t_dense})
+
+    # 1: tiny fp32
+    A, B = W.linear_small(1, device=dev)
+    linear_points(1, "fp32 64x256x256", A, B, [0.25, 0.5, 1.0])
+    # 2: Llama-3.1-8B MLP
+    for n in (1024, 2048, 4096):
+        for name, gen in (("up", W.mlp_up), ("down", W.mlp_down)):
+            A, B = gen(1, n=n, device=dev)
+            linear_points(2, name, A, B, [0.5, 0.7, 0.8, 1.0])
+            del A, B
+    # 3: QK^T, 32 heads / 8 KV heads, d_h = 128, causal
+    for n in (1024, 2048, 4096):
+        Q, K = W.attn_qk(1, n=n, device=dev)
+        Kt = K.repeat_interleave(4, dim=0).transpose(1, 2)
+        t_dense = lat(lambda: torch.matmul(Q, Kt))
+        for rho in (0.5, 0.8, 1.0):
+            k = retained(rho, 128)
+            t = lat(lambda: rmm.qk(Q, K, rho=rho, causal=True))
+            flops = 2.0 * n * k * n * 32
+            hbm = 32 * (2.0 * n * 128 + 2 * 2.0 * n * k + 2.0 * n * n) + 8 * 2.0 * n * 128
+            emit({"config": 3, "op": "qk", "n": n, "rho": rho, "k": k, "ms": t,
+                  "useful_tflops": flops / (t * 1e-3) / 1e12, "gbs": hbm / (t * 1e-3) / 1e9,
+                  "bound": "hbm", "frac": hbm / (t * 1e-3) / 1e9 / peak_gbs, "ms_dense_torch": t_dense})
+        del Q, K, Kt
+    # 4: PV, token selection
+    for n in (2048, 4096):
+        P, V = W.attn_pv(1, n=n, device=dev)
+        Vr = V.repeat_interleave(4, dim=0)
+        t_dense = lat(lambda: torch.matmul(P, Vr))
+        for rho in (0.5, 0.8, 1.0):
+            k = retained(rho, n)
+            t = lat(lambda: rmm.pv(P, V, rho=rho))
+            flops = 2.0 * n * k * 128 * 32
+            hbm = 32 * (2.0 * n * n + 2.0 * k * 128 + 2.0 * n * 128)  # P once, V rows, O
+            emit({"config": 4, "op": "pv", "n": n, "rho": rho, "k": k, "ms": t,
+                  "useful_tflops": flops / (t * 1e-3) / 1e12, "gbs": hbm / (t * 1e-3) / 1e9,
+                  "bound": "hbm", "frac": hbm / (t * 1e-3) / 1e9 / peak_gbs, "ms_dense_torch": t_dense})
+        del P, V, Vr
+    # 5: Llama-3-70B linear
+    for shape in ("up", "down", "qkv"):
+        for n in (1, 16, 512, 2048, 4096):
+            A, B = W.linear_70b(1, n=n, shape=shape, device=dev)
+            linear_points(5, shape, A, B, [0.5, 0.6, 0.7, 0.8, 1.0])
+            del A, B
+    if out:
+        out.close()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -436,7 +533,11 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="time every point of the five workloads")
+    ap.add_argument("--sweep-out", default=None)
     args = ap.parse_args(argv)
+    if args.sweep:
+        return run_sweep(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_rmm(args)

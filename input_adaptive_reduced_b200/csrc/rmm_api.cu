@@ -26,7 +26,7 @@
 namespace {
 
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
-constexpr size_t kFusedSelectBytes = size_t(1) << 20;  // per head
+constexpr size_t kFusedSelectBytes = size_t(128) << 10;  // per head: one CTA reads it all
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -59,7 +59,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // 3-D K-major map {K extent, rows, heads} with a {box_k, box_rows, 1} box,
 // 128-byte swizzle and zero fill outside the extents.
 bool encode_kmajor_map(CUtensorMap* map, int es, const void* base, int64_t kext, int64_t rows,
-                       int64_t heads, int64_t ld, int64_t stride_h, uint32_t box_k, uint32_t box_rows) {
+                       int64_t heads, int64_t ld, int64_t stride_h, uint32_t box_k, uint32_t box_rows,
+                       CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     const uint64_t row_bytes = static_cast<uint64_t>(ld) * es;
@@ -73,8 +74,7 @@ bool encode_kmajor_map(CUtensorMap* map, int es, const void* base, int64_t kext,
     cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r = enc(map, es == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                           swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -201,6 +201,54 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         }
     }
     if (p.n == 0 || p.m == 0) return RMM_OK;
+
+    if (plan->skinny) {
+        rmm::SkinnyParams sp;
+        std::memset(&sp, 0, sizeof(sp));
+        const uint32_t box_np = static_cast<uint32_t>(plan->sk_np);
+        if (!identity) {
+            rmm::PackArgs pa{};
+            pa.src = A;
+            pa.dtype = p.dtype;
+            pa.rows = p.n;
+            pa.d = p.d;
+            pa.ld_src = p.lda;
+            pa.stride_src = p.stride_a;
+            pa.group = 1;
+            pa.I = I;
+            pa.I_stride = k;
+            pa.k = k;
+            pa.dst = ws_at<void>(ws, plan->off_apack);
+            pa.ld_dst = plan->ldp;
+            pa.stride_dst = p.n * plan->ldp;
+            pa.heads = 1;
+            if (rmm::launch_pack(pa, stream) != cudaSuccess) return RMM_ERR_CUDA;
+            if (!encode_kmajor_map(&sp.map_a, 2, pa.dst, k, p.n, 1, plan->ldp, p.n * plan->ldp, 64, box_np))
+                return RMM_ERR_CUDA;
+        } else if (!encode_kmajor_map(&sp.map_a, 2, A, p.d, p.n, 1, p.lda, p.n * p.lda, 64, box_np)) {
+            return RMM_ERR_CUDA;
+        }
+        sp.B = B;
+        sp.ldb = p.ldb;
+        sp.I = identity ? nullptr : I;
+        sp.Y = Y;
+        sp.ldy = p.ldy;
+        sp.partials = ws_at<float>(ws, plan->off_bpack);
+        sp.alpha = p.alpha;
+        sp.n = static_cast<int32_t>(p.n);
+        sp.m = static_cast<int32_t>(p.m);
+        sp.k = static_cast<int32_t>(k);
+        sp.d = static_cast<int32_t>(p.d);
+        sp.np = plan->sk_np;
+        sp.m_tiles = static_cast<int32_t>((p.m + 127) / 128);
+        sp.splits = plan->sk_splits;
+        sp.err = ws_at<int>(ws, plan->off_err);
+        const bool traced = plan->product_start && plan->product_stop;
+        if (traced && cudaEventRecord(plan->product_start, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        if (rmm::launch_skinny(sp, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        if (traced && cudaEventRecord(plan->product_stop, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        return RMM_OK;
+    }
 
     // ---- stage the gathered A columns (and K columns in QK mode)
     rmm::GemmParams gp;
@@ -345,6 +393,10 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
     }
     gl.pair = pair_ok && gl.b_mode != rmm::kBGather;
     gp.m_tiles = static_cast<int32_t>(gl.pair ? (p.n + 255) / 256 : (p.n + 127) / 128);
+    // the pair kernel stores 32 x 32 output boxes by TMA (64- or 128-byte rows)
+    if (gl.pair && !encode_kmajor_map(&gp.map_y, es, Y, p.m, p.n, p.heads, p.ldy, p.stride_y, 32, 32,
+                                      es == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
+        return RMM_ERR_CUDA;
     const bool traced = plan->product_start && plan->product_stop;
     if (traced && cudaEventRecord(plan->product_start, stream) != cudaSuccess) return RMM_ERR_CUDA;
     if (rmm::launch_gemm(gp, gl, stream) != cudaSuccess) return RMM_ERR_CUDA;
@@ -359,6 +411,7 @@ int32_t launches_per_call(const rmm_plan* plan) {
     int32_t n = 0;
     if (!given && !identity) n += plan->fused_select ? 1 : 2;
     if (p.n == 0 || p.m == 0) return n;
+    if (plan->skinny) return n + (identity ? 0 : 1) + 1 + (plan->sk_splits > 1 ? 1 : 0);
     if (!identity) n += 1;                                   // pack A[:, I]
     if (p.mode == RMM_QK && !identity) n += 1;               // pack K[:, I]
     if (p.mode != RMM_QK && p.dtype == RMM_F32) n += 1;      // B[I, :] transposed for tf32
@@ -404,6 +457,15 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     plan->need_select = !given && plan->k < p->d;
     plan->bn = p->m <= 128 ? 128 : 256;
     plan->pack_b = p->mode != RMM_QK && p->dtype == RMM_BF16 && (plan->k < p->d || given);
+    // Few rows: the op is a stream of B[I, :]; gather it inside a split-K
+    // product with swapped operands instead of staging it.
+    plan->skinny = p->mode == RMM_LINEAR && p->dtype == RMM_BF16 && p->heads == 1 && p->n >= 1 && p->n <= 64 &&
+                   p->m >= 1;
+    if (plan->skinny) {
+        plan->pack_b = false;
+        plan->sk_np = rmm::skinny_pad(p->n);
+        plan->sk_splits = rmm::skinny_splits(p->m, plan->k, 0);  // fixed below once the SM count is known
+    }
 
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -413,6 +475,7 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
         return RMM_ERR_CUDA;
     }
     plan->num_sms = sms;
+    if (plan->skinny) plan->sk_splits = rmm::skinny_splits(p->m, plan->k, sms);
 
     // Selection kernels need every score of a head in shared memory.
     const bool select_possible = p->d <= rmm::kMaxSelectD;
@@ -457,7 +520,9 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     plan->off_apack = off;
     off += align256(static_cast<size_t>(p->heads) * p->n * plan->ldp * plan->es);
     plan->off_bpack = off;
-    if (p->mode == RMM_QK || p->dtype == RMM_F32)
+    if (plan->skinny)
+        off += align256(static_cast<size_t>(plan->sk_splits) * p->m * plan->sk_np * sizeof(float));
+    else if (p->mode == RMM_QK || p->dtype == RMM_F32)
         off += align256(static_cast<size_t>(p->heads) * p->m * plan->ldp * plan->es);
     else if (plan->pack_b || given)
         off += align256(static_cast<size_t>(p->heads) * plan->k * p->m * plan->es);

@@ -308,10 +308,39 @@ struct PairCfg {
     static constexpr int STAGES = 6;
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr int GROUP_BYTES = BK * 128;
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+    // epilogue staging: per epilogue warp two buffers of 32 rows x 32 columns
+    static constexpr int ROW_BYTES = 32 * ES;                 // 64 (bf16) or 128 (fp32)
+    static constexpr int OUT_BUF = 32 * ROW_BYTES;
+    static constexpr int OUT_BYTES = 4 * 2 * OUT_BUF;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + OUT_BYTES + 256;
     static_assert(!(TF32 && B_MN), "fp32 operands are staged K-major");
     static_assert(BMODE != kBGather, "indexed gathers use the single-CTA kernel");
 };
+
+// Write one thread's 32 output values (its row of a 32 x 32 chunk) into the
+// staging buffer in the layout of a 64-byte (bf16) or 128-byte (fp32)
+// swizzled TMA box: 16-byte granule g of row r sits at g ^ f(r).
+template <typename T>
+__device__ __forceinline__ void stage_row(uint8_t* buf, int r, const float (&v)[32]) {
+    uint8_t* row = buf + r * (32 * (int)sizeof(T));
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * g + 2 * i], v[8 * g + 2 * i + 1]);
+                w[i] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            *reinterpret_cast<uint4*>(row + ((g ^ ((r >> 1) & 3)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    } else {
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+            *reinterpret_cast<float4*>(row + ((g ^ (r & 7)) << 4)) =
+                make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+    }
+}
 
 template <typename T, int BMODE, int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -319,7 +348,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     using C = PairCfg<T, BMODE, BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::OUT_BYTES);
     uint64_t* empty = full + C::STAGES;
     uint64_t* tfull = empty + C::STAGES;
     uint64_t* tempty = tfull + 2;
@@ -433,52 +462,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
+        // Each warp owns 32 rows; per 32-column chunk it stages its rows in a
+        // swizzled shared buffer and one lane stores the 32 x 32 box by TMA
+        // (rows past n and columns past m are clipped by the store itself).
         const int q = warp & 3;
-        const int row_in_tile = (int)rank * kBM + q * 32 + lane;
+        const int row_base = (int)rank * kBM + q * 32;
         const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
         const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
-        uint32_t tcount = 0;
+        uint8_t* out = smem + C::STAGES * C::STAGE_BYTES + (q * 2) * C::OUT_BUF;
+        uint32_t tcount = 0, slot = 0;
         for (int t = cluster; t < total; t += nclusters) {
             const int mt = t % p.m_tiles, rest = t / p.m_tiles;
             const int nt = rest % p.n_tiles, h = rest / p.n_tiles;
             const int m0 = mt * 2 * kBM, n0 = nt * BN;
-            const int row = m0 + row_in_tile;
-            T* yrow = static_cast<T*>(p.Y) + (int64_t)h * p.stride_y + (int64_t)row * p.ldy;
-            if (p.causal && n0 > m0 + 2 * kBM - 1) {
-                if (row < p.n) {
-                    float v[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = -__int_as_float(0x7f800000);
-                    for (int ch = 0; ch < BN / 32; ++ch) store_chunk<T>(yrow, n0 + ch * 32, p.m, v);
-                }
-                continue;
+            const int row0 = m0 + row_base;
+            const int row = row0 + lane;
+            const bool skip = p.causal && n0 > m0 + 2 * kBM - 1;
+            uint32_t acc = 0, taddr = 0;
+            if (!skip) {
+                acc = tcount & 1u;
+                const uint32_t aph = (tcount >> 1) & 1u;
+                if (!mbar_wait(&tfull[acc], aph, abort_flag, p.err, kErrTimeoutEpilogue)) break;
+                tc_fence_after();
+                taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
             }
-            const uint32_t acc = tcount & 1u;
-            const uint32_t aph = (tcount >> 1) & 1u;
-            if (!mbar_wait(&tfull[acc], aph, abort_flag, p.err, kErrTimeoutEpilogue)) break;
-            tc_fence_after();
-            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+            if (row0 < p.n) {
 #pragma unroll 1
-            for (int ch = 0; ch < BN / 32; ++ch) {
-                uint32_t raw[32];
-                tmem_ld_32x32b_x32(taddr + ch * 32, raw);
-                tmem_ld_wait();
-                if (row < p.n) {
+                for (int ch = 0; ch < BN / 32; ++ch) {
                     const int col0 = n0 + ch * 32;
                     float v[32];
+                    if (skip) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float x = __uint_as_float(raw[i]) * p.alpha;
-                        v[i] = (p.causal && col0 + i > row) ? -__int_as_float(0x7f800000) : x;
+                        for (int i = 0; i < 32; ++i) v[i] = -__int_as_float(0x7f800000);
+                    } else {
+                        uint32_t raw[32];
+                        tmem_ld_32x32b_x32(taddr + ch * 32, raw);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float x = __uint_as_float(raw[i]) * p.alpha;
+                            v[i] = (p.causal && col0 + i > row) ? -__int_as_float(0x7f800000) : x;
+                        }
                     }
-                    store_chunk<T>(yrow, col0, p.m, v);
+                    if (col0 < p.m) {
+                        uint8_t* buf = out + slot * C::OUT_BUF;
+                        if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
+                        __syncwarp();
+                        stage_row<T>(buf, lane, v);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_3d(&p.map_y, buf, col0, row0, h);
+                            bulk_commit_group();
+                        }
+                        slot ^= 1u;
+                    }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
-            ++tcount;
+            if (!skip) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+                ++tcount;
+            }
         }
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
     }
 
     __syncwarp();

@@ -71,6 +71,7 @@ constexpr int kBGather = 2;  // tile::gather4 of indexed rows of a d x m matrix 
 struct __align__(64) GemmParams {
     CUtensorMap map_a;
     CUtensorMap map_b;          // kBKMajor: 3-D {K, m, heads}; kBRows/kBGather: 2-D {m, rows}
+    CUtensorMap map_y;          // CTA-pair kernel: 3-D {m, n, heads} store map, box {32, 32, 1}
     const int32_t* I;           // kBGather: [heads][I_stride] row indices
     int64_t I_stride;
     void* Y;
@@ -97,6 +98,25 @@ struct GemmLaunch {
 cudaError_t launch_gemm(const GemmParams& p, const GemmLaunch& l, cudaStream_t s);
 size_t gemm_smem_bytes(int dtype, int bn, bool pair);
 
+// ---------------------------------------------------------------- few rows
+// Product for n <= 64 with swapped operands (rmm_skinny.cu).
+struct __align__(64) SkinnyParams {
+    CUtensorMap map_a;      // A[:, I] (packed, or A itself when every index is kept):
+                            // 3-D {K extent, n, 1}, box {64, np, 1}
+    const void* B;          // row-major d x m bf16
+    int64_t ldb;
+    const int32_t* I;       // [k] retained rows of B, nullptr = every row in order
+    void* Y;                // n x m bf16
+    int64_t ldy;
+    float* partials;        // [splits][m][np] fp32 when splits > 1
+    float alpha;
+    int32_t n, m, k, d, np, m_tiles, splits;
+    int* err;
+};
+int skinny_pad(int64_t n);
+int skinny_splits(int64_t m, int64_t k, int num_sms);
+cudaError_t launch_skinny(const SkinnyParams& p, cudaStream_t s);
+
 }  // namespace rmm
 
 // The plan behind the opaque rmm_plan handle of include/rmm.h.
@@ -117,4 +137,6 @@ struct rmm_plan {
     size_t off_err, off_counters, off_partials, off_scores, off_I, off_apack, off_bpack, ws_bytes;
     size_t header_bytes;  // zeroed by rmm_workspace_init: error word + colnorm counters
     cudaEvent_t product_start, product_stop;  // tracing hook, may be null
+    bool skinny;        // n <= 64 bf16 LINEAR: swapped-operand split-K product
+    int sk_np, sk_splits;
 };

@@ -143,6 +143,48 @@ __global__ void __launch_bounds__(256) pack_rows_kernel(
     }
 }
 
+// Narrow variant (packed width <= kNarrowMax, e.g. attention heads with
+// d_h = 128): the CTA caches the head's indices in shared memory once and its
+// threads walk (row, 8-column chunk) pairs, so every thread has work.
+constexpr int kNarrowMax = 1024;
+constexpr int kNarrowRows = 64;
+
+template <typename T>
+__global__ void __launch_bounds__(256) pack_narrow_kernel(
+    const T* __restrict__ src, int64_t rows, int64_t d, int64_t ld_src, int64_t stride_src, int group,
+    const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
+    int64_t stride_dst) {
+    __shared__ int32_t sidx[kNarrowMax];
+    const int h = blockIdx.y;
+    const int cpr = (int)(ld_dst / 8);
+    for (int t = threadIdx.x; t < (int)ld_dst; t += 256) {
+        int32_t j = t < k ? __ldg(I + (int64_t)h * I_stride + t) : -1;
+        sidx[t] = j < 0 ? -1 : (j >= d ? (int32_t)(d - 1) : j);
+    }
+    __syncthreads();
+    const int64_t r0 = (int64_t)blockIdx.x * kNarrowRows;
+    const int nr = (int)min((int64_t)kNarrowRows, rows - r0);
+    const T* sh = src + (int64_t)(h / group) * stride_src;
+    T* dh = dst + (int64_t)h * stride_dst;
+    for (int e = threadIdx.x; e < nr * cpr; e += 256) {
+        const int r = e / cpr, c = e - r * cpr;
+        const T* srow = sh + (r0 + r) * ld_src;
+        __align__(16) T vals[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            const int32_t j = sidx[8 * c + v];
+            vals[v] = j >= 0 ? srow[j] : T(0.f);
+        }
+        T* o = dh + (r0 + r) * ld_dst + 8 * c;
+        if constexpr (sizeof(T) == 2) {
+            *reinterpret_cast<uint4*>(o) = *reinterpret_cast<const uint4*>(vals);
+        } else {
+            reinterpret_cast<uint4*>(o)[0] = reinterpret_cast<const uint4*>(vals)[0];
+            reinterpret_cast<uint4*>(o)[1] = reinterpret_cast<const uint4*>(vals)[1];
+        }
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_pack_rows(const PackArgs& a, int num_sms, cudaStream_t s) {
@@ -176,6 +218,19 @@ cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t s) {
+    if (a.ld_dst <= kNarrowMax) {
+        dim3 g((unsigned)((a.rows + kNarrowRows - 1) / kNarrowRows), (unsigned)a.heads);
+        if (g.x == 0) return cudaSuccess;
+        if (a.dtype == 1)
+            pack_narrow_kernel<float><<<g, 256, 0, s>>>((const float*)a.src, a.rows, a.d, a.ld_src, a.stride_src,
+                                                        a.group, a.I, a.I_stride, a.k, (float*)a.dst, a.ld_dst,
+                                                        a.stride_dst);
+        else
+            pack_narrow_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(
+                (const __nv_bfloat16*)a.src, a.rows, a.d, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k,
+                (__nv_bfloat16*)a.dst, a.ld_dst, a.stride_dst);
+        return cudaGetLastError();
+    }
     dim3 grid((unsigned)((a.ld_dst + 8 * kPackThreads - 1) / (8 * kPackThreads)),
               (unsigned)((a.rows + kPackRows - 1) / kPackRows), (unsigned)a.heads);
     if (grid.y == 0) return cudaSuccess;

@@ -484,16 +484,16 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
         return RMM_ERR_UNSUPPORTED;
     }
     const size_t head_bytes = static_cast<size_t>(p->n) * p->d * plan->es;
-    plan->fused_select = head_bytes <= kFusedSelectBytes && rmm::normselect_smem_bytes(p->d, p->dtype) <= 190 * 1024;
+    plan->fused_select = head_bytes <= kFusedSelectBytes && rmm::normselect_smem_bytes(p->d, p->dtype) <= 180 * 1024;
     // Row splits for the score pass: enough CTAs to keep HBM busy (about two
-    // per SM), at most kMaxSplitRows partials per column, at least 64 rows each.
+    // per SM), at most 16 partials per column, at least 64 rows each.
     const int vec = 16 / plan->es;
     const int64_t colblocks = (p->d + 32 * vec - 1) / (32 * vec);
     const int64_t target = 2LL * sms;
     int64_t nsplit = (target + colblocks * p->heads - 1) / (colblocks * p->heads);
     const int64_t max_split = (p->n + 63) / 64;
     if (nsplit > max_split) nsplit = max_split;
-    if (nsplit > rmm::kMaxSplitRows) nsplit = rmm::kMaxSplitRows;
+    if (nsplit > 16) nsplit = 16;
     if (nsplit < 1) nsplit = 1;
     int64_t rps = (p->n + nsplit - 1) / nsplit;
     rps = (rps + 7) / 8 * 8;

@@ -342,6 +342,23 @@ __device__ __forceinline__ void stage_row(uint8_t* buf, int r, const float (&v)[
     }
 }
 
+// Tile order of the CTA-pair kernel: within a head, groups of kGroupM
+// consecutive 256-row tiles sweep every column tile before the next group, so
+// that the A rows and B columns of one wave of tiles stay resident in L2.
+constexpr int kGroupM = 8;
+
+__device__ __forceinline__ void pair_tile(int t, const GemmParams& p, int& h, int& mt, int& nt) {
+    const int per_head = p.m_tiles * p.n_tiles;
+    h = t / per_head;
+    const int r = t - h * per_head;
+    const int group = r / (kGroupM * p.n_tiles);
+    const int within = r - group * (kGroupM * p.n_tiles);
+    const int left = p.m_tiles - group * kGroupM;
+    const int gm = left < kGroupM ? left : kGroupM;
+    mt = group * kGroupM + within % gm;
+    nt = within / gm;
+}
+
 template <typename T, int BMODE, int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     pair_gemm_kernel(const __grid_constant__ GemmParams p) {
@@ -391,8 +408,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int t = cluster; t < total && ok; t += nclusters) {
-                const int mt = t % p.m_tiles, rest = t / p.m_tiles;
-                const int nt = rest % p.n_tiles, h = rest / p.n_tiles;
+                int h, mt, nt;
+                pair_tile(t, p, h, mt, nt);
                 const int m0 = mt * 2 * kBM, n0 = nt * BN;
                 if (p.causal && n0 > m0 + 2 * kBM - 1) continue;
                 const int row_base = (h / p.group) * p.b_head_rows;
@@ -427,8 +444,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t it = 0, tcount = 0;
             bool ok = true;
             for (int t = cluster; t < total && ok; t += nclusters) {
-                const int mt = t % p.m_tiles, rest = t / p.m_tiles;
-                const int nt = rest % p.n_tiles;
+                int h, mt, nt;
+                pair_tile(t, p, h, mt, nt);
                 const int m0 = mt * 2 * kBM, n0 = nt * BN;
                 if (p.causal && n0 > m0 + 2 * kBM - 1) continue;
                 const uint32_t acc = tcount & 1u;
@@ -472,8 +489,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint8_t* out = smem + C::STAGES * C::STAGE_BYTES + (q * 2) * C::OUT_BUF;
         uint32_t tcount = 0, slot = 0;
         for (int t = cluster; t < total; t += nclusters) {
-            const int mt = t % p.m_tiles, rest = t / p.m_tiles;
-            const int nt = rest % p.n_tiles, h = rest / p.n_tiles;
+            int h, mt, nt;
+            pair_tile(t, p, h, mt, nt);
             const int m0 = mt * 2 * kBM, n0 = nt * BN;
             const int row0 = m0 + row_base;
             const int row = row0 + lane;

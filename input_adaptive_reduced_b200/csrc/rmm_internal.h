@@ -24,7 +24,7 @@ struct SelectArgs {
     int nsplit;          // 1 .. kMaxSplitRows
     int64_t rows_per_split;
 };
-constexpr int kMaxSplitRows = 16;
+constexpr int kMaxSplitRows = 64;
 
 // Column sums of squares in fp32: one partial per row split, then the last
 // CTA of each column block adds the partials in split order into `scores`.

@@ -55,7 +55,7 @@ struct Vec16<float> {
 // its columns in split order and writes the final fp32 scores, then resets
 // the counter for the next call.  The order of every sum is fixed and the
 // same for every column.
-constexpr int kMaxSplit = 16;
+constexpr int kMaxSplit = 64;
 
 template <typename T>
 __global__ void __launch_bounds__(256) colnorm_kernel(const T* __restrict__ A, int64_t n, int64_t d,
@@ -121,13 +121,15 @@ __global__ void __launch_bounds__(256) colnorm_kernel(const T* __restrict__ A, i
         const int64_t gcol = (int64_t)blockIdx.x * COLS + c;
         if (gcol >= d) continue;
         const float* pc = partials + (int64_t)h * nsplit * d + gcol;
-        float v[kMaxSplit];
+        float sum = 0.f;
+        for (int b = 0; b < nsplit; b += 16) {  // 16 independent loads in flight, added in split order
+            float v[16];
 #pragma unroll
-        for (int sp = 0; sp < kMaxSplit; ++sp) v[sp] = sp < nsplit ? __ldcg(pc + (int64_t)sp * d) : 0.f;
-        float sum = v[0];
+            for (int u = 0; u < 16; ++u) v[u] = b + u < nsplit ? __ldcg(pc + (int64_t)(b + u) * d) : 0.f;
 #pragma unroll
-        for (int sp = 1; sp < kMaxSplit; ++sp)
-            if (sp < nsplit) sum += v[sp];
+            for (int u = 0; u < 16; ++u)
+                if (b + u < nsplit) sum = (b + u == 0) ? v[u] : sum + v[u];
+        }
         s2[(int64_t)h * d + gcol] = sum;
     }
 }
@@ -137,8 +139,10 @@ __global__ void __launch_bounds__(256) colnorm_kernel(const T* __restrict__ A, i
 // 1024-thread block.  Three radix passes over bits [31:21], [20:10] and [9:0]
 // find the exact k-th largest key T and how many keys equal to T are kept;
 // then the indices are emitted in ascending order.
+constexpr int kSubHist = 4;  // warps w, w+4, ... share a histogram copy: 4x less atomic contention
+
 struct TopkShared {
-    uint32_t hist[2048];
+    uint32_t hist[kSubHist][2048];
     uint32_t warp_tot[32];
     uint32_t prefix;
     uint32_t remaining;
@@ -158,17 +162,22 @@ __device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k
     for (int pass = 0; pass < 3; ++pass) {
         const int shift = shifts[pass];
         const int nb = 1 << widths[pass];
-        for (int b = tid; b < nb; b += 1024) sh.hist[b] = 0;
+        for (int b = tid; b < kSubHist * 2048; b += 1024) (&sh.hist[0][0])[b] = 0;
         __syncthreads();
+        uint32_t* myhist = sh.hist[warp & (kSubHist - 1)];
         for (int64_t j = tid; j < d; j += 1024) {
             const uint32_t key = keys[j];
-            if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & (uint32_t)(nb - 1)], 1u);
+            if ((key & mask) == prefix) atomicAdd(&myhist[(key >> shift) & (uint32_t)(nb - 1)], 1u);
         }
         __syncthreads();
         // thread t owns bins nb-1-2t and nb-2-2t: a block scan in descending bin order
         const int b_hi = nb - 1 - 2 * tid, b_lo = b_hi - 1;
-        const uint32_t c0 = b_hi >= 0 ? sh.hist[b_hi] : 0u;
-        const uint32_t c1 = b_lo >= 0 ? sh.hist[b_lo] : 0u;
+        uint32_t c0 = 0, c1 = 0;
+#pragma unroll
+        for (int c = 0; c < kSubHist; ++c) {
+            if (b_hi >= 0) c0 += sh.hist[c][b_hi];
+            if (b_lo >= 0) c1 += sh.hist[c][b_lo];
+        }
         const uint32_t tot = c0 + c1;
         uint32_t incl = tot;
 #pragma unroll
@@ -268,7 +277,15 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
     __shared__ TopkShared sh;
     const int h = blockIdx.x;
     const float* p = scores + (int64_t)h * d;
-    for (int64_t j = threadIdx.x; j < d; j += 1024) keys[j] = __float_as_uint(p[j]);
+    // eight independent loads in flight per thread (the scores come from L2)
+    for (int64_t j0 = threadIdx.x; j0 < d; j0 += 8 * 1024) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = j0 + u * 1024 < d ? __ldcg(p + j0 + u * 1024) : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (j0 + u * 1024 < d) keys[j0 + u * 1024] = __float_as_uint(v[u]);
+    }
     __syncthreads();
     radix_select_and_emit(keys, d, k, I + (int64_t)h * k, sh);
 }

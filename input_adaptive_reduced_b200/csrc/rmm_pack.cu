@@ -15,13 +15,6 @@
 namespace rmm {
 namespace {
 
-__device__ __forceinline__ void cp_async_16_global(void* smem_dst, const void* gsrc) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                     static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
-                 "l"(gsrc)
-                 : "memory");
-}
-
 constexpr int kPackThreads = 256;
 constexpr int kPackRows = 16;  // rows per CTA; the 8 indices of a thread are reused across them
 
@@ -49,20 +42,19 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(
     T* dh = dst + (int64_t)h * stride_dst;
     const int64_t r_beg = (int64_t)blockIdx.y * kPackRows;
     const int64_t r_end = min(rows, r_beg + kPackRows);
-    // two rows per round: sixteen independent element loads in flight per thread
-    for (int64_t r = r_beg; r < r_end; r += 2) {
-        const bool two = r + 1 < r_end;
-        const T* s0 = sh + r * ld_src;
-        const T* s1 = sh + (two ? r + 1 : r) * ld_src;
-        __align__(16) T vals[2][8];
+    // four rows per round: thirty-two independent element loads in flight per thread
+    for (int64_t r = r_beg; r < r_end; r += 4) {
+        const int nq = (int)(r_end - r < 4 ? r_end - r : 4);
+        __align__(16) T vals[4][8];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-            vals[0][v] = live[v] ? s0[idx[v]] : T(0.f);
-            vals[1][v] = live[v] ? s1[idx[v]] : T(0.f);
+        for (int q = 0; q < 4; ++q) {
+            const T* sq = sh + (r + (q < nq ? q : 0)) * ld_src;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) vals[q][v] = live[v] ? sq[idx[v]] : T(0.f);
         }
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            if (q == 1 && !two) break;
+        for (int q = 0; q < 4; ++q) {
+            if (q >= nq) break;
             T* o = dh + (r + q) * ld_dst + t0;
             if constexpr (sizeof(T) == 2) {
                 *reinterpret_cast<uint4*>(o) = *reinterpret_cast<const uint4*>(vals[q]);
@@ -192,78 +184,7 @@ __global__ void __launch_bounds__(256) pack_narrow_kernel(
     }
 }
 
-// Wide variant for d < 65536: each CTA keeps the head's indices in shared
-// memory (16-bit) and streams whole source rows into shared memory with
-// 16-byte cp.async copies, double-buffered (the next row loads while this one
-// is gathered); the packed row is then built from shared memory and written
-// with 16-byte stores.  Reads of A are fully coalesced and many are in flight.
-constexpr int kStreamThreads = 256;
-
-template <typename T>
-__global__ void __launch_bounds__(kStreamThreads) pack_rowstream_kernel(
-    const T* __restrict__ src, int64_t rows, int64_t d, int64_t ld_src, int64_t stride_src, int group,
-    const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
-    int64_t stride_dst) {
-    constexpr int V = 16 / sizeof(T);
-    extern __shared__ __align__(16) uint8_t sm[];
-    uint16_t* sidx = reinterpret_cast<uint16_t*>(sm);
-    const int64_t idx_bytes = (ld_dst * 2 + 15) / 16 * 16;
-    const int64_t row_elems = (d + V - 1) / V * V;
-    T* rowbuf[2] = {reinterpret_cast<T*>(sm + idx_bytes), reinterpret_cast<T*>(sm + idx_bytes) + row_elems};
-    const int h = blockIdx.y;
-    for (int64_t t = threadIdx.x; t < ld_dst; t += kStreamThreads) {
-        int64_t j = t < k ? (int64_t)__ldg(I + (int64_t)h * I_stride + t) : -1;
-        sidx[t] = j < 0 ? (uint16_t)0xFFFFu : (uint16_t)(j >= d ? d - 1 : j);
-    }
-    const T* sh = src + (int64_t)(h / group) * stride_src;
-    T* dh = dst + (int64_t)h * stride_dst;
-    const int nvec = (int)(d / V);
-    auto issue_row = [&](int64_t r, T* buf) {
-        const T* srow = sh + r * ld_src;
-        for (int v = threadIdx.x; v < nvec; v += kStreamThreads)
-            cp_async_16_global(buf + (int64_t)v * V, srow + (int64_t)v * V);
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-    int64_t r = blockIdx.x;
-    int b = 0;
-    if (r < rows) issue_row(r, rowbuf[0]);
-    for (; r < rows; r += gridDim.x, b ^= 1) {
-        const int64_t rn = r + gridDim.x;
-        if (rn < rows) issue_row(rn, rowbuf[b ^ 1]);
-        if (rn < rows)
-            asm volatile("cp.async.wait_group 1;" ::: "memory");
-        else
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
-        __syncthreads();  // row r (and, the first time, the indices) visible to all threads
-        const T* buf = rowbuf[b];
-        T* o = dh + r * ld_dst;
-        for (int64_t c = threadIdx.x; c < ld_dst / 8; c += kStreamThreads) {
-            __align__(16) T vals[8];
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-                const uint16_t j = sidx[8 * c + v];
-                vals[v] = j == 0xFFFFu ? T(0.f) : buf[j];
-            }
-            if constexpr (sizeof(T) == 2) {
-                reinterpret_cast<uint4*>(o)[c] = *reinterpret_cast<const uint4*>(vals);
-            } else {
-                reinterpret_cast<uint4*>(o)[2 * c] = reinterpret_cast<const uint4*>(vals)[0];
-                reinterpret_cast<uint4*>(o)[2 * c + 1] = reinterpret_cast<const uint4*>(vals)[1];
-            }
-        }
-        __syncthreads();  // buffer b free for the row after next
-    }
-}
-
 }  // namespace
-
-size_t pack_rowstream_smem(int64_t d, int64_t ld_dst, int dtype) {
-    const int es = dtype == 1 ? 4 : 2;
-    const int V = 16 / es;
-    const int64_t idx_bytes = (ld_dst * 2 + 15) / 16 * 16;
-    const int64_t row_elems = (d + V - 1) / V * V;
-    return (size_t)(idx_bytes + 2 * row_elems * es);
-}
 
 cudaError_t launch_pack_rows(const PackArgs& a, int num_sms, cudaStream_t s) {
     (void)num_sms;
@@ -296,33 +217,6 @@ cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t s) {
-    const size_t stream_smem = pack_rowstream_smem(a.d, a.ld_dst, a.dtype);
-    if (a.ld_dst > kNarrowMax && a.d < 65535 && stream_smem <= 200 * 1024 && a.rows > 0) {
-        // as many CTAs as fit per SM (each keeps two rows in flight), at most 8
-        int per_sm = (int)((220 * 1024) / (stream_smem + 1024));
-        if (per_sm > 8) per_sm = 8;
-        if (per_sm < 1) per_sm = 1;
-        int64_t ctas = (int64_t)per_sm * 148;
-        if (ctas > a.rows) ctas = a.rows;
-        dim3 g((unsigned)ctas, (unsigned)a.heads);
-        cudaError_t e;
-        if (a.dtype == 1) {
-            e = cudaFuncSetAttribute(pack_rowstream_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)stream_smem);
-            if (e != cudaSuccess) return e;
-            pack_rowstream_kernel<float><<<g, kStreamThreads, stream_smem, s>>>(
-                (const float*)a.src, a.rows, a.d, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k,
-                (float*)a.dst, a.ld_dst, a.stride_dst);
-        } else {
-            e = cudaFuncSetAttribute(pack_rowstream_kernel<__nv_bfloat16>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)stream_smem);
-            if (e != cudaSuccess) return e;
-            pack_rowstream_kernel<__nv_bfloat16><<<g, kStreamThreads, stream_smem, s>>>(
-                (const __nv_bfloat16*)a.src, a.rows, a.d, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k,
-                (__nv_bfloat16*)a.dst, a.ld_dst, a.stride_dst);
-        }
-        return cudaGetLastError();
-    }
     if (a.ld_dst <= kNarrowMax) {
         dim3 g((unsigned)((a.rows + kNarrowRows - 1) / kNarrowRows), (unsigned)a.heads);
         if (g.x == 0) return cudaSuccess;

@@ -47,9 +47,9 @@ struct Vec16<float> {
 };
 
 // ------------------------------------------------------------------ colnorm
-// grid (ceil(d / (32*V)), nsplit, heads), 256 threads.  Warp w of split s sums
-// rows r0+w, r0+w+8, ... of its 32*V columns in increasing row order (eight
-// independent 16-byte loads in flight per thread); the 8 warp partials are
+// grid (ceil(d / (32*V)), nsplit, heads), 16 warps.  Warp w of split s sums
+// rows r0+w, r0+w+16, ... of its 32*V columns in increasing row order (eight
+// independent 16-byte loads in flight per thread); the 16 warp partials are
 // added in warp order and written as the split's partial.  The last CTA of a
 // column block to finish (device-scope counter) adds the nsplit partials of
 // its columns in split order and writes the final fp32 scores, then resets
@@ -57,8 +57,10 @@ struct Vec16<float> {
 // same for every column.
 constexpr int kMaxSplit = 64;
 
+constexpr int kColWarps = 16;
+
 template <typename T>
-__global__ void __launch_bounds__(256) colnorm_kernel(const T* __restrict__ A, int64_t n, int64_t d,
+__global__ void __launch_bounds__(32 * kColWarps) colnorm_kernel(const T* __restrict__ A, int64_t n, int64_t d,
                                                       int64_t lda, int64_t stride_a,
                                                       int64_t rows_per_split, int nsplit,
                                                       float* __restrict__ partials,
@@ -67,7 +69,8 @@ __global__ void __launch_bounds__(256) colnorm_kernel(const T* __restrict__ A, i
     constexpr int V = Vec16<T>::N;
     constexpr int COLS = 32 * V;
     constexpr int U = 8;
-    __shared__ float red[8][COLS];
+    constexpr int W = kColWarps;
+    __shared__ float red[W][COLS];
     __shared__ bool last;
     const int h = blockIdx.z, split = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -80,16 +83,16 @@ __global__ void __launch_bounds__(256) colnorm_kernel(const T* __restrict__ A, i
     if (col < d) {
         const T* base = A + (int64_t)h * stride_a + col;
         int64_t r = r0 + warp;
-        for (; r + 8 * (U - 1) < r1; r += 8 * U) {
+        for (; r + W * (U - 1) < r1; r += W * U) {
             float x[U][V];
 #pragma unroll
-            for (int u = 0; u < U; ++u) Vec16<T>::load(base + (r + 8 * u) * lda, x[u]);
+            for (int u = 0; u < U; ++u) Vec16<T>::load(base + (r + W * u) * lda, x[u]);
 #pragma unroll
             for (int u = 0; u < U; ++u)
 #pragma unroll
                 for (int v = 0; v < V; ++v) acc[v] = fmaf(x[u][v], x[u][v], acc[v]);
         }
-        for (; r < r1; r += 8) {
+        for (; r < r1; r += W) {
             float x0[V];
             Vec16<T>::load(base + r * lda, x0);
 #pragma unroll
@@ -99,10 +102,10 @@ __global__ void __launch_bounds__(256) colnorm_kernel(const T* __restrict__ A, i
 #pragma unroll
     for (int v = 0; v < V; ++v) red[warp][lane * V + v] = acc[v];
     __syncthreads();
-    for (int c = threadIdx.x; c < COLS; c += 256) {
+    for (int c = threadIdx.x; c < COLS; c += 32 * W) {
         float sum = red[0][c];
 #pragma unroll
-        for (int w = 1; w < 8; ++w) sum += red[w][c];
+        for (int w = 1; w < W; ++w) sum += red[w][c];
         const int64_t gcol = (int64_t)blockIdx.x * COLS + c;
         if (gcol < d) partials[((int64_t)h * nsplit + split) * d + gcol] = sum;
     }
@@ -117,7 +120,7 @@ __global__ void __launch_bounds__(256) colnorm_kernel(const T* __restrict__ A, i
     __syncthreads();
     if (!last) return;
     __threadfence();
-    for (int c = threadIdx.x; c < COLS; c += 256) {
+    for (int c = threadIdx.x; c < COLS; c += 32 * W) {
         const int64_t gcol = (int64_t)blockIdx.x * COLS + c;
         if (gcol >= d) continue;
         const float* pc = partials + (int64_t)h * nsplit * d + gcol;
@@ -387,11 +390,11 @@ cudaError_t launch_colnorm(const SelectArgs& a, cudaStream_t s) {
     const int V = a.dtype == 1 ? 4 : 8;
     dim3 grid((unsigned)((a.d + 32 * V - 1) / (32 * V)), (unsigned)a.nsplit, (unsigned)a.heads);
     if (a.dtype == 1)
-        colnorm_kernel<float><<<grid, 256, 0, s>>>((const float*)a.A, a.n, a.d, a.lda, a.stride_a,
+        colnorm_kernel<float><<<grid, 32 * kColWarps, 0, s>>>((const float*)a.A, a.n, a.d, a.lda, a.stride_a,
                                                    a.rows_per_split, a.nsplit, a.partials, a.counters,
                                                    a.scores);
     else
-        colnorm_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)a.A, a.n, a.d,
+        colnorm_kernel<__nv_bfloat16><<<grid, 32 * kColWarps, 0, s>>>((const __nv_bfloat16*)a.A, a.n, a.d,
                                                            a.lda, a.stride_a, a.rows_per_split,
                                                            a.nsplit, a.partials, a.counters, a.scores);
     return cudaGetLastError();

@@ -254,7 +254,10 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
     rmm::GemmParams gp;
     std::memset(&gp, 0, sizeof(gp));
     const uint32_t box_k = static_cast<uint32_t>(128 / es);
-    if (!identity) {
+    const bool qk_masked_path = p.mode == RMM_QK && !identity && p.d <= 1024;
+    if (qk_masked_path) {
+        // staged below together with B
+    } else if (!identity) {
         rmm::PackArgs pa{};
         pa.src = A;
         pa.dtype = p.dtype;
@@ -302,7 +305,36 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
     gp.err = ws_at<int>(ws, plan->off_err);
     gp.b_head_div = 1;
 
-    if (p.mode == RMM_QK) {
+    const bool qk_mask = p.mode == RMM_QK && !identity && p.d <= 1024;
+    if (qk_mask) {
+        // Attention scores are bound by writing S, not by the contraction: zero
+        // Q's features outside I_h and contract over all d_h with the shared K
+        // as it is (the zeroed terms add exact zeros, so the sum is the one
+        // over I_h) instead of packing Q and, per query head, K.
+        rmm::PackArgs pm{};
+        pm.src = A;
+        pm.dtype = p.dtype;
+        pm.rows = p.n;
+        pm.d = p.d;
+        pm.ld_src = p.lda;
+        pm.stride_src = p.stride_a;
+        pm.group = 1;
+        pm.I = I;
+        pm.I_stride = k;
+        pm.k = k;
+        pm.dst = ws_at<void>(ws, plan->off_apack);
+        pm.ld_dst = p.d;
+        pm.stride_dst = p.n * p.d;
+        pm.heads = static_cast<int>(p.heads);
+        if (rmm::launch_mask_columns(pm, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        if (!encode_kmajor_map(&gp.map_a, es, pm.dst, p.d, p.n, p.heads, p.d, p.n * p.d, box_k, 128))
+            return RMM_ERR_CUDA;
+        gp.k = static_cast<int32_t>(p.d);
+        gl.b_mode = rmm::kBKMajor;
+        if (!encode_kmajor_map(&gp.map_b, es, B, p.d, p.m, p.kv_heads, p.ldb, p.stride_b, box_k, kmajor_box_rows))
+            return RMM_ERR_CUDA;
+        gp.b_head_div = plan->group;
+    } else if (p.mode == RMM_QK) {
         gl.b_mode = rmm::kBKMajor;
         if (!identity) {
             rmm::PackArgs pb{};
@@ -393,6 +425,8 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
     }
     gl.pair = pair_ok && gl.b_mode != rmm::kBGather;
     gp.m_tiles = static_cast<int32_t>(gl.pair ? (p.n + 255) / 256 : (p.n + 127) / 128);
+    // rasterisation groups of 8 row tiles (measured best on the workloads' shapes)
+    gp.group_m = gp.m_tiles < 8 ? gp.m_tiles : 8;
     // the pair kernel stores 32 x 32 output boxes by TMA (64- or 128-byte rows)
     if (gl.pair && !encode_kmajor_map(&gp.map_y, es, Y, p.m, p.n, p.heads, p.ldy, p.stride_y, 32, 32,
                                       es == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
@@ -413,7 +447,7 @@ int32_t launches_per_call(const rmm_plan* plan) {
     if (p.n == 0 || p.m == 0) return n;
     if (plan->skinny) return n + (identity ? 0 : 1) + 1 + (plan->sk_splits > 1 ? 1 : 0);
     if (!identity) n += 1;                                   // pack A[:, I]
-    if (p.mode == RMM_QK && !identity) n += 1;               // pack K[:, I]
+    if (p.mode == RMM_QK && !identity && p.d > 1024) n += 1; // pack K[:, I] (else Q is masked in place of the A pack)
     if (p.mode != RMM_QK && p.dtype == RMM_F32) n += 1;      // B[I, :] transposed for tf32
     if (!identity && plan->pack_b) n += 1;                   // B[I, :] rows, contiguous
     return n + 1;                                            // the product
@@ -518,9 +552,12 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     plan->off_I = off;
     off += align256(static_cast<size_t>(p->heads) * plan->k * sizeof(int32_t));
     plan->off_apack = off;
-    off += align256(static_cast<size_t>(p->heads) * p->n * plan->ldp * plan->es);
+    const bool qk_mask = p->mode == RMM_QK && p->d <= 1024;  // Q masked at full width, K used as is
+    off += align256(static_cast<size_t>(p->heads) * p->n * (qk_mask ? p->d : plan->ldp) * plan->es);
     plan->off_bpack = off;
-    if (plan->skinny)
+    if (qk_mask) {
+        // no staged B
+    } else if (plan->skinny)
         off += align256(static_cast<size_t>(plan->sk_splits) * p->m * plan->sk_np * sizeof(float));
     else if (p->mode == RMM_QK || p->dtype == RMM_F32)
         off += align256(static_cast<size_t>(p->heads) * p->m * plan->ldp * plan->es);

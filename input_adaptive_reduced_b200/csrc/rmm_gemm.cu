@@ -308,10 +308,13 @@ struct PairCfg {
     static constexpr int STAGES = 6;
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr int GROUP_BYTES = BK * 128;
-    // epilogue staging: per epilogue warp two buffers of 32 rows x 32 columns
+    // epilogue: EPI_WARPS warps, two per TMEM lane quadrant for bf16 (each owns
+    // half of the tile's columns), with two staging buffers of 32 x 32 each
+    static constexpr int EPI_WARPS = (ES == 2) ? 8 : 4;
+    static constexpr int NT = 32 * (2 + EPI_WARPS);
     static constexpr int ROW_BYTES = 32 * ES;                 // 64 (bf16) or 128 (fp32)
     static constexpr int OUT_BUF = 32 * ROW_BYTES;
-    static constexpr int OUT_BYTES = 4 * 2 * OUT_BUF;
+    static constexpr int OUT_BYTES = EPI_WARPS * 2 * OUT_BUF;
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + OUT_BYTES + 256;
     static_assert(!(TF32 && B_MN), "fp32 operands are staged K-major");
     static_assert(BMODE != kBGather, "indexed gathers use the single-CTA kernel");
@@ -342,25 +345,28 @@ __device__ __forceinline__ void stage_row(uint8_t* buf, int r, const float (&v)[
     }
 }
 
-// Tile order of the CTA-pair kernel: within a head, groups of kGroupM
+// Tile order of the CTA-pair kernel: within a head, groups of p.group_m
 // consecutive 256-row tiles sweep every column tile before the next group, so
-// that the A rows and B columns of one wave of tiles stay resident in L2.
-constexpr int kGroupM = 8;
-
+// that the A rows of a group stay resident in L2 while B streams past.
 __device__ __forceinline__ void pair_tile(int t, const GemmParams& p, int& h, int& mt, int& nt) {
     const int per_head = p.m_tiles * p.n_tiles;
     h = t / per_head;
     const int r = t - h * per_head;
-    const int group = r / (kGroupM * p.n_tiles);
-    const int within = r - group * (kGroupM * p.n_tiles);
-    const int left = p.m_tiles - group * kGroupM;
-    const int gm = left < kGroupM ? left : kGroupM;
-    mt = group * kGroupM + within % gm;
+    const int G = p.group_m;
+    const int group = r / (G * p.n_tiles);
+    const int within = r - group * (G * p.n_tiles);
+    const int left = p.m_tiles - group * G;
+    const int gm = left < G ? left : G;
+    mt = group * G + within % gm;
     nt = within / gm;
 }
 
+// K loops of at most this many k-blocks make every epilogue warp poll the
+// accumulator barrier itself.
+constexpr int kAllPollMaxKb = 16;
+
 template <typename T, int BMODE, int BN>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN>::NT, 1)
     pair_gemm_kernel(const __grid_constant__ GemmParams p) {
     using C = PairCfg<T, BMODE, BN>;
     extern __shared__ uint8_t smem_raw[];
@@ -371,6 +377,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint64_t* tempty = tfull + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    volatile int* epi_go = reinterpret_cast<volatile int*>(tmem_holder + 2);  // accumulator ready (epilogue)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -383,7 +390,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);   // one multicast commit
-            mbar_init(&tempty[a], 8);  // 4 epilogue warps x 2 CTAs (used in the leader)
+            mbar_init(&tempty[a], 2 * C::EPI_WARPS);  // epilogue warps of both CTAs (used in the leader)
         }
         *abort_flag = 0;
         mbar_fence_init();
@@ -479,14 +486,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
-        // Each warp owns 32 rows; per 32-column chunk it stages its rows in a
-        // swizzled shared buffer and one lane stores the 32 x 32 box by TMA
-        // (rows past n and columns past m are clipped by the store itself).
+        // Warp e (of EPI_WARPS) owns TMEM lane quadrant q = (warp % 4), i.e. 32
+        // rows, and column chunks ch = half, half + H, ... of the tile (H = number
+        // of warps per quadrant).  Per 32-column chunk it stages its rows in a
+        // swizzled shared buffer and one lane stores the 32 x 32 box by TMA (rows
+        // past n and columns past m are clipped by the store itself).  Tiles the
+        // causal mask covers entirely store one -inf buffer repeatedly.
+        constexpr int H = C::EPI_WARPS / 4;
+        const int e = warp - 2;
         const int q = warp & 3;
+        const int half = e / 4;
         const int row_base = (int)rank * kBM + q * 32;
         const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
         const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
-        uint8_t* out = smem + C::STAGES * C::STAGE_BYTES + (q * 2) * C::OUT_BUF;
+        uint8_t* out = smem + C::STAGES * C::STAGE_BYTES + (e * 2) * C::OUT_BUF;
         uint32_t tcount = 0, slot = 0;
         for (int t = cluster; t < total; t += nclusters) {
             int h, mt, nt;
@@ -499,42 +512,65 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (!skip) {
                 acc = tcount & 1u;
                 const uint32_t aph = (tcount >> 1) & 1u;
-                if (!mbar_wait(&tfull[acc], aph, abort_flag, p.err, kErrTimeoutEpilogue)) break;
+                if (num_kb <= kAllPollMaxKb) {
+                    // short K loop: the epilogue is the critical path, every warp polls
+                    if (!mbar_wait(&tfull[acc], aph, abort_flag, p.err, kErrTimeoutEpilogue)) break;
+                } else {
+                    // long K loop: one warp polls so that the others leave the issue
+                    // slots to the producer and MMA warps; they sleep on a named barrier
+                    if (e == 0) *epi_go = mbar_wait(&tfull[acc], aph, abort_flag, p.err, kErrTimeoutEpilogue) ? 1 : 0;
+                    asm volatile("bar.sync 1, %0;" ::"n"(32 * C::EPI_WARPS) : "memory");
+                    if (!*epi_go) break;
+                }
                 tc_fence_after();
                 taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
             }
             if (row0 < p.n) {
+                bool inf_staged = false;
 #pragma unroll 1
-                for (int ch = 0; ch < BN / 32; ++ch) {
+                for (int ch = half; ch < BN / 32; ch += H) {
                     const int col0 = n0 + ch * 32;
-                    float v[32];
+                    if (col0 >= p.m) break;
+                    uint8_t* buf = out + slot * C::OUT_BUF;
                     if (skip) {
+                        if (!inf_staged) {
+                            float v[32];
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = -__int_as_float(0x7f800000);
-                    } else {
-                        uint32_t raw[32];
-                        tmem_ld_32x32b_x32(taddr + ch * 32, raw);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const float x = __uint_as_float(raw[i]) * p.alpha;
-                            v[i] = (p.causal && col0 + i > row) ? -__int_as_float(0x7f800000) : x;
+                            for (int i = 0; i < 32; ++i) v[i] = -__int_as_float(0x7f800000);
+                            if (lane == 0) bulk_wait_group_read<0>();
+                            __syncwarp();
+                            stage_row<T>(buf, lane, v);
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            inf_staged = true;
                         }
-                    }
-                    if (col0 < p.m) {
-                        uint8_t* buf = out + slot * C::OUT_BUF;
-                        if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
-                        __syncwarp();
-                        stage_row<T>(buf, lane, v);
-                        fence_proxy_async_smem();
-                        __syncwarp();
                         if (lane == 0) {
                             tma_store_3d(&p.map_y, buf, col0, row0, h);
                             bulk_commit_group();
                         }
-                        slot ^= 1u;
+                        continue;  // the same buffer serves every chunk of the tile
                     }
+                    uint32_t raw[32];
+                    tmem_ld_32x32b_x32(taddr + ch * 32, raw);
+                    float v[32];
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float x = __uint_as_float(raw[i]) * p.alpha;
+                        v[i] = (p.causal && col0 + i > row) ? -__int_as_float(0x7f800000) : x;
+                    }
+                    if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
+                    __syncwarp();
+                    stage_row<T>(buf, lane, v);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(&p.map_y, buf, col0, row0, h);
+                        bulk_commit_group();
+                    }
+                    slot ^= 1u;
                 }
+                if (skip) slot ^= 1u;  // the -inf buffer may still be read: use the other one next
             }
             if (!skip) {
                 tc_fence_before();
@@ -565,7 +601,7 @@ cudaError_t launch_pair(const GemmParams& p, int num_sms, cudaStream_t s) {
     const int total = p.heads * p.m_tiles * p.n_tiles;
     const int clusters = total < num_sms / 2 ? total : num_sms / 2;
     if (clusters <= 0) return cudaSuccess;
-    kern<<<2 * clusters, kThreads, C::SMEM, s>>>(p);
+    kern<<<2 * clusters, C::NT, C::SMEM, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -54,6 +54,10 @@ struct PackArgs {
     int heads;
 };
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t s);
+// dst[h][r][j] = src[h][r][j] if j is in I[h][0..k) else 0 (dst has the
+// source's shape; used for attention scores, where the product is bound by
+// its output and a zero-masked operand gives the same sum over I).
+cudaError_t launch_mask_columns(const PackArgs& a, cudaStream_t s);
 // dst[h][c][t] = src[h / group][I[h][t]][c]: gathered rows written K-major
 // (rows = number of source columns c; I == nullptr means I[t] = t).
 cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s);
@@ -82,6 +86,7 @@ struct __align__(64) GemmParams {
     int32_t b_rows_total;       // MN-major B: rows of the 2-D map (an out-of-range row reads zeros)
     int32_t b_head_div;         // kBKMajor: B head coordinate = h / b_head_div
     int32_t m_tiles, n_tiles;
+    int32_t group_m;            // CTA-pair kernel: 256-row tiles per rasterisation group
     float alpha;
     int32_t causal;
     int* err;

@@ -184,7 +184,58 @@ __global__ void __launch_bounds__(256) pack_narrow_kernel(
     }
 }
 
+// grid (ceil(rows / 64), heads), 256 threads: the head's index set becomes a
+// bit mask in shared memory; each thread copies 16-byte groups of a row,
+// zeroing the columns that are not kept.
+template <typename T>
+__global__ void __launch_bounds__(256) mask_columns_kernel(const T* __restrict__ src, int64_t rows, int64_t d,
+                                                           int64_t ld_src, int64_t stride_src,
+                                                           const int32_t* __restrict__ I, int64_t I_stride,
+                                                           int64_t k, T* __restrict__ dst, int64_t ld_dst,
+                                                           int64_t stride_dst) {
+    constexpr int V = 16 / sizeof(T);
+    __shared__ uint32_t keep[kNarrowMax / 32];
+    const int h = blockIdx.y;
+    for (int w = threadIdx.x; w < kNarrowMax / 32; w += 256) keep[w] = 0u;
+    __syncthreads();
+    for (int64_t t = threadIdx.x; t < k; t += 256) {
+        const int32_t j = __ldg(I + (int64_t)h * I_stride + t);
+        if (j >= 0 && j < d) atomicOr(&keep[j >> 5], 1u << (j & 31));
+    }
+    __syncthreads();
+    const int cpr = (int)(d / V);
+    const int64_t r0 = (int64_t)blockIdx.x * 64;
+    const int nr = (int)(rows - r0 < 64 ? rows - r0 : 64);
+    const T* sh = src + (int64_t)h * stride_src;
+    T* dh = dst + (int64_t)h * stride_dst;
+    for (int e = threadIdx.x; e < nr * cpr; e += 256) {
+        const int r = e / cpr, c = e - r * cpr;
+        uint4 v = __ldg(reinterpret_cast<const uint4*>(sh + (r0 + r) * ld_src) + c);
+        T* vals = reinterpret_cast<T*>(&v);
+#pragma unroll
+        for (int u = 0; u < V; ++u) {
+            const int j = c * V + u;
+            if (!((keep[j >> 5] >> (j & 31)) & 1u)) vals[u] = T(0.f);
+        }
+        reinterpret_cast<uint4*>(dh + (r0 + r) * ld_dst)[c] = v;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_mask_columns(const PackArgs& a, cudaStream_t s) {
+    if (a.d > kNarrowMax) return cudaErrorInvalidValue;
+    dim3 g((unsigned)((a.rows + 63) / 64), (unsigned)a.heads);
+    if (g.x == 0) return cudaSuccess;
+    if (a.dtype == 1)
+        mask_columns_kernel<float><<<g, 256, 0, s>>>((const float*)a.src, a.rows, a.d, a.ld_src, a.stride_src, a.I,
+                                                     a.I_stride, a.k, (float*)a.dst, a.ld_dst, a.stride_dst);
+    else
+        mask_columns_kernel<__nv_bfloat16><<<g, 256, 0, s>>>((const __nv_bfloat16*)a.src, a.rows, a.d, a.ld_src,
+                                                             a.stride_src, a.I, a.I_stride, a.k,
+                                                             (__nv_bfloat16*)a.dst, a.ld_dst, a.stride_dst);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_pack_rows(const PackArgs& a, int num_sms, cudaStream_t s) {
     (void)num_sms;

@@ -39,7 +39,7 @@ METRIC = "RMM op latency and useful TFLOP/s (2·n·⌈ρd⌉·m) vs ρ=1, % of b
 WORKLOAD = "llama3.1-8b-mlp-linear-rmm"
 SHAPES = {"up": (4096, 14336), "down": (14336, 4096)}
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gather_gemm_llama8b_mlp_n4096.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "pair_gemm_llama8b_mlp_n4096.md")
 GEMM_SOURCE = os.path.join(ROOT, "input_adaptive_reduced_b200", "csrc", "rmm_gemm.cu")
 
 

@@ -424,6 +424,10 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         if (!encode_rows_map(&gp.map_b, B, p.m, rows_total, p.ldb, row_tiles ? 64u : 1u)) return RMM_ERR_CUDA;
     }
     gl.pair = pair_ok && gl.b_mode != rmm::kBGather;
+    gp.split_tiles = gl.pair ? plan->split_tiles : 0;
+    gp.split_f = gl.pair ? plan->split_f : 1;
+    gp.split_partials = ws_at<float>(ws, plan->off_split);
+    gp.split_counters = ws_at<unsigned>(ws, plan->off_split_cnt);
     gp.m_tiles = static_cast<int32_t>(gl.pair ? (p.n + 255) / 256 : (p.n + 127) / 128);
     // rasterisation groups of 8 row tiles (measured best on the workloads' shapes)
     gp.group_m = gp.m_tiles < 8 ? gp.m_tiles : 8;
@@ -541,6 +545,18 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     off += 256;
     plan->off_counters = off;
     off += align256(static_cast<size_t>(p->heads) * colblocks * sizeof(unsigned));
+    // Split tail of the CTA-pair product (256-row tiles, more than one 128-row
+    // tile of work, no causal mask): its counters live in the header.
+    plan->split_tiles = 0;
+    plan->split_f = 1;
+    if (!plan->skinny && p->n > 128 && p->m > 0 && !(p->flags & RMM_FLAG_CAUSAL)) {
+        const int64_t k_eff = (p->mode == RMM_QK && p->d <= 1024) ? p->d : plan->k;
+        const int64_t bk = 128 / plan->es;
+        const int64_t tiles = p->heads * ((p->n + 255) / 256) * ((p->m + plan->bn - 1) / plan->bn);
+        rmm::pair_split_tail(tiles, (k_eff + bk - 1) / bk, sms / 2, &plan->split_tiles, &plan->split_f);
+    }
+    plan->off_split_cnt = off;
+    off += align256(static_cast<size_t>(plan->split_tiles) * 2 * rmm::kSplitCounterWarps * sizeof(unsigned));
     plan->header_bytes = off;
     plan->off_partials = off;
     plan->off_scores = off;
@@ -563,6 +579,8 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
         off += align256(static_cast<size_t>(p->heads) * p->m * plan->ldp * plan->es);
     else if (plan->pack_b || given)
         off += align256(static_cast<size_t>(p->heads) * plan->k * p->m * plan->es);
+    plan->off_split = off;
+    off += align256(static_cast<size_t>(plan->split_tiles) * plan->split_f * 256 * plan->bn * sizeof(float));
     plan->ws_bytes = off;
     if (workspace_bytes) *workspace_bytes = plan->ws_bytes;
     *out = plan;

@@ -361,11 +361,115 @@ __device__ __forceinline__ void pair_tile(int t, const GemmParams& p, int& h, in
     nt = within / gm;
 }
 
+// Work unit of the CTA-pair kernel: a whole tile, or K-part `part` of one of
+// the split tail tiles (k-blocks [kb0, kb1)).  Units before `whole` are the
+// tiles of the same index; the split tail follows, part-major within a tile.
+struct PairUnit {
+    int t, kb0, kb1, part;  // part < 0: whole tile
+};
+
+template <bool SPLIT>
+__device__ __forceinline__ PairUnit pair_unit(int u, int whole, int num_kb, const GemmParams& p) {
+    PairUnit w;
+    if (!SPLIT || u < whole) {
+        w.t = u;
+        w.kb0 = 0;
+        w.kb1 = num_kb;
+        w.part = -1;
+    } else {
+        const int v = u - whole;
+        w.t = whole + v / p.split_f;
+        w.part = v - (v / p.split_f) * p.split_f;
+        w.kb0 = w.part * num_kb / p.split_f;
+        w.kb1 = (w.part + 1) * num_kb / p.split_f;
+    }
+    return w;
+}
+
+// Epilogue of one K-part of a split tail tile, for one warp (its 32 rows x
+// the chunks ch = half, half + H, ...; TMEM address taddr).  The part's raw
+// fp32 accumulator goes to the workspace in chunk layout [ch][g][lane][4];
+// after a fence the warp counts the part, and the warp that counts the last
+// one adds the parts in part order (0, 1, ..., f - 1, so every call gives the
+// same bits), scales by alpha and stores the tile through the staging
+// buffers (slot: the next staging buffer; returns the one after the stores).
+// Split tails are planned only without the causal mask.  Kept out of line so
+// that it does not shape the whole-tile epilogue's code.
+template <typename T, int BN, int H>
+__device__ __noinline__ uint32_t split_part_epilogue(const GemmParams& p, uint32_t taddr, int si, int part, int rank,
+                                                     int q, int e, int half, int n0, int row0, int h, uint8_t* out,
+                                                     uint32_t slot) {
+    constexpr int OUT_BUF = 32 * 32 * (int)sizeof(T);
+    const int lane = threadIdx.x & 31;
+    const size_t tile_floats = (size_t)2 * kBM * BN;
+    float* parts = p.split_partials + (size_t)si * p.split_f * tile_floats + ((size_t)rank * kBM + (size_t)q * 32) * BN;
+#pragma unroll 1
+    for (int ch = half; ch < BN / 32; ch += H) {
+        if (n0 + ch * 32 >= p.m) break;
+        uint32_t raw[32];
+        tmem_ld_32x32b_x32(taddr + ch * 32, raw);
+        tmem_ld_wait();
+        float4* dst = reinterpret_cast<float4*>(parts + (size_t)part * tile_floats + ch * 1024) + lane;
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+            __stcg(dst + g * 32, make_float4(__uint_as_float(raw[4 * g]), __uint_as_float(raw[4 * g + 1]),
+                                             __uint_as_float(raw[4 * g + 2]), __uint_as_float(raw[4 * g + 3])));
+    }
+    __syncwarp();
+    unsigned* cnt = p.split_counters + ((size_t)si * 2 + rank) * kSplitCounterWarps + e;
+    unsigned done = 0;
+    if (lane == 0) {
+        __threadfence();  // this part's stores before its count
+        done = atomicAdd(cnt, 1u);
+    }
+    done = __shfl_sync(0xffffffffu, done, 0);
+    if (done != (unsigned)(p.split_f - 1)) return slot;
+    if (lane == 0) atomicExch(cnt, 0u);  // ready for the next launch
+    __threadfence();                     // the other parts' stores after their counts
+#pragma unroll 1
+    for (int ch = half; ch < BN / 32; ch += H) {
+        const int col0 = n0 + ch * 32;
+        if (col0 >= p.m) break;
+        uint32_t raw[32];
+        tmem_ld_32x32b_x32(taddr + ch * 32, raw);
+        tmem_ld_wait();
+        float v[32];
+#pragma unroll 1
+        for (int j = 0; j < p.split_f; ++j) {
+            const float4* src = reinterpret_cast<const float4*>(parts + (size_t)j * tile_floats + ch * 1024) + lane;
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+                const float4 x = j == part ? make_float4(__uint_as_float(raw[4 * g]), __uint_as_float(raw[4 * g + 1]),
+                                                         __uint_as_float(raw[4 * g + 2]), __uint_as_float(raw[4 * g + 3]))
+                                           : __ldcg(src + g * 32);
+                v[4 * g] = j == 0 ? x.x : v[4 * g] + x.x;
+                v[4 * g + 1] = j == 0 ? x.y : v[4 * g + 1] + x.y;
+                v[4 * g + 2] = j == 0 ? x.z : v[4 * g + 2] + x.z;
+                v[4 * g + 3] = j == 0 ? x.w : v[4 * g + 3] + x.w;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= p.alpha;
+        uint8_t* buf = out + slot * OUT_BUF;
+        if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
+        __syncwarp();
+        stage_row<T>(buf, lane, v);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_3d(&p.map_y, buf, col0, row0, h);
+            bulk_commit_group();
+        }
+        slot ^= 1u;
+    }
+    return slot;
+}
+
 // K loops of at most this many k-blocks make every epilogue warp poll the
 // accumulator barrier itself.
 constexpr int kAllPollMaxKb = 16;
 
-template <typename T, int BMODE, int BN>
+template <typename T, int BMODE, int BN, bool SPLIT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN>::NT, 1)
     pair_gemm_kernel(const __grid_constant__ GemmParams p) {
     using C = PairCfg<T, BMODE, BN>;
@@ -408,19 +512,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
 
     const int total = p.heads * p.m_tiles * p.n_tiles;  // 256-row tiles
     const int num_kb = (p.k + C::BK - 1) / C::BK;
+    const int whole = SPLIT ? total - p.split_tiles : total;
+    const int units = SPLIT ? whole + p.split_tiles * p.split_f : total;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
-            for (int t = cluster; t < total && ok; t += nclusters) {
+            for (int u = cluster; u < units && ok; u += nclusters) {
+                const PairUnit w = pair_unit<SPLIT>(u, whole, num_kb, p);
                 int h, mt, nt;
-                pair_tile(t, p, h, mt, nt);
+                pair_tile(w.t, p, h, mt, nt);
                 const int m0 = mt * 2 * kBM, n0 = nt * BN;
                 if (p.causal && n0 > m0 + 2 * kBM - 1) continue;
                 const int row_base = (h / p.group) * p.b_head_rows;
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
                     if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err, kErrTimeoutProducer)) {
@@ -450,9 +557,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
             constexpr uint32_t idesc = umma_idesc(C::TF32, C::B_MN, BN, 256);
             uint32_t it = 0, tcount = 0;
             bool ok = true;
-            for (int t = cluster; t < total && ok; t += nclusters) {
+            for (int u = cluster; u < units && ok; u += nclusters) {
+                const PairUnit w = pair_unit<SPLIT>(u, whole, num_kb, p);
                 int h, mt, nt;
-                pair_tile(t, p, h, mt, nt);
+                pair_tile(w.t, p, h, mt, nt);
                 const int m0 = mt * 2 * kBM, n0 = nt * BN;
                 if (p.causal && n0 > m0 + 2 * kBM - 1) continue;
                 const uint32_t acc = tcount & 1u;
@@ -460,7 +568,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
                 if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, p.err, kErrTimeoutMma)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
                     if (!mbar_wait(&full[s], ph, abort_flag, p.err, kErrTimeoutMma)) {
@@ -475,7 +583,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
                         const uint64_t adesc = sw128_desc(a_addr + kk * 32, 16, 1024);
                         const uint64_t bdesc = C::B_MN ? sw128_desc(b_addr + kk * C::UK * 128, C::GROUP_BYTES, 1024)
                                                        : sw128_desc(b_addr + kk * 32, 16, 1024);
-                        umma_pair<C::TF32>(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        umma_pair<C::TF32>(d_tmem, adesc, bdesc, idesc, (kb != w.kb0 || kk != 0) ? 1u : 0u);
                     }
                     umma_commit_pair(&empty[s], 0x3);
                 }
@@ -501,9 +609,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
         const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
         uint8_t* out = smem + C::STAGES * C::STAGE_BYTES + (e * 2) * C::OUT_BUF;
         uint32_t tcount = 0, slot = 0;
-        for (int t = cluster; t < total; t += nclusters) {
+        // Stage one thread's 32 values of a 32 x 32 chunk and store the chunk by TMA.
+        auto emit = [&](const float (&v)[32], int col0, int row0, int h) {
+            uint8_t* buf = out + slot * C::OUT_BUF;
+            if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
+            __syncwarp();
+            stage_row<T>(buf, lane, v);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(&p.map_y, buf, col0, row0, h);
+                bulk_commit_group();
+            }
+            slot ^= 1u;
+        };
+        for (int u = cluster; u < units; u += nclusters) {
+            const PairUnit w = pair_unit<SPLIT>(u, whole, num_kb, p);
             int h, mt, nt;
-            pair_tile(t, p, h, mt, nt);
+            pair_tile(w.t, p, h, mt, nt);
             const int m0 = mt * 2 * kBM, n0 = nt * BN;
             const int row0 = m0 + row_base;
             const int row = row0 + lane;
@@ -512,7 +635,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
             if (!skip) {
                 acc = tcount & 1u;
                 const uint32_t aph = (tcount >> 1) & 1u;
-                if (num_kb <= kAllPollMaxKb) {
+                if (w.kb1 - w.kb0 <= kAllPollMaxKb) {
                     // short K loop: the epilogue is the critical path, every warp polls
                     if (!mbar_wait(&tfull[acc], aph, abort_flag, p.err, kErrTimeoutEpilogue)) break;
                 } else {
@@ -525,14 +648,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
                 tc_fence_after();
                 taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
             }
-            if (row0 < p.n) {
+            if (SPLIT && row0 < p.n && w.part >= 0) {
+                slot = split_part_epilogue<T, BN, H>(p, taddr, w.t - whole, w.part, (int)rank, q, e, half, n0, row0,
+                                                     h, out, slot);
+            } else if (row0 < p.n) {
                 bool inf_staged = false;
 #pragma unroll 1
                 for (int ch = half; ch < BN / 32; ch += H) {
                     const int col0 = n0 + ch * 32;
                     if (col0 >= p.m) break;
-                    uint8_t* buf = out + slot * C::OUT_BUF;
                     if (skip) {
+                        uint8_t* buf = out + slot * C::OUT_BUF;
                         if (!inf_staged) {
                             float v[32];
 #pragma unroll
@@ -559,18 +685,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
                         const float x = __uint_as_float(raw[i]) * p.alpha;
                         v[i] = (p.causal && col0 + i > row) ? -__int_as_float(0x7f800000) : x;
                     }
-                    if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
-                    __syncwarp();
-                    stage_row<T>(buf, lane, v);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_3d(&p.map_y, buf, col0, row0, h);
-                        bulk_commit_group();
-                    }
-                    slot ^= 1u;
+                    emit(v, col0, row0, h);
                 }
-                if (skip) slot ^= 1u;  // the -inf buffer may still be read: use the other one next
+                if (skip && inf_staged) slot ^= 1u;  // the -inf buffer may still be read: use the other one next
             }
             if (!skip) {
                 tc_fence_before();
@@ -595,11 +712,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
 template <typename T, int BMODE, int BN>
 cudaError_t launch_pair(const GemmParams& p, int num_sms, cudaStream_t s) {
     using C = PairCfg<T, BMODE, BN>;
-    auto kern = pair_gemm_kernel<T, BMODE, BN>;
+    auto kern = p.split_tiles > 0 ? pair_gemm_kernel<T, BMODE, BN, true> : pair_gemm_kernel<T, BMODE, BN, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
     if (e != cudaSuccess) return e;
     const int total = p.heads * p.m_tiles * p.n_tiles;
-    const int clusters = total < num_sms / 2 ? total : num_sms / 2;
+    const int units = total - p.split_tiles + p.split_tiles * p.split_f;
+    const int clusters = units < num_sms / 2 ? units : num_sms / 2;
     if (clusters <= 0) return cudaSuccess;
     kern<<<2 * clusters, C::NT, C::SMEM, s>>>(p);
     return cudaGetLastError();
@@ -624,6 +742,22 @@ cudaError_t launch_bn(const GemmParams& p, const GemmLaunch& l, cudaStream_t s) 
 }
 
 }  // namespace
+
+void pair_split_tail(int64_t tiles, int64_t num_kb, int clusters, int* split_tiles, int* split_f) {
+    *split_tiles = 0;
+    *split_f = 1;
+    if (tiles <= 0 || clusters <= 0) return;
+    // The last wave holds tiles % clusters tiles; cut each into f K-parts so
+    // that the f-fold units still fit one wave, with at least 8 k-blocks a part.
+    const int64_t rem = tiles % clusters;
+    if (rem == 0) return;
+    int64_t f = clusters / rem;
+    if (f > 4) f = 4;
+    if (f > num_kb / 8) f = num_kb / 8;
+    if (f < 2) return;
+    *split_tiles = static_cast<int>(rem);
+    *split_f = static_cast<int>(f);
+}
 
 size_t gemm_smem_bytes(int dtype, int bn, bool pair) {
     if (pair) {

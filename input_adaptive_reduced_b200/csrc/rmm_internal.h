@@ -90,6 +90,14 @@ struct __align__(64) GemmParams {
     float alpha;
     int32_t causal;
     int* err;
+    // CTA-pair kernel, split tail: the last split_tiles tiles of the tile order
+    // are computed as split_f K-parts each (0 = none).  Part j of split tile i
+    // writes its fp32 accumulator to split_partials[(i * split_f + j)][256][BN];
+    // split_counters[i][2][8] counts the parts each epilogue warp has finished
+    // (zero between launches: the last part resets them).
+    int32_t split_tiles, split_f;
+    float* split_partials;
+    unsigned* split_counters;
 };
 
 struct GemmLaunch {
@@ -102,6 +110,11 @@ struct GemmLaunch {
 };
 cudaError_t launch_gemm(const GemmParams& p, const GemmLaunch& l, cudaStream_t s);
 size_t gemm_smem_bytes(int dtype, int bn, bool pair);
+// Split tail of the CTA-pair kernel for `tiles` 256-row tiles of `num_kb`
+// k-blocks on `clusters` pairs: sets *split_tiles and *split_f (0 and 1 when
+// the last wave is full or too short to split).
+void pair_split_tail(int64_t tiles, int64_t num_kb, int clusters, int* split_tiles, int* split_f);
+constexpr int kSplitCounterWarps = 8;  // counters per CTA per split tile (epilogue warps)
 
 // ---------------------------------------------------------------- few rows
 // Product for n <= 64 with swapped operands (rmm_skinny.cu).
@@ -144,4 +157,6 @@ struct rmm_plan {
     cudaEvent_t product_start, product_stop;  // tracing hook, may be null
     bool skinny;        // n <= 64 bf16 LINEAR: swapped-operand split-K product
     int sk_np, sk_splits;
+    int split_tiles, split_f;           // split tail of the CTA-pair product (0, 1: none)
+    size_t off_split_cnt, off_split;    // its counters (in the header) and fp32 partials
 };

@@ -153,6 +153,67 @@ def test_deterministic(rmm):
     assert torch.equal(I1, I2) and torch.equal(Y1, Y2)
 
 
+def _split_parts(tiles, num_kb):
+    """Parts per tile of the CTA-pair kernel's split tail on this GPU (1 = none):
+    the last wave's tiles are cut into f <= 4 K-parts that still fit one wave,
+    each at least 8 k-blocks long."""
+    clusters = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    rem = tiles % clusters
+    if rem == 0:
+        return 1
+    f = min(clusters // rem, 4, num_kb // 8)
+    return f if f >= 2 else 1
+
+
+# (n, d, m, rho): tiles of 256 x 256 and k-blocks of 64 that give split tails
+# of 4, 3 and 2 parts, one after a full wave of whole tiles
+SPLIT_SHAPES = [(300, 4096, 704, 0.6), (1024, 4096, 1280, 0.8), (1280, 4096, 1536, 0.5),
+                (2048, 2048, 2560, 0.7)]
+
+
+@pytest.mark.parametrize("n,d,m,rho", SPLIT_SHAPES)
+def test_split_tail_linear(rmm, n, d, m, rho):
+    """Tiles of the last wave computed as K-parts and added in part order."""
+    k = oracle.retained_count(rho, d)
+    tiles = -(-n // 256) * -(-m // 256)
+    assert _split_parts(tiles, -(-k // 64)) > 1
+    (A, B), _ = gap.enforce_boundary_gaps(lambda g: W.mlp_up(41, n=n, d=d, m=m, col_gain=g),
+                                          lambda x: gap.scores_2d(x[0]), [k])
+    Y1, _ = _linear_case(rmm, A, B, rho)
+    Y2 = rmm.matmul(A.cuda(), B.cuda(), rho=rho)  # counters were reset by the first call
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2)
+    rmm.check_workspaces()
+
+
+def test_split_tail_fp32(rmm):
+    n, d, m, rho = 300, 1024, 600, 0.5
+    k = oracle.retained_count(rho, d)
+    assert _split_parts(-(-n // 256) * -(-m // 256), -(-k // 32)) > 1
+    (A, B), _ = gap.enforce_boundary_gaps(
+        lambda g: W.mlp_up(42, n=n, d=d, m=m, col_gain=g, dtype=torch.float32),
+        lambda x: gap.scores_2d(x[0]), [k])
+    _linear_case(rmm, A, B, rho)
+    rmm.check_workspaces()
+
+
+def test_split_tail_pv(rmm):
+    H, Hkv, n, dv, rho = 2, 1, 2048, 128, 0.8
+    k = oracle.retained_count(rho, n)
+    assert _split_parts(H * (n // 256), -(-k // 64)) > 1
+    (P, V), _ = gap.enforce_boundary_gaps(
+        lambda g: W.attn_pv(43, n=n, heads=H, kv_heads=Hkv, v_dim=dv, col_gain=g),
+        lambda x: gap.scores_per_head(x[0]), [k])
+    O, T = rmm.pv(P.cuda(), V.cuda(), rho=rho, return_indices=True)
+    torch.cuda.synchronize()
+    O_ref, T_ref = oracle.rmm_pv(P, V, rho=rho)
+    assert_indices_equal(T, T_ref)
+    P64, V64 = oracle.as_f64(P), oracle.as_f64(V)
+    for h in range(H):
+        assert_product_close(O[h], O_ref[h], np.abs(P64[h][:, T_ref[h]]), np.abs(V64[0][T_ref[h]]))
+    rmm.check_workspaces()
+
+
 def _qk_check(rmm, Q, K, rho, causal):
     H, n, dh = Q.shape
     alpha = 1.0 / math.sqrt(dh)

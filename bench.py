@@ -326,7 +326,7 @@ def run_rmm(args):
                 "frac": achieved / peak_burst, "traffic": load_traffic(),
                 "peak_kind": f"{peak_src} cuBLAS bf16 burst",
                 "frac_of_sustained": (achieved / peak_sust) if peak_sust else None,
-                "kernel": "pair_gemm_kernel<bf16, kBRows, 256> (CTA pair, cta_group::2, 256x256 tile)",
+                "kernel": "pair_gemm_kernel<bf16, kBRows, 256, split> (CTA pair, cta_group::2, 256x256 tiles, split tail)",
                 "avg_launch_us": sum(gemm_ms) / len(gemm_ms) * 1e3}
 
     # per-op latency at rho and at rho = 1 (same kernels, identity I) and cuBLAS dense

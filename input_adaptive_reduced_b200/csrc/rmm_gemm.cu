@@ -133,6 +133,8 @@ __global__ void __launch_bounds__(kThreads, 1) gather_gemm_kernel(const __grid_c
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    pdl_wait();  // everything above touched only shared and tensor memory
+    pdl_trigger();
 
     const int total = p.heads * p.m_tiles * p.n_tiles;
     const int num_kb = (p.k + C::BK - 1) / C::BK;
@@ -509,6 +511,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
     cluster_sync_all();  // barriers of both CTAs initialised before any remote arrival
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    pdl_wait();  // everything above touched only shared and tensor memory
+    pdl_trigger();
 
     const int total = p.heads * p.m_tiles * p.n_tiles;  // 256-row tiles
     const int num_kb = (p.k + C::BK - 1) / C::BK;
@@ -719,8 +723,7 @@ cudaError_t launch_pair(const GemmParams& p, int num_sms, cudaStream_t s) {
     const int units = total - p.split_tiles + p.split_tiles * p.split_f;
     const int clusters = units < num_sms / 2 ? units : num_sms / 2;
     if (clusters <= 0) return cudaSuccess;
-    kern<<<2 * clusters, C::NT, C::SMEM, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(2 * clusters), dim3(C::NT), C::SMEM, s, p);
 }
 
 template <typename T, int BMODE, int BN>
@@ -732,8 +735,7 @@ cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t s) {
     const int total = p.heads * p.m_tiles * p.n_tiles;
     const int grid = total < num_sms ? total : num_sms;
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, kThreads, C::SMEM, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), C::SMEM, s, p);
 }
 
 template <typename T, int BMODE>

@@ -8,6 +8,36 @@
 
 namespace rmm {
 
+// ---------------------------------------------------------------- launches
+// Every kernel of the library is launched with programmatic stream
+// serialisation: it may be scheduled while the previous kernel on the stream
+// is still running, and it calls pdl_wait() before its first global memory
+// access (reads of what earlier work wrote, and writes that earlier work may
+// still read); pdl_wait() returns once every earlier kernel has completed and
+// its writes are visible.  pdl_trigger() lets the next kernel be scheduled.
+// Work before pdl_wait() touches only shared memory, tensor memory and the
+// kernel's parameters.
+#if defined(__CUDACC__)
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+#endif
+
+template <typename... Params, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // ---------------------------------------------------------------- selection
 struct SelectArgs {
     const void* A;       // [heads][n][lda]

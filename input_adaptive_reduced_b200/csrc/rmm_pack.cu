@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(
     const T* __restrict__ src, int64_t rows, int64_t d, int64_t ld_src, int64_t stride_src, int group,
     const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
     int64_t stride_dst) {
+    pdl_wait();
+    pdl_trigger();
     const int h = blockIdx.z;
     const int64_t t0 = ((int64_t)blockIdx.x * kPackThreads + threadIdx.x) * 8;
     if (t0 >= ld_dst) return;
@@ -74,6 +76,8 @@ __global__ void __launch_bounds__(256) pack_rows_transposed_kernel(
     const T* __restrict__ src, int64_t d, int64_t cols, int64_t ld_src, int64_t stride_src, int group,
     const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
     int64_t stride_dst) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ T tile[32][33];
     const int h = blockIdx.z;
     const int64_t t0 = (int64_t)blockIdx.x * 32, c0 = (int64_t)blockIdx.y * 32;
@@ -110,6 +114,8 @@ __global__ void __launch_bounds__(256) pack_rows_kernel(
     const T* __restrict__ src, int64_t d, int64_t cols, int64_t ld_src, int64_t stride_src, int group,
     const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
     int64_t stride_dst) {
+    pdl_wait();
+    pdl_trigger();
     constexpr int V = 16 / sizeof(T);
     const int h = blockIdx.y;
     const int cpr = (int)(cols / V);
@@ -153,6 +159,8 @@ __global__ void __launch_bounds__(256) pack_narrow_kernel(
     const T* __restrict__ src, int64_t rows, int64_t d, int64_t ld_src, int64_t stride_src, int group,
     const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
     int64_t stride_dst) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int32_t sidx[kNarrowMax];
     const int h = blockIdx.y;
     const int cpr = (int)(ld_dst / 8);
@@ -193,6 +201,8 @@ __global__ void __launch_bounds__(256) mask_columns_kernel(const T* __restrict__
                                                            const int32_t* __restrict__ I, int64_t I_stride,
                                                            int64_t k, T* __restrict__ dst, int64_t ld_dst,
                                                            int64_t stride_dst) {
+    pdl_wait();
+    pdl_trigger();
     constexpr int V = 16 / sizeof(T);
     __shared__ uint32_t keep[kNarrowMax / 32];
     const int h = blockIdx.y;
@@ -228,13 +238,11 @@ cudaError_t launch_mask_columns(const PackArgs& a, cudaStream_t s) {
     dim3 g((unsigned)((a.rows + 63) / 64), (unsigned)a.heads);
     if (g.x == 0) return cudaSuccess;
     if (a.dtype == 1)
-        mask_columns_kernel<float><<<g, 256, 0, s>>>((const float*)a.src, a.rows, a.d, a.ld_src, a.stride_src, a.I,
-                                                     a.I_stride, a.k, (float*)a.dst, a.ld_dst, a.stride_dst);
-    else
-        mask_columns_kernel<__nv_bfloat16><<<g, 256, 0, s>>>((const __nv_bfloat16*)a.src, a.rows, a.d, a.ld_src,
-                                                             a.stride_src, a.I, a.I_stride, a.k,
-                                                             (__nv_bfloat16*)a.dst, a.ld_dst, a.stride_dst);
-    return cudaGetLastError();
+        return launch_pdl(mask_columns_kernel<float>, g, dim3(256), 0, s, (const float*)a.src, a.rows, a.d, a.ld_src,
+                          a.stride_src, a.I, a.I_stride, a.k, (float*)a.dst, a.ld_dst, a.stride_dst);
+    return launch_pdl(mask_columns_kernel<__nv_bfloat16>, g, dim3(256), 0, s, (const __nv_bfloat16*)a.src, a.rows,
+                      a.d, a.ld_src, a.stride_src, a.I, a.I_stride, a.k, (__nv_bfloat16*)a.dst, a.ld_dst,
+                      a.stride_dst);
 }
 
 cudaError_t launch_pack_rows(const PackArgs& a, int num_sms, cudaStream_t s) {
@@ -242,14 +250,11 @@ cudaError_t launch_pack_rows(const PackArgs& a, int num_sms, cudaStream_t s) {
     if (a.k == 0 || a.rows == 0) return cudaSuccess;
     dim3 grid((unsigned)((a.k + kRowsPerCta - 1) / kRowsPerCta), (unsigned)a.heads);
     if (a.dtype == 1)
-        pack_rows_kernel<float><<<grid, 256, 0, s>>>((const float*)a.src, a.d, a.rows, a.ld_src, a.stride_src,
-                                                     a.group, a.I, a.I_stride, a.k, (float*)a.dst, a.ld_dst,
-                                                     a.stride_dst);
-    else
-        pack_rows_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            (const __nv_bfloat16*)a.src, a.d, a.rows, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k,
-            (__nv_bfloat16*)a.dst, a.ld_dst, a.stride_dst);
-    return cudaGetLastError();
+        return launch_pdl(pack_rows_kernel<float>, grid, dim3(256), 0, s, (const float*)a.src, a.d, a.rows, a.ld_src,
+                          a.stride_src, a.group, a.I, a.I_stride, a.k, (float*)a.dst, a.ld_dst, a.stride_dst);
+    return launch_pdl(pack_rows_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, (const __nv_bfloat16*)a.src, a.d,
+                      a.rows, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k, (__nv_bfloat16*)a.dst,
+                      a.ld_dst, a.stride_dst);
 }
 
 cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s) {
@@ -257,14 +262,12 @@ cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s) {
     dim3 grid((unsigned)((a.ld_dst + 31) / 32), (unsigned)((a.rows + 31) / 32), (unsigned)a.heads);
     if (grid.y == 0) return cudaSuccess;
     if (a.dtype == 1)
-        pack_rows_transposed_kernel<float><<<grid, 256, 0, s>>>(
-            (const float*)a.src, a.d, a.rows, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k,
-            (float*)a.dst, a.ld_dst, a.stride_dst);
-    else
-        pack_rows_transposed_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            (const __nv_bfloat16*)a.src, a.d, a.rows, a.ld_src, a.stride_src, a.group, a.I, a.I_stride,
-            a.k, (__nv_bfloat16*)a.dst, a.ld_dst, a.stride_dst);
-    return cudaGetLastError();
+        return launch_pdl(pack_rows_transposed_kernel<float>, grid, dim3(256), 0, s, (const float*)a.src, a.d,
+                          a.rows, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k, (float*)a.dst, a.ld_dst,
+                          a.stride_dst);
+    return launch_pdl(pack_rows_transposed_kernel<__nv_bfloat16>, grid, dim3(256), 0, s,
+                      (const __nv_bfloat16*)a.src, a.d, a.rows, a.ld_src, a.stride_src, a.group, a.I, a.I_stride,
+                      a.k, (__nv_bfloat16*)a.dst, a.ld_dst, a.stride_dst);
 }
 
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t s) {
@@ -272,27 +275,23 @@ cudaError_t launch_pack(const PackArgs& a, cudaStream_t s) {
         dim3 g((unsigned)((a.rows + kNarrowRows - 1) / kNarrowRows), (unsigned)a.heads);
         if (g.x == 0) return cudaSuccess;
         if (a.dtype == 1)
-            pack_narrow_kernel<float><<<g, 256, 0, s>>>((const float*)a.src, a.rows, a.d, a.ld_src, a.stride_src,
-                                                        a.group, a.I, a.I_stride, a.k, (float*)a.dst, a.ld_dst,
-                                                        a.stride_dst);
-        else
-            pack_narrow_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(
-                (const __nv_bfloat16*)a.src, a.rows, a.d, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k,
-                (__nv_bfloat16*)a.dst, a.ld_dst, a.stride_dst);
-        return cudaGetLastError();
+            return launch_pdl(pack_narrow_kernel<float>, g, dim3(256), 0, s, (const float*)a.src, a.rows, a.d,
+                              a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k, (float*)a.dst, a.ld_dst,
+                              a.stride_dst);
+        return launch_pdl(pack_narrow_kernel<__nv_bfloat16>, g, dim3(256), 0, s, (const __nv_bfloat16*)a.src, a.rows,
+                          a.d, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k, (__nv_bfloat16*)a.dst,
+                          a.ld_dst, a.stride_dst);
     }
     dim3 grid((unsigned)((a.ld_dst + 8 * kPackThreads - 1) / (8 * kPackThreads)),
               (unsigned)((a.rows + kPackRows - 1) / kPackRows), (unsigned)a.heads);
     if (grid.y == 0) return cudaSuccess;
     if (a.dtype == 1)
-        pack_kernel<float><<<grid, kPackThreads, 0, s>>>(
-            (const float*)a.src, a.rows, a.d, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k,
-            (float*)a.dst, a.ld_dst, a.stride_dst);
-    else
-        pack_kernel<__nv_bfloat16><<<grid, kPackThreads, 0, s>>>(
-            (const __nv_bfloat16*)a.src, a.rows, a.d, a.ld_src, a.stride_src, a.group, a.I,
-            a.I_stride, a.k, (__nv_bfloat16*)a.dst, a.ld_dst, a.stride_dst);
-    return cudaGetLastError();
+        return launch_pdl(pack_kernel<float>, grid, dim3(kPackThreads), 0, s, (const float*)a.src, a.rows, a.d,
+                          a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k, (float*)a.dst, a.ld_dst,
+                          a.stride_dst);
+    return launch_pdl(pack_kernel<__nv_bfloat16>, grid, dim3(kPackThreads), 0, s, (const __nv_bfloat16*)a.src, a.rows,
+                      a.d, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k, (__nv_bfloat16*)a.dst, a.ld_dst,
+                      a.stride_dst);
 }
 
 }  // namespace rmm

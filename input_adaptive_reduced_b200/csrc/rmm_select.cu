@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(32 * kColWarps) colnorm_kernel(const T* __rest
                                                       float* __restrict__ partials,
                                                       unsigned* __restrict__ counters,
                                                       float* __restrict__ s2) {
+    pdl_wait();
+    pdl_trigger();
     constexpr int V = Vec16<T>::N;
     constexpr int COLS = 32 * V;
     constexpr int U = 8;
@@ -276,6 +278,8 @@ __device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k
 // One 1024-thread CTA per head on the final scores written by colnorm.
 __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ scores, int64_t d, int64_t k,
                                                     int32_t* __restrict__ I) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ uint32_t keys[];
     __shared__ TopkShared sh;
     const int h = blockIdx.x;
@@ -302,6 +306,8 @@ __global__ void __launch_bounds__(1024) normselect_kernel(const T* __restrict__ 
                                                           int64_t d, int64_t lda, int64_t stride_a,
                                                           int rg, int64_t k, int32_t* __restrict__ I,
                                                           float* __restrict__ s2) {
+    pdl_wait();
+    pdl_trigger();
     constexpr int V = Vec16<T>::N;
     extern __shared__ uint32_t smem[];
     uint32_t* keys = smem;                                        // d
@@ -361,6 +367,8 @@ __global__ void __launch_bounds__(1024) normselect_kernel(const T* __restrict__ 
 }
 
 __global__ void identity_kernel(int32_t* __restrict__ I, int64_t k, int heads) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t total = k * heads;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
          i += (int64_t)gridDim.x * blockDim.x)
@@ -390,14 +398,10 @@ cudaError_t launch_colnorm(const SelectArgs& a, cudaStream_t s) {
     const int V = a.dtype == 1 ? 4 : 8;
     dim3 grid((unsigned)((a.d + 32 * V - 1) / (32 * V)), (unsigned)a.nsplit, (unsigned)a.heads);
     if (a.dtype == 1)
-        colnorm_kernel<float><<<grid, 32 * kColWarps, 0, s>>>((const float*)a.A, a.n, a.d, a.lda, a.stride_a,
-                                                   a.rows_per_split, a.nsplit, a.partials, a.counters,
-                                                   a.scores);
-    else
-        colnorm_kernel<__nv_bfloat16><<<grid, 32 * kColWarps, 0, s>>>((const __nv_bfloat16*)a.A, a.n, a.d,
-                                                           a.lda, a.stride_a, a.rows_per_split,
-                                                           a.nsplit, a.partials, a.counters, a.scores);
-    return cudaGetLastError();
+        return launch_pdl(colnorm_kernel<float>, grid, dim3(32 * kColWarps), 0, s, (const float*)a.A, a.n, a.d,
+                          a.lda, a.stride_a, a.rows_per_split, a.nsplit, a.partials, a.counters, a.scores);
+    return launch_pdl(colnorm_kernel<__nv_bfloat16>, grid, dim3(32 * kColWarps), 0, s, (const __nv_bfloat16*)a.A,
+                      a.n, a.d, a.lda, a.stride_a, a.rows_per_split, a.nsplit, a.partials, a.counters, a.scores);
 }
 
 cudaError_t launch_topk(const SelectArgs& a, cudaStream_t s) {
@@ -405,8 +409,7 @@ cudaError_t launch_topk(const SelectArgs& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    topk_kernel<<<a.heads, 1024, smem, s>>>(a.scores, a.d, a.k, a.I);
-    return cudaGetLastError();
+    return launch_pdl(topk_kernel, dim3(a.heads), dim3(1024), smem, s, (const float*)a.scores, a.d, a.k, a.I);
 }
 
 cudaError_t launch_normselect(const SelectArgs& a, cudaStream_t s) {
@@ -417,24 +420,23 @@ cudaError_t launch_normselect(const SelectArgs& a, cudaStream_t s) {
         e = cudaFuncSetAttribute(normselect_kernel<float>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        normselect_kernel<float><<<a.heads, 1024, smem, s>>>((const float*)a.A, a.n, a.d, a.lda,
-                                                             a.stride_a, rg, a.k, a.I, a.s2);
+        e = launch_pdl(normselect_kernel<float>, dim3(a.heads), dim3(1024), smem, s, (const float*)a.A, a.n, a.d,
+                       a.lda, a.stride_a, rg, a.k, a.I, a.s2);
     } else {
         e = cudaFuncSetAttribute(normselect_kernel<__nv_bfloat16>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        normselect_kernel<__nv_bfloat16><<<a.heads, 1024, smem, s>>>(
-            (const __nv_bfloat16*)a.A, a.n, a.d, a.lda, a.stride_a, rg, a.k, a.I, a.s2);
+        e = launch_pdl(normselect_kernel<__nv_bfloat16>, dim3(a.heads), dim3(1024), smem, s,
+                       (const __nv_bfloat16*)a.A, a.n, a.d, a.lda, a.stride_a, rg, a.k, a.I, a.s2);
     }
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_identity(int32_t* I, int64_t k, int heads, cudaStream_t s) {
     const int64_t total = k * heads;
     const int64_t want = (total + 255) / 256;
     const int blocks = (int)(want < 1024 ? (want > 0 ? want : 1) : 1024);
-    identity_kernel<<<blocks, 256, 0, s>>>(I, k, heads);
-    return cudaGetLastError();
+    return launch_pdl(identity_kernel, dim3(blocks), dim3(256), 0, s, I, k, heads);
 }
 
 }  // namespace rmm

@@ -90,6 +90,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    pdl_wait();  // everything above touched only shared and tensor memory
+    pdl_trigger();
     // this split's retained row indices, staged once (-1 past k)
     int32_t* sidx = reinterpret_cast<int32_t*>(smem + C::IDX_OFF);
     if (warp >= 6) {
@@ -216,6 +218,8 @@ template <int NP>
 __global__ void __launch_bounds__(256) skinny_reduce_kernel(const float* __restrict__ partials, int splits,
                                                             int n, int m, float alpha,
                                                             __nv_bfloat16* __restrict__ Y, int64_t ldy) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // over n x m, column fastest
     if (e >= (int64_t)n * m) return;
     const int i = (int)(e / m), c = (int)(e - (int64_t)i * m);
@@ -230,13 +234,11 @@ cudaError_t launch_np(const SkinnyParams& p, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(skinny_kernel<NP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::SMEM);
     if (e != cudaSuccess) return e;
-    skinny_kernel<NP><<<p.m_tiles * p.splits, kSkThreads, C::SMEM, s>>>(p);
-    e = cudaGetLastError();
+    e = launch_pdl(skinny_kernel<NP>, dim3(p.m_tiles * p.splits), dim3(kSkThreads), C::SMEM, s, p);
     if (e != cudaSuccess || p.splits == 1) return e;
     const int64_t total = (int64_t)p.n * p.m;
-    skinny_reduce_kernel<NP><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-        p.partials, p.splits, p.n, p.m, p.alpha, static_cast<__nv_bfloat16*>(p.Y), p.ldy);
-    return cudaGetLastError();
+    return launch_pdl(skinny_reduce_kernel<NP>, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, s, p.partials,
+                      p.splits, p.n, p.m, p.alpha, static_cast<__nv_bfloat16*>(p.Y), p.ldy);
 }
 
 }  // namespace

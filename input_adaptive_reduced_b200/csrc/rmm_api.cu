@@ -257,7 +257,7 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
     const bool qk_masked_path = p.mode == RMM_QK && !identity && p.d <= 1024;
     if (qk_masked_path) {
         // staged below together with B
-    } else if (!identity) {
+    } else if (!identity && !plan->pv_mask) {
         rmm::PackArgs pa{};
         pa.src = A;
         pa.dtype = p.dtype;
@@ -384,6 +384,32 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         if (!encode_kmajor_map(&gp.map_b, es, pb.dst, k, p.m, p.heads, plan->ldp, p.m * plan->ldp, box_k,
                                kmajor_box_rows))
             return RMM_ERR_CUDA;
+    } else if (plan->pv_mask) {
+        // V's rows outside each query head's T are zeroed in a per-head copy
+        // padded to whole K blocks; the product contracts over every token of P.
+        const int64_t d_pad = (p.d + 63) / 64 * 64;
+        rmm::PackArgs pb{};
+        pb.src = B;
+        pb.dtype = p.dtype;
+        pb.rows = p.m;
+        pb.d = p.d;
+        pb.ld_src = p.ldb;
+        pb.stride_src = p.stride_b;
+        pb.group = plan->group;
+        pb.I = I;
+        pb.I_stride = k;
+        pb.k = k;
+        pb.dst = ws_at<void>(ws, plan->off_bpack);
+        pb.ld_dst = p.m;
+        pb.stride_dst = d_pad * p.m;
+        pb.heads = static_cast<int>(p.heads);
+        if (rmm::launch_mask_rows(pb, d_pad, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        gl.b_mode = rmm::kBRows;
+        gp.k = static_cast<int32_t>(p.d);
+        gp.group = 1;
+        gp.b_head_rows = static_cast<int32_t>(d_pad);
+        gp.b_rows_total = static_cast<int32_t>(d_pad * p.heads);
+        if (!encode_rows_map(&gp.map_b, pb.dst, p.m, d_pad * p.heads, p.m, 64u)) return RMM_ERR_CUDA;
     } else if (!identity && plan->pack_b) {
         // The retained rows B[I, :] are copied into a contiguous k x m buffer per
         // head (a streaming copy at HBM rate), which the product then reads with
@@ -450,7 +476,7 @@ int32_t launches_per_call(const rmm_plan* plan) {
     if (!given && !identity) n += plan->fused_select ? 1 : 2;
     if (p.n == 0 || p.m == 0) return n;
     if (plan->skinny) return n + (identity ? 0 : 1) + 1 + (plan->sk_splits > 1 ? 1 : 0);
-    if (!identity) n += 1;                                   // pack A[:, I]
+    if (!identity) n += 1;                                   // pack A[:, I] (PV: mask V's rows instead)
     if (p.mode == RMM_QK && !identity && p.d > 1024) n += 1; // pack K[:, I] (else Q is masked in place of the A pack)
     if (p.mode != RMM_QK && p.dtype == RMM_F32) n += 1;      // B[I, :] transposed for tf32
     if (!identity && plan->pack_b) n += 1;                   // B[I, :] rows, contiguous
@@ -495,6 +521,10 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     plan->need_select = !given && plan->k < p->d;
     plan->bn = p->m <= 128 ? 128 : 256;
     plan->pack_b = p->mode != RMM_QK && p->dtype == RMM_BF16 && (plan->k < p->d || given);
+    // PV over short value heads is bound by reading P: instead of copying P's
+    // retained columns, zero V's unkept rows (per query head) and read P as is.
+    plan->pv_mask = p->mode == RMM_PV && p->dtype == RMM_BF16 && !given && plan->k < p->d && p->m <= 256;
+    if (plan->pv_mask) plan->pack_b = false;
     // Few rows: the op is a stream of B[I, :]; gather it inside a split-K
     // product with swapped operands instead of staging it.
     plan->skinny = p->mode == RMM_LINEAR && p->dtype == RMM_BF16 && p->heads == 1 && p->n >= 1 && p->n <= 64 &&
@@ -550,7 +580,7 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     plan->split_tiles = 0;
     plan->split_f = 1;
     if (!plan->skinny && p->n > 128 && p->m > 0 && !(p->flags & RMM_FLAG_CAUSAL)) {
-        const int64_t k_eff = (p->mode == RMM_QK && p->d <= 1024) ? p->d : plan->k;
+        const int64_t k_eff = ((p->mode == RMM_QK && p->d <= 1024) || plan->pv_mask) ? p->d : plan->k;
         const int64_t bk = 128 / plan->es;
         const int64_t tiles = p->heads * ((p->n + 255) / 256) * ((p->m + plan->bn - 1) / plan->bn);
         rmm::pair_split_tail(tiles, (k_eff + bk - 1) / bk, sms / 2, &plan->split_tiles, &plan->split_f);
@@ -569,7 +599,8 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     off += align256(static_cast<size_t>(p->heads) * plan->k * sizeof(int32_t));
     plan->off_apack = off;
     const bool qk_mask = p->mode == RMM_QK && p->d <= 1024;  // Q masked at full width, K used as is
-    off += align256(static_cast<size_t>(p->heads) * p->n * (qk_mask ? p->d : plan->ldp) * plan->es);
+    if (!plan->pv_mask)
+        off += align256(static_cast<size_t>(p->heads) * p->n * (qk_mask ? p->d : plan->ldp) * plan->es);
     plan->off_bpack = off;
     if (qk_mask) {
         // no staged B
@@ -577,6 +608,8 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
         off += align256(static_cast<size_t>(plan->sk_splits) * p->m * plan->sk_np * sizeof(float));
     else if (p->mode == RMM_QK || p->dtype == RMM_F32)
         off += align256(static_cast<size_t>(p->heads) * p->m * plan->ldp * plan->es);
+    else if (plan->pv_mask)
+        off += align256(static_cast<size_t>(p->heads) * ((p->d + 63) / 64 * 64) * p->m * plan->es);
     else if (plan->pack_b || given)
         off += align256(static_cast<size_t>(p->heads) * plan->k * p->m * plan->es);
     plan->off_split = off;

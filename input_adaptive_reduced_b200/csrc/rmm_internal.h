@@ -94,6 +94,11 @@ cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s);
 // dst[h][t][:] = src[h / group][I[h][t]][:] for t < k: the retained rows of a
 // row-major B, contiguous (a.rows = number of columns of B).
 cudaError_t launch_pack_rows(const PackArgs& a, int num_sms, cudaStream_t s);
+// dst[h][t][:] = src[h / group][t][:] if t is in I[h][0..k) (ascending, unique)
+// else 0, for t < rows_out (rows t >= a.d are zero); a.rows = columns of B.
+// Used for attention PV, where the product is bound by reading P and a
+// zero-masked V gives the same sum over I without a copy of P's columns.
+cudaError_t launch_mask_rows(const PackArgs& a, int64_t rows_out, cudaStream_t s);
 
 // ---------------------------------------------------------------- GEMM
 // How the B operand reaches shared memory (see rmm_gemm.cu).
@@ -187,6 +192,7 @@ struct rmm_plan {
     cudaEvent_t product_start, product_stop;  // tracing hook, may be null
     bool skinny;        // n <= 64 bf16 LINEAR: swapped-operand split-K product
     int sk_np, sk_splits;
+    bool pv_mask;       // bf16 PV with a selected T: V's unkept rows zeroed per query head, P read as stored
     int split_tiles, split_f;           // split tail of the CTA-pair product (0, 1: none)
     size_t off_split_cnt, off_split;    // its counters (in the header) and fp32 partials
 };

@@ -148,6 +148,50 @@ __global__ void __launch_bounds__(256) pack_rows_kernel(
     }
 }
 
+// Rows of B with the unkept ones zeroed, per query head: dst[h][t][:] =
+// src[h / group][t][:] if t is in I[h] (ascending, unique) else 0, for t <
+// rows_out (rows t >= d are zero).  grid (ceil(rows_out / 64), heads).  An
+// ascending set of unique indices in [0, d) has I[t] in [t, t + d - k], so the
+// indices that fall in rows [r0, r0 + 64) sit at positions [r0 - (d - k),
+// r0 + 64): the CTA scans that window with coalesced loads, marks its kept
+// rows, and reads only those.
+constexpr int kMaskRows = 64;
+
+template <typename T>
+__global__ void __launch_bounds__(256) mask_rows_kernel(
+    const T* __restrict__ src, int64_t d, int64_t cols, int64_t ld_src, int64_t stride_src, int group,
+    const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
+    int64_t stride_dst, int64_t rows_out) {
+    pdl_wait();
+    pdl_trigger();
+    constexpr int V = 16 / sizeof(T);
+    __shared__ int keep[kMaskRows];
+    const int h = blockIdx.y;
+    const int64_t r0 = (int64_t)blockIdx.x * kMaskRows;
+    const int32_t* Ih = I + (int64_t)h * I_stride;
+    if (threadIdx.x < kMaskRows) keep[threadIdx.x] = 0;
+    __syncthreads();
+    const int64_t t_beg = r0 - (d - k) > 0 ? r0 - (d - k) : 0;
+    const int64_t t_end = r0 + kMaskRows < k ? r0 + kMaskRows : k;
+    for (int64_t t = t_beg + threadIdx.x; t < t_end; t += 256) {
+        const int64_t j = __ldg(Ih + t);
+        if (j >= r0 && j < r0 + kMaskRows && j < d) keep[j - r0] = 1;
+    }
+    __syncthreads();
+    const int cpr = (int)(cols / V);
+    const int64_t left = rows_out - r0;
+    const int nrows = left < kMaskRows ? (int)left : kMaskRows;
+    const T* sh = src + (int64_t)(h / group) * stride_src;
+    T* dh = dst + (int64_t)h * stride_dst;
+    for (int idx = threadIdx.x; idx < nrows * cpr; idx += 256) {
+        const int r = idx / cpr;
+        const int c = idx - r * cpr;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (keep[r]) v = __ldg(reinterpret_cast<const uint4*>(sh + (r0 + r) * ld_src) + c);
+        *reinterpret_cast<uint4*>(dh + (r0 + r) * ld_dst + (int64_t)c * V) = v;
+    }
+}
+
 // Narrow variant (packed width <= kNarrowMax, e.g. attention heads with
 // d_h = 128): the CTA caches the head's indices in shared memory once and its
 // threads walk (row, 8-column chunk) pairs, so every thread has work.
@@ -255,6 +299,18 @@ cudaError_t launch_pack_rows(const PackArgs& a, int num_sms, cudaStream_t s) {
     return launch_pdl(pack_rows_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, (const __nv_bfloat16*)a.src, a.d,
                       a.rows, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k, (__nv_bfloat16*)a.dst,
                       a.ld_dst, a.stride_dst);
+}
+
+cudaError_t launch_mask_rows(const PackArgs& a, int64_t rows_out, cudaStream_t s) {
+    dim3 grid((unsigned)((rows_out + kMaskRows - 1) / kMaskRows), (unsigned)a.heads);
+    if (grid.x == 0 || a.rows == 0) return cudaSuccess;
+    if (a.dtype == 1)
+        return launch_pdl(mask_rows_kernel<float>, grid, dim3(256), 0, s, (const float*)a.src, a.d, a.rows, a.ld_src,
+                          a.stride_src, a.group, a.I, a.I_stride, a.k, (float*)a.dst, a.ld_dst, a.stride_dst,
+                          rows_out);
+    return launch_pdl(mask_rows_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, (const __nv_bfloat16*)a.src, a.d,
+                      a.rows, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k, (__nv_bfloat16*)a.dst,
+                      a.ld_dst, a.stride_dst, rows_out);
 }
 
 cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s) {

@@ -532,7 +532,7 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     if (plan->skinny) {
         plan->pack_b = false;
         plan->sk_np = rmm::skinny_pad(p->n);
-        plan->sk_splits = rmm::skinny_splits(p->m, plan->k, 0);  // fixed below once the SM count is known
+        plan->sk_splits = rmm::skinny_splits(p->m, plan->k, 0, plan->sk_np);  // fixed below once the SM count is known
     }
 
     int dev = 0, sms = 0;
@@ -543,7 +543,7 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
         return RMM_ERR_CUDA;
     }
     plan->num_sms = sms;
-    if (plan->skinny) plan->sk_splits = rmm::skinny_splits(p->m, plan->k, sms);
+    if (plan->skinny) plan->sk_splits = rmm::skinny_splits(p->m, plan->k, sms, plan->sk_np);
 
     // Selection kernels need every score of a head in shared memory.
     const bool select_possible = p->d <= rmm::kMaxSelectD;

@@ -161,13 +161,13 @@ struct __align__(64) SkinnyParams {
     const int32_t* I;       // [k] retained rows of B, nullptr = every row in order
     void* Y;                // n x m bf16
     int64_t ldy;
-    float* partials;        // [splits][m][np] fp32 when splits > 1
+    float* partials;        // [splits][np][m] fp32 when splits > 1
     float alpha;
     int32_t n, m, k, d, np, m_tiles, splits;
     int* err;
 };
 int skinny_pad(int64_t n);
-int skinny_splits(int64_t m, int64_t k, int num_sms);
+int skinny_splits(int64_t m, int64_t k, int num_sms, int np);
 cudaError_t launch_skinny(const SkinnyParams& p, cudaStream_t s);
 
 }  // namespace rmm

@@ -27,19 +27,20 @@ namespace rmm {
 namespace {
 
 constexpr int kSkThreads = 448;
-constexpr int kSkStages = 6;
 constexpr int kSkBK = 64;                     // bf16 K per stage (one 128-byte row)
 constexpr int kSkGatherBytes = kSkBK * 256;   // 64 rows x 128 columns x 2 B
 constexpr int kSkGroupBytes = kSkBK * 128;    // one 64-column group
 
-constexpr int kSkMaxSplitIdx = 8192;          // indices of one split staged in shared memory
+constexpr int kSkMaxSplitIdx = 4096;          // indices of one split staged in shared memory
 
 template <int NP>
 struct SkCfg {
     static constexpr int A_BYTES = NP * 128;  // the A[:, I] tile: NP rows x 128 B
     static constexpr int STAGE_BYTES = kSkGatherBytes + A_BYTES;
+    // two CTAs per SM (16 gather warps per SM): 4 stages, 3 when NP = 64
+    static constexpr int STAGES = NP == 64 ? 3 : 4;
     static constexpr int TMEM_COLS = NP < 32 ? 32 : NP;
-    static constexpr size_t IDX_OFF = (size_t)kSkStages * STAGE_BYTES + 256;
+    static constexpr size_t IDX_OFF = (size_t)STAGES * STAGE_BYTES + 256;
     static constexpr size_t SMEM = 1024 + IDX_OFF + kSkMaxSplitIdx * 4;
 };
 
@@ -54,13 +55,13 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 }
 
 template <int NP>
-__global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_constant__ SkinnyParams p) {
+__global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(const __grid_constant__ SkinnyParams p) {
     using C = SkCfg<NP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kSkStages * C::STAGE_BYTES);
-    uint64_t* empty = full + kSkStages;
-    uint64_t* tfull = empty + kSkStages;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+    uint64_t* empty = full + C::STAGES;
+    uint64_t* tfull = empty + C::STAGES;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tfull + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -73,7 +74,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
     const int kb_end = (int)((int64_t)nkb * (split + 1) / p.splits);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kSkStages; ++s) {
+        for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1 + 256);  // expect_tx arrival + 256 cp.async arrivals
             mbar_init(&empty[s], 1);
         }
@@ -112,8 +113,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
     if (warp == 0) {
         if (lane == 0) {
             for (int kb = kb_beg, it = 0; kb < kb_end; ++kb, ++it) {
-                const int s = it % kSkStages;
-                const uint32_t ph = (it / kSkStages) & 1u;
+                const int s = it % C::STAGES;
+                const uint32_t ph = (it / C::STAGES) & 1u;
                 if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err, kErrTimeoutProducer)) break;
                 uint8_t* sa = smem + s * C::STAGE_BYTES + kSkGatherBytes;
                 mbar_arrive_expect_tx(&full[s], C::A_BYTES);
@@ -127,8 +128,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
                                        ((uint32_t)(NP >> 3) << 17) | ((128u >> 4) << 24);
             bool ok = true;
             for (int kb = kb_beg, it = 0; kb < kb_end; ++kb, ++it) {
-                const int s = it % kSkStages;
-                const uint32_t ph = (it / kSkStages) & 1u;
+                const int s = it % C::STAGES;
+                const uint32_t ph = (it / C::STAGES) & 1u;
                 if (!mbar_wait(&full[s], ph, abort_flag, p.err, kErrTimeoutMma)) {
                     ok = false;
                     break;
@@ -154,26 +155,30 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
         const bool any_k = kb_end > kb_beg;
         if (!any_k || mbar_wait(tfull, 0, abort_flag, p.err, kErrTimeoutEpilogue)) {
             tc_fence_after();
-            float acc[NP];
-#pragma unroll
+            // 16 tokens at a time: TMEM columns c16*16 .. +15 of this lane's row
+#pragma unroll 1
             for (int c16 = 0; c16 < NP / 16; ++c16) {
                 uint32_t raw[16];
                 tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + c16 * 16, raw);
                 tmem_ld_wait();
+                if (col < p.m) {
+                    if (p.splits == 1) {
+                        __nv_bfloat16* Y = static_cast<__nv_bfloat16*>(p.Y);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) acc[c16 * 16 + i] = any_k ? __uint_as_float(raw[i]) : 0.f;
-            }
-            if (col < p.m) {
-                if (p.splits == 1) {
-                    __nv_bfloat16* Y = static_cast<__nv_bfloat16*>(p.Y);
+                        for (int i = 0; i < 16; ++i) {
+                            const int tok = c16 * 16 + i;
+                            const float v = any_k ? __uint_as_float(raw[i]) : 0.f;
+                            if (tok < p.n) Y[(int64_t)tok * p.ldy + col] = __float2bfloat16_rn(v * p.alpha);
+                        }
+                    } else {
+                        // [split][token][column]: a warp's lanes write consecutive columns
+                        float* dst = p.partials + (int64_t)split * NP * p.m + col;
 #pragma unroll
-                    for (int i = 0; i < NP; ++i)
-                        if (i < p.n) Y[(int64_t)i * p.ldy + col] = __float2bfloat16_rn(acc[i] * p.alpha);
-                } else {
-                    float4* dst = reinterpret_cast<float4*>(p.partials + ((int64_t)split * p.m + col) * NP);
-#pragma unroll
-                    for (int i = 0; i < NP / 4; ++i)
-                        dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+                        for (int i = 0; i < 16; ++i) {
+                            const int tok = c16 * 16 + i;
+                            if (tok < p.n) __stcg(dst + (int64_t)tok * p.m, any_k ? __uint_as_float(raw[i]) : 0.f);
+                        }
+                    }
                 }
             }
         }
@@ -183,8 +188,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) skinny_kernel(const __grid_cons
         const int ptid = threadIdx.x - 6 * 32;
         const __nv_bfloat16* B = static_cast<const __nv_bfloat16*>(p.B);
         for (int kb = kb_beg, it = 0; kb < kb_end; ++kb, ++it) {
-            const int s = it % kSkStages;
-            const uint32_t ph = (it / kSkStages) & 1u;
+            const int s = it % C::STAGES;
+            const uint32_t ph = (it / C::STAGES) & 1u;
             int32_t rowj[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) rowj[i] = sidx[it * kSkBK + (ptid >> 4) + 16 * i];
@@ -224,7 +229,7 @@ __global__ void __launch_bounds__(256) skinny_reduce_kernel(const float* __restr
     if (e >= (int64_t)n * m) return;
     const int i = (int)(e / m), c = (int)(e - (int64_t)i * m);
     float sum = 0.f;
-    for (int s = 0; s < splits; ++s) sum += __ldcg(partials + ((int64_t)s * m + c) * NP + i);
+    for (int s = 0; s < splits; ++s) sum += __ldcg(partials + ((int64_t)s * NP + i) * m + c);
     Y[(int64_t)i * ldy + c] = __float2bfloat16_rn(sum * alpha);
 }
 
@@ -245,15 +250,29 @@ cudaError_t launch_np(const SkinnyParams& p, cudaStream_t s) {
 
 int skinny_pad(int64_t n) { return n <= 16 ? 16 : (n <= 32 ? 32 : 64); }
 
-int skinny_splits(int64_t m, int64_t k, int num_sms) {
+int skinny_splits(int64_t m, int64_t k, int num_sms, int np) {
     const int64_t m_tiles = (m + 127) / 128;
     const int64_t nkb = (k + kSkBK - 1) / kSkBK;
-    int64_t s = (2LL * num_sms + m_tiles - 1) / m_tiles;
-    const int64_t min_s = (nkb * kSkBK + kSkMaxSplitIdx - kSkBK - 1) / (kSkMaxSplitIdx - kSkBK);
-    if (s < min_s) s = min_s;  // each split's indices fit the shared staging area
-    if (s > nkb) s = nkb;
-    if (s > 64) s = 64;
-    return s < 1 ? 1 : (int)s;
+    int64_t lo = (nkb * kSkBK + kSkMaxSplitIdx - kSkBK - 1) / (kSkMaxSplitIdx - kSkBK);
+    if (lo < 1) lo = 1;  // each split's indices fit the shared staging area
+    int64_t hi = nkb < 64 ? nkb : 64;
+    if (hi < lo) hi = lo;
+    if (num_sms <= 0) return (int)lo;
+    // Time in k-block units.  Two CTAs share an SM's bandwidth, so an SM's
+    // time follows the number of CTAs it runs: ceil(CTAs / SMs) times one
+    // CTA's share of K plus a fixed cost (prologue, pipeline fill, partials).
+    const int64_t slots = num_sms;
+    const int64_t fixed = 4 + np / 16;
+    int64_t best = lo, best_cost = -1;
+    for (int64_t sp = lo; sp <= hi; ++sp) {
+        const int64_t waves = (m_tiles * sp + slots - 1) / slots;
+        const int64_t cost = waves * ((nkb + sp - 1) / sp + fixed);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = sp;
+        }
+    }
+    return (int)best;
 }
 
 cudaError_t launch_skinny(const SkinnyParams& p, cudaStream_t s) {

@@ -489,7 +489,19 @@ def run_sweep(args):
     stream = torch.cuda.current_stream(dev)
     peak_tf, _, peak_gbs, _ = load_peaks()
     out = open(args.sweep_out, "w") if args.sweep_out else None
-    write_gbs = write_bandwidth(dev, stream)
+    # --sweep-only "cfg:op:n[:rho],...": run only the matching points
+    only = [tuple(x.split(":")) for x in args.sweep_only.split(",")] if args.sweep_only else None
+
+    def want(cfg, op, n, rho=None):
+        if only is None:
+            return True
+        for sel in only:
+            if (sel[0] == str(cfg) and (len(sel) < 2 or sel[1] == op) and (len(sel) < 3 or sel[2] == str(n))
+                    and (rho is None or len(sel) < 4 or abs(float(sel[3]) - rho) < 1e-9)):
+                return True
+        return False
+
+    write_gbs = write_bandwidth(dev, stream) if any(want(3, "qk", n) for n in (1024, 2048, 4096)) else None
 
     def lat(fn, iters=20):
         for _ in range(3):
@@ -515,6 +527,8 @@ def run_sweep(args):
         m = B.shape[1]
         t_dense = lat(lambda: torch.matmul(A, B))
         for rho in rhos:
+            if not want(cfg, name, n, rho):
+                continue
             k = retained(rho, d)
             t = lat(lambda: rmm.matmul(A, B, rho=rho))
             flops = 2.0 * n * k * m
@@ -526,20 +540,27 @@ def run_sweep(args):
                   "bound": bound, "frac": frac, "ms_dense_cublas": t_dense})
 
     # 1: tiny fp32
-    A, B = W.linear_small(1, device=dev)
-    linear_points(1, "fp32 64x256x256", A, B, [0.25, 0.5, 1.0])
+    if want(1, "fp32", 64):
+        A, B = W.linear_small(1, device=dev)
+        linear_points(1, "fp32", A, B, [0.25, 0.5, 1.0])
     # 2: Llama-3.1-8B MLP
     for n in (1024, 2048, 4096):
         for name, gen in (("up", W.mlp_up), ("down", W.mlp_down)):
+            if not want(2, name, n):
+                continue
             A, B = gen(1, n=n, device=dev)
             linear_points(2, name, A, B, [0.5, 0.7, 0.8, 1.0])
             del A, B
     # 3: QK^T, 32 heads / 8 KV heads, d_h = 128, causal
     for n in (1024, 2048, 4096):
+        if not want(3, "qk", n):
+            continue
         Q, K = W.attn_qk(1, n=n, device=dev)
         Kt = K.repeat_interleave(4, dim=0).transpose(1, 2)
         t_dense = lat(lambda: torch.matmul(Q, Kt))
         for rho in (0.5, 0.8, 1.0):
+            if not want(3, "qk", n, rho):
+                continue
             k = retained(rho, 128)
             t = lat(lambda: rmm.qk(Q, K, rho=rho, causal=True))
             flops = 2.0 * n * k * n * 32
@@ -555,10 +576,14 @@ def run_sweep(args):
         del Q, K, Kt
     # 4: PV, token selection
     for n in (2048, 4096):
+        if not want(4, "pv", n):
+            continue
         P, V = W.attn_pv(1, n=n, device=dev)
         Vr = V.repeat_interleave(4, dim=0)
         t_dense = lat(lambda: torch.matmul(P, Vr))
         for rho in (0.5, 0.8, 1.0):
+            if not want(4, "pv", n, rho):
+                continue
             k = retained(rho, n)
             t = lat(lambda: rmm.pv(P, V, rho=rho))
             flops = 2.0 * n * k * 128 * 32
@@ -570,6 +595,8 @@ def run_sweep(args):
     # 5: Llama-3-70B linear
     for shape in ("up", "down", "qkv"):
         for n in (1, 16, 512, 2048, 4096):
+            if not want(5, shape, n):
+                continue
             A, B = W.linear_70b(1, n=n, shape=shape, device=dev)
             linear_points(5, shape, A, B, [0.5, 0.6, 0.7, 0.8, 1.0])
             del A, B
@@ -591,6 +618,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="time every point of the five workloads")
     ap.add_argument("--sweep-out", default=None)
+    ap.add_argument("--sweep-only", default=None,
+                    help='comma-separated "config:op:n[:rho]" points, e.g. "5:down:16:0.8,3:qk:4096"')
     args = ap.parse_args(argv)
     if args.sweep:
         return run_sweep(args)

@@ -140,10 +140,11 @@ __global__ void __launch_bounds__(32 * kColWarps) colnorm_kernel(const T* __rest
 }
 
 // ------------------------------------------------------------------ TopK core
-// Works on keys[0..d) in shared memory (fp32 bit patterns of s^2 >= 0) with a
-// 1024-thread block.  Three radix passes over bits [31:21], [20:10] and [9:0]
-// find the exact k-th largest key T and how many keys equal to T are kept;
-// then the indices are emitted in ascending order.
+// Works on keys[0..d) in shared memory (fp32 bit patterns of s^2 >= 0; d a
+// multiple of 4, 16-byte aligned) with a 1024-thread block.  Three radix
+// passes over bits [31:21], [20:10] and [9:0] find the exact k-th largest key
+// T and how many keys equal to T are kept; then the indices are emitted in
+// ascending order.  Every pass reads four keys per 16-byte shared load.
 constexpr int kSubHist = 4;  // warps w, w+4, ... share a histogram copy: 4x less atomic contention
 
 struct TopkShared {
@@ -157,24 +158,48 @@ struct TopkShared {
     uint32_t sel_before[32];
 };
 
-__device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k, int32_t* out,
-                                      TopkShared& sh) {
+__device__ __forceinline__ void hist_clear(TopkShared& sh) {
+    for (int b = threadIdx.x; b < kSubHist * 2048; b += 1024) (&sh.hist[0][0])[b] = 0;
+}
+
+__device__ __forceinline__ void hist_add(uint32_t* myhist, uint32_t key, uint32_t mask, uint32_t prefix, int shift,
+                                         uint32_t bins) {
+    if ((key & mask) == prefix) atomicAdd(&myhist[(key >> shift) & (bins - 1)], 1u);
+}
+
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += y;
+    }
+    return v;
+}
+
+// first_done: the sub-histograms already hold the first pass over all keys.
+__device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k, int32_t* out, TopkShared& sh,
+                                      bool first_done) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint4* keys4 = reinterpret_cast<const uint4*>(keys);
+    const int64_t d4 = d >> 2;
     uint32_t prefix = 0, mask = 0, remaining = (uint32_t)k;
-    const int shifts[3] = {21, 10, 0};
-    const int widths[3] = {11, 11, 10};
 #pragma unroll 1
     for (int pass = 0; pass < 3; ++pass) {
-        const int shift = shifts[pass];
-        const int nb = 1 << widths[pass];
-        for (int b = tid; b < kSubHist * 2048; b += 1024) (&sh.hist[0][0])[b] = 0;
-        __syncthreads();
-        uint32_t* myhist = sh.hist[warp & (kSubHist - 1)];
-        for (int64_t j = tid; j < d; j += 1024) {
-            const uint32_t key = keys[j];
-            if ((key & mask) == prefix) atomicAdd(&myhist[(key >> shift) & (uint32_t)(nb - 1)], 1u);
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);  // bits [31:21], [20:10], [9:0]
+        const int nb = pass == 2 ? 1024 : 2048;
+        if (pass > 0 || !first_done) {
+            hist_clear(sh);
+            __syncthreads();
+            uint32_t* myhist = sh.hist[warp & (kSubHist - 1)];
+            for (int64_t q = tid; q < d4; q += 1024) {
+                const uint4 v = keys4[q];
+                hist_add(myhist, v.x, mask, prefix, shift, (uint32_t)nb);
+                hist_add(myhist, v.y, mask, prefix, shift, (uint32_t)nb);
+                hist_add(myhist, v.z, mask, prefix, shift, (uint32_t)nb);
+                hist_add(myhist, v.w, mask, prefix, shift, (uint32_t)nb);
+            }
+            __syncthreads();
         }
-        __syncthreads();
         // thread t owns bins nb-1-2t and nb-2-2t: a block scan in descending bin order
         const int b_hi = nb - 1 - 2 * tid, b_lo = b_hi - 1;
         uint32_t c0 = 0, c1 = 0;
@@ -184,23 +209,12 @@ __device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k
             if (b_lo >= 0) c1 += sh.hist[c][b_lo];
         }
         const uint32_t tot = c0 + c1;
-        uint32_t incl = tot;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += y;
-        }
+        const uint32_t incl = warp_incl_scan(tot, lane);
         if (lane == 31) sh.warp_tot[warp] = incl;
         __syncthreads();
         if (warp == 0) {
             const uint32_t w = sh.warp_tot[lane];
-            uint32_t wi = w;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xffffffffu, wi, off);
-                if (lane >= off) wi += y;
-            }
-            sh.warp_tot[lane] = wi - w;  // exclusive prefix of the warp totals
+            sh.warp_tot[lane] = warp_incl_scan(w, lane) - w;  // exclusive prefix of the warp totals
         }
         __syncthreads();
         const uint32_t excl = sh.warp_tot[warp] + incl - tot;
@@ -219,17 +233,22 @@ __device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k
     const uint32_t T = prefix;      // the k-th largest key
     const uint32_t r = remaining;   // how many keys equal to T are kept (lowest indices)
 
-    // Each warp owns a contiguous segment; count, scan over warps, then emit.
-    const int64_t seg = ((d + 31) / 32 + 31) / 32 * 32;
+    // Each warp owns a contiguous segment (a multiple of 128 keys).  It counts
+    // four keys per lane and step, and emits 32 keys per step in order.
+    const int64_t seg = ((d + 31) / 32 + 127) / 128 * 128;
     const int64_t beg = (int64_t)warp * seg;
     const int64_t end = min(d, beg + seg);
     uint32_t gt = 0, eq = 0;
-    for (int64_t j0 = beg; j0 < end; j0 += 32) {
-        const int64_t j = j0 + lane;
-        const uint32_t key = j < end ? keys[j] : 0u;
-        gt += __popc(__ballot_sync(0xffffffffu, j < end && key > T));
-        eq += __popc(__ballot_sync(0xffffffffu, j < end && key == T));
+    for (int64_t j0 = beg; j0 < end; j0 += 128) {
+        const int64_t j = j0 + 4 * lane;
+        if (j < end) {  // end is a multiple of 4: all four keys are in range
+            const uint4 v = keys4[j >> 2];
+            gt += (v.x > T) + (v.y > T) + (v.z > T) + (v.w > T);
+            eq += (v.x == T) + (v.y == T) + (v.z == T) + (v.w == T);
+        }
     }
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    eq = __reduce_add_sync(0xffffffffu, eq);
     if (lane == 0) {
         sh.warp_gt[warp] = gt;
         sh.warp_eq[warp] = eq;
@@ -237,23 +256,11 @@ __device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k
     __syncthreads();
     if (warp == 0) {
         const uint32_t e = sh.warp_eq[lane], g = sh.warp_gt[lane];
-        uint32_t incl = e;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += y;
-        }
-        const uint32_t eb = incl - e;
+        const uint32_t eb = warp_incl_scan(e, lane) - e;
         const uint32_t take_eq = eb >= r ? 0u : min(e, r - eb);
         const uint32_t sel = g + take_eq;
-        uint32_t sincl = sel;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, sincl, off);
-            if (lane >= off) sincl += y;
-        }
         sh.eq_before[lane] = eb;
-        sh.sel_before[lane] = sincl - sel;
+        sh.sel_before[lane] = warp_incl_scan(sel, lane) - sel;
     }
     __syncthreads();
     uint32_t eq_run = sh.eq_before[warp], sel_run = sh.sel_before[warp];
@@ -275,7 +282,9 @@ __device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k
 }
 
 // ------------------------------------------------------------------ TopK
-// One 1024-thread CTA per head on the final scores written by colnorm.
+// One 1024-thread CTA per head on the final scores written by colnorm (d a
+// multiple of 4): 16-byte loads, the first radix histogram built on the way
+// into shared memory.
 __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ scores, int64_t d, int64_t k,
                                                     int32_t* __restrict__ I) {
     pdl_wait();
@@ -283,18 +292,31 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
     extern __shared__ uint32_t keys[];
     __shared__ TopkShared sh;
     const int h = blockIdx.x;
-    const float* p = scores + (int64_t)h * d;
-    // eight independent loads in flight per thread (the scores come from L2)
-    for (int64_t j0 = threadIdx.x; j0 < d; j0 += 8 * 1024) {
-        float v[8];
+    const float4* p = reinterpret_cast<const float4*>(scores + (int64_t)h * d);
+    uint4* keys4 = reinterpret_cast<uint4*>(keys);
+    hist_clear(sh);
+    __syncthreads();
+    uint32_t* myhist = sh.hist[(threadIdx.x >> 5) & (kSubHist - 1)];
+    const int64_t d4 = d >> 2;
+    // four independent 16-byte loads in flight per thread (the scores come from L2)
+    for (int64_t q0 = threadIdx.x; q0 < d4; q0 += 4 * 1024) {
+        float4 v[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = j0 + u * 1024 < d ? __ldcg(p + j0 + u * 1024) : 0.f;
+        for (int u = 0; u < 4; ++u) v[u] = q0 + u * 1024 < d4 ? __ldcg(p + q0 + u * 1024) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-            if (j0 + u * 1024 < d) keys[j0 + u * 1024] = __float_as_uint(v[u]);
+        for (int u = 0; u < 4; ++u)
+            if (q0 + u * 1024 < d4) {
+                const uint4 w = make_uint4(__float_as_uint(v[u].x), __float_as_uint(v[u].y), __float_as_uint(v[u].z),
+                                           __float_as_uint(v[u].w));
+                keys4[q0 + u * 1024] = w;
+                atomicAdd(&myhist[w.x >> 21], 1u);
+                atomicAdd(&myhist[w.y >> 21], 1u);
+                atomicAdd(&myhist[w.z >> 21], 1u);
+                atomicAdd(&myhist[w.w >> 21], 1u);
+            }
     }
     __syncthreads();
-    radix_select_and_emit(keys, d, k, I + (int64_t)h * k, sh);
+    radix_select_and_emit(keys, d, k, I + (int64_t)h * k, sh, true);
 }
 
 // ------------------------------------------------------------------ fused
@@ -363,7 +385,7 @@ __global__ void __launch_bounds__(1024) normselect_kernel(const T* __restrict__ 
     if (s2) {
         for (int64_t j = threadIdx.x; j < d; j += 1024) s2[(int64_t)h * d + j] = __uint_as_float(keys[j]);
     }
-    radix_select_and_emit(keys, d, k, I + (int64_t)h * k, sh);
+    radix_select_and_emit(keys, d, k, I + (int64_t)h * k, sh, false);
 }
 
 __global__ void identity_kernel(int32_t* __restrict__ I, int64_t k, int heads) {

@@ -214,6 +214,62 @@ def test_split_tail_pv(rmm):
     rmm.check_workspaces()
 
 
+def test_cuda_graph_capture(rmm):
+    """Every kernel is launched with programmatic serialisation and the ops never
+    synchronise with the host: a CUDA graph of linear (CTA-pair product with a
+    split tail, and the small-n product), QK and PV calls replays to the same bits
+    as the eager calls."""
+    dev = torch.device("cuda")
+    s = torch.cuda.Stream()
+    cases = []
+    A, B = W.mlp_up(51, n=300, d=4096, m=704)
+    cases.append((rmm.RMM_LINEAR, A.to(dev), B.to(dev), 300, 4096, 704, 1, 1, 0.6))
+    A, B = W.mlp_down(52, n=16, d=4096, m=264)
+    cases.append((rmm.RMM_LINEAR, A.to(dev), B.to(dev), 16, 4096, 264, 1, 1, 0.7))
+    Q, K = W.attn_qk(53, n=200, heads=4, kv_heads=2, head_dim=128)
+    cases.append((rmm.RMM_QK, Q.to(dev), K.to(dev), 200, 128, 200, 4, 2, 0.5))
+    P, V = W.attn_pv(54, n=264, heads=4, kv_heads=2)
+    cases.append((rmm.RMM_PV, P.to(dev), V.to(dev), 264, 264, 128, 4, 2, 0.8))
+    runs = []
+    for mode, X, Z, n, d, m, H, Hkv, rho in cases:
+        p = rmm.rmm_problem_init(mode, rmm.RMM_BF16, n, d, m)
+        p.rho = rho
+        if H > 1:
+            p.heads, p.kv_heads = H, Hkv
+            p.stride_a, p.stride_b = X.stride(0), Z.stride(0)
+            p.ldy, p.stride_y = m, n * m
+        if mode == rmm.RMM_QK:
+            p.alpha = 1.0 / math.sqrt(d)
+            p.flags = rmm.RMM_FLAG_CAUSAL
+        plan = rmm.Plan(p)
+        ws = rmm.workspace_for(plan, dev, s)
+        Y = torch.empty((H, n, m) if H > 1 else (n, m), dtype=torch.bfloat16, device=dev)
+        I = torch.empty((H, plan.k) if H > 1 else (plan.k,), dtype=torch.int32, device=dev)
+        runs.append((plan, X, Z, Y, I, ws))
+    call = lambda r: rmm.rmm_matmul_batched(r[0], r[1], r[2], r[3], r[4], r[5], s)
+    with torch.cuda.stream(s):
+        for r in runs:
+            call(r)
+    torch.cuda.synchronize()
+    eager = [(r[3].clone(), r[4].clone()) for r in runs]
+    for r in runs:
+        r[3].zero_()
+        r[4].zero_()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for r in runs:
+            call(r)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    for (Ye, Ie), r in zip(eager, runs):
+        assert torch.equal(r[4], Ie)
+        assert torch.equal(r[3], Ye)
+    rmm.check_workspaces()
+    del g
+
+
 def _qk_check(rmm, Q, K, rho, causal):
     H, n, dh = Q.shape
     alpha = 1.0 / math.sqrt(dh)

@@ -581,16 +581,20 @@ def run_sweep(args):
         P, V = W.attn_pv(1, n=n, device=dev)
         Vr = V.repeat_interleave(4, dim=0)
         t_dense = lat(lambda: torch.matmul(P, Vr))
-        for rho in (0.5, 0.8, 1.0):
-            if not want(4, "pv", n, rho):
-                continue
-            k = retained(rho, n)
-            t = lat(lambda: rmm.pv(P, V, rho=rho))
-            flops = 2.0 * n * k * 128 * 32
-            hbm = 32 * (2.0 * n * n + 2.0 * k * 128 + 2.0 * n * 128)  # P once, V rows, O
-            emit({"config": 4, "op": "pv", "n": n, "rho": rho, "k": k, "ms": t,
-                  "useful_tflops": flops / (t * 1e-3) / 1e12, "gbs": hbm / (t * 1e-3) / 1e9,
-                  "bound": "hbm", "frac": hbm / (t * 1e-3) / 1e9 / peak_gbs, "ms_dense_torch": t_dense})
+        # P is a causal softmax: "pv" states it (RMM_FLAG_CAUSAL, the blocks above the
+        # diagonal are skipped); "pv_nocausal" reads all of P
+        for op, causal in (("pv", True), ("pv_nocausal", False)):
+            for rho in (0.5, 0.8, 1.0):
+                if not want(4, op, n, rho):
+                    continue
+                k = retained(rho, n)
+                t = lat(lambda: rmm.pv(P, V, rho=rho, causal=causal))
+                flops = 2.0 * n * k * 128 * 32
+                p_bytes = 2.0 * n * (n + 1) / 2 if causal else 2.0 * n * n  # P's nonzero part once
+                hbm = 32 * (p_bytes + 2.0 * k * 128 + 2.0 * n * 128)  # P once, V rows, O
+                emit({"config": 4, "op": op, "n": n, "rho": rho, "k": k, "ms": t,
+                      "useful_tflops": flops / (t * 1e-3) / 1e12, "gbs": hbm / (t * 1e-3) / 1e9,
+                      "bound": "hbm", "frac": hbm / (t * 1e-3) / 1e9 / peak_gbs, "ms_dense_torch": t_dense})
         del P, V, Vr
     # 5: Llama-3-70B linear
     for shape in ("up", "down", "qkv"):

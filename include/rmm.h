@@ -84,7 +84,12 @@ typedef enum rmm_mode {
     RMM_PV = 2
 } rmm_mode;
 
-/* Causal mask on the QK output: S[i][c] = -inf for c > i. */
+/* Causal structure.  QK: the output is masked, S[i][c] = -inf for c > i.
+   PV (n = d, query i is token i): the caller guarantees P[h][i][t] = 0 for
+   t > i, as a causal softmax leaves it; the op then skips the blocks of P that
+   lie entirely above the diagonal when it forms the token scores and the
+   product, which gives the same result as reading them.  Other modes:
+   RMM_ERR_INVALID_ARG. */
 #define RMM_FLAG_CAUSAL 1u
 /* rmm_matmul*: take I from the caller (I_inout, [heads][k], ascending,
    distinct, each in [0, d)) instead of computing it; no scores are formed. */

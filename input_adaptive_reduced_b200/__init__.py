@@ -378,9 +378,11 @@ def qk(Q, K, rho, alpha=None, causal=True, return_indices=False):
     return (S, I) if return_indices else S
 
 
-def pv(P, V, rho, return_indices=False):
+def pv(P, V, rho, return_indices=False, causal=False):
     """Token-reduced value product O[h] = P[h][:, T_h] V[g][T_h, :] for
-    P [H, n, n_k] and V [H_kv, n_k, d_v] (§3.3 "Attention", last sentence)."""
+    P [H, n, n_k] and V [H_kv, n_k, d_v] (§3.3 "Attention", last sentence).
+    causal=True states that P[h][i][t] = 0 for t > i (n = n_k): the op then
+    skips the blocks of P above the diagonal (same result)."""
     import torch
     _require_cuda(P, V)
     H, n, nk = P.shape
@@ -389,6 +391,7 @@ def pv(P, V, rho, return_indices=False):
     p.lda, p.ldb = _row_stride(P), _row_stride(V)
     p.heads, p.kv_heads = H, Hkv
     p.stride_a, p.stride_b = P.stride(0), V.stride(0)
+    p.flags = RMM_FLAG_CAUSAL if causal else 0
     _k_fields(p, rho, None)
     O = torch.empty((H, n, dv), dtype=P.dtype, device=P.device)
     p.ldy, p.stride_y = dv, n * dv

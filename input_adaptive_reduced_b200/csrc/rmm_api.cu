@@ -127,7 +127,8 @@ rmm_status validate_problem(const rmm_problem* p) {
         return RMM_ERR_INVALID_ARG;
     }
     if (p->flags & ~(RMM_FLAG_CAUSAL | RMM_FLAG_USE_GIVEN_INDICES)) return RMM_ERR_INVALID_ARG;
-    if ((p->flags & RMM_FLAG_CAUSAL) && p->mode != RMM_QK) return RMM_ERR_INVALID_ARG;
+    if ((p->flags & RMM_FLAG_CAUSAL) && !(p->mode == RMM_QK || (p->mode == RMM_PV && p->n == p->d)))
+        return RMM_ERR_INVALID_ARG;
     if (!std::isfinite(p->alpha)) return RMM_ERR_INVALID_ARG;
     return RMM_OK;
 }
@@ -166,6 +167,8 @@ rmm_status run_select(const rmm_plan* plan, const void* A, int32_t* I, float* s2
         a.scores = s2 ? s2 : ws_at<float>(ws, plan->off_scores);
         a.nsplit = plan->nsplit;
         a.rows_per_split = plan->rows_per_split;
+        // PV over a causal P: rows above a column block are zero there
+        a.causal_rows = p.mode == RMM_PV && (p.flags & RMM_FLAG_CAUSAL) ? 1 : 0;
         e = rmm::launch_colnorm(a, stream);
         if (e == cudaSuccess) e = rmm::launch_topk(a, stream);
     }
@@ -301,7 +304,10 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
 
     gp.n_tiles = static_cast<int32_t>((p.m + plan->bn - 1) / plan->bn);
     gp.alpha = p.alpha;
-    gp.causal = (p.flags & RMM_FLAG_CAUSAL) ? 1 : 0;
+    gp.causal = p.mode == RMM_QK && (p.flags & RMM_FLAG_CAUSAL) ? 1 : 0;
+    // PV over a causal P with the product's K axis on the tokens (every token
+    // kept, or V's unkept rows zeroed): a row tile stops at its last row
+    gp.causal_k = p.mode == RMM_PV && (p.flags & RMM_FLAG_CAUSAL) && (identity || plan->pv_mask) ? 1 : 0;
     gp.err = ws_at<int>(ws, plan->off_err);
     gp.b_head_div = 1;
 
@@ -561,6 +567,11 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     int64_t nsplit = (target + colblocks * p->heads - 1) / (colblocks * p->heads);
     const int64_t max_split = (p->n + 63) / 64;
     if (nsplit > max_split) nsplit = max_split;
+    // a causal P: splits of 512 rows, those above a column block end at once
+    if (p->mode == RMM_PV && (p->flags & RMM_FLAG_CAUSAL) && max_split > 1) {
+        const int64_t causal_split = (p->n + 511) / 512;
+        if (causal_split > nsplit) nsplit = causal_split;
+    }
     if (nsplit > 16) nsplit = 16;
     if (nsplit < 1) nsplit = 1;
     int64_t rps = (p->n + nsplit - 1) / nsplit;

@@ -351,6 +351,17 @@ __device__ __forceinline__ void stage_row(uint8_t* buf, int r, const float (&v)[
 // consecutive 256-row tiles sweep every column tile before the next group, so
 // that the A rows of a group stay resident in L2 while B streams past.
 __device__ __forceinline__ void pair_tile(int t, const GemmParams& p, int& h, int& mt, int& nt) {
+    if (p.causal_k) {
+        // row tiles carry K-work in proportion to their last row: visit every
+        // head's last row tile first, so that the round-robin over the pairs
+        // deals each pair one tile of every size band
+        const int band = p.heads * p.n_tiles;
+        mt = p.m_tiles - 1 - t / band;
+        const int r = t - (t / band) * band;
+        h = r / p.n_tiles;
+        nt = r - h * p.n_tiles;
+        return;
+    }
     const int per_head = p.m_tiles * p.n_tiles;
     h = t / per_head;
     const int r = t - h * per_head;
@@ -386,6 +397,16 @@ __device__ __forceinline__ PairUnit pair_unit(int u, int whole, int num_kb, cons
         w.kb1 = (w.part + 1) * num_kb / p.split_f;
     }
     return w;
+}
+
+// End of a unit's K loop: with a causal A (A[i][j] = 0 for j > i, the K axis
+// on the rows' positions), the k-blocks past the pair tile's last row are
+// zero and skipped.  Causal problems have no split tail.
+template <int BK>
+__device__ __forceinline__ int pair_kb_end(const GemmParams& p, const PairUnit& w, int m0) {
+    if (!p.causal_k) return w.kb1;
+    const int last = (m0 + 2 * kBM + BK - 1) / BK;
+    return last < w.kb1 ? last : w.kb1;
 }
 
 // Epilogue of one K-part of a split tail tile, for one warp (its 32 rows x
@@ -531,7 +552,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
                 const int m0 = mt * 2 * kBM, n0 = nt * BN;
                 if (p.causal && n0 > m0 + 2 * kBM - 1) continue;
                 const int row_base = (h / p.group) * p.b_head_rows;
-                for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+                const int kb_hi = pair_kb_end<C::BK>(p, w, m0);
+                for (int kb = w.kb0; kb < kb_hi; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
                     if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err, kErrTimeoutProducer)) {
@@ -572,7 +594,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
                 if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, p.err, kErrTimeoutMma)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
-                for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+                const int kb_hi = pair_kb_end<C::BK>(p, w, m0);
+                for (int kb = w.kb0; kb < kb_hi; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
                     if (!mbar_wait(&full[s], ph, abort_flag, p.err, kErrTimeoutMma)) {
@@ -639,7 +662,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
             if (!skip) {
                 acc = tcount & 1u;
                 const uint32_t aph = (tcount >> 1) & 1u;
-                if (w.kb1 - w.kb0 <= kAllPollMaxKb) {
+                if (pair_kb_end<C::BK>(p, w, m0) - w.kb0 <= kAllPollMaxKb) {
                     // short K loop: the epilogue is the critical path, every warp polls
                     if (!mbar_wait(&tfull[acc], aph, abort_flag, p.err, kErrTimeoutEpilogue)) break;
                 } else {

@@ -53,6 +53,7 @@ struct SelectArgs {
     float* scores;       // [heads][d] final fp32 scores (may alias s2)
     int nsplit;          // 1 .. kMaxSplitRows
     int64_t rows_per_split;
+    int causal_rows;     // A[i][j] = 0 for j > i: a column block skips the rows above it
 };
 constexpr int kMaxSplitRows = 64;
 
@@ -123,7 +124,9 @@ struct __align__(64) GemmParams {
     int32_t m_tiles, n_tiles;
     int32_t group_m;            // CTA-pair kernel: 256-row tiles per rasterisation group
     float alpha;
-    int32_t causal;
+    int32_t causal;             // QK: -inf above the diagonal of the output
+    int32_t causal_k;           // A[i][j] = 0 for j > i (K axis = rows' positions): a row tile's
+                                // K loop ends at its last row (CTA-pair kernel)
     int* err;
     // CTA-pair kernel, split tail: the last split_tiles tiles of the tile order
     // are computed as split_f K-parts each (0 = none).  Part j of split tile i

@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(32 * kColWarps) colnorm_kernel(const T* __rest
                                                       int64_t rows_per_split, int nsplit,
                                                       float* __restrict__ partials,
                                                       unsigned* __restrict__ counters,
-                                                      float* __restrict__ s2) {
+                                                      float* __restrict__ s2, int causal_rows) {
     pdl_wait();
     pdl_trigger();
     constexpr int V = Vec16<T>::N;
@@ -85,6 +85,12 @@ __global__ void __launch_bounds__(32 * kColWarps) colnorm_kernel(const T* __rest
     if (col < d) {
         const T* base = A + (int64_t)h * stride_a + col;
         int64_t r = r0 + warp;
+        // Rows above this column block are zero when A is causal: start at the
+        // first row of the warp's class (rows r0 + warp + W j) at or below the
+        // block's first column.  Skipped terms are exact zeros, so every sum
+        // keeps its value and order.
+        const int64_t c0 = (int64_t)blockIdx.x * COLS;
+        if (causal_rows && r < c0) r += (c0 - r + W - 1) / W * W;
         for (; r + W * (U - 1) < r1; r += W * U) {
             float x[U][V];
 #pragma unroll
@@ -421,9 +427,11 @@ cudaError_t launch_colnorm(const SelectArgs& a, cudaStream_t s) {
     dim3 grid((unsigned)((a.d + 32 * V - 1) / (32 * V)), (unsigned)a.nsplit, (unsigned)a.heads);
     if (a.dtype == 1)
         return launch_pdl(colnorm_kernel<float>, grid, dim3(32 * kColWarps), 0, s, (const float*)a.A, a.n, a.d,
-                          a.lda, a.stride_a, a.rows_per_split, a.nsplit, a.partials, a.counters, a.scores);
+                          a.lda, a.stride_a, a.rows_per_split, a.nsplit, a.partials, a.counters, a.scores,
+                          a.causal_rows);
     return launch_pdl(colnorm_kernel<__nv_bfloat16>, grid, dim3(32 * kColWarps), 0, s, (const __nv_bfloat16*)a.A,
-                      a.n, a.d, a.lda, a.stride_a, a.rows_per_split, a.nsplit, a.partials, a.counters, a.scores);
+                      a.n, a.d, a.lda, a.stride_a, a.rows_per_split, a.nsplit, a.partials, a.counters, a.scores,
+                      a.causal_rows);
 }
 
 cudaError_t launch_topk(const SelectArgs& a, cudaStream_t s) {

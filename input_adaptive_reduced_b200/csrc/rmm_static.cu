@@ -97,6 +97,7 @@ extern "C" rmm_status rmm_select_no_alloc(const rmm_plan* plan, const void* A, i
     a.scores = s2 ? s2 : reinterpret_cast<float*>(scratch + counter_bytes + partial_bytes);
     a.nsplit = plan->nsplit;
     a.rows_per_split = plan->rows_per_split;
+    a.causal_rows = p.mode == RMM_PV && (p.flags & RMM_FLAG_CAUSAL) ? 1 : 0;
     cudaError_t e = rmm::launch_colnorm(a, s);
     if (e == cudaSuccess) e = rmm::launch_topk(a, s);
     return e == cudaSuccess ? RMM_OK : RMM_ERR_CUDA;

@@ -75,6 +75,24 @@ def test_invalid_problems_are_rejected_on_the_host(field, value):
     assert _status(p) == rmm.RMM_ERR_INVALID_ARG
 
 
+def _pv(n, nk, flags):
+    p = rmm.rmm_problem_init(rmm.RMM_PV, rmm.RMM_BF16, n, nk, 128)
+    p.heads, p.kv_heads = 4, 2
+    p.stride_a, p.stride_b, p.stride_y = n * nk, nk * 128, n * 128
+    p.rho = 0.5
+    p.flags = flags
+    return p
+
+
+def test_causal_pv_needs_one_query_per_token():
+    """RMM_FLAG_CAUSAL on PV states P[i][t] = 0 for t > i, which needs n = n_k."""
+    import torch
+    assert _status(_pv(256, 512, rmm.RMM_FLAG_CAUSAL)) == rmm.RMM_ERR_INVALID_ARG
+    want = rmm.RMM_OK if torch.cuda.is_available() else rmm.RMM_ERR_CUDA
+    assert _status(_pv(512, 512, rmm.RMM_FLAG_CAUSAL)) == want
+    assert _status(_pv(256, 512, 0)) == want
+
+
 def test_valid_problem_reaches_the_device_query():
     # Validation passes, so the next step asks the CUDA runtime for the SM count:
     # OK on a GPU box, RMM_ERR_CUDA where there is no device.

@@ -87,8 +87,9 @@ def test_attention_qk_full(rmm, n):
         assert not bool(torch.isinf(S[:, ~upper]).any())
 
 
+@pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("n", [2048, 4096])
-def test_attention_pv_full(rmm, n):
+def test_attention_pv_full(rmm, n, causal):
     H, Hkv, dv = 32, 8, 128
     rhos = [0.5, 0.8]
     ks = [oracle.retained_count(r, n) for r in rhos]
@@ -101,7 +102,7 @@ def test_attention_pv_full(rmm, n):
     P64 = {h: oracle.as_f64(P[h]) for h in heads}
     V64 = oracle.as_f64(V)
     for rho in rhos:
-        O, T = rmm.pv(P, V, rho=rho, return_indices=True)
+        O, T = rmm.pv(P, V, rho=rho, return_indices=True, causal=causal)
         torch.cuda.synchronize()
         rmm.check_workspaces()
         k = oracle.retained_count(rho, n)

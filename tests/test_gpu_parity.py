@@ -296,14 +296,19 @@ def test_attention_qk(rmm, rho, causal):
     _qk_check(rmm, Q, K, rho, causal)
 
 
+@pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("rho", [0.5, 0.8, 1.0])
-def test_attention_pv(rmm, rho):
+def test_attention_pv(rmm, rho, causal):
+    """P is a causal softmax; causal=True lets the op skip the blocks above the
+    diagonal (here the second column block of the scores skips its first 256
+    rows, and the first 256-row tile drops its last k-block)."""
     H, Hkv, n, dv = 4, 2, 264, 128
     ks = [oracle.retained_count(r, n) for r in (0.5, 0.8)]
     (P, V), _ = gap.enforce_boundary_gaps(
         lambda g: W.attn_pv(31, n=n, heads=H, kv_heads=Hkv, v_dim=dv, col_gain=g),
         lambda x: gap.scores_per_head(x[0]), ks)
-    O, T = rmm.pv(P.cuda(), V.cuda(), rho=rho, return_indices=True)
+    assert not bool(torch.triu(P.float(), 1).any())
+    O, T = rmm.pv(P.cuda(), V.cuda(), rho=rho, return_indices=True, causal=causal)
     torch.cuda.synchronize()
     O_ref, T_ref = oracle.rmm_pv(P, V, rho=rho)
     assert_indices_equal(T, T_ref)

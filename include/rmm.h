@@ -189,6 +189,17 @@ RMM_API rmm_status rmm_workspace_init(const rmm_plan* plan, void* workspace, siz
    word is then cleared), or RMM_ERR_CUDA if the stream reports an error. */
 RMM_API rmm_status rmm_workspace_status(const rmm_plan* plan, void* workspace, void* stream);
 
+/* Self-test of the failure path (the pages have no counterpart): launches
+   one CTA on `stream` that waits, with the library's bounded wait, on a
+   barrier nothing ever completes.  After the wait limit (2 s) the CTA records
+   a timeout in the workspace's error word and exits, exactly as a kernel of
+   the op does when a peer stage never arrives; the context stays usable and
+   the next rmm_workspace_status reports RMM_ERR_TIMEOUT.  Errors: NULL plan or
+   workspace, or a workspace smaller than the plan's, RMM_ERR_WORKSPACE /
+   RMM_ERR_INVALID_ARG before any launch. */
+RMM_API rmm_status rmm_selftest_wait_timeout(const rmm_plan* plan, void* workspace, size_t workspace_bytes,
+                                             void* stream);
+
 /* Tracing hook.  When both are non-NULL, every later rmm_matmul* call with
    this plan records `start` immediately before and `stop` immediately after
    the launch of its reduced-product kernel, on the call's stream, so that

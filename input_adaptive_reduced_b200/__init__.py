@@ -24,6 +24,7 @@ __all__ = [
     "rmm_workspace_init", "rmm_workspace_status", "rmm_status_string", "rmm_version",
     "EXPORTED_SYMBOLS", "select", "matmul", "qk", "pv", "workspace_for", "check_workspaces",
     "rmm_plan_set_product_events", "rmm_plan_kernel_launches", "rmm_select_no_alloc",
+    "rmm_selftest_wait_timeout",
 ]
 
 RMM_OK, RMM_ERR_INVALID_ARG, RMM_ERR_UNSUPPORTED, RMM_ERR_WORKSPACE, RMM_ERR_CUDA, RMM_ERR_TIMEOUT = range(6)
@@ -36,7 +37,7 @@ EXPORTED_SYMBOLS = (
     "rmm_problem_init", "rmm_plan_create", "rmm_plan_destroy", "rmm_plan_k", "rmm_plan_workspace_size",
     "rmm_select", "rmm_matmul", "rmm_matmul_batched", "rmm_workspace_init", "rmm_workspace_status",
     "rmm_status_string", "rmm_version", "rmm_plan_set_product_events", "rmm_plan_kernel_launches",
-    "rmm_select_no_alloc",
+    "rmm_select_no_alloc", "rmm_selftest_wait_timeout",
 )
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librmm.so")
@@ -93,6 +94,8 @@ def _load_library():
     L.rmm_workspace_init.argtypes = [vp, vp, sz, vp]
     L.rmm_workspace_status.restype = st
     L.rmm_workspace_status.argtypes = [vp, vp, vp]
+    L.rmm_selftest_wait_timeout.restype = st
+    L.rmm_selftest_wait_timeout.argtypes = [vp, vp, sz, vp]
     L.rmm_plan_set_product_events.restype = st
     L.rmm_plan_set_product_events.argtypes = [vp, vp, vp]
     L.rmm_plan_kernel_launches.restype = ctypes.c_int32
@@ -200,6 +203,13 @@ def _ws(workspace):
 def rmm_workspace_init(plan: Plan, workspace, stream=None):
     wp, wb = _ws(workspace)
     _check(lib.rmm_workspace_init(plan.handle, wp, wb, _stream(stream)), "rmm_workspace_init")
+
+
+def rmm_selftest_wait_timeout(plan: Plan, workspace, stream=None):
+    """Make one bounded wait run out on purpose (see include/rmm.h); the next
+    rmm_workspace_status then reports RMM_ERR_TIMEOUT."""
+    wp, wb = _ws(workspace)
+    _check(lib.rmm_selftest_wait_timeout(plan.handle, wp, wb, _stream(stream)), "rmm_selftest_wait_timeout")
 
 
 def rmm_workspace_status(plan: Plan, workspace, stream=None) -> int:

@@ -318,6 +318,35 @@ def test_attention_pv(rmm, rho, causal):
         assert_product_close(O[h], O_ref[h], np.abs(P64[h][:, T_ref[h]]), np.abs(V64[g][T_ref[h]]))
 
 
+def test_bounded_wait_reports_timeout(rmm):
+    """A wait that nothing completes runs out after the limit, the status word
+    says so once, and the context stays usable: the next op matches the oracle."""
+    import time
+    n, d, m, rho = 200, 1024, 264, 0.5
+    k = oracle.retained_count(rho, d)
+    (A, B), _ = gap.enforce_boundary_gaps(lambda g: W.mlp_up(61, n=n, d=d, m=m, col_gain=g),
+                                          lambda x: gap.scores_2d(x[0]), [k])
+    p = rmm.rmm_problem_init(rmm.RMM_LINEAR, rmm.RMM_BF16, n, d, m)
+    p.rho = rho
+    plan = rmm.Plan(p)
+    ws = rmm.workspace_for(plan)
+    assert rmm.rmm_workspace_status(plan, ws) == rmm.RMM_OK
+    t0 = time.monotonic()
+    rmm.rmm_selftest_wait_timeout(plan, ws)
+    assert rmm.rmm_workspace_status(plan, ws) == rmm.RMM_ERR_TIMEOUT
+    assert time.monotonic() - t0 >= 1.5  # the wait gave up at its limit, not at once
+    assert rmm.rmm_workspace_status(plan, ws) == rmm.RMM_OK  # read once, then cleared
+    Ag, Bg = A.cuda(), B.cuda()
+    Y = torch.empty((n, m), dtype=torch.bfloat16, device="cuda")
+    I = torch.empty(plan.k, dtype=torch.int32, device="cuda")
+    rmm.rmm_matmul(plan, Ag, Bg, Y, I, ws)
+    assert rmm.rmm_workspace_status(plan, ws) == rmm.RMM_OK
+    I_ref, _ = oracle.select(A, rho=rho)
+    assert_indices_equal(I, I_ref)
+    A64, B64 = oracle.as_f64(A), oracle.as_f64(B)
+    assert_product_close(Y, oracle.reduced_product(A64, B64, I_ref), np.abs(A64[:, I_ref]), np.abs(B64[I_ref]))
+
+
 def test_workspace_status_clean(rmm):
     A, B = W.mlp_up(12, n=64, d=512, m=64)
     Ag, Bg = A.cuda(), B.cuda()

@@ -318,6 +318,29 @@ def test_attention_pv(rmm, rho, causal):
         assert_product_close(O[h], O_ref[h], np.abs(P64[h][:, T_ref[h]]), np.abs(V64[g][T_ref[h]]))
 
 
+def test_attention_fp32(rmm):
+    """fp32 attention (tf32 tensor cores): causal QK with GQA and PV."""
+    H, Hkv, n, dh = 4, 2, 200, 128
+    ks = [oracle.retained_count(0.5, dh)]
+    (Q, K), _ = gap.enforce_boundary_gaps(
+        lambda g: W.attn_qk(71, n=n, heads=H, kv_heads=Hkv, head_dim=dh, col_gain=g, dtype=torch.float32),
+        lambda x: gap.scores_per_head(x[0]), ks)
+    _qk_check(rmm, Q, K, 0.5, True)
+    n = 264
+    ks = [oracle.retained_count(0.8, n)]
+    (P, V), _ = gap.enforce_boundary_gaps(
+        lambda g: W.attn_pv(72, n=n, heads=H, kv_heads=Hkv, col_gain=g, dtype=torch.float32),
+        lambda x: gap.scores_per_head(x[0]), ks)
+    O, T = rmm.pv(P.cuda(), V.cuda(), rho=0.8, return_indices=True)
+    torch.cuda.synchronize()
+    O_ref, T_ref = oracle.rmm_pv(P, V, rho=0.8)
+    assert_indices_equal(T, T_ref)
+    P64, V64 = oracle.as_f64(P), oracle.as_f64(V)
+    for h in range(H):
+        g = oracle.kv_head_of(h, H, Hkv)
+        assert_product_close(O[h], O_ref[h], np.abs(P64[h][:, T_ref[h]]), np.abs(V64[g][T_ref[h]]))
+
+
 def test_bounded_wait_reports_timeout(rmm):
     """A wait that nothing completes runs out after the limit, the status word
     says so once, and the context stays usable: the next op matches the oracle."""

@@ -19,7 +19,8 @@
  *   - I is returned in ascending order, int32;
  *   - k = ceil(rho d), except that a product rho*d within 1e-9 d of an
  *     integer counts as that integer; k is clamped to [1, d];
- *   - the causal mask writes -inf where key index > query index;
+ *   - the causal mask writes -inf where key index > query index (QK); for
+ *     PV the same flag states that P is zero above its diagonal;
  *   - scores are accumulated in fp32 from the stored values; the product
  *     accumulates in fp32 (bf16 inputs) or tf32 (fp32 inputs) and is stored
  *     in the input dtype.
@@ -31,7 +32,10 @@
  *
  * Execution: compute calls only enqueue kernels on `stream` (a cudaStream_t
  * passed as void*; NULL = the legacy default stream) and return without
- * synchronising.  Argument errors are detected on the host before anything
+ * synchronising, so they can be captured in a CUDA graph.  Kernels are
+ * launched with programmatic stream serialisation: one may be scheduled while
+ * the work before it on the stream drains, and waits for that work to finish
+ * before it touches global memory.  Argument errors are detected on the host before anything
  * is enqueued; outputs are then untouched.  A kernel that gives up on an
  * internal wait (bounded at about two seconds) records it in the workspace;
  * rmm_workspace_status() reports it.  One plan and one workspace may be used
@@ -178,9 +182,10 @@ RMM_API rmm_status rmm_matmul_batched(const rmm_plan* plan, const void* A, const
                               int32_t* I_inout, void* workspace, size_t workspace_bytes,
                               void* stream);
 
-/* Zero the workspace's header (its error word and the score pass's
-   completion counters, which the kernels return to zero) on `stream`.  Call
-   once after allocating a workspace, before the first compute call. */
+/* Zero the workspace's header (its error word, the score pass's completion
+   counters and the product's split-tail counters, which the kernels return to
+   zero) on `stream`.  Call once after allocating a workspace, before the
+   first compute call. */
 RMM_API rmm_status rmm_workspace_init(const rmm_plan* plan, void* workspace, size_t workspace_bytes,
                               void* stream);
 

@@ -258,6 +258,7 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
     std::memset(&gp, 0, sizeof(gp));
     const uint32_t box_k = static_cast<uint32_t>(128 / es);
     const bool qk_masked_path = p.mode == RMM_QK && !identity && p.d <= 1024;
+    rmm::PackArgs pa_deferred{};
     if (qk_masked_path) {
         // staged below together with B
     } else if (!identity && !plan->pv_mask) {
@@ -276,7 +277,10 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         pa.ld_dst = plan->ldp;
         pa.stride_dst = p.n * plan->ldp;
         pa.heads = static_cast<int>(p.heads);
-        if (rmm::launch_pack(pa, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        if (plan->pack_ab)
+            pa_deferred = pa;  // launched together with the B row copy below
+        else if (rmm::launch_pack(pa, stream) != cudaSuccess)
+            return RMM_ERR_CUDA;
         if (!encode_kmajor_map(&gp.map_a, es, pa.dst, k, p.n, p.heads, plan->ldp, p.n * plan->ldp, box_k, 128))
             return RMM_ERR_CUDA;
     } else {
@@ -435,7 +439,9 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         pb.ld_dst = p.m;
         pb.stride_dst = k * p.m;
         pb.heads = static_cast<int>(p.heads);
-        if (rmm::launch_pack_rows(pb, plan->num_sms, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        const cudaError_t e = plan->pack_ab ? rmm::launch_pack_ab(pa_deferred, pb, stream)
+                                            : rmm::launch_pack_rows(pb, plan->num_sms, stream);
+        if (e != cudaSuccess) return RMM_ERR_CUDA;
         gl.b_mode = rmm::kBRows;
         gp.group = 1;
         gp.b_head_rows = static_cast<int32_t>(k);
@@ -485,7 +491,7 @@ int32_t launches_per_call(const rmm_plan* plan) {
     if (!identity) n += 1;                                   // pack A[:, I] (PV: mask V's rows instead)
     if (p.mode == RMM_QK && !identity && p.d > 1024) n += 1; // pack K[:, I] (else Q is masked in place of the A pack)
     if (p.mode != RMM_QK && p.dtype == RMM_F32) n += 1;      // B[I, :] transposed for tf32
-    if (!identity && plan->pack_b) n += 1;                   // B[I, :] rows, contiguous
+    if (!identity && plan->pack_b && !plan->pack_ab) n += 1; // B[I, :] rows, contiguous (else in the A pack's launch)
     return n + 1;                                            // the product
 }
 
@@ -540,6 +546,7 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
         plan->sk_np = rmm::skinny_pad(p->n);
         plan->sk_splits = rmm::skinny_splits(p->m, plan->k, 0, plan->sk_np);  // fixed below once the SM count is known
     }
+    plan->pack_ab = plan->pack_b && rmm::pack_ab_one_launch(p->dtype, plan->ldp);
 
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||

@@ -95,6 +95,11 @@ cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s);
 // dst[h][t][:] = src[h / group][I[h][t]][:] for t < k: the retained rows of a
 // row-major B, contiguous (a.rows = number of columns of B).
 cudaError_t launch_pack_rows(const PackArgs& a, int num_sms, cudaStream_t s);
+// launch_pack(a) and launch_pack_rows(b) as one launch, their CTAs interleaved
+// (bf16, packed A rows wider than the narrow variant's; pack_ab_one_launch says
+// whether an A pack qualifies).
+bool pack_ab_one_launch(int dtype, int64_t ld_a);
+cudaError_t launch_pack_ab(const PackArgs& a, const PackArgs& b, cudaStream_t s);
 // dst[h][t][:] = src[h / group][t][:] if t is in I[h][0..k) (ascending, unique)
 // else 0, for t < rows_out (rows t >= a.d are zero); a.rows = columns of B.
 // Used for attention PV, where the product is bound by reading P and a
@@ -189,6 +194,7 @@ struct rmm_plan {
     int64_t rows_per_split;
     int bn;
     bool pack_b;        // bf16 LINEAR/PV with k < d: stage B[I, :] contiguously
+    bool pack_ab;       // the A pack and the B row copy run as one launch
     int num_sms;
     size_t off_err, off_counters, off_partials, off_scores, off_I, off_apack, off_bpack, ws_bytes;
     size_t header_bytes;  // zeroed by rmm_workspace_init: error word + colnorm counters

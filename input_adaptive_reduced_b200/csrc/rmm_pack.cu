@@ -21,15 +21,13 @@ constexpr int kPackRows = 16;  // rows per CTA; the 8 indices of a thread are re
 // grid (ceil(ld_dst / (8*256)), ceil(rows / 16), heads).  Thread t owns output
 // columns [8t, 8t+8) of its CTA's slice; it loads their 8 source indices once
 // and writes 16-byte (bf16) or 2 x 16-byte (fp32) rows of the packed buffer.
+// The body of one CTA of the grid; (bx, by, h) is its block index.
 template <typename T>
-__global__ void __launch_bounds__(kPackThreads) pack_kernel(
-    const T* __restrict__ src, int64_t rows, int64_t d, int64_t ld_src, int64_t stride_src, int group,
-    const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
-    int64_t stride_dst) {
-    pdl_wait();
-    pdl_trigger();
-    const int h = blockIdx.z;
-    const int64_t t0 = ((int64_t)blockIdx.x * kPackThreads + threadIdx.x) * 8;
+__device__ __forceinline__ void pack_block(const T* __restrict__ src, int64_t rows, int64_t d, int64_t ld_src,
+                                           int64_t stride_src, int group, const int32_t* __restrict__ I,
+                                           int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
+                                           int64_t stride_dst, int64_t bx, int64_t by, int h) {
+    const int64_t t0 = (bx * kPackThreads + threadIdx.x) * 8;
     if (t0 >= ld_dst) return;
     int32_t idx[8];
     bool live[8];
@@ -42,7 +40,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(
     }
     const T* sh = src + (int64_t)(h / group) * stride_src;
     T* dh = dst + (int64_t)h * stride_dst;
-    const int64_t r_beg = (int64_t)blockIdx.y * kPackRows;
+    const int64_t r_beg = by * kPackRows;
     const int64_t r_end = min(rows, r_beg + kPackRows);
     // four rows per round: thirty-two independent element loads in flight per thread
     for (int64_t r = r_beg; r < r_end; r += 4) {
@@ -66,6 +64,17 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(
             }
         }
     }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kPackThreads) pack_kernel(
+    const T* __restrict__ src, int64_t rows, int64_t d, int64_t ld_src, int64_t stride_src, int group,
+    const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
+    int64_t stride_dst) {
+    pdl_wait();
+    pdl_trigger();
+    pack_block(src, rows, d, ld_src, stride_src, group, I, I_stride, k, dst, ld_dst, stride_dst, blockIdx.x,
+               blockIdx.y, (int)blockIdx.z);
 }
 
 // Transposing variant for fp32 operands: dst[h][c][t] = src[h / group][I[h][t]][c]
@@ -109,28 +118,25 @@ __global__ void __launch_bounds__(256) pack_rows_transposed_kernel(
 // so both sides are fully coalesced.
 constexpr int kRowsPerCta = 8;
 
-template <typename T>
-__global__ void __launch_bounds__(256) pack_rows_kernel(
-    const T* __restrict__ src, int64_t d, int64_t cols, int64_t ld_src, int64_t stride_src, int group,
-    const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
-    int64_t stride_dst) {
-    pdl_wait();
-    pdl_trigger();
+template <typename T, int U = 4>
+__device__ __forceinline__ void pack_rows_block(const T* __restrict__ src, int64_t d, int64_t cols, int64_t ld_src,
+                                                int64_t stride_src, int group, const int32_t* __restrict__ I,
+                                                int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
+                                                int64_t stride_dst, int64_t bx, int h) {
     constexpr int V = 16 / sizeof(T);
-    const int h = blockIdx.y;
     const int cpr = (int)(cols / V);
-    const int64_t t0 = (int64_t)blockIdx.x * kRowsPerCta;
+    const int64_t t0 = bx * kRowsPerCta;
     const int64_t left = k - t0;
     const int nrows = left < kRowsPerCta ? (int)left : kRowsPerCta;
     const int total = nrows * cpr;
     const T* sh = src + (int64_t)(h / group) * stride_src;
     T* dh = dst + (int64_t)h * stride_dst;
     const int32_t* Ih = I + (int64_t)h * I_stride + t0;
-    for (int base = threadIdx.x; base < total; base += 4 * 256) {
-        uint4 v[4];
-        int64_t out[4];
+    for (int base = threadIdx.x; base < total; base += U * 256) {
+        uint4 v[U];
+        int64_t out[U];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int idx = base + u * 256;
             out[u] = -1;
             if (idx < total) {
@@ -143,8 +149,43 @@ __global__ void __launch_bounds__(256) pack_rows_kernel(
             }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < U; ++u)
             if (out[u] >= 0) *reinterpret_cast<uint4*>(dh + out[u]) = v[u];
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) pack_rows_kernel(
+    const T* __restrict__ src, int64_t d, int64_t cols, int64_t ld_src, int64_t stride_src, int group,
+    const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
+    int64_t stride_dst) {
+    pdl_wait();
+    pdl_trigger();
+    pack_rows_block(src, d, cols, ld_src, stride_src, group, I, I_stride, k, dst, ld_dst, stride_dst, blockIdx.x,
+                    (int)blockIdx.y);
+}
+
+// Both staging copies of an op in one launch: the CTAs of pack_kernel's grid
+// (A[:, I]) first, then those of pack_rows_kernel's grid (B[I, :]), over one
+// 1-D grid.  The A gather runs while the score pass's reads of A may still sit
+// in L2, and the row copy's first CTAs fill the SMs that the gather's last wave
+// leaves idle, where a second launch would wait for the whole gather to end.
+// At this kernel's register count (3 CTAs per SM, against 8 for the lone row
+// copy) each row-copy thread keeps eight 16-byte loads in flight.
+template <typename T>
+__global__ void __launch_bounds__(256, 3) pack_ab_kernel(PackArgs a, PackArgs b, int64_t a_x, int64_t a_y, int64_t n_a,
+                                                         int64_t b_x) {
+    pdl_wait();
+    pdl_trigger();
+    const int64_t i = blockIdx.x;
+    if (i < n_a) {
+        const int64_t x = i % a_x, yz = i / a_x;
+        pack_block((const T*)a.src, a.rows, a.d, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k, (T*)a.dst,
+                   a.ld_dst, a.stride_dst, x, yz % a_y, (int)(yz / a_y));
+    } else {
+        const int64_t j = i - n_a;
+        pack_rows_block<T, 8>((const T*)b.src, b.d, b.rows, b.ld_src, b.stride_src, b.group, b.I, b.I_stride, b.k,
+                              (T*)b.dst, b.ld_dst, b.stride_dst, j % b_x, (int)(j / b_x));
     }
 }
 
@@ -299,6 +340,22 @@ cudaError_t launch_pack_rows(const PackArgs& a, int num_sms, cudaStream_t s) {
     return launch_pdl(pack_rows_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, (const __nv_bfloat16*)a.src, a.d,
                       a.rows, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k, (__nv_bfloat16*)a.dst,
                       a.ld_dst, a.stride_dst);
+}
+
+bool pack_ab_one_launch(int dtype, int64_t ld_a) { return dtype == 0 && ld_a > kNarrowMax; }
+
+cudaError_t launch_pack_ab(const PackArgs& a, const PackArgs& b, cudaStream_t s) {
+    if (!pack_ab_one_launch(a.dtype, a.ld_dst) || b.dtype != a.dtype) return cudaErrorInvalidValue;
+    const int64_t a_x = (a.ld_dst + 8 * kPackThreads - 1) / (8 * kPackThreads);
+    const int64_t a_y = (a.rows + kPackRows - 1) / kPackRows;
+    const int64_t n_a = a_x * a_y * a.heads;
+    const int64_t b_x = (b.k + kRowsPerCta - 1) / kRowsPerCta;
+    const int64_t n_b = b.rows == 0 ? 0 : b_x * b.heads;
+    const int64_t total = n_a + n_b;
+    if (total == 0) return cudaSuccess;
+    if (total > 0x7fffffff) return cudaErrorInvalidValue;
+    return launch_pdl(pack_ab_kernel<__nv_bfloat16>, dim3((unsigned)total), dim3(256), 0, s, a, b, a_x, a_y, n_a,
+                      b_x);
 }
 
 cudaError_t launch_mask_rows(const PackArgs& a, int64_t rows_out, cudaStream_t s) {

@@ -96,6 +96,34 @@ def test_linear_bf16(rmm, kind, n, d, m):
         _linear_case(rmm, A, B, rho)
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("rho", [0.2, 0.9])
+def test_wide_column_pack(rmm, dtype, rho):
+    """Packed A rows wider than 1024 columns: a CTA whose 2048 retained columns
+    span few source columns (rho = 0.9) copies the span through shared memory;
+    at rho = 0.2 the first CTA's span is too wide and it loads its columns one
+    by one (bf16, d = 14336: the ragged second CTA's span is staged)."""
+    n, d, m = 200, (14336 if dtype == torch.bfloat16 else 8192), 264
+    k = oracle.retained_count(rho, d)
+    assert k > 1024
+    (A, B), _ = gap.enforce_boundary_gaps(
+        lambda g: W.mlp_down(13, n=n, d=d, m=m, col_gain=g, dtype=dtype),
+        lambda x: gap.scores_2d(x[0]), [k])
+    _linear_case(rmm, A, B, rho)
+
+
+def test_wide_column_pack_given_span(rmm):
+    """A given index set whose first 2048 columns reach across the whole row
+    (the direct body) and whose rest is dense (the staged body)."""
+    n, d, m = 136, 14336, 264
+    A, B = W.mlp_down(14, n=n, d=d, m=m)
+    I = np.concatenate([np.arange(0, 1024), np.arange(d - 4096, d)]).astype(np.int32)
+    Y = rmm.matmul(A.cuda(), B.cuda(), indices=torch.from_numpy(I).cuda())
+    torch.cuda.synchronize()
+    A64, B64 = oracle.as_f64(A), oracle.as_f64(B)
+    assert_product_close(Y, oracle.reduced_product(A64, B64, I), np.abs(A64[:, I]), np.abs(B64[I]))
+
+
 def test_select_scores_and_indices(rmm):
     A, _ = W.mlp_up(3, n=300, d=4096, m=8)
     Ag = A.cuda()

@@ -158,6 +158,10 @@ rmm_status run_select(const rmm_plan* plan, const void* A, int32_t* I, float* s2
     a.k = plan->k;
     a.I = I;
     a.s2 = s2;
+    if (plan->decode && p.mode == RMM_PV) {  // the decode product reads membership words, not I
+        a.mask = ws_at<uint32_t>(ws, plan->off_dec_mask);
+        a.mask_words = (p.d + 31) / 32;
+    }
     cudaError_t e;
     if (plan->fused_select) {
         e = rmm::launch_normselect(a, stream);
@@ -204,6 +208,43 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         }
     }
     if (p.n == 0 || p.m == 0) return RMM_OK;
+
+    if (plan->decode) {
+        rmm::DecodeArgs da{};
+        da.A = static_cast<const __nv_bfloat16*>(A);
+        da.lda = p.lda;
+        da.stride_a = p.stride_a;
+        da.B = static_cast<const __nv_bfloat16*>(B);
+        da.ldb = p.ldb;
+        da.stride_b = p.stride_b;
+        da.Y = static_cast<__nv_bfloat16*>(Y);
+        da.ldy = p.ldy;
+        da.stride_y = p.stride_y;
+        da.k = k;
+        da.d = p.d;
+        da.m = p.m;
+        da.n = static_cast<int32_t>(p.n);
+        da.group = plan->group;
+        da.kv_heads = static_cast<int32_t>(p.kv_heads);
+        da.alpha = p.alpha;
+        const bool traced = plan->product_start && plan->product_stop;
+        if (traced && cudaEventRecord(plan->product_start, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        cudaError_t e;
+        if (p.mode == RMM_QK) {
+            da.I = identity ? nullptr : I;
+            e = rmm::launch_decode_qk(da, stream);
+        } else {
+            da.mask = identity ? nullptr : ws_at<uint32_t>(ws, plan->off_dec_mask);
+            da.mask_words = (p.d + 31) / 32;
+            da.partials = ws_at<float>(ws, plan->off_dec_part);
+            da.counters = ws_at<unsigned>(ws, plan->off_dec_cnt);
+            da.tokens = plan->dec_tokens;
+            e = rmm::launch_decode_pv(da, stream);
+        }
+        if (e != cudaSuccess) return RMM_ERR_CUDA;
+        if (traced && cudaEventRecord(plan->product_stop, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        return RMM_OK;
+    }
 
     if (plan->skinny) {
         rmm::SkinnyParams sp;
@@ -487,6 +528,7 @@ int32_t launches_per_call(const rmm_plan* plan) {
     int32_t n = 0;
     if (!given && !identity) n += plan->fused_select ? 1 : 2;
     if (p.n == 0 || p.m == 0) return n;
+    if (plan->decode) return n + 1;
     if (plan->skinny) return n + (identity ? 0 : 1) + 1 + (plan->sk_splits > 1 ? 1 : 0);
     if (!identity) n += 1;                                   // pack A[:, I] (PV: mask V's rows instead)
     if (p.mode == RMM_QK && !identity && p.d > 1024) n += 1; // pack K[:, I] (else Q is masked in place of the A pack)
@@ -546,6 +588,18 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
         plan->sk_np = rmm::skinny_pad(p->n);
         plan->sk_splits = rmm::skinny_splits(p->m, plan->k, 0, plan->sk_np);  // fixed below once the SM count is known
     }
+    // Decode step: a few query rows per head against cached keys / values;
+    // the group's query vectors are taken together (each cache row is read
+    // once per KV head).  PV needs the selection's membership words, so a
+    // given token set takes the general path.
+    const bool causal = (p->flags & RMM_FLAG_CAUSAL) != 0;
+    plan->decode = p->dtype == RMM_BF16 && !causal && p->n >= 1 && p->n * plan->group <= 8 &&
+                   ((p->mode == RMM_QK && rmm::decode_qk_supported(p->d)) ||
+                    (p->mode == RMM_PV && !given && rmm::decode_pv_supported(p->m)));
+    if (plan->decode) {
+        plan->pack_b = false;
+        plan->pv_mask = false;
+    }
     plan->pack_ab = plan->pack_b && rmm::pack_ab_one_launch(p->dtype, plan->ldp);
 
     int dev = 0, sms = 0;
@@ -557,6 +611,11 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     }
     plan->num_sms = sms;
     if (plan->skinny) plan->sk_splits = rmm::skinny_splits(p->m, plan->k, sms, plan->sk_np);
+    const bool dec_pv = plan->decode && p->mode == RMM_PV;
+    if (dec_pv) {
+        plan->dec_tokens = rmm::decode_pv_tokens(p->d, p->kv_heads, sms);
+        plan->dec_parts = static_cast<int>((p->d + plan->dec_tokens - 1) / plan->dec_tokens);
+    }
 
     // Selection kernels need every score of a head in shared memory.
     const bool select_possible = p->d <= rmm::kMaxSelectD;
@@ -605,6 +664,8 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     }
     plan->off_split_cnt = off;
     off += align256(static_cast<size_t>(plan->split_tiles) * 2 * rmm::kSplitCounterWarps * sizeof(unsigned));
+    plan->off_dec_cnt = off;
+    if (dec_pv) off += align256(static_cast<size_t>(p->kv_heads) * sizeof(unsigned));
     plan->header_bytes = off;
     plan->off_partials = off;
     plan->off_scores = off;
@@ -617,7 +678,7 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     off += align256(static_cast<size_t>(p->heads) * plan->k * sizeof(int32_t));
     plan->off_apack = off;
     const bool qk_mask = p->mode == RMM_QK && p->d <= 1024;  // Q masked at full width, K used as is
-    if (!plan->pv_mask)
+    if (!plan->pv_mask && !plan->decode)
         off += align256(static_cast<size_t>(p->heads) * p->n * (qk_mask ? p->d : plan->ldp) * plan->es);
     plan->off_bpack = off;
     if (qk_mask) {
@@ -632,6 +693,13 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
         off += align256(static_cast<size_t>(p->heads) * plan->k * p->m * plan->es);
     plan->off_split = off;
     off += align256(static_cast<size_t>(plan->split_tiles) * plan->split_f * 256 * plan->bn * sizeof(float));
+    plan->off_dec_mask = off;
+    plan->off_dec_part = off;
+    if (dec_pv) {
+        off += align256(static_cast<size_t>(p->heads) * ((p->d + 31) / 32) * sizeof(uint32_t));
+        plan->off_dec_part = off;
+        off += align256(static_cast<size_t>(p->kv_heads) * plan->dec_parts * 8 * p->m * sizeof(float));
+    }
     plan->ws_bytes = off;
     if (workspace_bytes) *workspace_bytes = plan->ws_bytes;
     *out = plan;

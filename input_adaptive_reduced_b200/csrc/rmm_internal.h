@@ -4,6 +4,7 @@
 
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace rmm {
@@ -54,6 +55,8 @@ struct SelectArgs {
     int nsplit;          // 1 .. kMaxSplitRows
     int64_t rows_per_split;
     int causal_rows;     // A[i][j] = 0 for j > i: a column block skips the rows above it
+    uint32_t* mask;      // [heads][mask_words] membership bits of I (bit j of word j / 32), or nullptr
+    int64_t mask_words;  // ceil(d / 32) when mask is set
 };
 constexpr int kMaxSplitRows = 64;
 
@@ -159,6 +162,35 @@ size_t gemm_smem_bytes(int dtype, int bn, bool pair);
 void pair_split_tail(int64_t tiles, int64_t num_kb, int clusters, int* split_tiles, int* split_f);
 constexpr int kSplitCounterWarps = 8;  // counters per CTA per split tile (epilogue warps)
 
+// ---------------------------------------------------------------- decode step
+// Attention with group * n <= 8 query vectors per KV head (rmm_decode.cu).
+struct DecodeArgs {
+    const __nv_bfloat16* A;  // qk: Q [heads][n][d]; pv: P [heads][n][t]
+    int64_t lda, stride_a;
+    const __nv_bfloat16* B;  // qk: K [kv_heads][t][d]; pv: V [kv_heads][t][d_v]
+    int64_t ldb, stride_b;
+    const int32_t* I;        // qk: [heads][k] kept features, nullptr = all
+    const uint32_t* mask;    // pv: [heads][mask_words] kept tokens (bit t of word t / 32), nullptr = all
+    int64_t mask_words;
+    __nv_bfloat16* Y;        // qk: S [heads][n][t]; pv: O [heads][n][d_v]
+    int64_t ldy, stride_y;
+    float* partials;         // pv: [kv_heads][token ranges][8][d_v] fp32
+    unsigned* counters;      // pv: [kv_heads], zero between launches
+    int64_t k;               // qk: entries of I per head
+    int64_t d;               // qk: features d_h; pv: tokens t
+    int64_t m;               // qk: keys t; pv: d_v
+    int32_t n, group, kv_heads;
+    int32_t tokens;          // pv: tokens per CTA (128, 256 or 512)
+    float alpha;             // qk: scale of the scores
+};
+bool decode_qk_supported(int64_t d);
+bool decode_pv_supported(int64_t dv);
+// tokens per CTA for t tokens on kv_heads heads: 512, halved while that
+// leaves fewer than two CTAs per SM (down to 128)
+int decode_pv_tokens(int64_t t, int64_t kv_heads, int num_sms);
+cudaError_t launch_decode_qk(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode_pv(const DecodeArgs& a, cudaStream_t s);
+
 // ---------------------------------------------------------------- few rows
 // Product for n <= 64 with swapped operands (rmm_skinny.cu).
 struct __align__(64) SkinnyParams {
@@ -204,4 +236,7 @@ struct rmm_plan {
     bool pv_mask;       // bf16 PV with a selected T: V's unkept rows zeroed per query head, P read as stored
     int split_tiles, split_f;           // split tail of the CTA-pair product (0, 1: none)
     size_t off_split_cnt, off_split;    // its counters (in the header) and fp32 partials
+    bool decode;        // bf16 attention with group * n <= 8 query vectors per KV head (rmm_decode.cu)
+    int dec_tokens, dec_parts;          // pv: tokens per CTA, token ranges per KV head
+    size_t off_dec_cnt, off_dec_mask, off_dec_part;  // pv: counters (header), membership words, partials
 };

@@ -183,8 +183,11 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
 }
 
 // first_done: the sub-histograms already hold the first pass over all keys.
+// mask_out (or nullptr): bit j of word j / 32 set iff column j is selected,
+// for the ceil(d / 32) words that cover [0, d); the emission's ballots over 32
+// consecutive columns are these words.
 __device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k, int32_t* out, TopkShared& sh,
-                                      bool first_done) {
+                                      bool first_done, uint32_t* mask_out) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint4* keys4 = reinterpret_cast<const uint4*>(keys);
     const int64_t d4 = d >> 2;
@@ -282,6 +285,7 @@ __device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k
         const unsigned sm = __ballot_sync(0xffffffffu, sel);
         const uint32_t pos = sel_run + __popc(sm & lt_mask);
         if (sel && pos < (uint32_t)k) out[pos] = (int32_t)j;
+        if (mask_out && lane == 0) mask_out[j0 >> 5] = sm;  // j0 is a multiple of 32 below end
         eq_run += __popc(em);
         sel_run += __popc(sm);
     }
@@ -292,7 +296,8 @@ __device__ void radix_select_and_emit(const uint32_t* keys, int64_t d, int64_t k
 // multiple of 4): 16-byte loads, the first radix histogram built on the way
 // into shared memory.
 __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ scores, int64_t d, int64_t k,
-                                                    int32_t* __restrict__ I) {
+                                                    int32_t* __restrict__ I, uint32_t* __restrict__ mask,
+                                                    int64_t mask_words) {
     pdl_wait();
     pdl_trigger();
     extern __shared__ uint32_t keys[];
@@ -322,7 +327,7 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ sc
             }
     }
     __syncthreads();
-    radix_select_and_emit(keys, d, k, I + (int64_t)h * k, sh, true);
+    radix_select_and_emit(keys, d, k, I + (int64_t)h * k, sh, true, mask ? mask + h * mask_words : nullptr);
 }
 
 // ------------------------------------------------------------------ fused
@@ -333,7 +338,8 @@ template <typename T>
 __global__ void __launch_bounds__(1024) normselect_kernel(const T* __restrict__ A, int64_t n,
                                                           int64_t d, int64_t lda, int64_t stride_a,
                                                           int rg, int64_t k, int32_t* __restrict__ I,
-                                                          float* __restrict__ s2) {
+                                                          float* __restrict__ s2, uint32_t* __restrict__ mask,
+                                                          int64_t mask_words) {
     pdl_wait();
     pdl_trigger();
     constexpr int V = Vec16<T>::N;
@@ -391,7 +397,7 @@ __global__ void __launch_bounds__(1024) normselect_kernel(const T* __restrict__ 
     if (s2) {
         for (int64_t j = threadIdx.x; j < d; j += 1024) s2[(int64_t)h * d + j] = __uint_as_float(keys[j]);
     }
-    radix_select_and_emit(keys, d, k, I + (int64_t)h * k, sh, false);
+    radix_select_and_emit(keys, d, k, I + (int64_t)h * k, sh, false, mask ? mask + h * mask_words : nullptr);
 }
 
 __global__ void identity_kernel(int32_t* __restrict__ I, int64_t k, int heads) {
@@ -439,7 +445,8 @@ cudaError_t launch_topk(const SelectArgs& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(topk_kernel, dim3(a.heads), dim3(1024), smem, s, (const float*)a.scores, a.d, a.k, a.I);
+    return launch_pdl(topk_kernel, dim3(a.heads), dim3(1024), smem, s, (const float*)a.scores, a.d, a.k, a.I, a.mask,
+                      a.mask_words);
 }
 
 cudaError_t launch_normselect(const SelectArgs& a, cudaStream_t s) {
@@ -451,13 +458,14 @@ cudaError_t launch_normselect(const SelectArgs& a, cudaStream_t s) {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         e = launch_pdl(normselect_kernel<float>, dim3(a.heads), dim3(1024), smem, s, (const float*)a.A, a.n, a.d,
-                       a.lda, a.stride_a, rg, a.k, a.I, a.s2);
+                       a.lda, a.stride_a, rg, a.k, a.I, a.s2, a.mask, a.mask_words);
     } else {
         e = cudaFuncSetAttribute(normselect_kernel<__nv_bfloat16>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         e = launch_pdl(normselect_kernel<__nv_bfloat16>, dim3(a.heads), dim3(1024), smem, s,
-                       (const __nv_bfloat16*)a.A, a.n, a.d, a.lda, a.stride_a, rg, a.k, a.I, a.s2);
+                       (const __nv_bfloat16*)a.A, a.n, a.d, a.lda, a.stride_a, rg, a.k, a.I, a.s2, a.mask,
+                       a.mask_words);
     }
     return e;
 }

@@ -52,6 +52,30 @@ def assert_product_close(Y_gpu, Y_ref, absA_I, absB_I, alpha=1.0, mask=None):
     return fro
 
 
+def assert_heads_close(Y_gpu, Y_ref, absA_I, absB_I, alpha=1.0):
+    """Batched output Y [H, n, m] against the oracle's: the relative Frobenius
+    bound on the op's whole output, the element bound per head with that head's
+    absA_I[h] (n x k) and absB_I[h] (k x m).  Rounding the output to bf16 alone
+    costs ~1.6e-3 of relative Frobenius error on average, so a head with a few
+    dozen outputs (one decode row) can exceed 2e-3 by rounding luck alone; the
+    bound is therefore taken over all heads together."""
+    Yg = np64(Y_gpu)
+    Yr = np.asarray(Y_ref, dtype=np.float64)
+    assert Yg.shape == Yr.shape, (Yg.shape, Yr.shape)
+    assert np.all(np.isfinite(Yg)), "non-finite values where finite ones are expected"
+    err = Yg - Yr
+    fro = np.linalg.norm(err) / max(np.linalg.norm(Yr), 1e-300)
+    assert fro <= REL_FRO, f"relative Frobenius error {fro:.3e} > {REL_FRO}"
+    for h in range(Yr.shape[0]):
+        bound = ELEM * abs(alpha) * (absA_I[h] @ absB_I[h])
+        over = np.abs(err[h]) > bound + 1e-30
+        if np.any(over):
+            i = np.argwhere(over)[0]
+            raise AssertionError(f"head {h}: {int(over.sum())} elements exceed 1e-2*(|A_I||B_I|); first at "
+                                 f"{i.tolist()}: err {err[h][tuple(i)]:.3e} bound {bound[tuple(i)]:.3e}")
+    return fro
+
+
 def sample_rows(n: int, seed: int = 0, per_tile: int = 2, tile: int = 128):
     """Two seeded rows from every 128-row tile (all rows when n is small)."""
     rng = np.random.default_rng(seed)

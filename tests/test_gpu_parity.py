@@ -14,7 +14,7 @@ import torch
 import oracle
 import workloads as W
 from tests import gap
-from tests.parity import assert_indices_equal, assert_product_close, np64
+from tests.parity import assert_heads_close, assert_indices_equal, assert_product_close, np64
 
 pytestmark = pytest.mark.gpu
 
@@ -414,3 +414,116 @@ def test_workspace_status_clean(rmm):
     with pytest.raises(rmm.RmmError) as e:
         rmm.rmm_matmul(plan, Ag[:, 1:], Bg, Y, None, ws)  # 2-byte offset: misaligned
     assert e.value.status == rmm.RMM_ERR_INVALID_ARG
+
+
+# Decode step: (batch, n, heads, kv_heads, head_dim = d_v, t).  n = 1 scores
+# are squares of bf16 values, exact in fp32 and fp64 alike, so equal scores
+# are ties on both sides and the lower index wins on both; n = 2 inputs get
+# the usual boundary gap.
+DECODE_CASES = [
+    (2, 1, 32, 8, 128, 1000),  # Llama-3.1-8B grouping, t not a multiple of the tiles
+    (1, 2, 32, 8, 128, 520),   # two query rows: 8 query vectors per KV head
+    (1, 1, 64, 8, 128, 264),   # groups of 8 query heads
+    (1, 1, 8, 4, 64, 96),      # d_h = d_v = 64, a single token range
+]
+
+
+def _decode_inputs(case, seed, which):
+    batch, n, H, Hkv, dh, t = case
+    make = lambda g: W.attn_decode(seed, t=t, batch=batch, n=n, heads=H, kv_heads=Hkv, head_dim=dh, v_dim=dh,
+                                   **({which: g} if g is not None else {}))
+    if n == 1:
+        return make(None)
+    d = dh if which == "q_gain" else t
+    ks = [oracle.retained_count(r, d) for r in (0.5, 0.8)]
+    idx = 0 if which == "q_gain" else 3
+    out, _ = gap.enforce_boundary_gaps(make, lambda x: gap.scores_per_head(x[idx]), ks)
+    return out
+
+
+def _decode_qk_close(S, S_ref, I_ref, q, K, alpha):
+    q64, K64 = oracle.as_f64(q), oracle.as_f64(K)
+    H, Hkv = q.shape[0], K.shape[0]
+    absA = [np.abs(q64[h][:, I_ref[h]]) for h in range(H)]
+    absB = [np.abs(K64[oracle.kv_head_of(h, H, Hkv)][:, I_ref[h]]).T for h in range(H)]
+    assert_heads_close(S, S_ref, absA, absB, alpha=alpha)
+
+
+def _decode_pv_close(O, O_ref, T_ref, P, V):
+    P64, V64 = oracle.as_f64(P), oracle.as_f64(V)
+    H, Hkv = P.shape[0], V.shape[0]
+    absA = [np.abs(P64[h][:, T_ref[h]]) for h in range(H)]
+    absB = [np.abs(V64[oracle.kv_head_of(h, H, Hkv)][T_ref[h]]) for h in range(H)]
+    assert_heads_close(O, O_ref, absA, absB)
+
+
+def _launches(rmm, mode, X, Z, m, rho):
+    H, n, d = X.shape
+    p = rmm.rmm_problem_init(mode, rmm.RMM_BF16, n, d, m)
+    p.rho = rho
+    p.heads, p.kv_heads = H, Z.shape[0]
+    p.lda, p.ldb = d, Z.shape[2]
+    p.stride_a, p.stride_b = X.stride(0), Z.stride(0)
+    p.ldy, p.stride_y = m, n * m
+    return rmm.Plan(p).kernel_launches
+
+
+@pytest.mark.parametrize("rho", [0.5, 0.8, 1.0])
+@pytest.mark.parametrize("case", DECODE_CASES)
+def test_decode_qk(rmm, case, rho):
+    """Scores of a decode step: the group's query vectors against each K row once."""
+    q, K, _, _ = _decode_inputs(case, 81, "q_gain")
+    H, n, dh = q.shape
+    assert _launches(rmm, rmm.RMM_QK, q, K, K.shape[1], rho) == (1 if rho < 1 else 0) + 1
+    alpha = 1.0 / math.sqrt(dh)
+    S, I = rmm.qk(q.cuda(), K.cuda(), rho=rho, alpha=alpha, causal=False, return_indices=True)
+    torch.cuda.synchronize()
+    S_ref, I_ref = oracle.rmm_qk(q, K, rho=rho, alpha=alpha, causal=False)
+    assert_indices_equal(I, I_ref)
+    _decode_qk_close(S, S_ref, I_ref, q, K, alpha)
+
+
+def test_decode_qk_head_dim_256(rmm):
+    q, K, _, _ = W.attn_decode(82, t=200, batch=1, n=1, heads=8, kv_heads=2, head_dim=256)
+    S, I = rmm.qk(q.cuda(), K.cuda(), rho=0.7, alpha=0.0625, causal=False, return_indices=True)
+    torch.cuda.synchronize()
+    S_ref, I_ref = oracle.rmm_qk(q, K, rho=0.7, alpha=0.0625, causal=False)
+    assert_indices_equal(I, I_ref)
+    _decode_qk_close(S, S_ref, I_ref, q, K, 0.0625)
+
+
+@pytest.mark.parametrize("rho", [0.5, 0.8, 1.0])
+@pytest.mark.parametrize("case", DECODE_CASES)
+def test_decode_pv(rmm, case, rho):
+    """Value product of a decode step: the union of the group's kept tokens is
+    read once per KV head, each weighed only for the heads that kept it."""
+    _, _, V, P = _decode_inputs(case, 91, "p_gain")
+    H, n, t = P.shape
+    Hkv = V.shape[0]
+    assert _launches(rmm, rmm.RMM_PV, P, V, V.shape[2], rho) == (1 if rho < 1 else 0) + 1
+    O, T = rmm.pv(P.cuda(), V.cuda(), rho=rho, return_indices=True)
+    torch.cuda.synchronize()
+    O_ref, T_ref = oracle.rmm_pv(P, V, rho=rho)
+    assert_indices_equal(T, T_ref)
+    _decode_pv_close(O, O_ref, T_ref, P, V)
+    O2 = rmm.pv(P.cuda(), V.cuda(), rho=rho)  # the token ranges' counters were reset
+    torch.cuda.synchronize()
+    assert torch.equal(O, O2)
+    rmm.check_workspaces()
+
+
+def test_decode_rows_past_the_group_take_the_general_path(rmm):
+    """group * n > 8 query vectors per KV head: the general kernels."""
+    case = (1, 4, 8, 2, 128, 264)
+    q, K, _, _ = _decode_inputs(case, 83, "q_gain")
+    _, _, V, P = _decode_inputs(case, 84, "p_gain")
+    assert _launches(rmm, rmm.RMM_QK, q, K, K.shape[1], 0.5) > 2
+    S, I = rmm.qk(q.cuda(), K.cuda(), rho=0.5, alpha=0.1, causal=False, return_indices=True)
+    O, T = rmm.pv(P.cuda(), V.cuda(), rho=0.5, return_indices=True)
+    torch.cuda.synchronize()
+    S_ref, I_ref = oracle.rmm_qk(q, K, rho=0.5, alpha=0.1, causal=False)
+    O_ref, T_ref = oracle.rmm_pv(P, V, rho=0.5)
+    assert_indices_equal(I, I_ref)
+    assert_indices_equal(T, T_ref)
+    _decode_qk_close(S, S_ref, I_ref, q, K, 0.1)
+    _decode_pv_close(O, O_ref, T_ref, P, V)

@@ -20,6 +20,11 @@ exp(N(0,1))):
                  V [H_kv][n][d_v] = N(0,1)
   linear_70b     bf16 B in {8192x28672, 28672x8192, 8192x10240} = N(0, 0.014);
                  A as mlp_up (d = 8192) or as mlp_down (d = 28672)
+  attn_decode    one decode step per sequence: q [B*H][n][d_h] and the K cache
+                 [B*H_kv][t][d_h] as attn_qk; V cache [B*H_kv][t][d_v] = N(0,1);
+                 P [B*H][n][t] = row softmax of N(0,2) logits (as attn_pv),
+                 each the sum of a draw shared by the query heads of one KV
+                 head and one of its own (correlation 0.5)
 These stand in for the Llama-family activations and weights the RMM paper
 evaluates on (none of which are available here).
 """
@@ -30,7 +35,7 @@ import math
 import torch
 
 __all__ = [
-    "gen", "linear_small", "mlp_up", "mlp_down", "attn_qk", "attn_pv", "linear_70b",
+    "gen", "linear_small", "mlp_up", "mlp_down", "attn_qk", "attn_pv", "attn_decode", "linear_70b",
     "duplicate_columns", "LLAMA8B_MLP", "LLAMA70B_LINEAR",
 ]
 
@@ -141,6 +146,36 @@ def attn_pv(seed: int, n: int, heads: int = 32, kv_heads: int = 8, v_dim: int = 
         del logits, p
     V = _normal((kv_heads, n, v_dim), g, device)
     return P, V.to(dtype).contiguous()
+
+
+def attn_decode(seed: int, t: int, batch: int = 1, n: int = 1, heads: int = 32, kv_heads: int = 8,
+                head_dim: int = 128, v_dim: int = 128, q_gain=None, p_gain=None, device="cpu",
+                dtype=torch.bfloat16):
+    """One decode step of `batch` sequences with t cached tokens each (query
+    heads of sequence b are b*heads .. b*heads + heads - 1, their KV heads
+    b*kv_heads ..).  Returns (q, K, V, P).  q_gain [batch*heads][head_dim]
+    scales q; p_gain [batch*heads][t] scales P after the softmax (both before
+    the final rounding)."""
+    g = gen(seed, device)
+    H, Hkv = batch * heads, batch * kv_heads
+    qs = torch.exp(_normal((H, 1, head_dim), g, device))
+    q = _normal((H, n, head_dim), g, device) * qs
+    ks = torch.exp(_normal((Hkv, 1, head_dim), g, device))
+    K = _normal((Hkv, t, head_dim), g, device) * ks
+    V = _normal((Hkv, t, v_dim), g, device)
+    group = heads // kv_heads
+    shared = _normal((Hkv, n, t), g, device).repeat_interleave(group, dim=0)
+    logits = 2.0 * math.sqrt(0.5) * (shared + _normal((H, n, t), g, device))
+    del shared
+    P = torch.softmax(logits, dim=-1)
+    del logits
+    if q_gain is not None:
+        gain = torch.as_tensor(q_gain, dtype=torch.float64).to(device)
+        q = (q.double() * gain[:, None, :]).float()
+    if p_gain is not None:
+        gain = torch.as_tensor(p_gain, dtype=torch.float64).to(device)
+        P = (P.double() * gain[:, None, :]).float()
+    return q.to(dtype).contiguous(), K.to(dtype).contiguous(), V.to(dtype).contiguous(), P.to(dtype).contiguous()
 
 
 def duplicate_columns(A: torch.Tensor, pairs) -> torch.Tensor:

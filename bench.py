@@ -596,6 +596,75 @@ def run_sweep(args):
                       "useful_tflops": flops / (t * 1e-3) / 1e12, "gbs": hbm / (t * 1e-3) / 1e9,
                       "bound": "hbm", "frac": hbm / (t * 1e-3) / 1e9 / peak_gbs, "ms_dense_torch": t_dense})
         del P, V, Vr
+    # decode step: one query row per head against t cached tokens (Llama-3.1-8B
+    # attention: 32 / 8 heads, d_h = d_v = 128, `batch` sequences); GPU time of
+    # 20 ops replayed from a CUDA graph, so that the host's launch cost is not
+    # what is timed
+    gs = torch.cuda.Stream(dev)
+
+    def graph_lat(fn, reps=20):
+        with torch.cuda.stream(gs):
+            for _ in range(3):
+                fn()
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=gs):
+            for _ in range(reps):
+                fn()
+        best = float("inf")
+        for _ in range(5):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(gs)
+            with torch.cuda.stream(gs):
+                g.replay()
+            b.record(gs)
+            torch.cuda.synchronize(dev)
+            best = min(best, a.elapsed_time(b) / reps)
+        del g
+        return best
+
+    for batch, t in ((1, 4096), (8, 4096), (8, 32768), (16, 32768)):
+        key = f"{batch}x{t}"
+        if not (want("decode", "qk", key) or want("decode", "pv", key)):
+            continue
+        q, K, V, P = W.attn_decode(1, t=t, batch=batch, device=dev)
+        H, Hkv = q.shape[0], K.shape[0]
+        for op, mode, X, Z, m in (("qk", rmm.RMM_QK, q, K, t), ("pv", rmm.RMM_PV, P, V, 128)):
+            for rho in (0.5, 0.8, 1.0):
+                if not want("decode", op, key, rho):
+                    continue
+                d = X.shape[2]
+                p = rmm.rmm_problem_init(mode, rmm.RMM_BF16, 1, d, m)
+                p.rho = rho
+                p.heads, p.kv_heads = H, Hkv
+                p.lda, p.ldb = d, Z.shape[2]
+                p.stride_a, p.stride_b = X.stride(0), Z.stride(0)
+                p.ldy, p.stride_y = m, m
+                if mode == rmm.RMM_QK:
+                    p.alpha = 1.0 / math.sqrt(d)
+                plan = rmm.Plan(p)
+                ws = rmm.workspace_for(plan, dev, gs)
+                Y = torch.empty((H, 1, m), dtype=torch.bfloat16, device=dev)
+                I = torch.empty((H, plan.k), dtype=torch.int32, device=dev)
+                t_op = graph_lat(lambda: rmm.rmm_matmul_batched(plan, X, Z, Y, I, ws, gs))
+                t_sel = graph_lat(lambda: rmm.rmm_select(plan, X, I, None, ws, gs)) if plan.k < d else 0.0
+                if mode == rmm.RMM_QK:
+                    # K in full (the scores need every key), q, S
+                    hbm = 2.0 * Hkv * t * d + 2.0 * H * d + 2.0 * H * t
+                    rec = {"kv_bytes_read": 2.0 * Hkv * t * d}
+                else:
+                    # P, the V rows of the union of each group's token sets, O
+                    grp = I.view(Hkv, -1)
+                    union = sum(int(torch.unique(grp[j]).numel()) for j in range(Hkv))
+                    hbm = 2.0 * H * t + 2.0 * union * m + 2.0 * H * m
+                    rec = {"v_rows_read": union, "v_rows_total": Hkv * t}
+                emit({"config": "decode", "op": op, "batch": batch, "t": t, "rho": rho, "k": plan.k,
+                      "ms": t_op, "ms_select": t_sel, "kernel_launches": plan.kernel_launches,
+                      "useful_gflop": 2.0 * H * plan.k * (t if mode == rmm.RMM_QK else m) / 1e9,
+                      "gbs": hbm / (t_op * 1e-3) / 1e9, "bound": "hbm",
+                      "frac": hbm / (t_op * 1e-3) / 1e9 / peak_gbs, **rec})
+        del q, K, V, P
     # 5: Llama-3-70B linear
     for shape in ("up", "down", "qkv"):
         for n in (1, 16, 512, 2048, 4096):

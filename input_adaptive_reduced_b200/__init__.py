@@ -332,6 +332,7 @@ def select(A, rho=None, k=None, return_scores=False):
     p.heads = heads
     p.kv_heads = 1
     p.stride_a = A.stride(0) if A.dim() == 3 else 0
+    p.ldy, p.stride_y = 8, n * 8  # no product: the output layout only has to be valid
     _k_fields(p, rho, k)
     plan = _plan_for(p)
     I = torch.empty((heads, plan.k) if A.dim() == 3 else (plan.k,), dtype=torch.int32, device=A.device)

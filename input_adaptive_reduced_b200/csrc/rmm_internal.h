@@ -67,6 +67,9 @@ cudaError_t launch_colnorm(const SelectArgs& a, cudaStream_t s);
 cudaError_t launch_topk(const SelectArgs& a, cudaStream_t s);
 // Scores and selection in one CTA per head (small inputs).
 cudaError_t launch_normselect(const SelectArgs& a, cudaStream_t s);
+// n = 1 bf16 rows (d <= 65535, a multiple of 8): a counting select over the
+// 15 magnitude bits, the same I as the fp32 score path.
+cudaError_t launch_select16(const SelectArgs& a, cudaStream_t s);
 // I[h][j] = j for j < k (k == d: every index kept).
 cudaError_t launch_identity(int32_t* I, int64_t k, int heads, cudaStream_t s);
 
@@ -222,6 +225,7 @@ struct rmm_plan {
     int group;          // heads / kv_heads
     bool need_select;   // scores + TopK on each call
     bool fused_select;  // one-kernel selection
+    bool select16;      // n = 1 bf16: the counting select over magnitude bits
     int nsplit;
     int64_t rows_per_split;
     int bn;

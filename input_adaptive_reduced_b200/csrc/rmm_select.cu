@@ -400,6 +400,158 @@ __global__ void __launch_bounds__(1024) normselect_kernel(const T* __restrict__ 
     radix_select_and_emit(keys, d, k, I + (int64_t)h * k, sh, false, mask ? mask + h * mask_words : nullptr);
 }
 
+// ------------------------------------------------------------------ one row
+// n = 1, bf16: column j's score is a_j^2, exact in fp32, so two scores are
+// equal exactly when |a_j| are, and they order as |a_j| does, i.e. as the 15
+// low bits of a_j's bf16 encoding (for NaN and infinity too).  The TopK is then
+// a counting select over 32768 keys: one pass of 16-bit counts (d <= 65535) in
+// 64 KiB of shared memory, the threshold key T from the counts, and the
+// emission of the kept indices in order (ties at T: the lowest indices), the
+// row re-read from L2.  One 512-thread CTA per head; three fit on an SM.
+constexpr int kSel16Threads = 512;
+constexpr int kSel16Words = 16384;  // 32768 16-bit counts
+
+__global__ void __launch_bounds__(kSel16Threads, 3) select16_kernel(const __nv_bfloat16* __restrict__ A, int64_t d,
+                                                                 int64_t stride_a, int64_t k,
+                                                                 int32_t* __restrict__ I, float* __restrict__ s2,
+                                                                 uint32_t* __restrict__ mask, int64_t mask_words) {
+    pdl_wait();
+    pdl_trigger();
+    extern __shared__ uint32_t cnt[];  // count of key 2w in the low half of word w, of key 2w+1 in the high half
+    __shared__ uint32_t part[kSel16Threads / 32];
+    __shared__ uint32_t s_T, s_gt;
+    __shared__ uint32_t warp_gt[kSel16Threads / 32], warp_eq[kSel16Threads / 32];
+    __shared__ uint32_t eq_before[kSel16Threads / 32], sel_before[kSel16Threads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int h = blockIdx.x;
+    const uint16_t* a = reinterpret_cast<const uint16_t*>(A + (int64_t)h * stride_a);
+    for (int w = tid; w < kSel16Words; w += kSel16Threads) cnt[w] = 0u;
+    __syncthreads();
+    // four 16-byte loads in flight per thread, then their 32 counts
+    const uint4* a4 = reinterpret_cast<const uint4*>(a);
+    for (int64_t q0 = tid; q0 < d / 8; q0 += 4 * kSel16Threads) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            v[u] = q0 + u * kSel16Threads < d / 8 ? __ldg(a4 + q0 + u * kSel16Threads) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (q0 + u * kSel16Threads >= d / 8) break;
+            const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const uint32_t k0 = w4[x] & 0x7fffu, k1 = (w4[x] >> 16) & 0x7fffu;
+                atomicAdd(&cnt[k0 >> 1], 1u << ((k0 & 1u) << 4));
+                atomicAdd(&cnt[k1 >> 1], 1u << ((k1 & 1u) << 4));
+            }
+        }
+    }
+    __syncthreads();
+    // thread t owns the 64 keys [32768 - 64 (t + 1), 32768 - 64 t), counted from the top
+    const int w_hi = kSel16Words - 32 * tid;  // its words are [w_hi - 32, w_hi)
+    uint32_t c = 0;
+    for (int w = w_hi - 32; w < w_hi; ++w) c += (cnt[w] & 0xffffu) + (cnt[w] >> 16);
+    const uint32_t incl = warp_incl_scan(c, lane);
+    if (lane == 31) part[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t v = lane < kSel16Threads / 32 ? part[lane] : 0u;
+        const uint32_t pi = warp_incl_scan(v, lane);
+        if (lane < kSel16Threads / 32) part[lane] = pi - v;
+    }
+    __syncthreads();
+    const uint32_t before = part[warp] + incl - c;  // keys above this thread's range
+    if (before < (uint32_t)k && (uint32_t)k <= before + c) {
+        uint32_t run = before;
+        for (int key = 2 * w_hi - 1; key >= 2 * (w_hi - 32); --key) {
+            const uint32_t ck = (cnt[key >> 1] >> ((key & 1) << 4)) & 0xffffu;
+            if (run + ck >= (uint32_t)k) {
+                s_T = (uint32_t)key;
+                s_gt = run;
+                break;
+            }
+            run += ck;
+        }
+    }
+    __syncthreads();
+    const uint32_t T = s_T, r = (uint32_t)k - s_gt;  // keys equal to T that are kept
+    // emission: warp w owns a segment of whole 32-key words
+    const int64_t seg = ((d + 31) / 32 + kSel16Threads / 32 - 1) / (kSel16Threads / 32) * 32;
+    const int64_t beg = (int64_t)warp * seg;
+    const int64_t end = min(d, beg + seg);
+    // the segment is walked in chunks of 16 steps: the chunk's 16 keys per lane
+    // are loaded together, then counted (and below emitted) from registers
+    constexpr int CH = 16;
+    uint32_t gt = 0, eq = 0;
+    for (int64_t c0 = beg; c0 < end; c0 += 32 * CH) {
+        uint16_t kk[CH];
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int64_t j = c0 + 32 * i + lane;
+            kk[i] = j < end ? a[j] : (uint16_t)0;
+        }
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const bool in = c0 + 32 * i + lane < end;
+            const uint32_t key = kk[i] & 0x7fffu;
+            gt += in && key > T;
+            eq += in && key == T;
+        }
+    }
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    eq = __reduce_add_sync(0xffffffffu, eq);
+    if (lane == 0) {
+        warp_gt[warp] = gt;
+        warp_eq[warp] = eq;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t e = lane < kSel16Threads / 32 ? warp_eq[lane] : 0u;
+        const uint32_t g = lane < kSel16Threads / 32 ? warp_gt[lane] : 0u;
+        const uint32_t eb = warp_incl_scan(e, lane) - e;
+        const uint32_t take = eb >= r ? 0u : min(e, r - eb);
+        const uint32_t sel = g + take;
+        const uint32_t sb = warp_incl_scan(sel, lane) - sel;
+        if (lane < kSel16Threads / 32) {
+            eq_before[lane] = eb;
+            sel_before[lane] = sb;
+        }
+    }
+    __syncthreads();
+    uint32_t eq_run = eq_before[warp], sel_run = sel_before[warp];
+    const uint32_t lt = (1u << lane) - 1u;
+    int32_t* Ih = I + (int64_t)h * k;
+    for (int64_t c0 = beg; c0 < end; c0 += 32 * CH) {
+        uint16_t kk[CH];
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int64_t j = c0 + 32 * i + lane;
+            kk[i] = j < end ? a[j] : (uint16_t)0;
+        }
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int64_t j0 = c0 + 32 * i;
+            if (j0 >= end) break;  // uniform over the warp
+            const int64_t j = j0 + lane;
+            const uint32_t key = kk[i] & 0x7fffu;
+            const bool is_gt = j < end && key > T;
+            const bool is_eq = j < end && key == T;
+            const unsigned em = __ballot_sync(0xffffffffu, is_eq);
+            const bool sel = is_gt || (is_eq && eq_run + __popc(em & lt) < r);
+            const unsigned sm = __ballot_sync(0xffffffffu, sel);
+            const uint32_t pos = sel_run + __popc(sm & lt);
+            if (sel && pos < (uint32_t)k) Ih[pos] = (int32_t)j;
+            if (mask && lane == 0) mask[(int64_t)h * mask_words + (j0 >> 5)] = sm;
+            if (s2 && j < end) {
+                const float x = __uint_as_float((uint32_t)kk[i] << 16);
+                s2[(int64_t)h * d + j] = x * x;
+            }
+            eq_run += __popc(em);
+            sel_run += __popc(sm);
+        }
+    }
+}
+
 __global__ void identity_kernel(int32_t* __restrict__ I, int64_t k, int heads) {
     pdl_wait();
     pdl_trigger();
@@ -468,6 +620,15 @@ cudaError_t launch_normselect(const SelectArgs& a, cudaStream_t s) {
                        a.mask_words);
     }
     return e;
+}
+
+cudaError_t launch_select16(const SelectArgs& a, cudaStream_t s) {
+    if (a.dtype != 0 || a.n != 1 || a.d > 65535 || a.d % 8 != 0) return cudaErrorInvalidValue;
+    const size_t smem = (size_t)kSel16Words * 4;
+    cudaError_t e = cudaFuncSetAttribute(select16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(select16_kernel, dim3(a.heads), dim3(kSel16Threads), smem, s, (const __nv_bfloat16*)a.A, a.d,
+                      a.stride_a, a.k, a.I, a.s2, a.mask, a.mask_words);
 }
 
 cudaError_t launch_identity(int32_t* I, int64_t k, int heads, cudaStream_t s) {

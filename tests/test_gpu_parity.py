@@ -138,6 +138,24 @@ def test_select_scores_and_indices(rmm):
         assert np.array_equal(I.cpu().numpy(), mine)
 
 
+@pytest.mark.parametrize("d", [4096, 32768])
+def test_one_row_select_ties(rmm, d):
+    """One row per head (n = 1): scores are squares of bf16 values, exact in
+    fp32, so classes of equal values are exact ties; the boundary falls inside
+    a class and its lowest indices are kept.  Values of both signs, zeros and
+    ragged k; several heads; scores returned as a_j^2."""
+    rng = np.random.default_rng(5)
+    vals = np.array([0.0, 0.5, -0.5, 1.0, -1.0, 1.5, 2.0, -2.0, 3.0, 0.125], dtype=np.float32)
+    A = torch.from_numpy(vals[rng.integers(0, len(vals), size=(3, 1, d))]).to(torch.bfloat16)
+    A64 = oracle.as_f64(A)
+    for k in (1, 7, d // 3, d // 2 + 5, d - 1):
+        I, s2 = rmm.select(A.cuda(), k=k, return_scores=True)
+        torch.cuda.synchronize()
+        for h in range(3):
+            assert np.array_equal(np64(s2[h]), oracle.column_scores_sq(A64[h]))
+            assert np.array_equal(I[h].cpu().numpy(), oracle.select(A64[h], k=k)[0])
+
+
 def test_given_indices(rmm):
     A, B = W.mlp_up(4, n=150, d=1024, m=264)
     rng = np.random.default_rng(0)

@@ -163,7 +163,9 @@ rmm_status run_select(const rmm_plan* plan, const void* A, int32_t* I, float* s2
         a.mask_words = (p.d + 31) / 32;
     }
     cudaError_t e;
-    if (plan->select16) {
+    if (plan->select_small) {
+        e = rmm::launch_select_small(a, stream);
+    } else if (plan->select16) {
         e = rmm::launch_select16(a, stream);
     } else if (plan->fused_select) {
         e = rmm::launch_normselect(a, stream);
@@ -528,7 +530,7 @@ int32_t launches_per_call(const rmm_plan* plan) {
     const bool given = (p.flags & RMM_FLAG_USE_GIVEN_INDICES) != 0;
     const bool identity = !given && plan->k == p.d;
     int32_t n = 0;
-    if (!given && !identity) n += (plan->fused_select || plan->select16) ? 1 : 2;
+    if (!given && !identity) n += (plan->fused_select || plan->select16 || plan->select_small) ? 1 : 2;
     if (p.n == 0 || p.m == 0) return n;
     if (plan->decode) return n + 1;
     if (plan->skinny) return n + (identity ? 0 : 1) + 1 + (plan->sk_splits > 1 ? 1 : 0);
@@ -629,6 +631,7 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     plan->fused_select = head_bytes <= kFusedSelectBytes && rmm::normselect_smem_bytes(p->d, p->dtype) <= 180 * 1024;
     // one bf16 row per head: a counting select over the magnitude bits
     plan->select16 = p->n == 1 && p->dtype == RMM_BF16 && p->d % 8 == 0 && p->d <= 65535;
+    plan->select_small = rmm::select_small_fits(p->n, p->d);
     // Row splits for the score pass: enough CTAs to keep HBM busy (about two
     // per SM), at most 16 partials per column, at least 64 rows each.
     const int vec = 16 / plan->es;
@@ -673,7 +676,7 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     plan->header_bytes = off;
     plan->off_partials = off;
     plan->off_scores = off;
-    if (select_possible && !plan->fused_select && !plan->select16) {
+    if (select_possible && !plan->fused_select && !plan->select16 && !plan->select_small) {
         off += align256(static_cast<size_t>(p->heads) * nsplit * p->d * sizeof(float));
         plan->off_scores = off;
         off += align256(static_cast<size_t>(p->heads) * p->d * sizeof(float));

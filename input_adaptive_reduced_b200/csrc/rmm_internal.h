@@ -67,6 +67,9 @@ cudaError_t launch_colnorm(const SelectArgs& a, cudaStream_t s);
 cudaError_t launch_topk(const SelectArgs& a, cudaStream_t s);
 // Scores and selection in one CTA per head (small inputs).
 cudaError_t launch_normselect(const SelectArgs& a, cudaStream_t s);
+// d <= 256 columns, n <= 8 rows: one warp per head ranks the columns.
+bool select_small_fits(int64_t n, int64_t d);
+cudaError_t launch_select_small(const SelectArgs& a, cudaStream_t s);
 // n = 1 bf16 rows (d <= 65535, a multiple of 8): a counting select over the
 // 15 magnitude bits, the same I as the fp32 score path.
 cudaError_t launch_select16(const SelectArgs& a, cudaStream_t s);
@@ -226,6 +229,7 @@ struct rmm_plan {
     bool need_select;   // scores + TopK on each call
     bool fused_select;  // one-kernel selection
     bool select16;      // n = 1 bf16: the counting select over magnitude bits
+    bool select_small;  // d <= 256, n <= 8: one warp per head ranks the columns
     int nsplit;
     int64_t rows_per_split;
     int bn;

@@ -400,6 +400,73 @@ __global__ void __launch_bounds__(1024) normselect_kernel(const T* __restrict__ 
     radix_select_and_emit(keys, d, k, I + (int64_t)h * k, sh, false, mask ? mask + h * mask_words : nullptr);
 }
 
+// ------------------------------------------------------------------ few features
+// d <= 256 columns and n <= 8 rows per head (attention heads at a decode
+// step): one warp per head.  The fp32 score of column j (sum of squares in row
+// order) goes to shared memory; column j is kept when its rank, the number of
+// columns with a larger score or an equal score at a lower index, is below k,
+// which is the TopK with ties to the lower index.  The kept columns are
+// emitted in order from one ballot per 32 columns.
+constexpr int kSmallMaxD = 256;
+constexpr int kSmallMaxRows = 8;
+constexpr int kSmallWarps = 8;
+
+__device__ __forceinline__ float to_float(float x) { return x; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// J: 32-column words per head (d <= 32 J)
+template <typename T, int J>
+__global__ void __launch_bounds__(32 * kSmallWarps) select_small_kernel(const T* __restrict__ A, int64_t n, int64_t d,
+                                                                       int64_t lda, int64_t stride_a, int heads,
+                                                                       int64_t k, int32_t* __restrict__ I,
+                                                                       float* __restrict__ s2, uint32_t* __restrict__ mask,
+                                                                       int64_t mask_words) {
+    pdl_wait();
+    pdl_trigger();
+    __shared__ uint32_t keys[kSmallWarps][kSmallMaxD];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int h = blockIdx.x * kSmallWarps + warp;
+    if (h >= heads) return;  // no block-wide barrier below
+    const T* Ah = A + (int64_t)h * stride_a;
+    uint32_t* key = keys[warp];
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const int f = lane + 32 * j;
+        if (f < d) {
+            float acc = 0.f;
+            for (int64_t r = 0; r < n; ++r) {
+                const float x = to_float(Ah[r * lda + f]);
+                acc = fmaf(x, x, acc);
+            }
+            key[f] = __float_as_uint(acc);
+            if (s2) s2[(int64_t)h * d + f] = acc;
+        }
+    }
+    __syncwarp();
+    uint32_t mine[J], rank[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        mine[j] = lane + 32 * j < d ? key[lane + 32 * j] : 0u;
+        rank[j] = 0u;
+    }
+    for (int f2 = 0; f2 < (int)d; ++f2) {
+        const uint32_t o = key[f2];  // the same word for every lane: a broadcast
+#pragma unroll
+        for (int j = 0; j < J; ++j) rank[j] += (o > mine[j]) || (o == mine[j] && f2 < lane + 32 * j);
+    }
+    int32_t* Ih = I + (int64_t)h * k;
+    uint32_t before = 0;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const int f = lane + 32 * j;
+        const bool kept = f < d && rank[j] < (uint32_t)k;
+        const unsigned b = __ballot_sync(0xffffffffu, kept);
+        if (kept) Ih[before + __popc(b & ((1u << lane) - 1u))] = f;
+        if (mask && lane == 0 && 32 * j < d) mask[(int64_t)h * mask_words + j] = b;
+        before += __popc(b);
+    }
+}
+
 // ------------------------------------------------------------------ one row
 // n = 1, bf16: column j's score is a_j^2, exact in fp32, so two scores are
 // equal exactly when |a_j| are, and they order as |a_j| does, i.e. as the 15
@@ -475,27 +542,36 @@ __global__ void __launch_bounds__(kSel16Threads, 3) select16_kernel(const __nv_b
     }
     __syncthreads();
     const uint32_t T = s_T, r = (uint32_t)k - s_gt;  // keys equal to T that are kept
-    // emission: warp w owns a segment of whole 32-key words
-    const int64_t seg = ((d + 31) / 32 + kSel16Threads / 32 - 1) / (kSel16Threads / 32) * 32;
+    // the counts are no longer needed: each warp stages a step's kept indices
+    // in 256 words of their space and writes them out contiguously
+    int32_t* wbuf = reinterpret_cast<int32_t*>(cnt) + warp * 256;
+    // Emission.  Warp w owns a segment of whole 256-key steps; in a step lane l
+    // holds keys [8l, 8l + 8) of it from one 16-byte load (d is a multiple of
+    // 8, so a lane's keys are all in range or all out).  Per lane, bit x of
+    // g / e marks key x above / equal to T; warp prefix sums place them.
+    const int64_t steps = (d + 255) / 256;
+    const int64_t seg = (steps + kSel16Threads / 32 - 1) / (kSel16Threads / 32) * 256;
     const int64_t beg = (int64_t)warp * seg;
     const int64_t end = min(d, beg + seg);
-    // the segment is walked in chunks of 16 steps: the chunk's 16 keys per lane
-    // are loaded together, then counted (and below emitted) from registers
-    constexpr int CH = 16;
-    uint32_t gt = 0, eq = 0;
-    for (int64_t c0 = beg; c0 < end; c0 += 32 * CH) {
-        uint16_t kk[CH];
+    auto bits_of = [&](const uint4& v, uint32_t& g, uint32_t& e) {
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        g = 0u;
+        e = 0u;
 #pragma unroll
-        for (int i = 0; i < CH; ++i) {
-            const int64_t j = c0 + 32 * i + lane;
-            kk[i] = j < end ? a[j] : (uint16_t)0;
+        for (int u = 0; u < 4; ++u) {
+            const uint32_t k0 = w4[u] & 0x7fffu, k1 = (w4[u] >> 16) & 0x7fffu;
+            g |= (uint32_t)(k0 > T) << (2 * u) | (uint32_t)(k1 > T) << (2 * u + 1);
+            e |= (uint32_t)(k0 == T) << (2 * u) | (uint32_t)(k1 == T) << (2 * u + 1);
         }
-#pragma unroll
-        for (int i = 0; i < CH; ++i) {
-            const bool in = c0 + 32 * i + lane < end;
-            const uint32_t key = kk[i] & 0x7fffu;
-            gt += in && key > T;
-            eq += in && key == T;
+    };
+    uint32_t gt = 0, eq = 0;
+    for (int64_t b0 = beg; b0 < end; b0 += 256) {
+        const int64_t j = b0 + 8 * lane;
+        if (j < end) {
+            uint32_t g, e;
+            bits_of(__ldg(reinterpret_cast<const uint4*>(a + j)), g, e);
+            gt += __popc(g);
+            eq += __popc(e);
         }
     }
     gt = __reduce_add_sync(0xffffffffu, gt);
@@ -519,35 +595,55 @@ __global__ void __launch_bounds__(kSel16Threads, 3) select16_kernel(const __nv_b
     }
     __syncthreads();
     uint32_t eq_run = eq_before[warp], sel_run = sel_before[warp];
-    const uint32_t lt = (1u << lane) - 1u;
     int32_t* Ih = I + (int64_t)h * k;
-    for (int64_t c0 = beg; c0 < end; c0 += 32 * CH) {
-        uint16_t kk[CH];
-#pragma unroll
-        for (int i = 0; i < CH; ++i) {
-            const int64_t j = c0 + 32 * i + lane;
-            kk[i] = j < end ? a[j] : (uint16_t)0;
+    for (int64_t b0 = beg; b0 < end; b0 += 256) {
+        const int64_t j = b0 + 8 * lane;
+        const bool in = j < end;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        uint32_t g = 0u, e = 0u;
+        if (in) {
+            v = __ldg(reinterpret_cast<const uint4*>(a + j));
+            bits_of(v, g, e);
         }
+        uint32_t sel = g;
+        if (__any_sync(0xffffffffu, e != 0u)) {  // ties at T: the lowest indices are kept
+            const uint32_t ec = __popc(e);
+            const uint32_t ei = warp_incl_scan(ec, lane);
+            uint32_t rank = eq_run + ei - ec;
 #pragma unroll
-        for (int i = 0; i < CH; ++i) {
-            const int64_t j0 = c0 + 32 * i;
-            if (j0 >= end) break;  // uniform over the warp
-            const int64_t j = j0 + lane;
-            const uint32_t key = kk[i] & 0x7fffu;
-            const bool is_gt = j < end && key > T;
-            const bool is_eq = j < end && key == T;
-            const unsigned em = __ballot_sync(0xffffffffu, is_eq);
-            const bool sel = is_gt || (is_eq && eq_run + __popc(em & lt) < r);
-            const unsigned sm = __ballot_sync(0xffffffffu, sel);
-            const uint32_t pos = sel_run + __popc(sm & lt);
-            if (sel && pos < (uint32_t)k) Ih[pos] = (int32_t)j;
-            if (mask && lane == 0) mask[(int64_t)h * mask_words + (j0 >> 5)] = sm;
-            if (s2 && j < end) {
-                const float x = __uint_as_float((uint32_t)kk[i] << 16);
-                s2[(int64_t)h * d + j] = x * x;
+            for (int x = 0; x < 8; ++x)
+                if ((e >> x) & 1u) {
+                    if (rank < r) sel |= 1u << x;
+                    ++rank;
+                }
+            eq_run += __shfl_sync(0xffffffffu, ei, 31);
+        }
+        const uint32_t sc = __popc(sel);
+        const uint32_t si = warp_incl_scan(sc, lane);
+        uint32_t pos = si - sc;
+#pragma unroll
+        for (int x = 0; x < 8; ++x)
+            if ((sel >> x) & 1u) wbuf[pos++] = (int32_t)(j + x);
+        __syncwarp();
+        const uint32_t nsel = __shfl_sync(0xffffffffu, si, 31);
+        for (uint32_t x = lane; x < nsel; x += 32) Ih[sel_run + x] = wbuf[x];
+        __syncwarp();  // wbuf is refilled by the next step
+        sel_run += nsel;
+        if (mask) {  // four lanes' 8 bits make one 32-key word
+            uint32_t w = sel << (8 * (lane & 3));
+            w |= __shfl_xor_sync(0xffffffffu, w, 1);
+            w |= __shfl_xor_sync(0xffffffffu, w, 2);
+            if (in && (lane & 3) == 0) mask[(int64_t)h * mask_words + (j >> 5)] = w;
+        }
+        if (s2 && in) {  // s2 is only 4-byte aligned
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            float* dst = s2 + (int64_t)h * d + j;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float x0 = __uint_as_float(w4[u] << 16), x1 = __uint_as_float(w4[u] & 0xffff0000u);
+                dst[2 * u] = x0 * x0;
+                dst[2 * u + 1] = x1 * x1;
             }
-            eq_run += __popc(em);
-            sel_run += __popc(sm);
         }
     }
 }
@@ -620,6 +716,27 @@ cudaError_t launch_normselect(const SelectArgs& a, cudaStream_t s) {
                        a.mask_words);
     }
     return e;
+}
+
+bool select_small_fits(int64_t n, int64_t d) { return n >= 1 && n <= kSmallMaxRows && d <= kSmallMaxD; }
+
+template <typename T, int J>
+cudaError_t launch_small_j(const SelectArgs& a, cudaStream_t s) {
+    const dim3 grid((unsigned)((a.heads + kSmallWarps - 1) / kSmallWarps));
+    return launch_pdl(select_small_kernel<T, J>, grid, dim3(32 * kSmallWarps), 0, s, (const T*)a.A, a.n, a.d, a.lda,
+                      a.stride_a, a.heads, a.k, a.I, a.s2, a.mask, a.mask_words);
+}
+
+template <typename T>
+cudaError_t launch_small_t(const SelectArgs& a, cudaStream_t s) {
+    if (a.d <= 64) return launch_small_j<T, 2>(a, s);
+    if (a.d <= 128) return launch_small_j<T, 4>(a, s);
+    return launch_small_j<T, 8>(a, s);
+}
+
+cudaError_t launch_select_small(const SelectArgs& a, cudaStream_t s) {
+    if (!select_small_fits(a.n, a.d)) return cudaErrorInvalidValue;
+    return a.dtype == 1 ? launch_small_t<float>(a, s) : launch_small_t<__nv_bfloat16>(a, s);
 }
 
 cudaError_t launch_select16(const SelectArgs& a, cudaStream_t s) {

@@ -138,7 +138,7 @@ def test_select_scores_and_indices(rmm):
         assert np.array_equal(I.cpu().numpy(), mine)
 
 
-@pytest.mark.parametrize("d", [4096, 32768])
+@pytest.mark.parametrize("d", [128, 4096, 32768, 40000])
 def test_one_row_select_ties(rmm, d):
     """One row per head (n = 1): scores are squares of bf16 values, exact in
     fp32, so classes of equal values are exact ties; the boundary falls inside
@@ -148,12 +148,27 @@ def test_one_row_select_ties(rmm, d):
     vals = np.array([0.0, 0.5, -0.5, 1.0, -1.0, 1.5, 2.0, -2.0, 3.0, 0.125], dtype=np.float32)
     A = torch.from_numpy(vals[rng.integers(0, len(vals), size=(3, 1, d))]).to(torch.bfloat16)
     A64 = oracle.as_f64(A)
-    for k in (1, 7, d // 3, d // 2 + 5, d - 1):
+    for k in sorted({1, 7, d // 3, d // 2 + 5, d - 1}):
         I, s2 = rmm.select(A.cuda(), k=k, return_scores=True)
         torch.cuda.synchronize()
         for h in range(3):
             assert np.array_equal(np64(s2[h]), oracle.column_scores_sq(A64[h]))
             assert np.array_equal(I[h].cpu().numpy(), oracle.select(A64[h], k=k)[0])
+
+
+def test_few_feature_select(rmm):
+    """d <= 256 columns and a few rows per head (one warp ranks a head's
+    columns): 5 heads of 3 x 200, the last 32-column word ragged."""
+    k = oracle.retained_count(0.6, 200)
+    (A, _), _ = gap.enforce_boundary_gaps(
+        lambda g: W.attn_qk(61, n=3, heads=5, kv_heads=5, head_dim=200, col_gain=g),
+        lambda x: gap.scores_per_head(x[0]), [k])
+    I, s2 = rmm.select(A.cuda(), k=k, return_scores=True)
+    torch.cuda.synchronize()
+    for h in range(5):
+        s2_ref = oracle.column_scores_sq(A[h])
+        assert np.max(np.abs(np64(s2[h]) - s2_ref) / np.maximum(s2_ref, 1e-30)) <= 3 * 2.0 ** -24 + 1e-7
+        assert np.array_equal(I[h].cpu().numpy(), oracle.select(A[h], k=k)[0])
 
 
 def test_given_indices(rmm):

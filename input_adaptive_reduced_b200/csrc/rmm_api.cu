@@ -230,6 +230,7 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         da.n = static_cast<int32_t>(p.n);
         da.group = plan->group;
         da.kv_heads = static_cast<int32_t>(p.kv_heads);
+        da.sms = plan->num_sms;
         da.alpha = p.alpha;
         const bool traced = plan->product_start && plan->product_stop;
         if (traced && cudaEventRecord(plan->product_start, stream) != cudaSuccess) return RMM_ERR_CUDA;

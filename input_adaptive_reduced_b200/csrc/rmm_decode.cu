@@ -80,14 +80,18 @@ __device__ __forceinline__ uint4 pack8(const float* y) {
 }
 
 // ------------------------------------------------------------------ qk
-// grid (ceil(t / ROWS), kv_heads), 4 warps.  Shared memory: the K tile
-// [ROWS][D + 8] (rows padded by 16 bytes: conflict-free ldmatrix), the 8
-// masked query vectors [8][D + 8] and the score tile [8][ROWS + 4] fp32.
+// grid (X, kv_heads), 4 warps, persistent: CTA x walks the KV head's ROWS-row
+// tiles x, x + X, ... with kQkStages tiles of K in flight, so that loads stay
+// in flight across tiles and the query setup is paid once.  Shared memory:
+// the K stages [kQkStages][ROWS][D + 8] (rows padded by 16 bytes:
+// conflict-free ldmatrix), the 8 masked query vectors [8][D + 8] and the
+// score tile [8][ROWS + 4] fp32.
+constexpr int kQkStages = 3;
 template <int D>
 __host__ __device__ constexpr int qk_rows() { return D == 256 ? 64 : 128; }
 template <int D>
 constexpr size_t qk_smem() {
-    return (size_t)(qk_rows<D>() + 8) * (D + 8) * 2 + (size_t)8 * (qk_rows<D>() + 4) * 4;
+    return (size_t)(kQkStages * qk_rows<D>() + 8) * (D + 8) * 2 + (size_t)8 * (qk_rows<D>() + 4) * 4;
 }
 
 template <int D>
@@ -99,20 +103,29 @@ __global__ void __launch_bounds__(128) decode_qk_kernel(const DecodeArgs a) {
     constexpr int KS = D / 16;      // MMA k-steps
     extern __shared__ __align__(16) unsigned char dsmem[];
     bf16* ks = reinterpret_cast<bf16*>(dsmem);
-    bf16* qs = ks + ROWS * LDS;
+    bf16* qs = ks + kQkStages * ROWS * LDS;
     float* ys = reinterpret_cast<float*>(qs + 8 * LDS);
     const int g = blockIdx.y;
-    const int64_t j0 = (int64_t)blockIdx.x * ROWS;
+    const int64_t tiles = (a.m + ROWS - 1) / ROWS;
     const int qvn = a.group * a.n;
     pdl_wait();
     const bf16* Kg = a.B + (int64_t)g * a.stride_b;
-    for (int c = threadIdx.x; c < ROWS * CPR; c += 128) {
-        const int r = c / CPR, q = c - r * CPR;
-        const int64_t j = j0 + r;
-        const bool in = j < a.m;
-        cp_async16(ks + r * LDS + q * 8, Kg + (in ? j : 0) * a.ldb + q * 8, in ? 16 : 0);
+    auto issue = [&](int64_t tile, int stage) {
+        bf16* dst = ks + stage * ROWS * LDS;
+        const int64_t j0 = tile * ROWS;
+        for (int c = threadIdx.x; c < ROWS * CPR; c += 128) {
+            const int r = c / CPR, q = c - r * CPR;
+            const int64_t j = j0 + r;
+            const bool in = j < a.m;
+            cp_async16(dst + r * LDS + q * 8, Kg + (in ? j : 0) * a.ldb + q * 8, in ? 16 : 0);
+        }
+    };
+#pragma unroll
+    for (int i = 0; i < kQkStages - 1; ++i) {
+        const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
+        if (tile < tiles) issue(tile, i);
+        cp_async_commit();
     }
-    cp_async_commit();
     pdl_trigger();
     // The query vectors with the features outside I_h zeroed.  One round of
     // loads: the group's query rows into registers and, from I, a flag per
@@ -169,13 +182,20 @@ __global__ void __launch_bounds__(128) decode_qk_kernel(const DecodeArgs a) {
         bq[s][0] = *reinterpret_cast<const uint32_t*>(qs + (lane >> 2) * LDS + s * 16 + (lane & 3) * 2);
         bq[s][1] = *reinterpret_cast<const uint32_t*>(qs + (lane >> 2) * LDS + s * 16 + 8 + (lane & 3) * 2);
     }
-    cp_async_wait<0>();
-    __syncthreads();
+    int it = 0;
+    for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+    const int64_t ahead = tile + (int64_t)(kQkStages - 1) * gridDim.x;
+    if (ahead < tiles) issue(ahead, (it + kQkStages - 1) % kQkStages);
+    cp_async_commit();
+    cp_async_wait<kQkStages - 1>();
+    __syncthreads();  // this tile's K is in; the previous tile's scores are stored
+    const bf16* kt = ks + (it % kQkStages) * ROWS * LDS;
+    const int64_t j0 = tile * ROWS;
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
         const int r0 = warp * (ROWS / 4) + mt * 16;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        const bf16* arow = ks + (r0 + (lane & 7) + ((lane >> 3) & 1) * 8) * LDS + (lane >> 4) * 8;
+        const bf16* arow = kt + (r0 + (lane & 7) + ((lane >> 3) & 1) * 8) * LDS + (lane >> 4) * 8;
 #pragma unroll
         for (int s = 0; s < KS; ++s) {
             uint32_t af[4];
@@ -188,7 +208,7 @@ __global__ void __launch_bounds__(128) decode_qk_kernel(const DecodeArgs a) {
         ys[qv * (ROWS + 4) + r + 8] = acc[2] * a.alpha;
         ys[(qv + 1) * (ROWS + 4) + r + 8] = acc[3] * a.alpha;
     }
-    __syncthreads();
+    __syncthreads();  // the scores are in ys; this stage is free for the next issue
     for (int c = threadIdx.x; c < qvn * (ROWS / 8); c += 128) {
         const int qv = c / (ROWS / 8), q = c - qv * (ROWS / 8);
         const int64_t j = j0 + q * 8;
@@ -196,6 +216,7 @@ __global__ void __launch_bounds__(128) decode_qk_kernel(const DecodeArgs a) {
         const int hl = qv / a.n, i = qv - hl * a.n;
         bf16* out = a.Y + (int64_t)(g * a.group + hl) * a.stride_y + (int64_t)i * a.ldy + j;
         *reinterpret_cast<uint4*>(out) = pack8(ys + qv * (ROWS + 4) + q * 8);
+    }
     }
 }
 
@@ -409,22 +430,25 @@ int decode_pv_tokens(int64_t t, int64_t kv_heads, int num_sms) {
     return tokens;
 }
 
+template <int D>
+cudaError_t launch_qk_d(const DecodeArgs& a, cudaStream_t s) {
+    const int64_t tiles = (a.m + qk_rows<D>() - 1) / qk_rows<D>();
+    // one persistent wave: about two CTAs per SM over all KV heads
+    int64_t x = 2LL * (a.sms > 0 ? a.sms : 1) / a.kv_heads;
+    x = x < 1 ? 1 : (x > tiles ? tiles : x);
+    const cudaError_t e = cudaFuncSetAttribute(decode_qk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)qk_smem<D>());
+    if (e != cudaSuccess) return e;
+    return launch_pdl(decode_qk_kernel<D>, dim3((unsigned)x, (unsigned)a.kv_heads), dim3(128), qk_smem<D>(), s, a);
+}
+
 cudaError_t launch_decode_qk(const DecodeArgs& a, cudaStream_t s) {
     if (a.m == 0) return cudaSuccess;
     switch (a.d) {
-        case 64:
-            return launch_pdl(decode_qk_kernel<64>, dim3((unsigned)((a.m + qk_rows<64>() - 1) / qk_rows<64>()), a.kv_heads),
-                              dim3(128), qk_smem<64>(), s, a);
-        case 128:
-            return launch_pdl(decode_qk_kernel<128>,
-                              dim3((unsigned)((a.m + qk_rows<128>() - 1) / qk_rows<128>()), a.kv_heads), dim3(128),
-                              qk_smem<128>(), s, a);
-        case 256:
-            return launch_pdl(decode_qk_kernel<256>,
-                              dim3((unsigned)((a.m + qk_rows<256>() - 1) / qk_rows<256>()), a.kv_heads), dim3(128),
-                              qk_smem<256>(), s, a);
-        default:
-            return cudaErrorInvalidValue;
+        case 64: return launch_qk_d<64>(a, s);
+        case 128: return launch_qk_d<128>(a, s);
+        case 256: return launch_qk_d<256>(a, s);
+        default: return cudaErrorInvalidValue;
     }
 }
 

@@ -187,6 +187,7 @@ struct DecodeArgs {
     int64_t m;               // qk: keys t; pv: d_v
     int32_t n, group, kv_heads;
     int32_t tokens;          // pv: tokens per CTA (128, 256 or 512)
+    int32_t sms;             // qk: SMs of the device (persistent grid)
     float alpha;             // qk: scale of the scores
 };
 bool decode_qk_supported(int64_t d);

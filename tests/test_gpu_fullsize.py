@@ -113,3 +113,40 @@ def test_attention_pv_full(rmm, n, causal):
             O_ref = oracle.reduced_product(P64[h], V64[g], T_ref[h], rows)
             assert_product_close(O[h][rows], O_ref, np.abs(P64[h][rows][:, T_ref[h]]),
                                  np.abs(V64[g][T_ref[h]]))
+
+
+@pytest.mark.parametrize("rho", [0.5, 0.8])
+def test_decode_full(rmm, rho):
+    """Decode step at the largest measured point: 16 sequences x 32768 cached
+    tokens, Llama-3.1-8B heads (512 query heads, 128 KV heads).  The index
+    sets of every head are compared with the oracle's (n = 1: exact squares of
+    bf16 values on both sides); scores and outputs of 16 sampled heads in full."""
+    from tests.parity import assert_heads_close
+    dev = torch.device("cuda")
+    q, K, V, P = W.attn_decode(111, t=32768, batch=16, device=dev)
+    H, Hkv = q.shape[0], K.shape[0]
+    alpha = 1.0 / math.sqrt(128)
+    S, I = rmm.qk(q, K, rho=rho, alpha=alpha, causal=False, return_indices=True)
+    O, T = rmm.pv(P, V, rho=rho, return_indices=True)
+    torch.cuda.synchronize()
+    rmm.check_workspaces()
+    q64, P64 = oracle.as_f64(q.cpu()), oracle.as_f64(P.cpu())
+    kf, kt = oracle.retained_count(rho, 128), oracle.retained_count(rho, 32768)
+    I_ref = np.stack([oracle.select(q64[h], k=kf)[0] for h in range(H)])
+    T_ref = np.stack([oracle.select(P64[h], k=kt)[0] for h in range(H)])
+    assert_indices_equal(I, I_ref)
+    assert_indices_equal(T, T_ref)
+    heads = sorted(np.random.default_rng(7).choice(H, size=16, replace=False).tolist())
+    S_ref, O_ref, aS, bS, aO, bO = [], [], [], [], [], []
+    for h in heads:
+        g = oracle.kv_head_of(h, H, Hkv)
+        K64, V64 = oracle.as_f64(K[g].cpu()), oracle.as_f64(V[g].cpu())
+        S_ref.append(oracle.reduced_scores(q64[h], K64, I_ref[h], alpha, False))
+        aS.append(np.abs(q64[h][:, I_ref[h]]))
+        bS.append(np.abs(K64[:, I_ref[h]]).T)
+        O_ref.append(oracle.reduced_product(P64[h], V64, T_ref[h]))
+        aO.append(np.abs(P64[h][:, T_ref[h]]))
+        bO.append(np.abs(V64[T_ref[h]]))
+    idx = torch.tensor(heads, device=dev)
+    assert_heads_close(S[idx], np.stack(S_ref), aS, bS, alpha=alpha)
+    assert_heads_close(O[idx], np.stack(O_ref), aO, bO)

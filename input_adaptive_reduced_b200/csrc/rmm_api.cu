@@ -202,7 +202,7 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
     // ---- index set
     int32_t* I = I_inout ? I_inout : ws_at<int32_t>(ws, plan->off_I);
     const bool identity = !given && k == p.d;
-    if (!given) {
+    if (!given && !plan->decode_select) {
         if (identity) {
             if (I_inout && rmm::launch_identity(I_inout, k, static_cast<int>(p.heads), stream) != cudaSuccess)
                 return RMM_ERR_CUDA;
@@ -236,7 +236,9 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         if (traced && cudaEventRecord(plan->product_start, stream) != cudaSuccess) return RMM_ERR_CUDA;
         cudaError_t e;
         if (p.mode == RMM_QK) {
-            da.I = identity ? nullptr : I;
+            da.I = identity || plan->decode_select ? nullptr : I;
+            da.fused_select = plan->decode_select ? 1 : 0;
+            da.I_out = plan->decode_select ? I_inout : nullptr;
             e = rmm::launch_decode_qk(da, stream);
         } else {
             da.mask = identity ? nullptr : ws_at<uint32_t>(ws, plan->off_dec_mask);
@@ -531,7 +533,8 @@ int32_t launches_per_call(const rmm_plan* plan) {
     const bool given = (p.flags & RMM_FLAG_USE_GIVEN_INDICES) != 0;
     const bool identity = !given && plan->k == p.d;
     int32_t n = 0;
-    if (!given && !identity) n += (plan->fused_select || plan->select16 || plan->select_small) ? 1 : 2;
+    if (!given && !identity && !plan->decode_select)
+        n += (plan->fused_select || plan->select16 || plan->select_small) ? 1 : 2;
     if (p.n == 0 || p.m == 0) return n;
     if (plan->decode) return n + 1;
     if (plan->skinny) return n + (identity ? 0 : 1) + 1 + (plan->sk_splits > 1 ? 1 : 0);
@@ -605,6 +608,7 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
         plan->pack_b = false;
         plan->pv_mask = false;
     }
+    plan->decode_select = plan->decode && p->mode == RMM_QK && plan->need_select;
     plan->pack_ab = plan->pack_b && rmm::pack_ab_one_launch(p->dtype, plan->ldp);
 
     int dev = 0, sms = 0;

@@ -165,6 +165,58 @@ __global__ void __launch_bounds__(128) decode_qk_kernel(const DecodeArgs a) {
         const int e = threadIdx.x + j * 128;
         if (e < nI && fk[j] >= 0 && fk[j] < D) kept[e / (int)a.k][fk[j]] = 1;
     }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (a.fused_select) {
+        // The selection of each head's k features, in the CTA: the raw query
+        // rows go to shared memory, warp w ranks the features of heads w, w + 4
+        // (fp32 sums of squares in row order; rank = #{larger score, or equal
+        // at a lower index}; kept iff rank < k) and the first CTA of the KV head
+        // writes I in order.
+        __shared__ uint32_t keyf[4][D];  // one head's scores per warp (two CTAs still fit an SM)
+#pragma unroll
+        for (int j = 0; j < QPT; ++j) {
+            const int e = threadIdx.x + j * 128;
+            const int qv = e / (D / 2), f = (e - qv * (D / 2)) * 2;
+            *reinterpret_cast<uint32_t*>(qs + qv * LDS + f) = qreg[j];
+        }
+        __syncthreads();
+        constexpr int J = D / 32;
+        for (int hl = warp; hl < a.group; hl += 4) {
+            uint32_t mine[J], rank[J];
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                const int f = lane + 32 * j;
+                float sc = 0.f;
+                for (int i = 0; i < a.n; ++i) {
+                    const float x = __bfloat162float(qs[(hl * a.n + i) * LDS + f]);
+                    sc = fmaf(x, x, sc);
+                }
+                mine[j] = __float_as_uint(sc);
+                keyf[warp][f] = mine[j];
+                rank[j] = 0u;
+            }
+            __syncwarp();
+            for (int f2 = 0; f2 < D; ++f2) {
+                const uint32_t o = keyf[warp][f2];  // one word for every lane: a broadcast
+#pragma unroll
+                for (int j = 0; j < J; ++j) rank[j] += (o > mine[j]) || (o == mine[j] && f2 < lane + 32 * j);
+            }
+            uint32_t before = 0;
+            const bool emit = a.I_out && blockIdx.x == 0;
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                const int f = lane + 32 * j;
+                const bool kp = rank[j] < (uint32_t)a.k;
+                kept[hl][f] = kp ? 1 : 0;
+                if (emit) {
+                    const unsigned b = __ballot_sync(0xffffffffu, kp);
+                    if (kp) a.I_out[(int64_t)(g * a.group + hl) * a.k + before + __popc(b & ((1u << lane) - 1u))] = f;
+                    before += __popc(b);
+                }
+            }
+            __syncwarp();  // keyf[warp] holds the next head's scores next
+        }
+    }
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < QPT; ++j) {
@@ -175,7 +227,6 @@ __global__ void __launch_bounds__(128) decode_qk_kernel(const DecodeArgs a) {
         *reinterpret_cast<uint32_t*>(qs + qv * LDS + f) = qreg[j] & (lo | hi);
     }
     __syncthreads();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t bq[KS][2];
 #pragma unroll
     for (int s = 0; s < KS; ++s) {

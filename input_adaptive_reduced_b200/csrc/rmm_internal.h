@@ -175,7 +175,8 @@ struct DecodeArgs {
     int64_t lda, stride_a;
     const __nv_bfloat16* B;  // qk: K [kv_heads][t][d]; pv: V [kv_heads][t][d_v]
     int64_t ldb, stride_b;
-    const int32_t* I;        // qk: [heads][k] kept features, nullptr = all
+    const int32_t* I;        // qk: [heads][k] kept features, nullptr = all (or selected in the kernel)
+    int32_t* I_out;          // qk with fused_select: where the selected I goes, or nullptr
     const uint32_t* mask;    // pv: [heads][mask_words] kept tokens (bit t of word t / 32), nullptr = all
     int64_t mask_words;
     __nv_bfloat16* Y;        // qk: S [heads][n][t]; pv: O [heads][n][d_v]
@@ -188,6 +189,7 @@ struct DecodeArgs {
     int32_t n, group, kv_heads;
     int32_t tokens;          // pv: tokens per CTA (128, 256 or 512)
     int32_t sms;             // qk: SMs of the device (persistent grid)
+    int32_t fused_select;    // qk: select each head's k features in the kernel (I unused)
     float alpha;             // qk: scale of the scores
 };
 bool decode_qk_supported(int64_t d);
@@ -246,6 +248,7 @@ struct rmm_plan {
     int split_tiles, split_f;           // split tail of the CTA-pair product (0, 1: none)
     size_t off_split_cnt, off_split;    // its counters (in the header) and fp32 partials
     bool decode;        // bf16 attention with group * n <= 8 query vectors per KV head (rmm_decode.cu)
+    bool decode_select; // decode QK: the features are selected inside the product kernel
     int dec_tokens, dec_parts;          // pv: tokens per CTA, token ranges per KV head
     size_t off_dec_cnt, off_dec_mask, off_dec_part;  // pv: counters (header), membership words, partials
 };

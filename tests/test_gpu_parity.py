@@ -504,10 +504,11 @@ def _launches(rmm, mode, X, Z, m, rho):
 @pytest.mark.parametrize("rho", [0.5, 0.8, 1.0])
 @pytest.mark.parametrize("case", DECODE_CASES)
 def test_decode_qk(rmm, case, rho):
-    """Scores of a decode step: the group's query vectors against each K row once."""
+    """Scores of a decode step: the group's query vectors against each K row once,
+    the features selected inside the same kernel (one launch)."""
     q, K, _, _ = _decode_inputs(case, 81, "q_gain")
     H, n, dh = q.shape
-    assert _launches(rmm, rmm.RMM_QK, q, K, K.shape[1], rho) == (1 if rho < 1 else 0) + 1
+    assert _launches(rmm, rmm.RMM_QK, q, K, K.shape[1], rho) == 1
     alpha = 1.0 / math.sqrt(dh)
     S, I = rmm.qk(q.cuda(), K.cuda(), rho=rho, alpha=alpha, causal=False, return_indices=True)
     torch.cuda.synchronize()

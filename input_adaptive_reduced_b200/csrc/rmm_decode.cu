@@ -17,7 +17,9 @@
 // qk: S[h][i][j] = alpha * sum_{f in I_h} Q[h][i][f] K[g][j][f].  The query
 //   vectors, with the features outside I_h set to zero, are the MMA's 8-column
 //   operand; K as stored is the 16-row operand, so the contraction runs over
-//   every feature and each zeroed term adds an exact zero.
+//   every feature and each zeroed term adds an exact zero.  I_h is selected in
+//   the kernel from the query rows it loads (each CTA ranks its group's d_h
+//   features; the first CTA of a KV head writes I), unless a given I is passed.
 // pv: O[h][i][:] = sum_{t in T_h} P[h][i][t] V[g][t][:].  A CTA takes a range of
 //   tokens, forms the union of the group's token sets over it from the
 //   selection's membership bits, gathers only those V rows, and weighs row t

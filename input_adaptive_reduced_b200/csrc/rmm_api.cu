@@ -207,7 +207,11 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
             if (I_inout && rmm::launch_identity(I_inout, k, static_cast<int>(p.heads), stream) != cudaSuccess)
                 return RMM_ERR_CUDA;
         } else {
-            st = run_select(plan, A, I, nullptr, ws, stream);
+            // the decode PV product reads the membership words only: without
+            // I_inout the one-row select writes no index list
+            const bool words_only =
+                plan->decode && p.mode == RMM_PV && plan->select16 && !plan->select_small && !I_inout;
+            st = run_select(plan, A, words_only ? nullptr : I, nullptr, ws, stream);
             if (st != RMM_OK) return st;
         }
     }

@@ -595,7 +595,7 @@ __global__ void __launch_bounds__(kSel16Threads, 3) select16_kernel(const __nv_b
     }
     __syncthreads();
     uint32_t eq_run = eq_before[warp], sel_run = sel_before[warp];
-    int32_t* Ih = I + (int64_t)h * k;
+    int32_t* Ih = I ? I + (int64_t)h * k : nullptr;  // nullptr: only the membership words are wanted
     for (int64_t b0 = beg; b0 < end; b0 += 256) {
         const int64_t j = b0 + 8 * lane;
         const bool in = j < end;
@@ -618,17 +618,19 @@ __global__ void __launch_bounds__(kSel16Threads, 3) select16_kernel(const __nv_b
                 }
             eq_run += __shfl_sync(0xffffffffu, ei, 31);
         }
-        const uint32_t sc = __popc(sel);
-        const uint32_t si = warp_incl_scan(sc, lane);
-        uint32_t pos = si - sc;
+        if (Ih) {
+            const uint32_t sc = __popc(sel);
+            const uint32_t si = warp_incl_scan(sc, lane);
+            uint32_t pos = si - sc;
 #pragma unroll
-        for (int x = 0; x < 8; ++x)
-            if ((sel >> x) & 1u) wbuf[pos++] = (int32_t)(j + x);
-        __syncwarp();
-        const uint32_t nsel = __shfl_sync(0xffffffffu, si, 31);
-        for (uint32_t x = lane; x < nsel; x += 32) Ih[sel_run + x] = wbuf[x];
-        __syncwarp();  // wbuf is refilled by the next step
-        sel_run += nsel;
+            for (int x = 0; x < 8; ++x)
+                if ((sel >> x) & 1u) wbuf[pos++] = (int32_t)(j + x);
+            __syncwarp();
+            const uint32_t nsel = __shfl_sync(0xffffffffu, si, 31);
+            for (uint32_t x = lane; x < nsel; x += 32) Ih[sel_run + x] = wbuf[x];
+            __syncwarp();  // wbuf is refilled by the next step
+            sel_run += nsel;
+        }
         if (mask) {  // four lanes' 8 bits make one 32-key word
             uint32_t w = sel << (8 * (lane & 3));
             w |= __shfl_xor_sync(0xffffffffu, w, 1);

@@ -91,3 +91,45 @@ def test_pv_dense_special_case_and_bound():
             bound = np.sum(np.linalg.norm(P[h][:, drop], axis=0) *
                            np.linalg.norm(V[h // 2][drop, :], axis=1))
             assert np.linalg.norm(P[h] @ V[h // 2] - O[h]) <= bound * (1 + 1e-12) + 1e-15
+
+
+def test_decode_one_row_selection_is_a_magnitude_sort():
+    """Appendix D.1, the decode case: one query row per head.  With n = 1 the
+    column norm of column j is |a_j|, so the oracle's TopK must equal the k
+    largest magnitudes in a stable library sort (equal magnitudes in index
+    order, which is the lower-index tie rule), returned ascending.  Values of
+    both signs, zeros and exact ties."""
+    rng = np.random.default_rng(17)
+    vals = np.array([0.0, 0.5, -0.5, 1.0, -1.0, 2.0, -3.0, 0.25])
+    for d in (7, 64, 1000):
+        a = vals[rng.integers(0, len(vals), size=(1, d))]
+        for k in sorted({1, 3, d // 2, d - 1}):
+            order = np.argsort(-np.abs(a[0]), kind="stable")
+            expect = np.sort(order[:k]).astype(np.int32)
+            got, _ = oracle.select(a, k=k)
+            assert np.array_equal(np.asarray(got), expect), (d, k)
+
+
+def test_decode_group_scores_and_values():
+    """Decode-step forms on the oracle's per-head functions: with one query row,
+    QK's scores at rho = 1 equal alpha * q K^T (numpy) for every KV head's
+    query heads, and PV's output at rho = 1 equals P V (numpy); below rho = 1
+    the PV error obeys the bound of Prop. 1 per head."""
+    rng = np.random.default_rng(23)
+    H, Hkv, t, dh = 8, 2, 40, 16
+    q = rng.standard_normal((H, 1, dh))
+    K = rng.standard_normal((Hkv, t, dh))
+    V = rng.standard_normal((Hkv, t, dh))
+    P = rng.random((H, 1, t))
+    S, _ = oracle.rmm_qk(q, K, rho=1.0, alpha=0.25, causal=False)
+    O, _ = oracle.rmm_pv(P, V, rho=1.0)
+    for h in range(H):
+        g = h // (H // Hkv)
+        np.testing.assert_allclose(S[h], 0.25 * q[h] @ K[g].T, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(O[h], P[h] @ V[g], rtol=1e-12, atol=1e-12)
+    O5, T5 = oracle.rmm_pv(P, V, rho=0.5)
+    for h in range(H):
+        g = h // (H // Hkv)
+        drop = np.setdiff1d(np.arange(t), T5[h])
+        bound = sum(np.abs(P[h][0, j]) * np.linalg.norm(V[g][j]) for j in drop)
+        assert np.linalg.norm(P[h] @ V[g] - O5[h]) <= bound * (1 + 1e-12) + 1e-12

@@ -15,6 +15,7 @@ import ctypes
 import math
 import os
 import threading
+import weakref
 
 __all__ = [
     "RMM_OK", "RMM_ERR_INVALID_ARG", "RMM_ERR_UNSUPPORTED", "RMM_ERR_WORKSPACE", "RMM_ERR_CUDA",
@@ -148,6 +149,7 @@ class Plan:
         self.workspace_bytes = int(ws.value)
         self.k = int(lib.rmm_plan_k(h))
         self.kernel_launches = int(lib.rmm_plan_kernel_launches(h))
+        self._ws = {}  # (device index, stream) -> workspace; released with the plan
 
     def set_product_events(self, start=None, stop=None):
         """Bracket the reduced-product kernel of later calls with torch.cuda.Event
@@ -246,7 +248,7 @@ def rmm_matmul_batched(plan: Plan, A, B, Y, I=None, workspace=None, stream=None)
 # ----------------------------------------------------------------------------
 _cache_lock = threading.Lock()
 _plans: dict = {}
-_workspaces: dict = {}
+_ws_plans = weakref.WeakSet()  # plans that own a workspace (for check_workspaces)
 
 
 def _dtype_code(t) -> int:
@@ -285,18 +287,22 @@ def _plan_for(p: rmm_problem) -> Plan:
 
 
 def workspace_for(plan: Plan, device=None, stream=None):
-    """A zero-initialised workspace for a plan, cached per (plan, device, stream)."""
+    """A zero-initialised workspace for a plan, kept on the plan per (device,
+    stream): it lives as long as the plan, and a later plan never inherits it
+    (its counters are laid out for this plan)."""
     import torch
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     s = torch.cuda.current_stream(dev) if stream is None else stream
-    key = (id(plan), dev.index, s.cuda_stream)
+    key = (dev.index, s.cuda_stream)
     with _cache_lock:
-        ws = _workspaces.get(key)
+        ws = plan._ws.get(key)
     if ws is None or ws.numel() < plan.workspace_bytes:
         ws = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device=dev)
+        ws.record_stream(s)  # used on s: not reused before s's work on it is done
         rmm_workspace_init(plan, ws, s)
         with _cache_lock:
-            _workspaces[key] = ws
+            plan._ws[key] = ws
+            _ws_plans.add(plan)
     return ws
 
 
@@ -304,12 +310,9 @@ def check_workspaces():
     """Synchronise and read the error word of every workspace this module
     allocated; raise RmmError(RMM_ERR_TIMEOUT) if a kernel gave up on a wait."""
     with _cache_lock:
-        items = list(_workspaces.items())
-        plans = {id(p): p for p in _plans.values()}
-    for (pid, _dev, _s), ws in items:
-        plan = plans.get(pid)
-        if plan is not None:
-            _check(rmm_workspace_status(plan, ws), "kernel wait")
+        items = [(p, ws) for p in list(_ws_plans) for ws in list(p._ws.values())]
+    for plan, ws in items:
+        _check(rmm_workspace_status(plan, ws), "kernel wait")
 
 
 def _k_fields(p: rmm_problem, rho, k):

@@ -561,3 +561,60 @@ def test_decode_rows_past_the_group_take_the_general_path(rmm):
     assert_indices_equal(T, T_ref)
     _decode_qk_close(S, S_ref, I_ref, q, K, 0.1)
     _decode_pv_close(O, O_ref, T_ref, P, V)
+
+
+def test_decode_strided_views(rmm):
+    """Decode ops on views with padded rows and head strides (q and the K / V
+    caches 136 wide holding d_h = 128, P 8 tokens longer than t): the kernels
+    use the leading dimensions and head strides they are given."""
+    t, H, Hkv = 1000, 32, 8
+    q, K, V, P = W.attn_decode(85, t=t, batch=1)
+    dev = torch.device("cuda")
+    def padded(x, extra):
+        big = torch.zeros(x.shape[:-1] + (x.shape[-1] + extra,), dtype=x.dtype, device=dev)
+        big[..., : x.shape[-1]] = x.to(dev)
+        return big[..., : x.shape[-1]]
+    qv, Kv, Vv, Pv = padded(q, 8), padded(K, 8), padded(V, 8), padded(P, 8)
+    assert Kv.stride(1) == 136 and Pv.stride(0) == t + 8
+    alpha = 1.0 / math.sqrt(128)
+    S, I = rmm.qk(qv, Kv, rho=0.5, alpha=alpha, causal=False, return_indices=True)
+    O, T = rmm.pv(Pv, Vv, rho=0.5, return_indices=True)
+    torch.cuda.synchronize()
+    S_ref, I_ref = oracle.rmm_qk(q, K, rho=0.5, alpha=alpha, causal=False)
+    O_ref, T_ref = oracle.rmm_pv(P, V, rho=0.5)
+    assert_indices_equal(I, I_ref)
+    assert_indices_equal(T, T_ref)
+    _decode_qk_close(S, S_ref, I_ref, q, K, alpha)
+    _decode_pv_close(O, O_ref, T_ref, P, V)
+
+
+def test_workspace_belongs_to_its_plan(rmm):
+    """A plan's workspace is zero-initialised for that plan's layout and dies
+    with it: a new plan, even one that takes a dead plan's Python id, gets its
+    own workspace, and the decode PV op (whose range counters sit in the
+    workspace header) still matches the oracle."""
+    import gc
+    q, K, V, P = W.attn_decode(86, t=1000, batch=1)
+    Pg, Vg = P.cuda(), V.cuda()
+    seen = []
+    for rho in (0.5, 0.8, 0.5, 0.7):
+        p = rmm.rmm_problem_init(rmm.RMM_PV, rmm.RMM_BF16, 1, 1000, 128)
+        p.rho = rho
+        p.heads, p.kv_heads = 32, 8
+        p.lda, p.ldb = 1000, 128
+        p.stride_a, p.stride_b = Pg.stride(0), Vg.stride(0)
+        p.ldy, p.stride_y = 128, 128
+        plan = rmm.Plan(p)
+        ws = rmm.workspace_for(plan)
+        assert all(ws is not w for w in seen)
+        seen.append(ws)
+        O = torch.empty((32, 1, 128), dtype=torch.bfloat16, device="cuda")
+        T = torch.empty((32, plan.k), dtype=torch.int32, device="cuda")
+        rmm.rmm_matmul_batched(plan, Pg, Vg, O, T, ws)
+        torch.cuda.synchronize()
+        O_ref, T_ref = oracle.rmm_pv(P, V, rho=rho)
+        assert_indices_equal(T, T_ref)
+        _decode_pv_close(O, O_ref, T_ref, P, V)
+        del plan, ws
+        gc.collect()
+    rmm.check_workspaces()

@@ -275,6 +275,27 @@ def test_split_tail_pv(rmm):
     rmm.check_workspaces()
 
 
+@pytest.mark.parametrize("rho", [0.5, 0.9])
+def test_attention_pv_wide_values(rmm, rho):
+    """PV with value heads wider than 256 (no masked-V path): P's kept columns
+    are packed and V's kept rows copied per query head (grouped-query V heads);
+    at rho = 0.9 (k = 1080 > 1024) both in one launch, at 0.5 the narrow pack."""
+    H, Hkv, n, dv = 4, 2, 1200, 320
+    ks = [oracle.retained_count(r, n) for r in (0.5, 0.9)]
+    (P, V), _ = gap.enforce_boundary_gaps(
+        lambda g: W.attn_pv(44, n=n, heads=H, kv_heads=Hkv, v_dim=dv, col_gain=g),
+        lambda x: gap.scores_per_head(x[0]), ks)
+    O, T = rmm.pv(P.cuda(), V.cuda(), rho=rho, return_indices=True)
+    torch.cuda.synchronize()
+    O_ref, T_ref = oracle.rmm_pv(P, V, rho=rho)
+    assert_indices_equal(T, T_ref)
+    P64, V64 = oracle.as_f64(P), oracle.as_f64(V)
+    for h in range(H):
+        g = oracle.kv_head_of(h, H, Hkv)
+        assert_product_close(O[h], O_ref[h], np.abs(P64[h][:, T_ref[h]]), np.abs(V64[g][T_ref[h]]))
+    rmm.check_workspaces()
+
+
 def test_cuda_graph_capture(rmm):
     """Every kernel is launched with programmatic serialisation and the ops never
     synchronise with the host: a CUDA graph of linear (CTA-pair product with a

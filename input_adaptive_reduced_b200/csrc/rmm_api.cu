@@ -492,7 +492,7 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         pb.stride_dst = k * p.m;
         pb.heads = static_cast<int>(p.heads);
         const cudaError_t e = plan->pack_ab ? rmm::launch_pack_ab(pa_deferred, pb, stream)
-                                            : rmm::launch_pack_rows(pb, plan->num_sms, stream);
+                                            : rmm::launch_pack_rows(pb, stream);
         if (e != cudaSuccess) return RMM_ERR_CUDA;
         gl.b_mode = rmm::kBRows;
         gp.group = 1;

@@ -103,10 +103,10 @@ cudaError_t launch_mask_columns(const PackArgs& a, cudaStream_t s);
 cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s);
 // dst[h][t][:] = src[h / group][I[h][t]][:] for t < k: the retained rows of a
 // row-major B, contiguous (a.rows = number of columns of B).
-cudaError_t launch_pack_rows(const PackArgs& a, int num_sms, cudaStream_t s);
-// launch_pack(a) and launch_pack_rows(b) as one launch, their CTAs interleaved
-// (bf16, packed A rows wider than the narrow variant's; pack_ab_one_launch says
-// whether an A pack qualifies).
+cudaError_t launch_pack_rows(const PackArgs& a, cudaStream_t s);
+// launch_pack(a) and launch_pack_rows(b) as one launch: the A pack's CTAs, then
+// the row copy's (bf16, packed A rows wider than the narrow variant's;
+// pack_ab_one_launch says whether an A pack qualifies).
 bool pack_ab_one_launch(int dtype, int64_t ld_a);
 cudaError_t launch_pack_ab(const PackArgs& a, const PackArgs& b, cudaStream_t s);
 // dst[h][t][:] = src[h / group][t][:] if t is in I[h][0..k) (ascending, unique)

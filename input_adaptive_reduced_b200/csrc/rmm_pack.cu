@@ -330,8 +330,7 @@ cudaError_t launch_mask_columns(const PackArgs& a, cudaStream_t s) {
                       a.stride_dst);
 }
 
-cudaError_t launch_pack_rows(const PackArgs& a, int num_sms, cudaStream_t s) {
-    (void)num_sms;
+cudaError_t launch_pack_rows(const PackArgs& a, cudaStream_t s) {
     if (a.k == 0 || a.rows == 0) return cudaSuccess;
     dim3 grid((unsigned)((a.k + kRowsPerCta - 1) / kRowsPerCta), (unsigned)a.heads);
     if (a.dtype == 1)

@@ -282,9 +282,15 @@ __global__ void __launch_bounds__(128) decode_qk_kernel(const DecodeArgs a) {
 // accumulates a 16 x DV tile (rows = query vectors, 8 used) over them.
 constexpr int kPvMaxTok = 512;
 constexpr int kPvStages = 2;
+// dynamic shared memory: the per-warp V stages (reused for the warp sums), then
+// the staged P rows of the qvn query vectors over a range of `tokens`
 template <int DV>
-constexpr size_t pv_smem() {
-    return (size_t)4 * kPvStages * 16 * (DV + 8) * 2;  // per-warp V stages; reused for the warp sums
+__host__ __device__ constexpr size_t pv_stage_bytes() {
+    return (size_t)4 * kPvStages * 16 * (DV + 8) * 2;
+}
+template <int DV>
+size_t pv_smem(int qvn, int tokens) {
+    return pv_stage_bytes<DV>() + (size_t)qvn * (tokens + 8) * 2;
 }
 
 template <int DV>
@@ -295,7 +301,7 @@ __global__ void __launch_bounds__(128) decode_pv_kernel(const DecodeArgs a) {
     extern __shared__ __align__(16) unsigned char dsmem[];
     bf16* vs = reinterpret_cast<bf16*>(dsmem);           // [4 warps][stages][16][LDS]
     float* red = reinterpret_cast<float*>(dsmem);        // [4 warps][8][DV] after the loop
-    __shared__ __align__(16) bf16 ps[8][kPvMaxTok + 8];  // P rows of the query vectors over the range
+    bf16* ps = reinterpret_cast<bf16*>(dsmem + pv_stage_bytes<DV>());  // [qvn][tokens + 8]
     __shared__ uint32_t mw[8][kPvMaxTok / 32];           // membership words per group head
     __shared__ int32_t tok[kPvMaxTok];                   // union of the group's tokens, ascending
     __shared__ uint8_t bits[kPvMaxTok];                  // which group heads kept each listed token
@@ -313,7 +319,7 @@ __global__ void __launch_bounds__(128) decode_pv_kernel(const DecodeArgs a) {
     for (int c = threadIdx.x; c < qvn * (tn / 8); c += 128) {
         const int qv = c / (tn / 8), q = c - qv * (tn / 8);
         const int hl = qv / a.n, i = qv - hl * a.n;
-        cp_async16(&ps[qv][q * 8], a.A + (int64_t)(g * a.group + hl) * a.stride_a + (int64_t)i * a.lda + t0 + q * 8,
+        cp_async16(ps + qv * (a.tokens + 8) + q * 8, a.A + (int64_t)(g * a.group + hl) * a.stride_a + (int64_t)i * a.lda + t0 + q * 8,
                    16);
     }
     cp_async_commit();
@@ -392,7 +398,7 @@ __global__ void __launch_bounds__(128) decode_pv_kernel(const DecodeArgs a) {
             for (int u = 0; u < 2; ++u) {
                 const int pos = s * 16 + kk + half * 8 + u;
                 bf16 w = __float2bfloat16_rn(0.f);
-                if (qv < qvn && pos < nu && ((bits[pos] >> hl) & 1u)) w = ps[qv][tok[pos] - (int)t0];
+                if (qv < qvn && pos < nu && ((bits[pos] >> hl) & 1u)) w = ps[qv * (a.tokens + 8) + tok[pos] - (int)t0];
                 e[u] = w;
             }
             v[half] = pack_bf16x2(e[0], e[1]);
@@ -508,8 +514,9 @@ cudaError_t launch_decode_qk(const DecodeArgs& a, cudaStream_t s) {
 cudaError_t launch_decode_pv(const DecodeArgs& a, cudaStream_t s) {
     if (a.d == 0 || a.tokens <= 0 || a.tokens > kPvMaxTok) return cudaErrorInvalidValue;
     const dim3 grid((unsigned)((a.d + a.tokens - 1) / a.tokens), a.kv_heads);
-    if (a.m == 64) return launch_pdl(decode_pv_kernel<64>, grid, dim3(128), pv_smem<64>(), s, a);
-    if (a.m == 128) return launch_pdl(decode_pv_kernel<128>, grid, dim3(128), pv_smem<128>(), s, a);
+    const int qvn = a.group * a.n;
+    if (a.m == 64) return launch_pdl(decode_pv_kernel<64>, grid, dim3(128), pv_smem<64>(qvn, a.tokens), s, a);
+    if (a.m == 128) return launch_pdl(decode_pv_kernel<128>, grid, dim3(128), pv_smem<128>(qvn, a.tokens), s, a);
     return cudaErrorInvalidValue;
 }
 

@@ -51,3 +51,33 @@ def test_boundary_gap_enforcement():
     s2 = oracle.column_scores_sq(A)
     for k in ks:
         assert gap.boundary_gap(s2, k) >= 1e-3
+
+
+def test_attn_decode_shapes_and_structure():
+    """The decode-step generator: shapes for `batch` sequences, seeded, P rows
+    summing to one, the gains applied where documented, and the query heads of
+    one KV head weighing tokens more alike than heads of different KV heads
+    (the shared half of their logits)."""
+    q, K, V, P = W.attn_decode(3, t=512, batch=2, n=1, heads=8, kv_heads=2, head_dim=64, v_dim=32)
+    assert q.shape == (16, 1, 64) and K.shape == (4, 512, 64) and V.shape == (4, 512, 32)
+    assert P.shape == (16, 1, 512) and P.dtype == torch.bfloat16
+    q2, K2, V2, P2 = W.attn_decode(3, t=512, batch=2, n=1, heads=8, kv_heads=2, head_dim=64, v_dim=32)
+    assert all(torch.equal(a, b) for a, b in ((q, q2), (K, K2), (V, V2), (P, P2)))
+    assert torch.allclose(P.float().sum(-1), torch.ones(16, 1), atol=2e-2)
+    # logits' correlation: heads 0-3 share KV head 0, heads 4-7 KV head 1
+    lg = torch.log(P.float().clamp_min(1e-30))[:, 0]
+    lg = lg - lg.mean(-1, keepdim=True)
+    c = (lg @ lg.T) / (lg.norm(dim=-1)[:, None] * lg.norm(dim=-1)[None, :])
+    same = float(c[0, 1:4].mean())
+    other = float(c[0, 4:8].mean())
+    assert same > 0.35 and abs(other) < 0.2, (same, other)
+    g = np.ones((16, 64))
+    g[:, 5] = 4.0
+    qg = W.attn_decode(3, t=512, batch=2, n=1, heads=8, kv_heads=2, head_dim=64, v_dim=32, q_gain=g)[0]
+    assert torch.allclose(qg.float()[:, :, 5], (4.0 * q.float()[:, :, 5]).to(torch.bfloat16).float())
+    assert torch.equal(qg[:, :, 6], q[:, :, 6])
+    gp = np.ones((16, 512))
+    gp[:, 7] = 0.5
+    Pg = W.attn_decode(3, t=512, batch=2, n=1, heads=8, kv_heads=2, head_dim=64, v_dim=32, p_gain=gp)[3]
+    assert torch.equal(Pg[:, :, 8], P[:, :, 8])
+    assert torch.allclose(Pg.float()[:, :, 7], 0.5 * P.float()[:, :, 7], rtol=1e-2)

@@ -57,3 +57,33 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     monkeypatch.setattr(bench, "cpu_inputs", lambda *a, **k: called.append(1))
     assert bench.main(["--impl", "reference", "--gpus", "2", "--steps", "3", "--warmup", "3"]) == 0
     assert not called
+
+
+def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
+    """Rank 0 of the reference arm times the oracle and prints one JSON line with
+    the contract's keys (shrunken inputs so that it runs in a moment)."""
+    import json
+
+    import numpy as np
+
+    import bench
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    rng = np.random.default_rng(0)
+    small = {"up": (rng.standard_normal((64, 64)), rng.standard_normal((64, 32))),
+             "down": (rng.standard_normal((64, 64)), rng.standard_normal((64, 32)))}
+    monkeypatch.setattr(bench, "SHAPES", {"up": (64, 32), "down": (64, 32)})
+    monkeypatch.setattr(bench, "cpu_inputs", lambda *a, **k: small)
+    assert bench.main(["--impl", "reference", "--steps", "2", "--warmup", "1"]) == 0
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    r = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in r, key
+    assert r["impl"] == "reference" and r["steps"] == 2 and r["warmup"] == 1
+    assert r["value"] > 0 and r["cpu_baseline"]["kind"] == "oracle" and r["cpu_baseline"]["cores"] >= 1
+    assert r["cpu_baseline"]["value"] == r["value"]
+    assert r["e2e"]["h2d_bytes_per_step"] == 0 and r["e2e"]["d2h_bytes_per_step"] == 0
+    assert r["e2e"]["value"] == r["value"] and r["e2e"]["unit"] == r["unit"]

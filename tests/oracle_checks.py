@@ -212,6 +212,24 @@ def check_one_row_ties(impl):
         assert np.asarray(impl.topk_indices(s2, k)).tolist() == w, k
 
 
+def check_grouped_heads(impl, seed=17):
+    """§3.3 Attention with grouped-query heads: query head h reads K / V head
+    h // (H / H_kv).  At rho = 1 the per-head forms equal numpy's products with
+    that mapping (QK: alpha Q_h K_g^T; PV: P_h V_g)."""
+    rng = _rng(seed)
+    H, Hkv, n, t, dh = 8, 2, 3, 20, 16
+    Q = rng.standard_normal((H, n, dh))
+    K = rng.standard_normal((Hkv, t, dh))
+    P = rng.random((H, n, t))
+    V = rng.standard_normal((Hkv, t, dh))
+    S, _ = impl.rmm_qk(Q, K, 1.0, 0.5, causal=False)
+    O, _ = impl.rmm_pv(P, V, 1.0)
+    for h in range(H):
+        g = h // (H // Hkv)
+        np.testing.assert_allclose(S[h], 0.5 * Q[h] @ K[g].T, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(O[h], P[h] @ V[g], rtol=1e-12, atol=1e-12)
+
+
 ALL_CHECKS = [
     check_retained_counts,
     check_scores_closed_forms,
@@ -222,4 +240,5 @@ ALL_CHECKS = [
     check_minimax_worst_case,
     check_invariants,
     check_one_row_ties,
+    check_grouped_heads,
 ]

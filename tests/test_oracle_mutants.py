@@ -20,6 +20,8 @@ def _mutant(**overrides):
         column_scores_sq=oracle.column_scores_sq,
         topk_indices=oracle.topk_indices,
         reduced_product=oracle.reduced_product,
+        rmm_qk=oracle.rmm_qk,
+        rmm_pv=oracle.rmm_pv,
     )
     for k, v in overrides.items():
         setattr(m, k, v)
@@ -74,6 +76,25 @@ def _product_wrong_sign(A, B, I, rows=None):
     return Y
 
 
+def _qk_interleaved(Q, K, rho, alpha, causal=True, heads=None, rows=None):
+    """Grouped-query heads mapped h -> h % H_kv instead of h // (H / H_kv)."""
+    Q, K = oracle.as_f64(Q), oracle.as_f64(K)
+    H, Hkv = Q.shape[0], K.shape[0]
+    k = oracle.retained_count(rho, Q.shape[2])
+    I = np.stack([oracle.select(Q[h], k=k)[0] for h in range(H)])
+    S = np.stack([oracle.reduced_scores(Q[h], K[h % Hkv], I[h], alpha, causal) for h in range(H)])
+    return S, I
+
+
+def _pv_interleaved(P, V, rho, heads=None, rows=None):
+    P, V = oracle.as_f64(P), oracle.as_f64(V)
+    H, Hkv = P.shape[0], V.shape[0]
+    k = oracle.retained_count(rho, P.shape[2])
+    T = np.stack([oracle.select(P[h], k=k)[0] for h in range(H)])
+    O = np.stack([oracle.reduced_product(P[h], V[h % Hkv], T[h]) for h in range(H)])
+    return O, T
+
+
 def _count_floor(rho, d):
     return max(1, int(math.floor(rho * d)))
 
@@ -93,6 +114,7 @@ MUTANTS = {
     "product_sign_error": _mutant(reduced_product=_product_wrong_sign),
     "k_floor_not_ceil": _mutant(retained_count=_count_floor),
     "k_no_rounding_snap": _mutant(retained_count=_count_no_snap),
+    "gqa_heads_interleaved": _mutant(rmm_qk=_qk_interleaved, rmm_pv=_pv_interleaved),
 }
 
 

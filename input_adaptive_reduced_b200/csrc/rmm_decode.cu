@@ -170,11 +170,10 @@ __global__ void __launch_bounds__(128) decode_qk_kernel(const DecodeArgs a) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (a.fused_select) {
         // The selection of each head's k features, in the CTA: the raw query
-        // rows go to shared memory, warp w ranks the features of heads w, w + 4
-        // (fp32 sums of squares in row order; rank = #{larger score, or equal
-        // at a lower index}; kept iff rank < k) and the first CTA of the KV head
+        // rows go to shared memory, warp w selects the features of heads w,
+        // w + 4 (fp32 sums of squares in row order; warp_topk_bits: the k
+        // largest, ties to the lower feature) and the first CTA of the KV head
         // writes I in order.
-        __shared__ uint32_t keyf[4][D];  // one head's scores per warp (two CTAs still fit an SM)
 #pragma unroll
         for (int j = 0; j < QPT; ++j) {
             const int e = threadIdx.x + j * 128;
@@ -184,7 +183,8 @@ __global__ void __launch_bounds__(128) decode_qk_kernel(const DecodeArgs a) {
         __syncthreads();
         constexpr int J = D / 32;
         for (int hl = warp; hl < a.group; hl += 4) {
-            uint32_t mine[J], rank[J];
+            uint32_t key[J];
+            bool valid[J];
 #pragma unroll
             for (int j = 0; j < J; ++j) {
                 const int f = lane + 32 * j;
@@ -193,22 +193,16 @@ __global__ void __launch_bounds__(128) decode_qk_kernel(const DecodeArgs a) {
                     const float x = __bfloat162float(qs[(hl * a.n + i) * LDS + f]);
                     sc = fmaf(x, x, sc);
                 }
-                mine[j] = __float_as_uint(sc);
-                keyf[warp][f] = mine[j];
-                rank[j] = 0u;
+                key[j] = __float_as_uint(sc);
+                valid[j] = true;
             }
-            __syncwarp();
-            for (int f2 = 0; f2 < D; ++f2) {
-                const uint32_t o = keyf[warp][f2];  // one word for every lane: a broadcast
-#pragma unroll
-                for (int j = 0; j < J; ++j) rank[j] += (o > mine[j]) || (o == mine[j] && f2 < lane + 32 * j);
-            }
+            const uint32_t kept_bits = warp_topk_bits<J>(key, valid, (uint32_t)a.k, lane);
             uint32_t before = 0;
             const bool emit = a.I_out && blockIdx.x == 0;
 #pragma unroll
             for (int j = 0; j < J; ++j) {
                 const int f = lane + 32 * j;
-                const bool kp = rank[j] < (uint32_t)a.k;
+                const bool kp = (kept_bits >> j) & 1u;
                 kept[hl][f] = kp ? 1 : 0;
                 if (emit) {
                     const unsigned b = __ballot_sync(0xffffffffu, kp);
@@ -216,7 +210,6 @@ __global__ void __launch_bounds__(128) decode_qk_kernel(const DecodeArgs a) {
                     before += __popc(b);
                 }
             }
-            __syncwarp();  // keyf[warp] holds the next head's scores next
         }
     }
     __syncthreads();

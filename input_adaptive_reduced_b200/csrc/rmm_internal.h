@@ -21,6 +21,41 @@ namespace rmm {
 #if defined(__CUDACC__)
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// TopK of 32 J keys held by one warp (lane l holds the keys of columns
+// l + 32 j; keys are the bit patterns of non-negative fp32 scores, which order
+// as the scores do): bit j of the result is set when column lane + 32 j is
+// among the k largest, ties going to the lower column.  The k-th largest key
+// T is found bit by bit (the largest T with at least k keys >= T); the keys
+// equal to T are then kept in column order until k are kept.  Columns past
+// the end must hold key 0 and `valid` false.
+template <int J>
+__device__ __forceinline__ uint32_t warp_topk_bits(const uint32_t (&key)[J], const bool (&valid)[J], uint32_t k,
+                                                   int lane) {
+    uint32_t T = 0u;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = T | (1u << bit);
+        uint32_t c = 0u;
+#pragma unroll
+        for (int j = 0; j < J; ++j) c += (valid[j] && key[j] >= cand) ? 1u : 0u;
+        if (__reduce_add_sync(0xffffffffu, c) >= k) T = cand;
+    }
+    uint32_t gt = 0u;
+#pragma unroll
+    for (int j = 0; j < J; ++j) gt += (valid[j] && key[j] > T) ? 1u : 0u;
+    const uint32_t r = k - __reduce_add_sync(0xffffffffu, gt);  // keys equal to T that are kept
+    uint32_t kept = 0u, eq_before = 0u;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const bool eq = valid[j] && key[j] == T;
+        const unsigned b = __ballot_sync(0xffffffffu, eq);
+        const uint32_t rank = eq_before + __popc(b & ((1u << lane) - 1u));
+        if ((valid[j] && key[j] > T) || (eq && rank < r)) kept |= 1u << j;
+        eq_before += __popc(b);
+    }
+    return kept;
+}
 #endif
 
 template <typename... Params, typename... Args>

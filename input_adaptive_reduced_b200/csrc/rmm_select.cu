@@ -402,11 +402,9 @@ __global__ void __launch_bounds__(1024) normselect_kernel(const T* __restrict__ 
 
 // ------------------------------------------------------------------ few features
 // d <= 256 columns and n <= 8 rows per head (attention heads at a decode
-// step): one warp per head.  The fp32 score of column j (sum of squares in row
-// order) goes to shared memory; column j is kept when its rank, the number of
-// columns with a larger score or an equal score at a lower index, is below k,
-// which is the TopK with ties to the lower index.  The kept columns are
-// emitted in order from one ballot per 32 columns.
+// step): one warp per head.  Lane l sums the squares of columns l + 32 j in
+// row order (fp32); warp_topk_bits finds the k largest, ties to the lower
+// column, and the kept columns are emitted in order from one ballot per 32.
 constexpr int kSmallMaxD = 256;
 constexpr int kSmallMaxRows = 8;
 constexpr int kSmallWarps = 8;
@@ -423,43 +421,33 @@ __global__ void __launch_bounds__(32 * kSmallWarps) select_small_kernel(const T*
                                                                        int64_t mask_words) {
     pdl_wait();
     pdl_trigger();
-    __shared__ uint32_t keys[kSmallWarps][kSmallMaxD];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int h = blockIdx.x * kSmallWarps + warp;
     if (h >= heads) return;  // no block-wide barrier below
     const T* Ah = A + (int64_t)h * stride_a;
-    uint32_t* key = keys[warp];
+    uint32_t key[J];
+    bool valid[J];
 #pragma unroll
     for (int j = 0; j < J; ++j) {
         const int f = lane + 32 * j;
-        if (f < d) {
-            float acc = 0.f;
+        valid[j] = f < d;
+        float acc = 0.f;
+        if (valid[j]) {
             for (int64_t r = 0; r < n; ++r) {
                 const float x = to_float(Ah[r * lda + f]);
                 acc = fmaf(x, x, acc);
             }
-            key[f] = __float_as_uint(acc);
             if (s2) s2[(int64_t)h * d + f] = acc;
         }
+        key[j] = __float_as_uint(acc);
     }
-    __syncwarp();
-    uint32_t mine[J], rank[J];
-#pragma unroll
-    for (int j = 0; j < J; ++j) {
-        mine[j] = lane + 32 * j < d ? key[lane + 32 * j] : 0u;
-        rank[j] = 0u;
-    }
-    for (int f2 = 0; f2 < (int)d; ++f2) {
-        const uint32_t o = key[f2];  // the same word for every lane: a broadcast
-#pragma unroll
-        for (int j = 0; j < J; ++j) rank[j] += (o > mine[j]) || (o == mine[j] && f2 < lane + 32 * j);
-    }
+    const uint32_t kept_bits = warp_topk_bits<J>(key, valid, (uint32_t)k, lane);
     int32_t* Ih = I + (int64_t)h * k;
     uint32_t before = 0;
 #pragma unroll
     for (int j = 0; j < J; ++j) {
         const int f = lane + 32 * j;
-        const bool kept = f < d && rank[j] < (uint32_t)k;
+        const bool kept = (kept_bits >> j) & 1u;
         const unsigned b = __ballot_sync(0xffffffffu, kept);
         if (kept) Ih[before + __popc(b & ((1u << lane) - 1u))] = f;
         if (mask && lane == 0 && 32 * j < d) mask[(int64_t)h * mask_words + j] = b;

@@ -87,3 +87,16 @@ def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
     assert r["cpu_baseline"]["value"] == r["value"]
     assert r["e2e"]["h2d_bytes_per_step"] == 0 and r["e2e"]["d2h_bytes_per_step"] == 0
     assert r["e2e"]["value"] == r["value"] and r["e2e"]["unit"] == r["unit"]
+
+
+def test_traffic_figure_only_while_the_kernel_is_unchanged(monkeypatch, tmp_path):
+    """roofline.traffic comes from the committed ncu summary of the product
+    kernel, and only while the kernel source still hashes to the value recorded
+    there: a changed kernel reports null."""
+    import bench
+    t = bench.load_traffic()
+    assert t is not None and t > 0
+    changed = tmp_path / "rmm_gemm.cu"
+    changed.write_bytes(open(bench.GEMM_SOURCE, "rb").read() + b"\n// changed\n")
+    monkeypatch.setattr(bench, "GEMM_SOURCE", str(changed))
+    assert bench.load_traffic() is None

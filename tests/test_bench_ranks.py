@@ -100,3 +100,13 @@ def test_traffic_figure_only_while_the_kernel_is_unchanged(monkeypatch, tmp_path
     changed.write_bytes(open(bench.GEMM_SOURCE, "rb").read() + b"\n// changed\n")
     monkeypatch.setattr(bench, "GEMM_SOURCE", str(changed))
     assert bench.load_traffic() is None
+
+
+def test_metric_counts_the_methods_k():
+    """The useful-FLOP count of every reported point uses k = ceil(rho * d) as
+    the oracle states it (pinned to the paper's worked counts)."""
+    import bench
+    import oracle
+    for d in (128, 256, 4096, 8192, 14336, 28672, 32768):
+        for rho in (0.25, 0.5, 0.6, 0.7, 0.8, 0.9, 1.0):
+            assert bench.retained(rho, d) == oracle.retained_count(rho, d), (rho, d)

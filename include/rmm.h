@@ -153,20 +153,25 @@ RMM_API rmm_status rmm_select(const rmm_plan* plan, const void* A, int32_t* I, f
    this is a deployment convenience.  Same result as rmm_select (I ascending,
    optional fp32 s2), for callers that cannot allocate device memory when they
    need an index set (a frozen or captured memory pool, a plugin inside
-   another runtime's allocator, a process with a fixed memory budget).  The
-   scratch of the score pass (partials, completion counters, final scores)
-   lives in one 8 MiB file-scope device array inside this library, held by
-   every GPU that loads it until the process exits; the caller passes only A,
-   I and s2.  Limits: heads * d * 4 * (nsplit + 1) bytes plus the counters
-   must fit in 8 MiB (nsplit <= 16, chosen by the plan; e.g. d = 28672 with one
-   head fits), else RMM_ERR_UNSUPPORTED and nothing is launched.  The first
-   call on a device looks up the array's device address (cudaGetSymbolAddress)
-   with that device current; make that first call before any stream capture.
-   Every call reuses the same array and it keeps the last call's contents (the
-   counters are cleared on the stream at the start of each call): calls that
-   overlap on the GPU -- two streams, or two host threads -- race and corrupt
-   each other's results; serialise them.  Calls no cudaMalloc, cudaFree or
-   other allocating routine. */
+   another runtime's allocator, a process with a fixed memory budget).  Plans
+   whose selection runs in one kernel per head (few rows, one row, or a small
+   head; the same kernel rmm_select takes) use no scratch at all.  Otherwise
+   the scratch of the score pass (partials, completion counters, final
+   scores) lives in one 8 MiB file-scope device array inside this library,
+   held by every GPU that loads it until the process exits; the caller passes
+   only A, I and s2.  Limits: heads * d * 4 * (nsplit + 1) bytes plus the
+   counters must fit in 8 MiB (nsplit <= 16, chosen by the plan; e.g.
+   d = 28672 with one head fits), else RMM_ERR_UNSUPPORTED and nothing is
+   launched.  The array's device address is looked up (cudaGetSymbolAddress)
+   with the calling thread's current device and context on the first such call
+   in that context, and again whenever the context changes (e.g. after
+   cudaDeviceReset); make that first call before any stream capture.  `stream`
+   must belong to the current device (RMM_ERR_INVALID_ARG otherwise: the
+   address is that device's).  Every call reuses the same array and it keeps
+   the last call's contents (the counters are cleared on the stream at the
+   start of each call): calls that overlap on the GPU -- two streams, or two
+   host threads -- race and corrupt each other's results; serialise them.
+   Calls no cudaMalloc, cudaFree or other allocating routine. */
 RMM_API rmm_status rmm_select_no_alloc(const rmm_plan* plan, const void* A, int32_t* I, float* s2,
                                        void* stream);
 

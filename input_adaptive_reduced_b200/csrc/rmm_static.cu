@@ -12,6 +12,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "rmm.h"
@@ -28,25 +29,63 @@ static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchB
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+struct ScratchSlot {
+    unsigned long long ctx_id;  // the CUDA context the address was looked up in
+    void* addr;
+};
+ScratchSlot g_scratch[kMaxDevices] = {};
 
-// Device address of g_select_scratch on the current device (looked up on the
-// first call for that device).
+// Unique id of the calling thread's current CUDA context (driver API, looked
+// up once through the runtime's entry-point query), or 0 if unavailable.
+unsigned long long current_context_id() {
+    using GetCurrent = CUresult (*)(CUcontext*);
+    using GetId = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static bool looked_up = false;
+    if (!looked_up) {
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f1, 12000, cudaEnableDefault, &q1) == cudaSuccess &&
+            q1 == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPointByVersion("cuCtxGetId", &f2, 12000, cudaEnableDefault, &q2) == cudaSuccess &&
+            q2 == cudaDriverEntryPointSuccess) {
+            get_current = reinterpret_cast<GetCurrent>(f1);
+            get_id = reinterpret_cast<GetId>(f2);
+        }
+        cudaGetLastError();
+        looked_up = true;
+    }
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of g_select_scratch on the current device and context.  It
+// is looked up with cudaGetSymbolAddress on the first call in a context and
+// looked up again when the context changes (after cudaDeviceReset, for
+// example, the device's primary context and the address are new).
 rmm_status scratch_address(void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return RMM_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return RMM_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    ScratchSlot& slot = g_scratch[dev];
+    if (!slot.addr || ctx == 0 || slot.ctx_id != ctx) {
         void* p = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&p, g_select_scratch);
         if (e != cudaSuccess || p == nullptr) {
             cudaGetLastError();
             return RMM_ERR_CUDA;
         }
-        g_scratch_addr[dev] = p;
+        slot.addr = p;
+        slot.ctx_id = ctx;
     }
-    *out = g_scratch_addr[dev];
+    *out = slot.addr;
     return RMM_OK;
 }
 
@@ -63,24 +102,7 @@ extern "C" rmm_status rmm_select_no_alloc(const rmm_plan* plan, const void* A, i
     const rmm_problem& p = plan->p;
     if (p.d > rmm::kMaxSelectD) return RMM_ERR_UNSUPPORTED;
 
-    // Scratch layout: completion counters | split partials | final scores.
-    const int vec = 16 / plan->es;
-    const int64_t colblocks = (p.d + 32 * vec - 1) / (32 * vec);
-    const size_t counter_bytes = align256(static_cast<size_t>(p.heads) * colblocks * sizeof(unsigned));
-    const size_t partial_bytes = align256(static_cast<size_t>(p.heads) * plan->nsplit * p.d * sizeof(float));
-    const size_t score_bytes = align256(static_cast<size_t>(p.heads) * p.d * sizeof(float));
-    if (counter_bytes + partial_bytes + score_bytes > kNoAllocScratchBytes) return RMM_ERR_UNSUPPORTED;
-
-    void* base = nullptr;
-    const rmm_status st = scratch_address(&base);
-    if (st != RMM_OK) return st;
-    unsigned char* scratch = static_cast<unsigned char*>(base);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-
-    // The counters must start at zero; the partials and scores are fully
-    // overwritten by every call.
-    if (cudaMemsetAsync(scratch, 0, counter_bytes, s) != cudaSuccess) return RMM_ERR_CUDA;
-
     rmm::SelectArgs a{};
     a.A = A;
     a.dtype = p.dtype;
@@ -92,6 +114,41 @@ extern "C" rmm_status rmm_select_no_alloc(const rmm_plan* plan, const void* A, i
     a.k = plan->k;
     a.I = I;
     a.s2 = s2;
+    // Selections done inside one kernel per head need no scratch at all: take
+    // the same kernel as rmm_select for the plan.
+    if (plan->select_small || plan->select16 || plan->fused_select) {
+        cudaError_t e = plan->select_small ? rmm::launch_select_small(a, s)
+                        : plan->select16   ? rmm::launch_select16(a, s)
+                                           : rmm::launch_normselect(a, s);
+        return e == cudaSuccess ? RMM_OK : RMM_ERR_CUDA;
+    }
+
+    // Scratch layout: completion counters | split partials | final scores.
+    const int vec = 16 / plan->es;
+    const int64_t colblocks = (p.d + 32 * vec - 1) / (32 * vec);
+    const size_t counter_bytes = align256(static_cast<size_t>(p.heads) * colblocks * sizeof(unsigned));
+    const size_t partial_bytes = align256(static_cast<size_t>(p.heads) * plan->nsplit * p.d * sizeof(float));
+    const size_t score_bytes = align256(static_cast<size_t>(p.heads) * p.d * sizeof(float));
+    if (counter_bytes + partial_bytes + score_bytes > kNoAllocScratchBytes) return RMM_ERR_UNSUPPORTED;
+
+    // The scratch address belongs to the current device: the stream must be
+    // one of that device's streams.
+    int cur = -1, sdev = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess || cudaStreamGetDevice(s, &sdev) != cudaSuccess) {
+        cudaGetLastError();
+        return RMM_ERR_CUDA;
+    }
+    if (sdev != cur) return RMM_ERR_INVALID_ARG;
+
+    void* base = nullptr;
+    const rmm_status st = scratch_address(&base);
+    if (st != RMM_OK) return st;
+    unsigned char* scratch = static_cast<unsigned char*>(base);
+
+    // The counters must start at zero; the partials and scores are fully
+    // overwritten by every call.
+    if (cudaMemsetAsync(scratch, 0, counter_bytes, s) != cudaSuccess) return RMM_ERR_CUDA;
+
     a.counters = reinterpret_cast<unsigned*>(scratch);
     a.partials = reinterpret_cast<float*>(scratch + counter_bytes);
     a.scores = s2 ? s2 : reinterpret_cast<float*>(scratch + counter_bytes + partial_bytes);

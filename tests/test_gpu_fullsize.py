@@ -40,25 +40,29 @@ def _linear_full(rmm, gen, n, rhos, seed, **kw):
         assert_product_close(Y[rows], Y_ref, np.abs(A64[rows][:, I_ref]), np.abs(B64[I_ref]))
 
 
-@pytest.mark.parametrize("n", [1024, 4096])
-def test_llama8b_up_gate(rmm, n):
-    _linear_full(rmm, W.mlp_up, n, [0.5, 0.8] if n == 4096 else [0.7], seed=101)
+@pytest.mark.parametrize("n,rhos", [(1024, [0.7]), (2048, [0.8]), (4096, [0.5, 0.8])])
+def test_llama8b_up_gate(rmm, n, rhos):
+    _linear_full(rmm, W.mlp_up, n, rhos, seed=101)
 
 
-@pytest.mark.parametrize("n", [2048, 4096])
-def test_llama8b_down(rmm, n):
-    _linear_full(rmm, W.mlp_down, n, [0.7] if n == 4096 else [0.5, 0.8], seed=102)
+@pytest.mark.parametrize("n,rhos", [(2048, [0.5, 0.8]), (4096, [0.7, 0.8])])
+def test_llama8b_down(rmm, n, rhos):
+    """n = 4096, rho = 0.8 is the benchmark's down-projection point."""
+    _linear_full(rmm, W.mlp_down, n, rhos, seed=102)
 
 
 @pytest.mark.parametrize("shape,n,rhos", [
     ("up", 1, [0.5, 0.8]), ("up", 16, [0.6, 1.0]), ("down", 16, [0.7]), ("qkv", 16, [0.8]),
     ("down", 1, [0.6]), ("qkv", 512, [0.5, 0.7]), ("up", 2048, [0.8]),
+    # the longest K loops (k up to 22938) and the largest A packs of the suite
+    ("down", 512, [0.5, 0.8]), ("down", 2048, [0.5, 0.8]), ("down", 4096, [0.5, 0.8]),
+    ("up", 4096, [0.8]), ("qkv", 4096, [0.8]),
 ])
 def test_llama70b_linear(rmm, shape, n, rhos):
     _linear_full(rmm, W.linear_70b, n, rhos, seed=103, shape=shape)
 
 
-@pytest.mark.parametrize("n", [1024, 4096])
+@pytest.mark.parametrize("n", [1024, 2048, 4096])
 def test_attention_qk_full(rmm, n):
     H, Hkv, dh = 32, 8, 128
     rhos = [0.5, 0.8]

@@ -76,6 +76,94 @@ def test_exact_tie_lower_index_wins(rmm, rho, direction):
     assert lo in got and hi not in got
 
 
+def _tie_pair(s2, k, direction, other_block_of=None):
+    """(src, dst): src is the last kept column; dst a dropped column above
+    (copy_up) or below (copy_down) it, in another 256-column block when
+    other_block_of is set.  None when there is no such column."""
+    order = gap.descending_order(s2)
+    src = int(order[k - 1])
+    for j in order[k:].tolist():
+        if (j > src) != (direction == "copy_up"):
+            continue
+        if other_block_of is not None and j // other_block_of == src // other_block_of:
+            continue
+        return src, int(j)
+    return None
+
+
+@pytest.mark.parametrize("direction", ["copy_up", "copy_down"])
+@pytest.mark.parametrize("kind,d", [("up", 4096), ("down", 14336)])
+def test_exact_tie_across_column_blocks(rmm, kind, d, direction):
+    """Duplicated bf16 columns in different 256-column blocks of the score pass,
+    at n = 1024 where every column block is summed in several row splits (16 at
+    d = 4096, 6 at d = 14336) and the last CTA of the block adds the split
+    partials: equal columns must get bit-equal scores wherever they sit, and
+    the lower index of the tied pair is the one kept."""
+    n, m, rho = 1024, 264, 0.8
+    k = oracle.retained_count(rho, d)
+    gen = W.mlp_up if kind == "up" else W.mlp_down
+    (A, B), _ = gap.enforce_boundary_gaps(lambda g: gen(21, n=n, d=d, m=m, col_gain=g),
+                                          lambda x: gap.scores_2d(x[0]), [k])
+    pair = _tie_pair(oracle.column_scores_sq(A), k, direction, other_block_of=256)
+    if pair is None:
+        pytest.skip("no dropped column on that side in another column block")
+    src, dst = pair
+    A2 = W.duplicate_columns(A, [(src, dst)])
+    s2b = oracle.column_scores_sq(A2)
+    assert s2b[src] == s2b[dst]
+    Y, I = _linear_case(rmm, A2, B, rho, rows=list(range(0, n, 37)))
+    got = set(I.cpu().tolist())
+    assert min(src, dst) in got and max(src, dst) not in got
+
+
+@pytest.mark.parametrize("n", [2, 4, 512, 1024])
+def test_exact_tie_per_head_features(rmm, n):
+    """Per-head feature selection with the boundary feature of every head
+    duplicated over a dropped one (even heads above it, odd heads below it),
+    through each selection path the heads take: n = 2 the decode QK kernel
+    selects in-kernel, n = 4 the one-warp-per-head select (select() on
+    [heads, 4, 128]), n = 512 the one-CTA score+select, n = 1024 the score pass
+    and the radix select."""
+    H, Hkv, dh, rho = 8, 2, 128, 0.8
+    k = oracle.retained_count(rho, dh)
+    nk = max(n, 64)  # keys: a multiple of 8
+
+    def make(g):
+        Qf, Kf = W.attn_qk(22, n=nk, heads=H, kv_heads=Hkv, head_dim=dh, col_gain=g)
+        return Qf[:, :n].contiguous(), Kf
+
+    (Q, K), _ = gap.enforce_boundary_gaps(make, lambda x: gap.scores_per_head(x[0]), [k])
+    pairs = []
+    for h in range(H):
+        pr = _tie_pair(oracle.column_scores_sq(Q[h]), k, "copy_up" if h % 2 == 0 else "copy_down")
+        if pr is None:
+            pr = _tie_pair(oracle.column_scores_sq(Q[h]), k, "copy_down" if h % 2 == 0 else "copy_up")
+        pairs.append(pr)
+        Q[h] = W.duplicate_columns(Q[h], [pr])
+    dev = torch.device("cuda")
+    if n == 4:
+        I = rmm.select(Q.to(dev), rho=rho)
+    else:
+        causal = n > 8  # the decode kernels take the non-causal form
+        S, I = rmm.qk(Q.to(dev), K.to(dev), rho=rho, causal=causal, return_indices=True)
+    torch.cuda.synchronize()
+    I_ref = np.stack([oracle.select(Q[h], k=k)[0] for h in range(H)])
+    assert_indices_equal(I, I_ref)
+    for h, (src, dst) in enumerate(pairs):
+        got = set(I[h].cpu().tolist())
+        assert min(src, dst) in got and max(src, dst) not in got, h
+    if n != 4:
+        alpha = 1.0 / math.sqrt(dh)
+        rows = list(range(n)) if n <= 8 else list(range(0, n, 61))
+        S_ref, _ = oracle.rmm_qk(Q, K, rho=rho, alpha=alpha, causal=causal, heads=[0, 5], rows=rows)
+        Q64, K64 = oracle.as_f64(Q), oracle.as_f64(K)
+        mask = (np.arange(nk)[None, :] > np.asarray(rows)[:, None]) if causal else None
+        for i, h in enumerate([0, 5]):
+            g = oracle.kv_head_of(h, H, Hkv)
+            assert_product_close(S[h][rows], S_ref[i], np.abs(Q64[h][rows][:, I_ref[h]]),
+                                 np.abs(K64[g][:, I_ref[h]]).T, alpha=alpha, mask=mask)
+
+
 LINEAR_SHAPES = [
     ("up", 200, 4096, 520),
     ("down", 136, 14336, 264),

@@ -16,6 +16,9 @@ calls it.  Every function pins to the paper as follows (tests/test_oracle_pins.p
                          Eq. 17 bounds; equality in the rank-one construction
   reduced_scores      -- rho=1 equals alpha*Q K^T; causal entries are -inf
   rmm_qk / rmm_pv     -- per-head bounds and rho=1 dense special cases
+  softmax_rows        -- closed forms (uniform row, two-key logistic), masked
+                         entries exactly 0, rows sum to 1 and not columns,
+                         per-row shift invariance, large logits stay finite
 No function here is "parity unpinned".
 """
 from __future__ import annotations
@@ -63,6 +66,8 @@ def _load():
             lib.rmm_oracle_reduced_product.restype = None
             lib.rmm_oracle_reduced_product.argtypes = [_f64p, _i64, _f64p, _i64, _i64, _i64,
                                                        _i32p, _i64, _f64p, _i64]
+            lib.rmm_oracle_softmax_rows.restype = ctypes.c_int
+            lib.rmm_oracle_softmax_rows.argtypes = [_f64p, _i64, _i64, _i64, _f64p, _i64]
             lib.rmm_oracle_reduced_scores.restype = None
             lib.rmm_oracle_reduced_scores.argtypes = [_f64p, _i64, _f64p, _i64, _i64, _i64, _i64,
                                                       _i32p, _i64, ctypes.c_double, ctypes.c_int,
@@ -161,6 +166,20 @@ def reduced_scores(Q, K, I, alpha: float, causal: bool, rows=None) -> np.ndarray
                                       1, nk, int(r), _p(I, _i32p), I.size, float(alpha),
                                       int(bool(causal)), _p(out[r_out:], _f64p), nk)
     return out
+
+
+def softmax_rows(S) -> np.ndarray:
+    """Attention weights P = softmax(S + M) over the key axis of each row, the
+    mask M given as -inf entries of S [RMM paper, §3.3 "Attention"].  S is
+    [n, t] or [heads, n, t]; fp64 out."""
+    S = as_f64(S)
+    if S.ndim == 3:
+        return np.stack([softmax_rows(S[h]) for h in range(S.shape[0])])
+    n, t = S.shape
+    P = np.empty((n, t), dtype=np.float64)
+    if _load().rmm_oracle_softmax_rows(_p(S, _f64p), t, n, t, _p(P, _f64p), t) != 0:
+        raise ValueError("a row of S has no finite entry")
+    return P
 
 
 def kv_head_of(h: int, heads: int, kv_heads: int) -> int:

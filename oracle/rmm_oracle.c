@@ -176,3 +176,41 @@ void rmm_oracle_reduced_scores(const double *Q, int64_t ldq,
         }
     }
 }
+
+/*
+ * Attention weights of one head, P = softmax(S + M)  [RMM paper, §3.3
+ * "Attention": P = softmax(S~ + M), M the optional causal or attention mask;
+ * the softmax normalises each query row over the key axis].  The mask is
+ * already in S as -inf entries (the causal form written by
+ * rmm_oracle_reduced_scores), and such entries get weight exactly 0.
+ * Row i, with mu_i = max_c S[i,c]:
+ *   P[i,c] = exp(S[i,c] - mu_i) / sum over c' of exp(S[i,c'] - mu_i).
+ * Subtracting mu_i changes nothing in exact arithmetic and keeps every exp
+ * finite.  Returns 0, or -1 when some row has no finite entry (out of
+ * contract: the mask leaves every query at least its own key).
+ */
+int rmm_oracle_softmax_rows(const double *S, int64_t lds, int64_t n, int64_t t,
+                            double *P, int64_t ldp)
+{
+    int bad = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        const double *s = S + i * lds;
+        double *p = P + i * ldp;
+        double mu = -INFINITY;
+        for (int64_t c = 0; c < t; ++c)
+            if (s[c] > mu) mu = s[c];
+        if (!(mu > -INFINITY)) {
+            bad = 1;
+            continue;
+        }
+        double sum = 0.0;
+        for (int64_t c = 0; c < t; ++c) {
+            double e = (s[c] == -INFINITY) ? 0.0 : exp(s[c] - mu);
+            p[c] = e;
+            sum += e;
+        }
+        for (int64_t c = 0; c < t; ++c)
+            p[c] = p[c] / sum;
+    }
+    return bad ? -1 : 0;
+}

@@ -230,6 +230,39 @@ def check_grouped_heads(impl, seed=17):
         np.testing.assert_allclose(O[h], P[h] @ V[g], rtol=1e-12, atol=1e-12)
 
 
+def check_softmax(impl, seed=18):
+    """P = softmax(S + M) over the key axis of each row [§3.3 "Attention"]:
+    a constant row gives 1/t; two keys give the logistic function of their
+    difference; -inf (masked) entries weigh exactly 0 and a causal first row is
+    one-hot; every row sums to 1 while columns of a wide S do not; adding a
+    constant to a row changes nothing; logits of 1000 stay finite."""
+    sm = impl.softmax_rows
+    t = 7
+    got = sm(np.full((3, t), 2.5))
+    assert np.array_equal(got, np.full((3, t), 1.0 / t)), got
+    for x in (-3.0, 0.0, 0.7, 5.0):
+        got = sm(np.array([[0.0, x]]))
+        lo = 1.0 / (1.0 + np.exp(x))
+        assert abs(got[0, 0] - lo) <= 1e-15 and abs(got[0, 1] - (1.0 - lo)) <= 1e-15, (x, got)
+    rng = _rng(seed)
+    n, w = 6, 10
+    S = rng.standard_normal((n, w)) * 3.0
+    causal = np.triu(np.ones((n, w), dtype=bool), 1)
+    Sm = np.where(causal, -np.inf, S)
+    P = sm(Sm)
+    assert np.all(P[causal] == 0.0)
+    assert P[0, 0] == 1.0 and np.all(P[~causal] > 0.0)
+    assert np.allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+    Pw = sm(S)
+    assert np.allclose(Pw.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+    assert not np.allclose(Pw.sum(axis=0), 1.0, atol=1e-3)
+    shift = rng.standard_normal((n, 1)) * 50.0
+    assert np.allclose(sm(S + shift), Pw, rtol=1e-12, atol=1e-15)
+    big = sm(np.array([[1000.0, 999.0, 0.0]]))
+    assert np.all(np.isfinite(big))
+    assert abs(big[0, 0] - 1.0 / (1.0 + np.exp(-1.0) + np.exp(-1000.0))) <= 1e-15
+
+
 ALL_CHECKS = [
     check_retained_counts,
     check_scores_closed_forms,
@@ -241,4 +274,5 @@ ALL_CHECKS = [
     check_invariants,
     check_one_row_ties,
     check_grouped_heads,
+    check_softmax,
 ]

@@ -93,9 +93,16 @@ def test_traffic_figure_only_while_the_kernel_is_unchanged(monkeypatch, tmp_path
     """roofline.traffic comes from the committed ncu summary of the product
     kernel, and only while the kernel source still hashes to the value recorded
     there: a changed kernel reports null."""
+    import hashlib
+    import re
     import bench
     t = bench.load_traffic()
-    assert t is not None and t > 0
+    recorded = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", open(bench.TRAFFIC_FILE).read()).group(1)
+    current = hashlib.sha256(open(bench.GEMM_SOURCE, "rb").read()).hexdigest()
+    if recorded == current:
+        assert t is not None and t > 0
+    else:  # the kernel changed after the capture: no figure until it is recaptured
+        assert t is None
     changed = tmp_path / "rmm_gemm.cu"
     changed.write_bytes(open(bench.GEMM_SOURCE, "rb").read() + b"\n// changed\n")
     monkeypatch.setattr(bench, "GEMM_SOURCE", str(changed))

@@ -22,6 +22,7 @@ def _mutant(**overrides):
         reduced_product=oracle.reduced_product,
         rmm_qk=oracle.rmm_qk,
         rmm_pv=oracle.rmm_pv,
+        softmax_rows=oracle.softmax_rows,
     )
     for k, v in overrides.items():
         setattr(m, k, v)
@@ -95,6 +96,29 @@ def _pv_interleaved(P, V, rho, heads=None, rows=None):
     return O, T
 
 
+def _softmax_no_max_shift(S):
+    with np.errstate(over="ignore", invalid="ignore"):
+        E = np.exp(oracle.as_f64(S))
+        return E / E.sum(axis=1, keepdims=True)
+
+
+def _softmax_over_columns(S):
+    S = oracle.as_f64(S)
+    E = np.exp(S - S.max(axis=0, keepdims=True))
+    return E / E.sum(axis=0, keepdims=True)
+
+
+def _softmax_mask_as_zero_logit(S):
+    S = oracle.as_f64(S)
+    return oracle.softmax_rows(np.where(np.isneginf(S), 0.0, S))
+
+
+def _softmax_linear(S):
+    S = oracle.as_f64(S)
+    E = np.where(np.isneginf(S), 0.0, S - S.min(axis=1, keepdims=True, initial=np.inf, where=~np.isneginf(S)) + 1.0)
+    return E / E.sum(axis=1, keepdims=True)
+
+
 def _count_floor(rho, d):
     return max(1, int(math.floor(rho * d)))
 
@@ -115,6 +139,10 @@ MUTANTS = {
     "k_floor_not_ceil": _mutant(retained_count=_count_floor),
     "k_no_rounding_snap": _mutant(retained_count=_count_no_snap),
     "gqa_heads_interleaved": _mutant(rmm_qk=_qk_interleaved, rmm_pv=_pv_interleaved),
+    "softmax_without_max_shift": _mutant(softmax_rows=_softmax_no_max_shift),
+    "softmax_over_the_query_axis": _mutant(softmax_rows=_softmax_over_columns),
+    "softmax_mask_as_zero_logit": _mutant(softmax_rows=_softmax_mask_as_zero_logit),
+    "softmax_without_exp": _mutant(softmax_rows=_softmax_linear),
 }
 
 
@@ -125,6 +153,6 @@ def test_pins_catch_mutant(name):
     for check in oc.ALL_CHECKS:
         try:
             check(impl)
-        except (AssertionError, ValueError, IndexError):
+        except (AssertionError, ValueError, IndexError, FloatingPointError):
             caught.append(check.__name__)
     assert caught, f"no pin catches the planted mistake '{name}'"

@@ -16,6 +16,8 @@ calls it.  Every function pins to the paper as follows (tests/test_oracle_pins.p
                          Eq. 17 bounds; equality in the rank-one construction
   reduced_scores      -- rho=1 equals alpha*Q K^T; causal entries are -inf
   rmm_qk / rmm_pv     -- per-head bounds and rho=1 dense special cases
+  decode_e4m3         -- hand-worked codes (golden file) and every code against
+                         torch's float8_e4m3fn conversion
   softmax_rows        -- closed forms (uniform row, two-key logistic), masked
                          entries exactly 0, rows sum to 1 and not columns,
                          per-row shift invariance, large logits stay finite
@@ -66,6 +68,8 @@ def _load():
             lib.rmm_oracle_reduced_product.restype = None
             lib.rmm_oracle_reduced_product.argtypes = [_f64p, _i64, _f64p, _i64, _i64, _i64,
                                                        _i32p, _i64, _f64p, _i64]
+            lib.rmm_oracle_decode_e4m3.restype = ctypes.c_int
+            lib.rmm_oracle_decode_e4m3.argtypes = [ctypes.POINTER(ctypes.c_uint8), _i64, _f64p]
             lib.rmm_oracle_softmax_rows.restype = ctypes.c_int
             lib.rmm_oracle_softmax_rows.argtypes = [_f64p, _i64, _i64, _i64, _f64p, _i64]
             lib.rmm_oracle_reduced_scores.restype = None
@@ -165,6 +169,20 @@ def reduced_scores(Q, K, I, alpha: float, causal: bool, rows=None) -> np.ndarray
         lib.rmm_oracle_reduced_scores(_p(q, _f64p), Q.shape[1], _p(K, _f64p), K.shape[1],
                                       1, nk, int(r), _p(I, _i32p), I.size, float(alpha),
                                       int(bool(causal)), _p(out[r_out:], _f64p), nk)
+    return out
+
+
+def decode_e4m3(codes) -> np.ndarray:
+    """Exact fp64 values of E4M3 (OCP 8-bit float, e4m3fn) codes: uint8 array
+    or a torch float8_e4m3fn tensor (its bytes).  The low-bit form of RMM
+    stores A and B in this format (see rmm_oracle.c)."""
+    if hasattr(codes, "detach"):
+        codes = codes.detach().to("cpu").contiguous().view(__import__("torch").uint8).numpy()
+    c = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
+    out = np.empty(c.shape, dtype=np.float64)
+    if _load().rmm_oracle_decode_e4m3(c.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), c.size,
+                                      _p(out, _f64p)) != 0:
+        raise ValueError("NaN code in an E4M3 operand")
     return out
 
 

@@ -214,3 +214,36 @@ int rmm_oracle_softmax_rows(const double *S, int64_t lds, int64_t n, int64_t t,
     }
     return bad ? -1 : 0;
 }
+
+/*
+ * Exact value of 8-bit floating-point codes in the E4M3 format of the OCP
+ * 8-bit floating point specification (the "e4m3fn" variant: no infinities,
+ * the all-ones exponent and mantissa is NaN, largest magnitude 448).  The
+ * RMM paper runs RMM alongside 8-bit weight quantization (App. B.6) and names
+ * dedicated low-bit kernels as future work (App. B.7); the low-bit form here
+ * stores A and B in this format with per-tensor scales folded into the
+ * output scale alpha, and the method's arithmetic (scores, TopK, product)
+ * runs on the exact decoded values.
+ * Bit layout: sign s (bit 7), exponent e (bits 6..3, bias 7), mantissa f
+ * (bits 2..0).  e = 0: (-1)^s * f * 2^-9 (subnormal); otherwise
+ * (-1)^s * 2^(e-7) * (1 + f/8).  Returns 0, or -1 if a code is NaN.
+ */
+int rmm_oracle_decode_e4m3(const uint8_t *codes, int64_t count, double *out)
+{
+    int bad = 0;
+    for (int64_t i = 0; i < count; ++i) {
+        unsigned b = codes[i];
+        unsigned s = b >> 7, e = (b >> 3) & 15u, f = b & 7u;
+        double v;
+        if (e == 15u && f == 7u) {
+            v = NAN;
+            bad = 1;
+        } else if (e == 0u) {
+            v = ldexp((double)f, -9);
+        } else {
+            v = ldexp(1.0 + (double)f / 8.0, (int)e - 7);
+        }
+        out[i] = s ? -v : v;
+    }
+    return bad ? -1 : 0;
+}

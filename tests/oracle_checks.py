@@ -263,6 +263,24 @@ def check_softmax(impl, seed=18):
     assert abs(big[0, 0] - 1.0 / (1.0 + np.exp(-1.0) + np.exp(-1000.0))) <= 1e-15
 
 
+def check_e4m3_decoding(impl):
+    """Exact E4M3 values (the low-bit operand format) against codes worked by
+    hand from the OCP 8-bit floating point layout, and every non-NaN code
+    against torch's float8_e4m3fn conversion (a library routine)."""
+    import torch
+    with open(os.path.join(GOLDEN, "e4m3_codes.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if not line:
+                continue
+            code, want = line.split()
+            got = impl.decode_e4m3(np.array([int(code, 16)], dtype=np.uint8))[0]
+            assert got == float(want) and np.signbit(got) == np.signbit(float(want)), (code, got, want)
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(impl.decode_e4m3(codes), lib)
+
+
 ALL_CHECKS = [
     check_retained_counts,
     check_scores_closed_forms,
@@ -275,4 +293,5 @@ ALL_CHECKS = [
     check_one_row_ties,
     check_grouped_heads,
     check_softmax,
+    check_e4m3_decoding,
 ]

@@ -23,6 +23,7 @@ def _mutant(**overrides):
         rmm_qk=oracle.rmm_qk,
         rmm_pv=oracle.rmm_pv,
         softmax_rows=oracle.softmax_rows,
+        decode_e4m3=oracle.decode_e4m3,
     )
     for k, v in overrides.items():
         setattr(m, k, v)
@@ -119,6 +120,17 @@ def _softmax_linear(S):
     return E / E.sum(axis=1, keepdims=True)
 
 
+def _e4m3_bias_8(codes):
+    c = np.asarray(codes, dtype=np.uint8)
+    return oracle.decode_e4m3(c) / 2.0
+
+
+def _e4m3_no_subnormals(codes):
+    c = np.asarray(codes, dtype=np.uint8)
+    v = oracle.decode_e4m3(c)
+    return np.where((c & 0x78) == 0, 0.0 * v, v)
+
+
 def _count_floor(rho, d):
     return max(1, int(math.floor(rho * d)))
 
@@ -143,6 +155,8 @@ MUTANTS = {
     "softmax_over_the_query_axis": _mutant(softmax_rows=_softmax_over_columns),
     "softmax_mask_as_zero_logit": _mutant(softmax_rows=_softmax_mask_as_zero_logit),
     "softmax_without_exp": _mutant(softmax_rows=_softmax_linear),
+    "e4m3_exponent_bias_8": _mutant(decode_e4m3=_e4m3_bias_8),
+    "e4m3_subnormals_flushed": _mutant(decode_e4m3=_e4m3_no_subnormals),
 }
 
 

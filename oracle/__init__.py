@@ -18,6 +18,9 @@ calls it.  Every function pins to the paper as follows (tests/test_oracle_pins.p
   rmm_qk / rmm_pv     -- per-head bounds and rho=1 dense special cases
   decode_e4m3         -- hand-worked codes (golden file) and every code against
                          torch's float8_e4m3fn conversion
+  rmm_attention       -- rho = 1 equals scipy's softmax attention; the token step
+                         obeys Proposition 1 on P V; its sets are the TopK of
+                         the oracle's own column norms
   softmax_rows        -- closed forms (uniform row, two-key logistic), masked
                          entries exactly 0, rows sum to 1 and not columns,
                          per-row shift invariance, large logits stay finite
@@ -225,6 +228,25 @@ def rmm_qk(Q, K, rho: float, alpha: float, causal: bool = True, heads=None, rows
     S = np.stack([reduced_scores(Q[h], K[kv_head_of(h, H, Hkv)], I[h], alpha, causal, rows)
                   for h in hs])
     return S, I
+
+
+def rmm_attention(Q, K, V, rho_d: float, rho_t: float, alpha: float, causal: bool = True):
+    """RMM attention of every head [RMM paper, §3.3 "Attention"], the three steps
+    in the paper's order: features I_h = TopK of Q_h's column norms (rho_d)
+    and S_h = alpha Q_h[:, I_h] K_g[:, I_h]^T + M; P_h = softmax(S_h) over each
+    row; tokens T_h = TopK of P_h's column norms (rho_t) and
+    O_h = P_h[:, T_h] V_g[T_h, :].  Q [H, n, d_h], K [H_kv, n_k, d_h],
+    V [H_kv, n_k, d_v].  Returns (O [H, n, d_v], I [H, k_d], T [H, k_t], P [H, n, n_k]),
+    all fp64 (I, T int32)."""
+    Q, K, V = as_f64(Q), as_f64(K), as_f64(V)
+    H = Q.shape[0]
+    Hkv = K.shape[0]
+    S, I = rmm_qk(Q, K, rho=rho_d, alpha=alpha, causal=causal)
+    P = softmax_rows(S)
+    kt = retained_count(rho_t, P.shape[2])
+    T = np.stack([select(P[h], k=kt)[0] for h in range(H)])
+    O = np.stack([reduced_product(P[h], V[kv_head_of(h, H, Hkv)], T[h]) for h in range(H)])
+    return O, I, T, P
 
 
 def rmm_pv(P, V, rho: float, heads=None, rows=None):

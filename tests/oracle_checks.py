@@ -281,6 +281,38 @@ def check_e4m3_decoding(impl):
     assert np.array_equal(impl.decode_e4m3(codes), lib)
 
 
+def check_attention(impl, seed=19):
+    """RMM attention [§3.3 "Attention"]: with every feature and token kept it is
+    softmax(alpha Q K^T + M) V per head with grouped-query K/V (scipy's softmax,
+    a library routine); with tokens dropped the error of O_h obeys
+    Proposition 1 (Eq. 12) for the product P_h V_g, and T_h is the TopK of
+    P_h's column norms."""
+    import scipy.special
+    rng = _rng(seed)
+    H, Hkv, n, dh, dv = 4, 2, 12, 8, 6
+    Q = rng.standard_normal((H, n, dh)) * np.exp(rng.standard_normal((H, 1, dh)))
+    K = rng.standard_normal((Hkv, n, dh))
+    V = rng.standard_normal((Hkv, n, dv))
+    alpha = 1.0 / np.sqrt(dh)
+    mask = np.triu(np.ones((n, n), dtype=bool), 1)
+    O, I, T, P = impl.rmm_attention(Q, K, V, 1.0, 1.0, alpha, True)
+    for h in range(H):
+        g = h // (H // Hkv)
+        logits = np.where(mask, -np.inf, alpha * Q[h] @ K[g].T)
+        ref = scipy.special.softmax(logits, axis=1) @ V[g]
+        assert np.allclose(O[h], ref, rtol=1e-12, atol=1e-14), h
+    O, I, T, P = impl.rmm_attention(Q, K, V, 0.5, 0.5, alpha, True)
+    kt = impl.retained_count(0.5, n)
+    for h in range(H):
+        g = h // (H // Hkv)
+        s2 = (P[h] ** 2).sum(axis=0)
+        assert np.array_equal(T[h], impl.topk_indices(s2, kt))
+        full = P[h] @ V[g]
+        dropped = np.setdiff1d(np.arange(n), T[h])
+        bound = sum(np.linalg.norm(P[h][:, j]) * np.linalg.norm(V[g][j]) for j in dropped)
+        assert np.linalg.norm(full - O[h]) <= bound * (1 + 1e-12) + 1e-15
+
+
 ALL_CHECKS = [
     check_retained_counts,
     check_scores_closed_forms,
@@ -294,4 +326,5 @@ ALL_CHECKS = [
     check_grouped_heads,
     check_softmax,
     check_e4m3_decoding,
+    check_attention,
 ]

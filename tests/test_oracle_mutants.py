@@ -24,6 +24,7 @@ def _mutant(**overrides):
         rmm_pv=oracle.rmm_pv,
         softmax_rows=oracle.softmax_rows,
         decode_e4m3=oracle.decode_e4m3,
+        rmm_attention=oracle.rmm_attention,
     )
     for k, v in overrides.items():
         setattr(m, k, v)
@@ -131,6 +132,23 @@ def _e4m3_no_subnormals(codes):
     return np.where((c & 0x78) == 0, 0.0 * v, v)
 
 
+def _attention_tokens_from_scores(Q, K, V, rho_d, rho_t, alpha, causal=True):
+    """Token set chosen from the column norms of the scores S instead of P."""
+    Q, K, V = oracle.as_f64(Q), oracle.as_f64(K), oracle.as_f64(V)
+    H, Hkv = Q.shape[0], K.shape[0]
+    S, I = oracle.rmm_qk(Q, K, rho=rho_d, alpha=alpha, causal=causal)
+    P = oracle.softmax_rows(S)
+    kt = oracle.retained_count(rho_t, P.shape[2])
+    Sf = np.where(np.isneginf(S), 0.0, S)
+    T = np.stack([oracle.topk_indices((Sf[h] ** 2).sum(axis=0), kt) for h in range(H)])
+    O = np.stack([oracle.reduced_product(P[h], V[h // (H // Hkv)], T[h]) for h in range(H)])
+    return O, I, T, P
+
+
+def _attention_unscaled(Q, K, V, rho_d, rho_t, alpha, causal=True):
+    return oracle.rmm_attention(Q, K, V, rho_d, rho_t, 1.0, causal)
+
+
 def _count_floor(rho, d):
     return max(1, int(math.floor(rho * d)))
 
@@ -157,6 +175,8 @@ MUTANTS = {
     "softmax_without_exp": _mutant(softmax_rows=_softmax_linear),
     "e4m3_exponent_bias_8": _mutant(decode_e4m3=_e4m3_bias_8),
     "e4m3_subnormals_flushed": _mutant(decode_e4m3=_e4m3_no_subnormals),
+    "attention_tokens_from_scores": _mutant(rmm_attention=_attention_tokens_from_scores),
+    "attention_without_scale": _mutant(rmm_attention=_attention_unscaled),
 }
 
 

@@ -355,6 +355,11 @@ def run_rmm(args):
                         "ms_cublas_dense": t_cb, "speedup_vs_rho1": t_1 / t_r,
                         "kernel_launches": e["rmm"]["plan"].kernel_launches}
 
+    # more evidence timed by the same run (outside the headline timed region):
+    # the Llama-3-70B MLP ops and the attention forms at n = 4096
+    if not args.no_extra_points:
+        points.update(extra_points(dev, stream, rho, op_latency))
+
     # end to end through the public API with host buffers (pinned), copies timed
     e2e = None
     if not args.no_e2e:
@@ -453,6 +458,90 @@ def run_rmm(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def extra_points(dev, stream, rho, op_latency):
+    """Per-op latency at rho, at rho = 1 and of the dense torch product for the
+    Llama-3-70B up / down projections at n = 4096 and for causal attention
+    (32 query heads, 8 KV heads, L = 4096, d_h = 128): QK^T, PV scoring P
+    itself, and PV taking the token scores written by the softmax kernel that
+    produced P (producer-fused scoring; the softmax timed on its own)."""
+    import torch
+    import input_adaptive_reduced_b200 as rmm
+    import workloads as W
+    out = {}
+    n = 4096
+    for shape in ("up", "down"):
+        A, B = W.linear_70b(1, n=n, shape=shape, device=dev)
+        d, m = A.shape[1], B.shape[1]
+        k = retained(rho, d)
+        t_r = op_latency(lambda: rmm.matmul(A, B, rho=rho))
+        t_1 = op_latency(lambda: rmm.matmul(A, B, rho=1.0))
+        t_cb = op_latency(lambda: torch.matmul(A, B))
+        out[f"70b_{shape}"] = {"n": n, "d": d, "m": m, "k": k, "ms": t_r,
+                               "useful_tflops": 2.0 * n * k * m / (t_r * 1e-3) / 1e12, "ms_rho1": t_1,
+                               "ms_cublas_dense": t_cb, "speedup_vs_rho1": t_1 / t_r}
+        del A, B
+        torch.cuda.empty_cache()
+    H, Hkv, dh = 32, 8, 128
+    Q, K = W.attn_qk(1, n=n, device=dev)
+    Kt = K.repeat_interleave(H // Hkv, dim=0).transpose(1, 2)
+    t_r = op_latency(lambda: rmm.qk(Q, K, rho=rho, causal=True))
+    t_1 = op_latency(lambda: rmm.qk(Q, K, rho=1.0, causal=True))
+    t_d = op_latency(lambda: torch.matmul(Q, Kt))
+    out["qk_causal"] = {"heads": H, "kv_heads": Hkv, "L": n, "d_h": dh, "k": retained(rho, dh), "ms": t_r,
+                        "ms_rho1": t_1, "ms_torch_dense": t_d, "speedup_vs_rho1": t_1 / t_r}
+    # scores of the causal attention for the softmax (bf16, -inf above the diagonal)
+    S = rmm.qk(Q, K, rho=1.0, causal=True)
+    del Q, K, Kt
+    torch.cuda.empty_cache()
+    V = (torch.randn((Hkv, n, 128), generator=W.gen(2, dev), device=dev)).to(torch.bfloat16)
+    t_sm = op_latency(lambda: rmm.softmax_scores(S, causal=True))
+    P, s2 = rmm.softmax_scores(S, causal=True)
+    del S
+    torch.cuda.empty_cache()
+    Vr = V.repeat_interleave(H // Hkv, dim=0)
+    k = retained(rho, n)
+    t_r = op_latency(lambda: rmm.pv(P, V, rho=rho, causal=True))
+    t_g = op_latency(lambda: rmm.pv(P, V, rho=rho, causal=True, scores=s2))
+    t_1 = op_latency(lambda: rmm.pv(P, V, rho=1.0, causal=True))
+    t_d = op_latency(lambda: torch.matmul(P, Vr))
+    out["pv_causal"] = {"heads": H, "kv_heads": Hkv, "L": n, "d_v": 128, "k": k, "ms": t_r,
+                        "ms_given_scores": t_g, "ms_rho1": t_1, "ms_torch_dense": t_d,
+                        "ms_softmax_with_scores": t_sm, "speedup_vs_rho1": t_1 / t_r,
+                        "speedup_vs_rho1_given_scores": t_1 / t_g}
+    del P, V, Vr, s2
+    torch.cuda.empty_cache()
+    # fused RMM attention (features rho, tokens rho) against the same three steps as
+    # separate ops (scores written, softmax with token scores, PV on the given
+    # scores) and torch's dense causal attention (scaled_dot_product_attention)
+    Q, K = W.attn_qk(1, n=n, device=dev)
+    V = (torch.randn((Hkv, n, 128), generator=W.gen(2, dev), device=dev)).to(torch.bfloat16)
+    alpha = 1.0 / math.sqrt(dh)
+    t_f = op_latency(lambda: rmm.attention(Q, K, V, rho, rho, causal=True, alpha=alpha))
+    t_f1 = op_latency(lambda: rmm.attention(Q, K, V, 1.0, 1.0, causal=True, alpha=alpha))
+
+    def unfused():
+        S = rmm.qk(Q, K, rho=rho, alpha=alpha, causal=True)
+        P, s2 = rmm.softmax_scores(S, causal=True)
+        return rmm.pv(P, V, rho=rho, causal=True, scores=s2)
+    t_u = op_latency(unfused)
+    t_sdpa = None
+    try:
+        Kr, Vr = K.repeat_interleave(H // Hkv, dim=0), V.repeat_interleave(H // Hkv, dim=0)
+        t_sdpa = op_latency(lambda: torch.nn.functional.scaled_dot_product_attention(
+            Q[None], Kr[None], Vr[None], is_causal=True))
+        del Kr, Vr
+    except Exception:
+        pass
+    flops_qk = 2.0 * H * retained(rho, dh) * n * (n + 1) / 2  # causal half of the scores, per pass
+    out["attention_fused_causal"] = {"heads": H, "kv_heads": Hkv, "L": n, "d_h": dh, "rho_d": rho, "rho_t": rho,
+                                     "ms": t_f, "ms_rho1": t_f1, "ms_unfused_ops": t_u,
+                                     "ms_torch_sdpa_dense": t_sdpa, "passes_over_the_scores": 3,
+                                     "score_tflops_per_pass": flops_qk / (t_f * 1e-3) / 1e12}
+    del Q, K, V
+    torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------------------- sweep
@@ -665,6 +754,60 @@ def run_sweep(args):
                       "gbs": hbm / (t_op * 1e-3) / 1e9, "bound": "hbm",
                       "frac": hbm / (t_op * 1e-3) / 1e9 / peak_gbs, **rec})
         del q, K, V, P
+    # fused RMM attention (features and tokens at rho) against the three steps as
+    # separate ops, and the softmax that writes P with its token scores
+    for n in (1024, 2048, 4096):
+        if not (want("attn", "fused", n) or want("attn", "softmax", n)):
+            continue
+        H, Hkv, dh = 32, 8, 128
+        Q, K = W.attn_qk(1, n=n, device=dev)
+        V = (torch.randn((Hkv, n, 128), generator=W.gen(2, dev), device=dev)).to(torch.bfloat16)
+        alpha = 1.0 / math.sqrt(dh)
+        if want("attn", "softmax", n):
+            S = rmm.qk(Q, K, rho=1.0, alpha=alpha, causal=True)
+            t = lat(lambda: rmm.softmax_scores(S, causal=True))
+            moved = 32 * (2.0 * n * (n + 1) / 2 + 2.0 * n * n)  # causal half of S read, P written in full
+            emit({"config": "attn", "op": "softmax", "n": n, "ms": t, "gbs": moved / (t * 1e-3) / 1e9,
+                  "bound": "hbm", "frac": moved / (t * 1e-3) / 1e9 / peak_gbs})
+            del S
+        for rho in (0.5, 0.8, 1.0):
+            if not want("attn", "fused", n, rho):
+                continue
+            t = lat(lambda: rmm.attention(Q, K, V, rho, rho, causal=True, alpha=alpha))
+            flops = 2.0 * H * retained(rho, dh) * n * (n + 1) / 2  # one causal pass over the reduced scores
+            emit({"config": "attn", "op": "fused", "n": n, "rho": rho, "ms": t, "bound": "tensor",
+                  "score_tflops_per_pass": flops / (t * 1e-3) / 1e12, "passes": 3})
+        del Q, K, V
+    # low-bit form: E4M3 operands with per-tensor scales, bf16 output, on the
+    # Llama-3.1-8B MLP shapes; dense reference: torch's scaled fp8 matmul
+    for n in (2048, 4096):
+        for name, gen in (("up", W.mlp_up), ("down", W.mlp_down)):
+            if not want("fp8", name, n):
+                continue
+            A, B = gen(1, n=n, device=dev)
+            Aq, sa = W.quantize_e4m3(A)
+            Bq, sb = W.quantize_e4m3(B)
+            del A, B
+            d, m = Aq.shape[1], Bq.shape[1]
+            t_dense = None
+            try:
+                Bcm = Bq.t().contiguous().t()
+                one = torch.ones((), device=dev)
+                t_dense = lat(lambda: torch._scaled_mm(Aq, Bcm, scale_a=one * sa, scale_b=one * sb,
+                                                       out_dtype=torch.bfloat16))
+            except Exception:
+                pass
+            for rho in (0.5, 0.8, 1.0):
+                if not want("fp8", name, n, rho):
+                    continue
+                k = retained(rho, d)
+                t = lat(lambda: rmm.matmul(Aq, Bq, rho=rho, alpha=sa * sb))
+                flops = 2.0 * n * k * m
+                emit({"config": "fp8", "op": name, "n": n, "d": d, "m": m, "rho": rho, "k": k, "ms": t,
+                      "useful_tflops": flops / (t * 1e-3) / 1e12, "bound": "tensor",
+                      "frac_of_bf16_peak": flops / (t * 1e-3) / 1e12 / peak_tf,
+                      "ms_dense_scaled_mm": t_dense})
+            del Aq, Bq
     # 5: Llama-3-70B linear
     for shape in ("up", "down", "qkv"):
         for n in (1, 16, 512, 2048, 4096):
@@ -689,6 +832,8 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=64)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-extra-points", action="store_true",
+                    help="skip the 70B and attention points timed after the headline")
     ap.add_argument("--sweep", action="store_true", help="time every point of the five workloads")
     ap.add_argument("--sweep-out", default=None)
     ap.add_argument("--sweep-only", default=None,

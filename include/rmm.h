@@ -68,7 +68,19 @@ typedef enum rmm_status {
 
 typedef enum rmm_dtype {
     RMM_BF16 = 0, /* bfloat16 storage, fp32 accumulation (tcgen05 kind::f16) */
-    RMM_F32 = 1   /* fp32 storage, tf32 products with fp32 accumulation (tcgen05 kind::tf32) */
+    RMM_F32 = 1,  /* fp32 storage, tf32 products with fp32 accumulation (tcgen05 kind::tf32) */
+    /* Low-bit form (the RMM paper runs RMM next to 8-bit weight quantization,
+       App. B.6, and names dedicated low-bit kernels as future work, App. B.7):
+       A and B hold 8-bit E4M3 codes (OCP 8-bit floating point, e4m3fn: no
+       infinities, largest magnitude 448), Y is bfloat16.  Per-tensor scales go
+       into alpha: Y = alpha * A[:, I] B[I, :] over the decoded codes, so a
+       caller with A = sa * Aq and B = sb * Bq passes alpha = sa * sb.  Scores
+       are sums of squares of the decoded codes (a positive per-tensor scale
+       does not change I); products on tcgen05 kind::f8f6f4 with fp32
+       accumulation.  LINEAR with one head only, n = 0 or n > 128
+       (RMM_ERR_UNSUPPORTED otherwise); d, m, lda and ldb multiples of 16;
+       ldy a multiple of 8 (bf16 elements). */
+    RMM_FP8_E4M3 = 2
 } rmm_dtype;
 
 typedef enum rmm_mode {
@@ -98,6 +110,20 @@ typedef enum rmm_mode {
 /* rmm_matmul*: take I from the caller (I_inout, [heads][k], ascending,
    distinct, each in [0, d)) instead of computing it; no scores are formed. */
 #define RMM_FLAG_USE_GIVEN_INDICES 2u
+/* Producer-fused scoring (the RMM paper §3.3 "Attention" scores tokens by the
+   column norms of P, and Appendix D.1 "Practical implications" asks for the
+   norms to be computed efficiently).  rmm_matmul_ex only:
+   RMM_FLAG_GIVEN_SCORES -- take the column scores of A from the caller
+   (s2_in[h][j] = fp32 sum_i A[h][i][j]^2, as written by the op that produced
+   A: RMM_FLAG_EMIT_SCORES of an earlier product, or rmm_softmax_scores)
+   instead of reading A for them; I = TopK of s2_in, exactly as if the op had
+   computed those scores.  Not with RMM_FLAG_USE_GIVEN_INDICES.
+   RMM_FLAG_EMIT_SCORES -- also write the column scores of this op's output,
+   s2_out[h][c] = fp32 sum_i Y[h][i][c]^2 over the stored (rounded) values,
+   summed in a fixed order (the same bits on every call), so that an op
+   taking Y as its A can skip its score pass.  LINEAR and PV only. */
+#define RMM_FLAG_GIVEN_SCORES 4u
+#define RMM_FLAG_EMIT_SCORES 8u
 
 /* One problem shape.  All sizes and strides count ELEMENTS.  Heads: query
    head h (0 <= h < heads) reads A, I and Y at offset h * stride_{a,y} and B at
@@ -105,7 +131,7 @@ typedef enum rmm_mode {
    kv_heads = heads means one B per head, kv_heads = 1 one shared B). */
 typedef struct rmm_problem {
     int32_t mode;      /* rmm_mode */
-    int32_t dtype;     /* rmm_dtype of A, B and Y */
+    int32_t dtype;     /* rmm_dtype of A, B and Y (E4M3: A and B; Y is bf16) */
     int64_t n;         /* rows of A and Y (tokens / queries), >= 0 */
     int64_t d;         /* contraction size, >= 1, multiple of 8 (bf16) or 4 (fp32) */
     int64_t m;         /* columns of Y, >= 0, multiple of 8 (bf16) or 4 (fp32) */
@@ -182,10 +208,48 @@ RMM_API rmm_status rmm_select_no_alloc(const rmm_plan* plan, const void* A, int3
 RMM_API rmm_status rmm_matmul(const rmm_plan* plan, const void* A, const void* B, void* Y,
                       int32_t* I_inout, void* workspace, size_t workspace_bytes, void* stream);
 
-/* Same as rmm_matmul for any number of heads; I_inout is [heads][k]. */
+/* Same as rmm_matmul for any number of heads; I_inout is [heads][k].
+   rmm_matmul and rmm_matmul_batched return RMM_ERR_INVALID_ARG for a plan
+   with RMM_FLAG_GIVEN_SCORES or RMM_FLAG_EMIT_SCORES (use rmm_matmul_ex). */
 RMM_API rmm_status rmm_matmul_batched(const rmm_plan* plan, const void* A, const void* B, void* Y,
                               int32_t* I_inout, void* workspace, size_t workspace_bytes,
                               void* stream);
+
+/* rmm_matmul_batched with producer-fused scoring.  s2_in: device fp32
+   [heads][d], the column scores of A; required with RMM_FLAG_GIVEN_SCORES,
+   else ignored.  s2_out: device fp32 [heads][m], receives the column scores
+   of Y; required with RMM_FLAG_EMIT_SCORES, else ignored.  On the CTA-pair
+   product (more than 128 rows) the scores come from the product's epilogue:
+   each warp squares its 32 x 32 block of stored outputs, sums the 32 rows of
+   each column, and the last block of a column adds the row blocks' sums in
+   row order; other shapes add one score pass over Y after the product.
+   Errors: a required pointer NULL or not 4-byte aligned, RMM_ERR_INVALID_ARG. */
+RMM_API rmm_status rmm_matmul_ex(const rmm_plan* plan, const void* A, const void* B, void* Y,
+                                 int32_t* I_inout, const float* s2_in, float* s2_out, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* Attention weights with producer-fused token scores: the op that produces
+   P for an RMM PV call (the RMM paper §3.3 "Attention": P = softmax(S~ + M);
+   the PV product then keeps the tokens with the largest a_t = ||P[:, t]||).
+   For each head h and row i of S[h] (n x t bf16, row stride lds, head
+   stride stride_s, -inf entries are masked keys) it writes
+     P[h][i][c] = exp(S[h][i][c] - max_c' S[h][i][c']) / sum_c' exp(...)
+   rounded to bf16 (row stride ldp, head stride stride_p), and
+     s2[h][c] = fp32 sum over i of P[h][i][c]^2 of the stored values,
+   each thread's rows summed in row order and the row blocks in block order
+   (the same bits on every call); pass s2 as s2_in of an RMM_PV plan with
+   RMM_FLAG_GIVEN_SCORES.  flags: RMM_FLAG_CAUSAL states S[h][i][c] = -inf
+   for c > i (those entries are not read; P is written as 0 there).  Every
+   row needs a finite entry.  Sizes: t a multiple of 8, t <= 8192; strides
+   multiples of 8 elements, lds and ldp >= t.  workspace: device memory of
+   rmm_softmax_workspace_size(heads, n, t) bytes, 256-byte aligned, zeroed
+   once (cudaMemsetAsync) before its first use; the kernel leaves its
+   counters at zero.  Errors: RMM_ERR_INVALID_ARG / RMM_ERR_UNSUPPORTED /
+   RMM_ERR_WORKSPACE before any launch. */
+RMM_API size_t rmm_softmax_workspace_size(int64_t heads, int64_t n, int64_t t);
+RMM_API rmm_status rmm_softmax_scores(const void* S, void* P, float* s2, int64_t heads, int64_t n, int64_t t,
+                                      int64_t lds, int64_t stride_s, int64_t ldp, int64_t stride_p, uint32_t flags,
+                                      void* workspace, size_t workspace_bytes, void* stream);
 
 /* Zero the workspace's header (its error word, the score pass's completion
    counters and the product's split-tail counters, which the kernels return to
@@ -221,6 +285,47 @@ RMM_API rmm_status rmm_plan_set_product_events(rmm_plan* plan, void* start, void
 
 /* Number of kernels one rmm_matmul* call of this plan launches (-1 for NULL). */
 RMM_API int32_t rmm_plan_kernel_launches(const rmm_plan* plan);
+
+/* Fused RMM attention (self-attention, one call for all heads): the RMM
+   paper's three steps of §3.3 "Attention" without writing the score matrix
+   or the weights.  Per query head h (grouped-query K/V head g = h / (heads /
+   kv_heads)): I_h = TopK of Q[h]'s column norms, k_d = ceil(rho_d d_h);
+   S = alpha Q[h][:, I_h] K[g][:, I_h]^T (-inf above the diagonal with
+   RMM_FLAG_CAUSAL); P = softmax(S) over each row; T_h = TopK of P's column
+   norms, k_t = ceil(rho_t n); O[h] = P[:, T_h] V[g][T_h, :].  The scores are
+   recomputed in three passes (row statistics; token scores, which need every
+   row's final normalisation; the output over the key blocks that hold a kept
+   token), on the tensor cores; the token scores are fp32 sums of P^2 of the
+   fp32 weights, and the product rounds P to bf16.  Ties keep the lower index;
+   I and T are ascending.  The pages' own attention kernels were not fully
+   fused (App. B.7); this form has no counterpart there beyond the method. */
+typedef struct rmm_attn_problem {
+    int64_t heads, kv_heads;  /* query heads; K/V heads, dividing heads */
+    int64_t n;                /* queries = keys per head, a multiple of 8, <= 49152 */
+    int64_t d_h, d_v;         /* both 128 (RMM_ERR_UNSUPPORTED otherwise) */
+    int64_t ldq, ldk, ldv, ldo;                      /* row strides, multiples of 8 elements */
+    int64_t stride_q, stride_k, stride_v, stride_o;  /* head strides (elements) */
+    double rho_d, rho_t;      /* feature and token retention ratios in (0, 1] */
+    float alpha;              /* score scale; the paper's 1/sqrt(d_h) */
+    uint32_t flags;           /* RMM_FLAG_CAUSAL or 0 */
+} rmm_attn_problem;
+
+/* Workspace bytes rmm_attention needs for *p (0 for an invalid problem).
+   Reads the current device's SM count. */
+RMM_API size_t rmm_attention_workspace_size(const rmm_attn_problem* p);
+
+/* Q [heads][n][d_h], K [kv_heads][n][d_h], V [kv_heads][n][d_v], O
+   [heads][n][d_v]: bf16 device memory, 16-byte aligned.  I_out ([heads][k_d])
+   and T_out ([heads][k_t]) receive the index sets when not NULL.  workspace:
+   device memory of rmm_attention_workspace_size(p) bytes, 256-byte aligned,
+   zeroed once (cudaMemsetAsync) before its first use; the kernels return its
+   counters to zero, and a kernel that gives up on a wait (about two seconds)
+   writes a nonzero code into its first word.  Asynchronous on `stream`.
+   Errors: RMM_ERR_INVALID_ARG / RMM_ERR_UNSUPPORTED / RMM_ERR_WORKSPACE before
+   any launch, RMM_ERR_CUDA if a launch fails. */
+RMM_API rmm_status rmm_attention(const rmm_attn_problem* p, const void* Q, const void* K, const void* V, void* O,
+                                 int32_t* I_out, int32_t* T_out, void* workspace, size_t workspace_bytes,
+                                 void* stream);
 
 /* Static string naming a status code. */
 RMM_API const char* rmm_status_string(rmm_status s);

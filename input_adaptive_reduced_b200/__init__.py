@@ -19,26 +19,31 @@ import weakref
 
 __all__ = [
     "RMM_OK", "RMM_ERR_INVALID_ARG", "RMM_ERR_UNSUPPORTED", "RMM_ERR_WORKSPACE", "RMM_ERR_CUDA",
-    "RMM_ERR_TIMEOUT", "RMM_BF16", "RMM_F32", "RMM_LINEAR", "RMM_QK", "RMM_PV", "RMM_FLAG_CAUSAL",
+    "RMM_ERR_TIMEOUT", "RMM_BF16", "RMM_F32", "RMM_FP8_E4M3", "RMM_LINEAR", "RMM_QK", "RMM_PV", "RMM_FLAG_CAUSAL",
     "RMM_FLAG_USE_GIVEN_INDICES", "RmmError", "rmm_problem", "Plan", "lib", "library_path",
     "rmm_problem_init", "rmm_plan_create", "rmm_select", "rmm_matmul", "rmm_matmul_batched",
     "rmm_workspace_init", "rmm_workspace_status", "rmm_status_string", "rmm_version",
     "EXPORTED_SYMBOLS", "select", "matmul", "qk", "pv", "workspace_for", "check_workspaces",
     "rmm_plan_set_product_events", "rmm_plan_kernel_launches", "rmm_select_no_alloc",
-    "rmm_selftest_wait_timeout",
+    "rmm_selftest_wait_timeout", "RMM_FLAG_GIVEN_SCORES", "RMM_FLAG_EMIT_SCORES", "rmm_matmul_ex",
+    "rmm_softmax_scores", "rmm_softmax_workspace_size", "softmax_scores", "rmm_attn_problem",
+    "rmm_attention", "rmm_attention_workspace_size", "attention",
 ]
 
 RMM_OK, RMM_ERR_INVALID_ARG, RMM_ERR_UNSUPPORTED, RMM_ERR_WORKSPACE, RMM_ERR_CUDA, RMM_ERR_TIMEOUT = range(6)
-RMM_BF16, RMM_F32 = 0, 1
+RMM_BF16, RMM_F32, RMM_FP8_E4M3 = 0, 1, 2
 RMM_LINEAR, RMM_QK, RMM_PV = 0, 1, 2
 RMM_FLAG_CAUSAL = 1
 RMM_FLAG_USE_GIVEN_INDICES = 2
+RMM_FLAG_GIVEN_SCORES = 4
+RMM_FLAG_EMIT_SCORES = 8
 
 EXPORTED_SYMBOLS = (
     "rmm_problem_init", "rmm_plan_create", "rmm_plan_destroy", "rmm_plan_k", "rmm_plan_workspace_size",
     "rmm_select", "rmm_matmul", "rmm_matmul_batched", "rmm_workspace_init", "rmm_workspace_status",
     "rmm_status_string", "rmm_version", "rmm_plan_set_product_events", "rmm_plan_kernel_launches",
-    "rmm_select_no_alloc", "rmm_selftest_wait_timeout",
+    "rmm_select_no_alloc", "rmm_selftest_wait_timeout", "rmm_matmul_ex", "rmm_softmax_workspace_size",
+    "rmm_softmax_scores", "rmm_attention_workspace_size", "rmm_attention",
 )
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librmm.so")
@@ -59,6 +64,17 @@ class rmm_problem(ctypes.Structure):
         ("stride_a", ctypes.c_int64), ("stride_b", ctypes.c_int64), ("stride_y", ctypes.c_int64),
         ("rho", ctypes.c_double), ("k", ctypes.c_int64), ("alpha", ctypes.c_float),
         ("flags", ctypes.c_uint32),
+    ]
+
+
+class rmm_attn_problem(ctypes.Structure):
+    _fields_ = [
+        ("heads", ctypes.c_int64), ("kv_heads", ctypes.c_int64), ("n", ctypes.c_int64),
+        ("d_h", ctypes.c_int64), ("d_v", ctypes.c_int64),
+        ("ldq", ctypes.c_int64), ("ldk", ctypes.c_int64), ("ldv", ctypes.c_int64), ("ldo", ctypes.c_int64),
+        ("stride_q", ctypes.c_int64), ("stride_k", ctypes.c_int64), ("stride_v", ctypes.c_int64),
+        ("stride_o", ctypes.c_int64), ("rho_d", ctypes.c_double), ("rho_t", ctypes.c_double),
+        ("alpha", ctypes.c_float), ("flags", ctypes.c_uint32),
     ]
 
 
@@ -101,6 +117,16 @@ def _load_library():
     L.rmm_plan_set_product_events.argtypes = [vp, vp, vp]
     L.rmm_plan_kernel_launches.restype = ctypes.c_int32
     L.rmm_plan_kernel_launches.argtypes = [vp]
+    L.rmm_matmul_ex.restype = st
+    L.rmm_matmul_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.rmm_softmax_workspace_size.restype = sz
+    L.rmm_softmax_workspace_size.argtypes = [i64, i64, i64]
+    L.rmm_softmax_scores.restype = st
+    L.rmm_softmax_scores.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, ctypes.c_uint32, vp, sz, vp]
+    L.rmm_attention_workspace_size.restype = sz
+    L.rmm_attention_workspace_size.argtypes = [ctypes.POINTER(rmm_attn_problem)]
+    L.rmm_attention.restype = st
+    L.rmm_attention.argtypes = [ctypes.POINTER(rmm_attn_problem), vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.rmm_select_no_alloc.restype = st
     L.rmm_select_no_alloc.argtypes = [vp, vp, vp, vp, vp]
     L.rmm_status_string.restype = ctypes.c_char_p
@@ -243,6 +269,35 @@ def rmm_matmul_batched(plan: Plan, A, B, Y, I=None, workspace=None, stream=None)
                                   _stream(stream)), "rmm_matmul_batched")
 
 
+def rmm_matmul_ex(plan: Plan, A, B, Y, I=None, s2_in=None, s2_out=None, workspace=None, stream=None):
+    """rmm_matmul_batched with producer-fused scoring: s2_in (fp32 [heads][d])
+    with RMM_FLAG_GIVEN_SCORES, s2_out (fp32 [heads][m]) with RMM_FLAG_EMIT_SCORES."""
+    wp, wb = _ws(workspace)
+    _check(lib.rmm_matmul_ex(plan.handle, _ptr(A), _ptr(B), _ptr(Y), _ptr(I), _ptr(s2_in), _ptr(s2_out), wp, wb,
+                             _stream(stream)), "rmm_matmul_ex")
+
+
+def rmm_softmax_workspace_size(heads: int, n: int, t: int) -> int:
+    return int(lib.rmm_softmax_workspace_size(heads, n, t))
+
+
+def rmm_softmax_scores(S, P, s2, heads, n, t, lds, stride_s, ldp, stride_p, flags=0, workspace=None,
+                       stream=None):
+    wp, wb = _ws(workspace)
+    _check(lib.rmm_softmax_scores(_ptr(S), _ptr(P), _ptr(s2), heads, n, t, lds, stride_s, ldp, stride_p,
+                                  int(flags), wp, wb, _stream(stream)), "rmm_softmax_scores")
+
+
+def rmm_attention_workspace_size(problem: rmm_attn_problem) -> int:
+    return int(lib.rmm_attention_workspace_size(ctypes.byref(problem)))
+
+
+def rmm_attention(problem: rmm_attn_problem, Q, K, V, O, I=None, T=None, workspace=None, stream=None):
+    wp, wb = _ws(workspace)
+    _check(lib.rmm_attention(ctypes.byref(problem), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(I), _ptr(T), wp, wb,
+                             _stream(stream)), "rmm_attention")
+
+
 # ----------------------------------------------------------------------------
 # Convenience layer over torch tensors (still marshalling only).
 # ----------------------------------------------------------------------------
@@ -257,7 +312,9 @@ def _dtype_code(t) -> int:
         return RMM_BF16
     if t.dtype == torch.float32:
         return RMM_F32
-    raise TypeError(f"RMM supports bfloat16 and float32 tensors, not {t.dtype}")
+    if t.dtype == torch.float8_e4m3fn:
+        return RMM_FP8_E4M3
+    raise TypeError(f"RMM supports bfloat16, float32 and float8_e4m3fn tensors, not {t.dtype}")
 
 
 def _require_cuda(*ts):
@@ -345,29 +402,46 @@ def select(A, rho=None, k=None, return_scores=False):
     return (I, s2) if return_scores else I
 
 
-def matmul(A, B, rho=None, k=None, indices=None, return_indices=False, out=None):
-    """RMM_rho(A, B) = A[:, I] B[I, :] for A [n, d], B [d, m] (§3.2)."""
+def matmul(A, B, rho=None, k=None, indices=None, return_indices=False, out=None, scores=None,
+           emit_scores=False, alpha=1.0):
+    """RMM_rho(A, B) = alpha A[:, I] B[I, :] for A [n, d], B [d, m] (§3.2).
+    scores: A's column scores from the op that produced A (fp32 [d]); the op
+    then selects from them instead of reading A for them.  emit_scores=True
+    also returns Y's column scores (fp32 [m]) for the op that takes Y next.
+    float8_e4m3fn A and B (the low-bit form) give a bf16 Y; pass their
+    per-tensor scales as alpha = scale_A * scale_B."""
     import torch
-    _require_cuda(A, B, out, indices)
+    _require_cuda(A, B, out, indices, scores)
     n, d = A.shape
     m = B.shape[1]
     if B.shape[0] != d or B.dtype != A.dtype:
         raise ValueError("A is n x d and B is d x m with the same dtype")
     p = rmm_problem_init(RMM_LINEAR, _dtype_code(A), n, d, m)
     p.lda, p.ldb = _row_stride(A), _row_stride(B)
+    p.alpha = float(alpha)
     if indices is not None:
         p.k = indices.numel()
         p.flags |= RMM_FLAG_USE_GIVEN_INDICES
     else:
         _k_fields(p, rho, k)
-    Y = torch.empty((n, m), dtype=A.dtype, device=A.device) if out is None else out
+    if scores is not None:
+        p.flags |= RMM_FLAG_GIVEN_SCORES
+    if emit_scores:
+        p.flags |= RMM_FLAG_EMIT_SCORES
+    y_dtype = torch.bfloat16 if A.dtype == torch.float8_e4m3fn else A.dtype
+    Y = torch.empty((n, m), dtype=y_dtype, device=A.device) if out is None else out
     p.ldy = _row_stride(Y)
     plan = _plan_for(p)
     I = indices
     if I is None and return_indices:
         I = torch.empty(plan.k, dtype=torch.int32, device=A.device)
-    rmm_matmul(plan, A, B, Y, I, workspace_for(plan))
-    return (Y, I) if return_indices else Y
+    if scores is None and not emit_scores:
+        rmm_matmul(plan, A, B, Y, I, workspace_for(plan))
+        return (Y, I) if return_indices else Y
+    s2 = torch.empty(m, dtype=torch.float32, device=A.device) if emit_scores else None
+    rmm_matmul_ex(plan, A, B, Y, I, scores, s2, workspace_for(plan))
+    out_t = (Y,) + ((I,) if return_indices else ()) + ((s2,) if emit_scores else ())
+    return out_t if len(out_t) > 1 else Y
 
 
 def qk(Q, K, rho, alpha=None, causal=True, return_indices=False):
@@ -392,11 +466,94 @@ def qk(Q, K, rho, alpha=None, causal=True, return_indices=False):
     return (S, I) if return_indices else S
 
 
-def pv(P, V, rho, return_indices=False, causal=False):
+def softmax_scores(S, causal=False):
+    """Attention weights P = softmax(S) over each row of S [H, n, t] (bf16,
+    -inf = masked), with the token scores s2[h][t] = sum_i P[h][i][t]^2 of the
+    stored weights (the op producing P scores its columns, §3.3 "Attention").
+    Returns (P, s2)."""
+    import torch
+    _require_cuda(S)
+    if S.dtype != torch.bfloat16:
+        raise TypeError("softmax_scores takes bf16 scores")
+    H, n, t = S.shape
+    P = torch.empty_like(S)
+    s2 = torch.empty((H, t), dtype=torch.float32, device=S.device)
+    key = ("softmax", H, n, t, S.device.index)
+    with _cache_lock:
+        ws = _plans.get(key)
+    if ws is None:
+        ws = torch.zeros(max(rmm_softmax_workspace_size(H, n, t), 256), dtype=torch.uint8, device=S.device)
+        with _cache_lock:
+            _plans[key] = ws
+    rmm_softmax_scores(S, P, s2, H, n, t, _row_stride(S), S.stride(0), _row_stride(P), P.stride(0),
+                       RMM_FLAG_CAUSAL if causal else 0, ws)
+    return P, s2
+
+
+def attention(Q, K, V, rho_d, rho_t, causal=True, alpha=None, return_sets=False):
+    """Fused RMM attention (§3.3 "Attention"): features of Q per head (rho_d),
+    softmax of the reduced scores, tokens by P's column norms (rho_t), output
+    over the kept tokens -- without writing S or P.  Q [H, n, 128],
+    K and V [H_kv, n, 128], bf16.  Returns O (and I, T with return_sets)."""
+    import torch
+    _require_cuda(Q, K, V)
+    H, n, dh = Q.shape
+    Hkv, _, dv = V.shape
+    p = rmm_attn_problem()
+    p.heads, p.kv_heads, p.n, p.d_h, p.d_v = H, Hkv, n, dh, dv
+    p.ldq, p.ldk, p.ldv = _row_stride(Q), _row_stride(K), _row_stride(V)
+    p.stride_q, p.stride_k, p.stride_v = Q.stride(0), K.stride(0), V.stride(0)
+    O = torch.empty((H, n, dv), dtype=Q.dtype, device=Q.device)
+    p.ldo, p.stride_o = dv, n * dv
+    p.rho_d, p.rho_t = float(rho_d), float(rho_t)
+    p.alpha = 1.0 / math.sqrt(dh) if alpha is None else float(alpha)
+    p.flags = RMM_FLAG_CAUSAL if causal else 0
+    size = rmm_attention_workspace_size(p)
+    if size == 0:
+        raise RmmError(RMM_ERR_INVALID_ARG, "rmm_attention_workspace_size")
+    key = ("attention", H, Hkv, n, float(rho_d), float(rho_t), Q.device.index)
+    with _cache_lock:
+        ws = _plans.get(key)
+    if ws is None or ws.numel() < size:
+        ws = torch.zeros(max(size, 256), dtype=torch.uint8, device=Q.device)
+        with _cache_lock:
+            _plans[key] = ws
+    kd = _retained(float(rho_d), dh)
+    kt = _retained(float(rho_t), n)
+    I = torch.empty((H, kd), dtype=torch.int32, device=Q.device) if return_sets else None
+    T = torch.empty((H, kt), dtype=torch.int32, device=Q.device) if return_sets else None
+    rmm_attention(p, Q, K, V, O, I, T, ws)
+    return (O, I, T) if return_sets else O
+
+
+def attention_status(Q, K, V, rho_d, rho_t) -> int:
+    """The error word of the workspace attention() used for these sizes: 0, or
+    the code of a kernel that gave up on a wait (synchronises)."""
+    import torch
+    H, n = Q.shape[0], Q.shape[1]
+    key = ("attention", H, K.shape[0], n, float(rho_d), float(rho_t), Q.device.index)
+    with _cache_lock:
+        ws = _plans.get(key)
+    if ws is None:
+        return 0
+    torch.cuda.synchronize()
+    return int(ws[:4].view(torch.int32).item())
+
+
+def _retained(rho: float, d: int) -> int:
+    x = rho * d
+    r = round(x)
+    k = r if abs(x - r) <= 1e-9 * d else math.ceil(x)
+    return max(1, min(d, int(k)))
+
+
+def pv(P, V, rho, return_indices=False, causal=False, scores=None):
     """Token-reduced value product O[h] = P[h][:, T_h] V[g][T_h, :] for
     P [H, n, n_k] and V [H_kv, n_k, d_v] (§3.3 "Attention", last sentence).
     causal=True states that P[h][i][t] = 0 for t > i (n = n_k): the op then
-    skips the blocks of P above the diagonal (same result)."""
+    skips the blocks of P above the diagonal (same result).  scores: P's token
+    scores from the op that produced P (softmax_scores), fp32 [H, n_k]; the
+    op then selects from them instead of reading P for them."""
     import torch
     _require_cuda(P, V)
     H, n, nk = P.shape
@@ -406,10 +563,16 @@ def pv(P, V, rho, return_indices=False, causal=False):
     p.heads, p.kv_heads = H, Hkv
     p.stride_a, p.stride_b = P.stride(0), V.stride(0)
     p.flags = RMM_FLAG_CAUSAL if causal else 0
+    if scores is not None:
+        _require_cuda(scores)
+        p.flags |= RMM_FLAG_GIVEN_SCORES
     _k_fields(p, rho, None)
     O = torch.empty((H, n, dv), dtype=P.dtype, device=P.device)
     p.ldy, p.stride_y = dv, n * dv
     plan = _plan_for(p)
     T = torch.empty((H, plan.k), dtype=torch.int32, device=P.device) if return_indices else None
-    rmm_matmul_batched(plan, P, V, O, T, workspace_for(plan))
+    if scores is None:
+        rmm_matmul_batched(plan, P, V, O, T, workspace_for(plan))
+    else:
+        rmm_matmul_ex(plan, P, V, O, T, scores, None, workspace_for(plan))
     return (O, T) if return_indices else O

@@ -72,23 +72,28 @@ bool encode_kmajor_map(CUtensorMap* map, int es, const void* base, int64_t kext,
     cuuint64_t strides[2] = {row_bytes, head_bytes};
     cuuint32_t box[3] = {box_k, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = enc(map, es == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+    const CUtensorMapDataType dt = es == 4   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                   : es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                             : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const CUresult r = enc(map, dt, 3,
                            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
 // 2-D row-major map {m columns, rows} of an MN-major B operand with a
-// {64, box_rows} box (128 bytes of columns), 128-byte swizzle, zero fill.
+// {128 bytes of columns, box_rows} box, 128-byte swizzle, zero fill; es is the
+// element size (2: bf16, 1: E4M3 codes).
 bool encode_rows_map(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int64_t ld,
-                     uint32_t box_rows) {
+                     uint32_t box_rows, int es = 2) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
-    cuuint32_t box[2] = {64, box_rows};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * es};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), box_rows};
     cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+    const CUresult r = enc(map, es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                           const_cast<void*>(base), dims, strides, box,
                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -97,21 +102,22 @@ bool encode_rows_map(CUtensorMap* map, const void* base, int64_t cols, int64_t r
 rmm_status validate_problem(const rmm_problem* p) {
     if (!p) return RMM_ERR_INVALID_ARG;
     if (p->mode < RMM_LINEAR || p->mode > RMM_PV) return RMM_ERR_INVALID_ARG;
-    if (p->dtype != RMM_BF16 && p->dtype != RMM_F32) return RMM_ERR_INVALID_ARG;
-    const int es = p->dtype == RMM_F32 ? 4 : 2;
-    const int vec = 16 / es;
+    if (p->dtype != RMM_BF16 && p->dtype != RMM_F32 && p->dtype != RMM_FP8_E4M3) return RMM_ERR_INVALID_ARG;
+    const int es = p->dtype == RMM_F32 ? 4 : p->dtype == RMM_FP8_E4M3 ? 1 : 2;
+    const int vec = 16 / es;                               // input elements per 16 bytes
+    const int vec_y = p->dtype == RMM_FP8_E4M3 ? 8 : vec;  // output elements per 16 bytes (E4M3 -> bf16)
     if (p->n < 0 || p->m < 0 || p->d < 1) return RMM_ERR_INVALID_ARG;
     if (p->n > kMaxDim || p->m > kMaxDim || p->d > kMaxDim) return RMM_ERR_UNSUPPORTED;
     if (p->d % vec != 0 || p->m % vec != 0) return RMM_ERR_INVALID_ARG;
     if (p->heads < 1 || p->kv_heads < 1 || p->heads % p->kv_heads != 0) return RMM_ERR_INVALID_ARG;
     if (p->heads > 65535) return RMM_ERR_UNSUPPORTED;
     if (p->lda < p->d || p->lda % vec != 0) return RMM_ERR_INVALID_ARG;
-    if (p->ldy < p->m || p->ldy % vec != 0) return RMM_ERR_INVALID_ARG;
+    if (p->ldy < p->m || p->ldy % vec_y != 0) return RMM_ERR_INVALID_ARG;
     const int64_t b_cols = p->mode == RMM_QK ? p->d : p->m;
     if (p->ldb < b_cols || p->ldb % vec != 0) return RMM_ERR_INVALID_ARG;
     if (p->heads > 1) {
         if (p->stride_a < 0 || p->stride_a % vec != 0) return RMM_ERR_INVALID_ARG;
-        if (p->stride_y % vec != 0 || (p->n > 0 && p->stride_y < p->n * p->ldy)) return RMM_ERR_INVALID_ARG;
+        if (p->stride_y % vec_y != 0 || (p->n > 0 && p->stride_y < p->n * p->ldy)) return RMM_ERR_INVALID_ARG;
     }
     if (p->kv_heads > 1 && (p->stride_b < 0 || p->stride_b % vec != 0)) return RMM_ERR_INVALID_ARG;
     // bf16 row gathers address every B head through one 2-D map: heads must sit
@@ -126,10 +132,16 @@ rmm_status validate_problem(const rmm_problem* p) {
     } else if (p->k < 0 || p->k > p->d) {
         return RMM_ERR_INVALID_ARG;
     }
-    if (p->flags & ~(RMM_FLAG_CAUSAL | RMM_FLAG_USE_GIVEN_INDICES)) return RMM_ERR_INVALID_ARG;
+    if (p->flags & ~(RMM_FLAG_CAUSAL | RMM_FLAG_USE_GIVEN_INDICES | RMM_FLAG_GIVEN_SCORES | RMM_FLAG_EMIT_SCORES))
+        return RMM_ERR_INVALID_ARG;
+    if ((p->flags & RMM_FLAG_GIVEN_SCORES) && (p->flags & RMM_FLAG_USE_GIVEN_INDICES)) return RMM_ERR_INVALID_ARG;
+    if ((p->flags & RMM_FLAG_EMIT_SCORES) && p->mode == RMM_QK) return RMM_ERR_INVALID_ARG;
     if ((p->flags & RMM_FLAG_CAUSAL) && !(p->mode == RMM_QK || (p->mode == RMM_PV && p->n == p->d)))
         return RMM_ERR_INVALID_ARG;
     if (!std::isfinite(p->alpha)) return RMM_ERR_INVALID_ARG;
+    // The low-bit form runs on the CTA-pair product only: linear ops of more than 128 rows.
+    if (p->dtype == RMM_FP8_E4M3 && (p->mode != RMM_LINEAR || p->heads != 1 || (p->n > 0 && p->n <= 128)))
+        return RMM_ERR_UNSUPPORTED;
     return RMM_OK;
 }
 
@@ -145,7 +157,7 @@ T* ws_at(void* ws, size_t off) {
 }
 
 rmm_status run_select(const rmm_plan* plan, const void* A, int32_t* I, float* s2, void* ws,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, const float* given = nullptr) {
     const rmm_problem& p = plan->p;
     rmm::SelectArgs a{};
     a.A = A;
@@ -163,7 +175,11 @@ rmm_status run_select(const rmm_plan* plan, const void* A, int32_t* I, float* s2
         a.mask_words = (p.d + 31) / 32;
     }
     cudaError_t e;
-    if (plan->select_small) {
+    if (given) {
+        // producer-fused scoring: the scores come from the op that produced A
+        a.scores = const_cast<float*>(given);
+        e = rmm::launch_topk(a, stream);
+    } else if (plan->select_small) {
         e = rmm::launch_select_small(a, stream);
     } else if (plan->select16) {
         e = rmm::launch_select16(a, stream);
@@ -183,9 +199,50 @@ rmm_status run_select(const rmm_plan* plan, const void* A, int32_t* I, float* s2
     return e == cudaSuccess ? RMM_OK : RMM_ERR_CUDA;
 }
 
+rmm_status run_product(const rmm_plan* plan, const void* A, const void* B, void* Y, int32_t* I_inout,
+                       float* s2_out, bool* scores_done, void* ws, size_t ws_bytes, void* stream_v,
+                       const float* s2_in);
+
+// Column scores of the output by a score pass over Y (shapes whose product has
+// no epilogue form of the emission).
+rmm_status emit_scores_pass(const rmm_plan* plan, const void* Y, float* s2_out, void* ws, cudaStream_t stream) {
+    const rmm_problem& p = plan->p;
+    rmm::SelectArgs a{};
+    a.A = Y;
+    a.dtype = p.dtype == RMM_FP8_E4M3 ? RMM_BF16 : p.dtype;  // the stored output's type
+    a.n = p.n;
+    a.d = p.m;
+    a.lda = p.ldy;
+    a.stride_a = p.stride_y;
+    a.heads = static_cast<int>(p.heads);
+    a.partials = ws_at<float>(ws, plan->off_emit_ypart);
+    a.counters = ws_at<unsigned>(ws, plan->off_emit_ycnt);
+    a.scores = s2_out;
+    a.nsplit = plan->emit_nsplit;
+    a.rows_per_split = plan->emit_rows_per_split;
+    return rmm::launch_colnorm(a, stream) == cudaSuccess ? RMM_OK : RMM_ERR_CUDA;
+}
+
 rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* Y, int32_t* I_inout,
-                      void* ws, size_t ws_bytes, void* stream_v) {
+                      const float* s2_in, float* s2_out, void* ws, size_t ws_bytes, void* stream_v) {
     if (!plan) return RMM_ERR_INVALID_ARG;
+    const rmm_problem& p = plan->p;
+    if (plan->given_scores && (!s2_in || (reinterpret_cast<uintptr_t>(s2_in) & 3u))) return RMM_ERR_INVALID_ARG;
+    if (plan->emit_scores && (!s2_out || (reinterpret_cast<uintptr_t>(s2_out) & 3u))) return RMM_ERR_INVALID_ARG;
+    bool scores_done = false;
+    const rmm_status st = run_product(plan, A, B, Y, I_inout, plan->emit_scores ? s2_out : nullptr, &scores_done, ws,
+                                      ws_bytes, stream_v, plan->given_scores ? s2_in : nullptr);
+    if (st != RMM_OK || !plan->emit_scores || scores_done || p.m == 0) return st;
+    if (p.n == 0) return cudaMemsetAsync(s2_out, 0, static_cast<size_t>(p.heads) * p.m * sizeof(float),
+                                         static_cast<cudaStream_t>(stream_v)) == cudaSuccess
+                             ? RMM_OK
+                             : RMM_ERR_CUDA;
+    return emit_scores_pass(plan, Y, s2_out, ws, static_cast<cudaStream_t>(stream_v));
+}
+
+rmm_status run_product(const rmm_plan* plan, const void* A, const void* B, void* Y, int32_t* I_inout,
+                       float* s2_out, bool* scores_done, void* ws, size_t ws_bytes, void* stream_v,
+                       const float* s2_in) {
     const rmm_problem& p = plan->p;
     const bool given = (p.flags & RMM_FLAG_USE_GIVEN_INDICES) != 0;
     const bool empty = p.n == 0 || p.m == 0;  // nothing to read or write but I
@@ -210,8 +267,8 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
             // the decode PV product reads the membership words only: without
             // I_inout the one-row select writes no index list
             const bool words_only =
-                plan->decode && p.mode == RMM_PV && plan->select16 && !plan->select_small && !I_inout;
-            st = run_select(plan, A, words_only ? nullptr : I, nullptr, ws, stream);
+                plan->decode && p.mode == RMM_PV && plan->select16 && !plan->select_small && !I_inout && !s2_in;
+            st = run_select(plan, A, words_only ? nullptr : I, nullptr, ws, stream, s2_in);
             if (st != RMM_OK) return st;
         }
     }
@@ -465,7 +522,11 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         pb.ld_dst = p.m;
         pb.stride_dst = d_pad * p.m;
         pb.heads = static_cast<int>(p.heads);
-        if (rmm::launch_mask_rows(pb, d_pad, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        uint8_t* kb_keep = ws_at<uint8_t>(ws, plan->off_kb_keep);
+        if (rmm::launch_mask_rows(pb, d_pad, stream, kb_keep) != cudaSuccess) return RMM_ERR_CUDA;
+        // 64-token blocks without a kept token contribute zeros: the product skips them
+        gp.kb_keep = kb_keep;
+        gp.kb_keep_stride = static_cast<int32_t>(d_pad / 64);
         gl.b_mode = rmm::kBRows;
         gp.k = static_cast<int32_t>(p.d);
         gp.group = 1;
@@ -498,12 +559,13 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         gp.group = 1;
         gp.b_head_rows = static_cast<int32_t>(k);
         gp.b_rows_total = static_cast<int32_t>(k * p.heads);
-        if (!encode_rows_map(&gp.map_b, pb.dst, p.m, k * p.heads, p.m, 64u)) return RMM_ERR_CUDA;
+        if (!encode_rows_map(&gp.map_b, pb.dst, p.m, k * p.heads, p.m, static_cast<uint32_t>(box_k), es))
+            return RMM_ERR_CUDA;
     } else {
         // Plain row tiles only where rows past d are out of the map (one B head)
         // or never reached (d a whole number of K blocks); otherwise rows are
         // fetched four at a time through the index set with tile::gather4.
-        const bool row_tiles = identity && (p.kv_heads == 1 || p.d % 64 == 0);
+        const bool row_tiles = identity && (p.kv_heads == 1 || p.d % box_k == 0);
         gl.b_mode = row_tiles ? rmm::kBRows : rmm::kBGather;
         const int64_t head_rows = p.kv_heads > 1 ? p.stride_b / p.ldb : p.d;
         const int64_t rows_total = (p.kv_heads - 1) * head_rows + p.d;
@@ -511,9 +573,16 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
         gp.b_rows_total = static_cast<int32_t>(rows_total);
         gp.I = identity ? nullptr : I;
         gp.I_stride = k;
-        if (!encode_rows_map(&gp.map_b, B, p.m, rows_total, p.ldb, row_tiles ? 64u : 1u)) return RMM_ERR_CUDA;
+        if (!encode_rows_map(&gp.map_b, B, p.m, rows_total, p.ldb, row_tiles ? static_cast<uint32_t>(box_k) : 1u, es))
+            return RMM_ERR_CUDA;
     }
     gl.pair = pair_ok && gl.b_mode != rmm::kBGather;
+    if (gl.pair && s2_out) {
+        gp.emit_s2 = s2_out;
+        gp.emit_partials = ws_at<float>(ws, plan->off_emit_part);
+        gp.emit_counters = ws_at<unsigned>(ws, plan->off_emit_cnt);
+        *scores_done = true;
+    }
     gp.split_tiles = gl.pair ? plan->split_tiles : 0;
     gp.split_f = gl.pair ? plan->split_f : 1;
     gp.split_partials = ws_at<float>(ws, plan->off_split);
@@ -522,8 +591,8 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
     // rasterisation groups of 8 row tiles (measured best on the workloads' shapes)
     gp.group_m = gp.m_tiles < 8 ? gp.m_tiles : 8;
     // the pair kernel stores 32 x 32 output boxes by TMA (64- or 128-byte rows)
-    if (gl.pair && !encode_kmajor_map(&gp.map_y, es, Y, p.m, p.n, p.heads, p.ldy, p.stride_y, 32, 32,
-                                      es == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
+    if (gl.pair && !encode_kmajor_map(&gp.map_y, plan->es_out, Y, p.m, p.n, p.heads, p.ldy, p.stride_y, 32, 32,
+                                      plan->es_out == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
         return RMM_ERR_CUDA;
     const bool traced = plan->product_start && plan->product_stop;
     if (traced && cudaEventRecord(plan->product_start, stream) != cudaSuccess) return RMM_ERR_CUDA;
@@ -532,13 +601,25 @@ rmm_status run_matmul(const rmm_plan* plan, const void* A, const void* B, void* 
     return RMM_OK;
 }
 
+// Whether the product runs on the CTA-pair kernel (run_product's choice),
+// where emitted column scores come from the epilogue.
+bool product_on_pairs(const rmm_plan* plan) {
+    const rmm_problem& p = plan->p;
+    if (plan->decode || plan->skinny || p.n <= 128) return false;
+    const bool given = (p.flags & RMM_FLAG_USE_GIVEN_INDICES) != 0;
+    const bool identity = !given && plan->k == p.d;
+    const bool gather = p.mode != RMM_QK && p.dtype == RMM_BF16 && identity && p.kv_heads > 1 && p.d % 64 != 0;
+    return !gather;
+}
+
 int32_t launches_per_call(const rmm_plan* plan) {
     const rmm_problem& p = plan->p;
     const bool given = (p.flags & RMM_FLAG_USE_GIVEN_INDICES) != 0;
     const bool identity = !given && plan->k == p.d;
     int32_t n = 0;
     if (!given && !identity && !plan->decode_select)
-        n += (plan->fused_select || plan->select16 || plan->select_small) ? 1 : 2;
+        n += (plan->given_scores || plan->fused_select || plan->select16 || plan->select_small) ? 1 : 2;
+    if (plan->emit_scores && p.m > 0 && p.n > 0 && !product_on_pairs(plan)) n += 1;  // score pass over Y
     if (p.n == 0 || p.m == 0) return n;
     if (plan->decode) return n + 1;
     if (plan->skinny) return n + (identity ? 0 : 1) + 1 + (plan->sk_splits > 1 ? 1 : 0);
@@ -579,14 +660,17 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     if (!plan) return RMM_ERR_UNSUPPORTED;
     std::memset(plan, 0, sizeof(*plan));
     plan->p = *p;
-    plan->es = p->dtype == RMM_F32 ? 4 : 2;
+    plan->es = p->dtype == RMM_F32 ? 4 : p->dtype == RMM_FP8_E4M3 ? 1 : 2;
+    plan->es_out = p->dtype == RMM_FP8_E4M3 ? 2 : plan->es;
     plan->k = p->k > 0 ? p->k : retained_count(p->rho, p->d);
-    plan->ldp = (plan->k + 7) / 8 * 8;
+    // packed rows: whole groups of 8 elements (the packs write 8 at a time) and whole 16-byte granules
+    const int64_t pack_group = plan->es == 1 ? 16 : 8;
+    plan->ldp = (plan->k + pack_group - 1) / pack_group * pack_group;
     plan->group = static_cast<int>(p->heads / p->kv_heads);
     const bool given = (p->flags & RMM_FLAG_USE_GIVEN_INDICES) != 0;
     plan->need_select = !given && plan->k < p->d;
     plan->bn = p->m <= 128 ? 128 : 256;
-    plan->pack_b = p->mode != RMM_QK && p->dtype == RMM_BF16 && (plan->k < p->d || given);
+    plan->pack_b = p->mode != RMM_QK && (p->dtype == RMM_BF16 || p->dtype == RMM_FP8_E4M3) && (plan->k < p->d || given);
     // PV over short value heads is bound by reading P: instead of copying P's
     // retained columns, zero V's unkept rows (per query head) and read P as is.
     plan->pv_mask = p->mode == RMM_PV && p->dtype == RMM_BF16 && !given && plan->k < p->d && p->m <= 256;
@@ -612,7 +696,9 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
         plan->pack_b = false;
         plan->pv_mask = false;
     }
-    plan->decode_select = plan->decode && p->mode == RMM_QK && plan->need_select;
+    plan->given_scores = (p->flags & RMM_FLAG_GIVEN_SCORES) != 0;
+    plan->emit_scores = (p->flags & RMM_FLAG_EMIT_SCORES) != 0;
+    plan->decode_select = plan->decode && p->mode == RMM_QK && plan->need_select && !plan->given_scores;
     plan->pack_ab = plan->pack_b && rmm::pack_ab_one_launch(p->dtype, plan->ldp);
 
     int dev = 0, sms = 0;
@@ -637,7 +723,8 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
         return RMM_ERR_UNSUPPORTED;
     }
     const size_t head_bytes = static_cast<size_t>(p->n) * p->d * plan->es;
-    plan->fused_select = head_bytes <= kFusedSelectBytes && rmm::normselect_smem_bytes(p->d, p->dtype) <= 180 * 1024;
+    plan->fused_select = p->dtype != RMM_FP8_E4M3 && head_bytes <= kFusedSelectBytes &&
+                         rmm::normselect_smem_bytes(p->d, p->dtype) <= 180 * 1024;
     // one bf16 row per head: a counting select over the magnitude bits
     plan->select16 = p->n == 1 && p->dtype == RMM_BF16 && p->d % 8 == 0 && p->d <= 65535;
     plan->select_small = rmm::select_small_fits(p->n, p->d);
@@ -672,7 +759,7 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     // tile of work, no causal mask): its counters live in the header.
     plan->split_tiles = 0;
     plan->split_f = 1;
-    if (!plan->skinny && p->n > 128 && p->m > 0 && !(p->flags & RMM_FLAG_CAUSAL)) {
+    if (!plan->skinny && p->n > 128 && p->m > 0 && !(p->flags & RMM_FLAG_CAUSAL) && !plan->emit_scores) {
         const int64_t k_eff = ((p->mode == RMM_QK && p->d <= 1024) || plan->pv_mask) ? p->d : plan->k;
         const int64_t bk = 128 / plan->es;
         const int64_t tiles = p->heads * ((p->n + 255) / 256) * ((p->m + plan->bn - 1) / plan->bn);
@@ -682,6 +769,17 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     off += align256(static_cast<size_t>(plan->split_tiles) * 2 * rmm::kSplitCounterWarps * sizeof(unsigned));
     plan->off_dec_cnt = off;
     if (dec_pv) off += align256(static_cast<size_t>(p->kv_heads) * sizeof(unsigned));
+    // Producer-fused scoring of the output: counters of the epilogue form
+    // (per 32-column chunk) and of the score pass over Y (per column block).
+    const int vec_y = 16 / plan->es_out;
+    const int64_t y_colblocks = (p->m + 32 * vec_y - 1) / (32 * vec_y);
+    plan->off_emit_cnt = off;
+    plan->off_emit_ycnt = off;
+    if (plan->emit_scores) {
+        off += align256(static_cast<size_t>(p->heads) * ((p->m + 255) / 256) * 8 * sizeof(unsigned));
+        plan->off_emit_ycnt = off;
+        off += align256(static_cast<size_t>(p->heads) * y_colblocks * sizeof(unsigned));
+    }
     plan->header_bytes = off;
     plan->off_partials = off;
     plan->off_scores = off;
@@ -709,12 +807,34 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
         off += align256(static_cast<size_t>(p->heads) * plan->k * p->m * plan->es);
     plan->off_split = off;
     off += align256(static_cast<size_t>(plan->split_tiles) * plan->split_f * 256 * plan->bn * sizeof(float));
+    plan->off_kb_keep = off;
+    if (plan->pv_mask) off += align256(static_cast<size_t>(p->heads) * ((p->d + 63) / 64));
     plan->off_dec_mask = off;
     plan->off_dec_part = off;
     if (dec_pv) {
         off += align256(static_cast<size_t>(p->heads) * ((p->d + 31) / 32) * sizeof(uint32_t));
         plan->off_dec_part = off;
         off += align256(static_cast<size_t>(p->kv_heads) * plan->dec_parts * 8 * p->m * sizeof(float));
+    }
+    plan->off_emit_part = off;
+    plan->off_emit_ypart = off;
+    if (plan->emit_scores) {
+        // epilogue form: row groups of 32 rows x m per head
+        off += align256(static_cast<size_t>(p->heads) * 8 * ((p->n + 255) / 256) * p->m * sizeof(float));
+        // score-pass form: row splits as for a score pass over A
+        int64_t ens = (2LL * sms + y_colblocks * p->heads - 1) / (y_colblocks * p->heads);
+        const int64_t emax = (p->n + 63) / 64;
+        if (ens > emax) ens = emax;
+        if (ens > 16) ens = 16;
+        if (ens < 1) ens = 1;
+        int64_t erps = (p->n + ens - 1) / ens;
+        erps = (erps + 7) / 8 * 8;
+        if (erps < 8) erps = 8;
+        ens = p->n > 0 ? (p->n + erps - 1) / erps : 1;
+        plan->emit_nsplit = static_cast<int>(ens);
+        plan->emit_rows_per_split = erps;
+        plan->off_emit_ypart = off;
+        off += align256(static_cast<size_t>(p->heads) * ens * p->m * sizeof(float));
     }
     plan->ws_bytes = off;
     if (workspace_bytes) *workspace_bytes = plan->ws_bytes;
@@ -745,13 +865,20 @@ rmm_status rmm_select(const rmm_plan* plan, const void* A, int32_t* I, float* s2
 rmm_status rmm_matmul(const rmm_plan* plan, const void* A, const void* B, void* Y, int32_t* I_inout, void* ws,
                       size_t ws_bytes, void* stream) {
     if (!plan) return RMM_ERR_INVALID_ARG;
-    if (plan->p.heads != 1) return RMM_ERR_INVALID_ARG;
-    return run_matmul(plan, A, B, Y, I_inout, ws, ws_bytes, stream);
+    if (plan->p.heads != 1 || plan->given_scores || plan->emit_scores) return RMM_ERR_INVALID_ARG;
+    return run_matmul(plan, A, B, Y, I_inout, nullptr, nullptr, ws, ws_bytes, stream);
 }
 
 rmm_status rmm_matmul_batched(const rmm_plan* plan, const void* A, const void* B, void* Y, int32_t* I_inout,
                               void* ws, size_t ws_bytes, void* stream) {
-    return run_matmul(plan, A, B, Y, I_inout, ws, ws_bytes, stream);
+    if (!plan) return RMM_ERR_INVALID_ARG;
+    if (plan->given_scores || plan->emit_scores) return RMM_ERR_INVALID_ARG;
+    return run_matmul(plan, A, B, Y, I_inout, nullptr, nullptr, ws, ws_bytes, stream);
+}
+
+rmm_status rmm_matmul_ex(const rmm_plan* plan, const void* A, const void* B, void* Y, int32_t* I_inout,
+                         const float* s2_in, float* s2_out, void* ws, size_t ws_bytes, void* stream) {
+    return run_matmul(plan, A, B, Y, I_inout, s2_in, s2_out, ws, ws_bytes, stream);
 }
 
 rmm_status rmm_workspace_init(const rmm_plan* plan, void* ws, size_t ws_bytes, void* stream) {

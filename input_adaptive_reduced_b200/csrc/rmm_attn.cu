@@ -1,0 +1,670 @@
+// rmm_attn.cu -- fused RMM attention: the three steps of "Reduced Matrix
+// Multiplication: Input-Adaptive Matrix-Product Reduction for LLM Inference"
+// §3.3 "Attention" without writing the score matrix S or the weights P:
+//   features  I_h = TopK of Q_h's column norms;  S = alpha Q_h[:, I_h] K_g[:, I_h]^T + M
+//   weights   P = softmax(S) over each query row
+//   tokens    T_h = TopK of P's column norms;    O_h = P[:, T_h] V_g[T_h, :]
+// Token selection needs the column norms of the final P before any output is
+// formed, and every row's normalisation before any column norm, so the score
+// blocks are recomputed in three passes of one kernel (the paper's own
+// kernels were not fully fused; App. B.7):
+//   kRowStats  per query row the maximum m_i and the exponential sum l_i of
+//              its scaled scores (online over the key blocks);
+//   kColScores per key the sum over 32 rows of P[i][t]^2 with
+//              P = exp(S - m_i) / l_i, written per 32-row slice; a second
+//              kernel adds the slices in order, and TopK picks T_h;
+//   kOutput    O = sum over the key blocks holding a kept token of
+//              (P masked to T_h, rounded to bf16) V, on the tensor cores.
+// Masked features are zeroed in a copy of Q (the contraction then runs over
+// all d_h with exact zeros), as the library's QK op does.
+//
+// One CTA computes 128 query rows of one head: warp 0 loads by TMA (Q once,
+// then K and V blocks of 128 keys, two stages), warp 1 issues tcgen05.mma
+// (S = Q K^T into one of two TMEM buffers; O += P V into a third), and 16
+// row warps, four per TMEM lane quadrant, each own 32 rows x 32 keys of every
+// block (one row per thread): they read their S chunk from TMEM and write P
+// into a swizzled shared tile for the PV product.  Every wait is bounded.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "rmm.h"
+#include "rmm_device.cuh"
+#include "rmm_internal.h"
+
+namespace rmm {
+namespace {
+
+constexpr int kRowStats = 0;
+constexpr int kColScores = 1;
+constexpr int kOutput = 2;
+
+constexpr int BQ = 128;    // query rows per CTA
+constexpr int BKEY = 128;  // keys per block
+constexpr int DH = 128;    // head dimension of Q and K
+constexpr int DV = 128;    // value dimension
+constexpr int kRowWarps = 16;                 // 4 per TMEM lane quadrant, 32 keys each
+constexpr int kThreads = 32 * (2 + kRowWarps);
+constexpr int ATOM = 128 * 128;  // one 64-column swizzle atom of 128 rows (bytes)
+constexpr int TILE = 2 * ATOM;   // a 128 x 128 bf16 operand tile
+
+struct __align__(64) AttnParams {
+    CUtensorMap map_q;  // masked Q: {d_h, n, heads}, box {64, 128, 1}
+    CUtensorMap map_k;  // K: {d_h, n, kv_heads}, box {64, 128, 1}
+    CUtensorMap map_v;  // V: {d_v, n, kv_heads}, box {64, 128, 1}
+    __nv_bfloat16* O;   // [heads][n][ldo]
+    int64_t ldo, stride_o;
+    float* row_m;       // [heads][n]: maximum of the row's scaled scores (base-2 units)
+    float* row_l;       // [heads][n]: sum over the row of 2^(x - m)
+    float* col_part;    // [heads][4 q_blocks][n]: per 32-row slice, sum of P^2 per key
+    const uint32_t* tok_mask;  // [heads][mask_words]: bit t set iff token t is kept
+    int64_t mask_words;
+    int n, heads, group, q_blocks, k_blocks, causal;
+    float scale_log2;   // alpha * log2(e): the scores are taken in base 2
+    int* err;
+};
+
+template <int MODE>
+struct AttnCfg {
+    static constexpr bool OUT = MODE == kOutput;
+    static constexpr int KV_BYTES = OUT ? 2 * TILE : TILE;  // K (and V) of one key block
+    static constexpr int STAT_BYTES = MODE == kRowStats ? 2 * 4 * BQ * 4 : 0;  // per-quarter (m, l) of each row
+    static constexpr size_t SMEM = 1024 + TILE + 2 * (size_t)KV_BYTES + (OUT ? 2 * TILE : 0) + STAT_BYTES + 256;
+    static constexpr uint32_t TMEM_COLS = OUT ? 512 : 256;  // two S buffers (+ O)
+};
+
+// Query block of CTA b: the longest causal key ranges first.
+__device__ __forceinline__ void attn_block(const AttnParams& p, int& h, int& qb) {
+    const int b = blockIdx.x;
+    const int r = b / p.heads;
+    h = b - r * p.heads;
+    qb = p.causal ? p.q_blocks - 1 - r : r;
+}
+
+// Whether key block kb takes part for query block qb: inside the causal
+// range, and in the output pass only if one of its tokens is kept.
+template <int MODE>
+__device__ __forceinline__ bool key_block_used(const AttnParams& p, int h, int qb, int kb) {
+    if (p.causal && kb > qb) return false;
+    if constexpr (MODE == kOutput) {
+        const uint32_t* w = p.tok_mask + (int64_t)h * p.mask_words;
+        uint32_t any = 0;
+#pragma unroll
+        for (int i = 0; i < BKEY / 32; ++i) {
+            const int64_t wi = (int64_t)kb * (BKEY / 32) + i;
+            if (wi < p.mask_words) any |= __ldg(w + wi);
+        }
+        return any != 0;
+    }
+    return true;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_constant__ AttnParams p) {
+    using C = AttnCfg<MODE>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = smem;
+    uint8_t* sKV = sQ + TILE;                         // 2 stages: K tile (then V tile)
+    uint8_t* sP = sKV + 2 * C::KV_BYTES;              // 2 P tiles (output pass)
+    float* stat = reinterpret_cast<float*>(sP + (C::OUT ? 2 * TILE : 0));  // [2][4][BQ] (row statistics)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stat) + C::STAT_BYTES);
+    uint64_t* q_full = bars;
+    uint64_t* kv_full = bars + 1;
+    uint64_t* kv_empty = bars + 3;
+    uint64_t* s_full = bars + 5;
+    uint64_t* s_empty = bars + 7;
+    uint64_t* p_full = bars + 9;
+    uint64_t* p_empty = bars + 11;
+    uint64_t* o_full = bars + 13;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_empty[s], kRowWarps);  // one arrival per row warp
+            mbar_init(&p_full[s], kRowWarps);
+            mbar_init(&p_empty[s], 1);
+        }
+        mbar_init(o_full, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+        tma_prefetch_map(&p.map_q);
+        tma_prefetch_map(&p.map_k);
+        if (C::OUT) tma_prefetch_map(&p.map_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    pdl_wait();
+    pdl_trigger();
+
+    int h, qb;
+    attn_block(p, h, qb);
+    const int g = h / p.group;
+    const int q0 = qb * BQ;
+    const int kb_end = p.causal ? min(qb + 1, p.k_blocks) : p.k_blocks;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- loads
+        if (lane == 0) {
+            mbar_arrive_expect_tx(q_full, TILE);
+            tma_load_3d(sQ, &p.map_q, q_full, 0, q0, h);
+            tma_load_3d(sQ + ATOM, &p.map_q, q_full, 64, q0, h);
+            uint32_t it = 0;
+            for (int kb = 0; kb < kb_end; ++kb) {
+                if (!key_block_used<MODE>(p, h, qb, kb)) continue;
+                const int s = it & 1;
+                const uint32_t ph = (it >> 1) & 1u;
+                ++it;
+                if (!mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, p.err, kErrTimeoutProducer)) break;
+                uint8_t* dst = sKV + s * C::KV_BYTES;
+                mbar_arrive_expect_tx(&kv_full[s], C::KV_BYTES);
+                tma_load_3d(dst, &p.map_k, &kv_full[s], 0, kb * BKEY, g);
+                tma_load_3d(dst + ATOM, &p.map_k, &kv_full[s], 64, kb * BKEY, g);
+                if constexpr (C::OUT) {
+                    tma_load_3d(dst + TILE, &p.map_v, &kv_full[s], 0, kb * BKEY, g);
+                    tma_load_3d(dst + TILE + ATOM, &p.map_v, &kv_full[s], 64, kb * BKEY, g);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = umma_idesc(kKindF16, false, BKEY, 128);  // S = Q K^T
+            constexpr uint32_t idesc_o = umma_idesc(kKindF16, true, DV, 128);     // O += P V (V MN-major)
+            const uint32_t q_addr = smem_u32(sQ);
+            // O += P_j V_j for the j-th used block (P tile j % 2, K/V stage j % 2)
+            auto pv = [&](uint32_t j) -> bool {
+                const int pb = j & 1;
+                if (!mbar_wait(&p_full[pb], (j >> 1) & 1u, abort_flag, p.err, kErrTimeoutMma)) return false;
+                tc_fence_after();
+                const uint32_t p_addr = smem_u32(sP + pb * TILE);
+                const uint32_t v_addr = smem_u32(sKV + pb * C::KV_BYTES + TILE);
+#pragma unroll
+                for (int kk = 0; kk < BKEY / 16; ++kk) {
+                    const uint64_t adesc = sw128_desc(p_addr + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bdesc = sw128_desc(v_addr + kk * 16 * 128, ATOM, 1024);
+                    umma<kKindF16>(tmem_base + 256, adesc, bdesc, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&p_empty[pb]);
+                umma_commit(&kv_empty[pb]);
+                return true;
+            };
+            bool ok = mbar_wait(q_full, 0u, abort_flag, p.err, kErrTimeoutMma);
+            uint32_t it = 0;
+            for (int kb = 0; kb < kb_end && ok; ++kb) {
+                if (!key_block_used<MODE>(p, h, qb, kb)) continue;
+                const int s = it & 1;
+                const uint32_t ph = (it >> 1) & 1u;
+                if (!mbar_wait(&kv_full[s], ph, abort_flag, p.err, kErrTimeoutMma) ||
+                    !mbar_wait(&s_empty[s], ph ^ 1u, abort_flag, p.err, kErrTimeoutMma)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t k_addr = smem_u32(sKV + s * C::KV_BYTES);
+                const uint32_t d_tmem = tmem_base + s * BKEY;
+#pragma unroll
+                for (int kk = 0; kk < DH / 16; ++kk) {
+                    const uint64_t adesc = sw128_desc(q_addr + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bdesc = sw128_desc(k_addr + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
+                    umma<kKindF16>(d_tmem, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[s]);
+                if constexpr (C::OUT) {
+                    if (it > 0 && !pv(it - 1)) ok = false;
+                } else {
+                    umma_commit(&kv_empty[s]);  // K consumed by this block's scores
+                }
+                ++it;
+            }
+            if constexpr (C::OUT) {
+                if (ok && it > 0) ok = pv(it - 1);
+                umma_commit(o_full);
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- rows
+        const int quad = warp & 3;         // TMEM lane quadrant: rows quad*32 .. +32
+        const int cq = (warp - 2) >> 2;    // key quarter: keys cq*32 .. +32 of every block
+        const int r_loc = quad * 32 + lane;
+        const int row = q0 + r_loc;
+        const bool row_ok = row < p.n;
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+        // rows past n: m = 0 and 1/l = 0, so that every weight is 2^-inf * 0 = 0
+        float m = MODE == kRowStats ? -INFINITY : 0.f, l = 0.f, inv_l = 0.f;
+        if (MODE != kRowStats && row_ok) {
+            m = p.row_m[(int64_t)h * p.n + row];
+            l = p.row_l[(int64_t)h * p.n + row];
+            inv_l = l > 0.f ? 1.0f / l : 0.f;
+        }
+        const uint32_t* mask_h = p.tok_mask ? p.tok_mask + (int64_t)h * p.mask_words : nullptr;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int kb = 0; kb < kb_end && ok; ++kb) {
+            if (!key_block_used<MODE>(p, h, qb, kb)) continue;
+            const int sb = it & 1;
+            const uint32_t ph = (it >> 1) & 1u;
+            ++it;
+            if (!mbar_wait(&s_full[sb], ph, abort_flag, p.err, kErrTimeoutEpilogue)) {
+                ok = false;
+                break;
+            }
+            if constexpr (C::OUT) {
+                if (!mbar_wait(&p_empty[sb], ph ^ 1u, abort_flag, p.err, kErrTimeoutEpilogue)) {
+                    ok = false;
+                    break;
+                }
+            }
+            tc_fence_after();
+            const int k0 = kb * BKEY + cq * 32;  // this warp's first key
+            // which of the 32 keys of this row count: all, none, or some (the
+            // diagonal block and the last block)
+            const bool all_in = row_ok && k0 + 31 < p.n && (!p.causal || k0 + 31 <= row);
+            const bool none_in = !row_ok || k0 >= p.n || (p.causal && k0 > row);
+            uint32_t raw[32];
+            tmem_ld_32x32b_x32(tmem_base + lane_base + sb * BKEY + cq * 32, raw);
+            tmem_ld_wait();
+            float x[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const bool valid = all_in || (!none_in && k0 + i < p.n && (!p.causal || k0 + i <= row));
+                x[i] = valid ? __uint_as_float(raw[i]) * p.scale_log2 : -INFINITY;
+            }
+            if constexpr (MODE == kRowStats) {
+                if (!none_in) {
+                    float mc = -INFINITY;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) mc = fmaxf(mc, x[i]);
+                    const float mn = fmaxf(m, mc);
+                    float acc = l * exp2f(m - mn);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc += exp2f(x[i] - mn);  // 2^-inf = 0
+                    l = acc;
+                    m = mn;
+                }
+            } else if constexpr (MODE == kColScores) {
+                float z = 0.f;
+                if (__any_sync(0xffffffffu, !none_in)) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float pr = exp2f(x[i] - m) * inv_l;  // 0 where masked
+                        x[i] = pr * pr;
+                    }
+                    z = warp_column_sums(x, lane);  // this warp's 32 rows, summed per key
+                }
+                const int key = k0 + lane;
+                if (key < p.n) p.col_part[((int64_t)h * p.q_blocks * 4 + qb * 4 + quad) * p.n + key] = z;
+            } else {
+                // P masked to the kept tokens, rounded to bf16, into the swizzled P tile
+                const int64_t wi = (int64_t)k0 >> 5;
+                const uint32_t keep_bits = (!none_in && wi < p.mask_words) ? __ldg(mask_h + wi) : 0u;
+                uint8_t* prow = sP + sb * TILE + (cq >> 1) * ATOM + r_loc * 128;
+#pragma unroll
+                for (int gi = 0; gi < 4; ++gi) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i0 = gi * 8 + 2 * e;
+                        const float p0 = ((keep_bits >> i0) & 1u) ? exp2f(x[i0] - m) * inv_l : 0.f;
+                        const float p1 = ((keep_bits >> (i0 + 1)) & 1u) ? exp2f(x[i0 + 1] - m) * inv_l : 0.f;
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+                        w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                    }
+                    const int gran = (cq & 1) * 4 + gi;
+                    *reinterpret_cast<uint4*>(prow + ((gran ^ (r_loc & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            // this S buffer may be overwritten
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[sb]);
+            if constexpr (C::OUT) {
+                fence_proxy_async_smem();  // the P tile's generic stores before the MMA reads it
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[sb]);
+            }
+        }
+        if constexpr (MODE == kRowStats) {
+            // the four key quarters' (m, l) of each row, combined in quarter order;
+            // every row warp reaches this barrier once, whether or not a wait gave up
+            stat[cq * BQ + r_loc] = m;
+            stat[4 * BQ + cq * BQ + r_loc] = l;
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * kRowWarps) : "memory");
+            if (cq == 0 && row_ok) {
+                float mr = stat[r_loc];
+#pragma unroll
+                for (int j = 1; j < 4; ++j) mr = fmaxf(mr, stat[j * BQ + r_loc]);
+                float lr = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float mj = stat[j * BQ + r_loc];
+                    if (mj > -INFINITY) lr += stat[4 * BQ + j * BQ + r_loc] * exp2f(mj - mr);
+                }
+                p.row_m[(int64_t)h * p.n + row] = mr;
+                p.row_l[(int64_t)h * p.n + row] = lr;
+            }
+        }
+        if constexpr (C::OUT) {
+            __nv_bfloat16* orow = p.O + (int64_t)h * p.stride_o + (int64_t)row * p.ldo + cq * 32;
+            const bool have = ok && it > 0;
+            if (have && !mbar_wait(o_full, 0u, abort_flag, p.err, kErrTimeoutEpilogue)) ok = false;
+            tc_fence_after();
+            uint32_t raw[32];
+            if (have && ok) {
+                tmem_ld_32x32b_x32(tmem_base + lane_base + 256 + cq * 32, raw);
+                tmem_ld_wait();
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) raw[i] = 0u;  // no kept token in this row's range
+            }
+            if (row_ok) {
+#pragma unroll
+                for (int gi = 0; gi < 4; ++gi) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(raw[gi * 8 + 2 * e]),
+                                                                        __uint_as_float(raw[gi * 8 + 2 * e + 1]));
+                        w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                    }
+                    *reinterpret_cast<uint4*>(orow + gi * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// a2[h][t] = sum over the 32-row slices (in row order) of their P^2 sums;
+// with the causal mask only the slices of the blocks at or below key t's
+// block hold any.
+__global__ void __launch_bounds__(256) attn_colscore_reduce_kernel(const float* __restrict__ part,
+                                                                   float* __restrict__ a2, int n, int q_blocks,
+                                                                   int causal) {
+    pdl_wait();
+    pdl_trigger();
+    const int h = blockIdx.y;
+    const int t = blockIdx.x * 256 + threadIdx.x;
+    if (t >= n) return;
+    const int s0 = causal ? (t / BKEY) * 4 : 0;
+    const float* ph = part + (int64_t)h * q_blocks * 4 * n + t;
+    float z = 0.f;
+    for (int sl = s0; sl < 4 * q_blocks; ++sl) z += ph[(int64_t)sl * n];
+    a2[(int64_t)h * n + t] = z;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 3-D bf16 map {cols, rows, heads} with a {64, 128, 1} box and 128-byte swizzle.
+bool encode_map(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int64_t heads, int64_t ld,
+                int64_t stride_h) {
+    auto enc = encoder();
+    if (!enc) return false;
+    uint64_t head_bytes = heads > 1 ? static_cast<uint64_t>(stride_h) * 2 : static_cast<uint64_t>(ld) * 2 * rows;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(heads)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * 2, head_bytes};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_pass(const AttnParams& p, cudaStream_t s) {
+    using C = AttnCfg<MODE>;
+    cudaError_t e = cudaFuncSetAttribute(attn_pass_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::SMEM);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(attn_pass_kernel<MODE>, dim3((unsigned)(p.q_blocks * p.heads)), dim3(kThreads), C::SMEM, s, p);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int64_t retained(double rho, int64_t d) {
+    const double x = rho * static_cast<double>(d);
+    const double r = std::nearbyint(x);
+    int64_t k = (std::fabs(x - r) <= 1e-9 * static_cast<double>(d)) ? static_cast<int64_t>(r)
+                                                                      : static_cast<int64_t>(std::ceil(x));
+    return k < 1 ? 1 : (k > d ? d : k);
+}
+
+// Workspace layout of one problem (offsets in bytes, 256-aligned).
+struct AttnLayout {
+    int64_t kd, kt, q_blocks, mask_words;
+    int nsplit;
+    int64_t rows_per_split;
+    bool fused_select;
+    size_t err, cnt, part, scores, I, T, qm, rm, rl, cpart, a2, mask, total;
+};
+
+AttnLayout attn_layout(const rmm_attn_problem* p, int sms) {
+    AttnLayout L{};
+    L.kd = retained(p->rho_d, p->d_h);
+    L.kt = retained(p->rho_t, p->n);
+    L.q_blocks = (p->n + BQ - 1) / BQ;
+    L.mask_words = (p->n + 31) / 32;
+    L.fused_select = p->n * p->d_h * 2 <= (int64_t(128) << 10);
+    int64_t ns = (2LL * sms + p->heads - 1) / p->heads;
+    const int64_t mx = (p->n + 63) / 64;
+    if (ns > mx) ns = mx;
+    if (ns > 16) ns = 16;
+    if (ns < 1) ns = 1;
+    int64_t rps = (p->n + ns - 1) / ns;
+    rps = (rps + 7) / 8 * 8;
+    if (rps < 8) rps = 8;
+    L.nsplit = static_cast<int>((p->n + rps - 1) / rps);
+    L.rows_per_split = rps;
+    size_t off = 0;
+    L.err = off;  // error word: a kernel that gave up on a wait records its code
+    off += 256;
+    L.cnt = off;  // score-pass counters of the feature selection (zero between calls)
+    off += align256(static_cast<size_t>(p->heads) * sizeof(unsigned));
+    L.part = off;
+    off += align256(static_cast<size_t>(p->heads) * L.nsplit * p->d_h * sizeof(float));
+    L.scores = off;
+    off += align256(static_cast<size_t>(p->heads) * p->d_h * sizeof(float));
+    L.I = off;
+    off += align256(static_cast<size_t>(p->heads) * L.kd * sizeof(int32_t));
+    L.T = off;
+    off += align256(static_cast<size_t>(p->heads) * L.kt * sizeof(int32_t));
+    L.qm = off;
+    off += align256(static_cast<size_t>(p->heads) * p->n * p->d_h * 2);
+    L.rm = off;
+    off += align256(static_cast<size_t>(p->heads) * p->n * sizeof(float));
+    L.rl = off;
+    off += align256(static_cast<size_t>(p->heads) * p->n * sizeof(float));
+    L.cpart = off;
+    off += align256(static_cast<size_t>(p->heads) * 4 * L.q_blocks * p->n * sizeof(float));
+    L.a2 = off;
+    off += align256(static_cast<size_t>(p->heads) * p->n * sizeof(float));
+    L.mask = off;
+    off += align256(static_cast<size_t>(p->heads) * L.mask_words * sizeof(uint32_t));
+    L.total = off;
+    return L;
+}
+
+rmm_status validate_attn(const rmm_attn_problem* p) {
+    if (!p) return RMM_ERR_INVALID_ARG;
+    if (p->heads < 1 || p->kv_heads < 1 || p->heads % p->kv_heads != 0 || p->n < 0) return RMM_ERR_INVALID_ARG;
+    if (p->d_h != DH || p->d_v != DV) return RMM_ERR_UNSUPPORTED;
+    if (p->heads > 65535 || p->n > kMaxSelectD) return RMM_ERR_UNSUPPORTED;
+    if (p->n % 8 != 0) return RMM_ERR_INVALID_ARG;  // token scores are selected in 16-byte groups
+    if (p->ldq < p->d_h || p->ldk < p->d_h || p->ldv < p->d_v || p->ldo < p->d_v) return RMM_ERR_INVALID_ARG;
+    if (p->ldq % 8 || p->ldk % 8 || p->ldv % 8 || p->ldo % 8) return RMM_ERR_INVALID_ARG;
+    if (p->heads > 1 && (p->stride_q % 8 || p->stride_o % 8 || p->stride_q < p->n * p->ldq ||
+                         p->stride_o < p->n * p->ldo))
+        return RMM_ERR_INVALID_ARG;
+    if (p->kv_heads > 1 && (p->stride_k % 8 || p->stride_v % 8 || p->stride_k < p->n * p->ldk ||
+                            p->stride_v < p->n * p->ldv))
+        return RMM_ERR_INVALID_ARG;
+    if (!(p->rho_d > 0.0) || p->rho_d > 1.0 || !(p->rho_t > 0.0) || p->rho_t > 1.0) return RMM_ERR_INVALID_ARG;
+    if (!std::isfinite(p->alpha)) return RMM_ERR_INVALID_ARG;
+    if (p->flags & ~RMM_FLAG_CAUSAL) return RMM_ERR_INVALID_ARG;
+    return RMM_OK;
+}
+
+int device_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return sms;
+}
+
+}  // namespace
+}  // namespace rmm
+
+extern "C" {
+
+size_t rmm_attention_workspace_size(const rmm_attn_problem* p) {
+    if (rmm::validate_attn(p) != RMM_OK) return 0;
+    const int sms = rmm::device_sms();
+    return rmm::attn_layout(p, sms > 0 ? sms : 148).total;
+}
+
+rmm_status rmm_attention(const rmm_attn_problem* p, const void* Q, const void* K, const void* V, void* O,
+                         int32_t* I_out, int32_t* T_out, void* ws, size_t ws_bytes, void* stream) {
+    using namespace rmm;
+    rmm_status st = validate_attn(p);
+    if (st != RMM_OK) return st;
+    if (p->n == 0) return RMM_OK;
+    if (!Q || !K || !V || !O) return RMM_ERR_INVALID_ARG;
+    for (const void* ptr : {Q, K, V, static_cast<const void*>(O)})
+        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return RMM_ERR_INVALID_ARG;
+    if ((I_out && (reinterpret_cast<uintptr_t>(I_out) & 3u)) || (T_out && (reinterpret_cast<uintptr_t>(T_out) & 3u)))
+        return RMM_ERR_INVALID_ARG;
+    const int sms = device_sms();
+    if (sms <= 0) return RMM_ERR_CUDA;
+    const AttnLayout L = attn_layout(p, sms);
+    if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return RMM_ERR_WORKSPACE;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int H = static_cast<int>(p->heads);
+    const int64_t n = p->n;
+    int32_t* I = I_out ? I_out : reinterpret_cast<int32_t*>(w + L.I);
+    int32_t* T = T_out ? T_out : reinterpret_cast<int32_t*>(w + L.T);
+
+    // 1. features: I_h = TopK of Q_h's column norms
+    SelectArgs sa{};
+    sa.A = Q;
+    sa.dtype = RMM_BF16;
+    sa.n = n;
+    sa.d = p->d_h;
+    sa.lda = p->ldq;
+    sa.stride_a = p->stride_q;
+    sa.heads = H;
+    sa.k = L.kd;
+    sa.I = I;
+    cudaError_t e;
+    if (L.kd == p->d_h) {
+        e = launch_identity(I, L.kd, H, s);
+    } else if (L.fused_select) {
+        e = launch_normselect(sa, s);
+    } else {
+        sa.partials = reinterpret_cast<float*>(w + L.part);
+        sa.counters = reinterpret_cast<unsigned*>(w + L.cnt);
+        sa.scores = reinterpret_cast<float*>(w + L.scores);
+        sa.nsplit = L.nsplit;
+        sa.rows_per_split = L.rows_per_split;
+        e = launch_colnorm(sa, s);
+        if (e == cudaSuccess) e = launch_topk(sa, s);
+    }
+    if (e != cudaSuccess) return RMM_ERR_CUDA;
+    // 2. Q with the unkept features zeroed
+    __nv_bfloat16* Qm = reinterpret_cast<__nv_bfloat16*>(w + L.qm);
+    PackArgs pm{};
+    pm.src = Q;
+    pm.dtype = RMM_BF16;
+    pm.rows = n;
+    pm.d = p->d_h;
+    pm.ld_src = p->ldq;
+    pm.stride_src = p->stride_q;
+    pm.group = 1;
+    pm.I = I;
+    pm.I_stride = L.kd;
+    pm.k = L.kd;
+    pm.dst = Qm;
+    pm.ld_dst = p->d_h;
+    pm.stride_dst = n * p->d_h;
+    pm.heads = H;
+    if (launch_mask_columns(pm, s) != cudaSuccess) return RMM_ERR_CUDA;
+
+    AttnParams ap;
+    std::memset(&ap, 0, sizeof(ap));
+    if (!encode_map(&ap.map_q, Qm, p->d_h, n, H, p->d_h, n * p->d_h) ||
+        !encode_map(&ap.map_k, K, p->d_h, n, p->kv_heads, p->ldk, p->stride_k) ||
+        !encode_map(&ap.map_v, V, p->d_v, n, p->kv_heads, p->ldv, p->stride_v))
+        return RMM_ERR_CUDA;
+    ap.O = static_cast<__nv_bfloat16*>(O);
+    ap.ldo = p->ldo;
+    ap.stride_o = p->stride_o;
+    ap.row_m = reinterpret_cast<float*>(w + L.rm);
+    ap.row_l = reinterpret_cast<float*>(w + L.rl);
+    ap.col_part = reinterpret_cast<float*>(w + L.cpart);
+    ap.tok_mask = reinterpret_cast<const uint32_t*>(w + L.mask);
+    ap.mask_words = L.mask_words;
+    ap.n = static_cast<int>(n);
+    ap.heads = H;
+    ap.group = static_cast<int>(p->heads / p->kv_heads);
+    ap.q_blocks = static_cast<int>(L.q_blocks);
+    ap.k_blocks = static_cast<int>(L.q_blocks);
+    ap.causal = (p->flags & RMM_FLAG_CAUSAL) ? 1 : 0;
+    ap.scale_log2 = p->alpha * 1.4426950408889634f;
+    ap.err = reinterpret_cast<int*>(w + L.err);
+    // 3. row statistics, 4. token scores, 5. T_h, 6. the output
+    if (launch_pass<kRowStats>(ap, s) != cudaSuccess) return RMM_ERR_CUDA;
+    if (launch_pass<kColScores>(ap, s) != cudaSuccess) return RMM_ERR_CUDA;
+    float* a2 = reinterpret_cast<float*>(w + L.a2);
+    if (launch_pdl(attn_colscore_reduce_kernel, dim3((unsigned)((n + 255) / 256), (unsigned)H), dim3(256), 0, s,
+                   static_cast<const float*>(ap.col_part), a2, ap.n, ap.q_blocks, ap.causal) != cudaSuccess)
+        return RMM_ERR_CUDA;
+    SelectArgs ta{};
+    ta.d = n;
+    ta.heads = H;
+    ta.k = L.kt;
+    ta.I = T;
+    ta.scores = a2;
+    ta.mask = reinterpret_cast<uint32_t*>(w + L.mask);
+    ta.mask_words = L.mask_words;
+    if (launch_topk(ta, s) != cudaSuccess) return RMM_ERR_CUDA;
+    if (launch_pass<kOutput>(ap, s) != cudaSuccess) return RMM_ERR_CUDA;
+    return RMM_OK;
+}
+
+}  // extern "C"

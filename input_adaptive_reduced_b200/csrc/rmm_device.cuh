@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "rmm_internal.h"
@@ -90,6 +91,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
             }
         }
     }
+}
+
+// a[i] of every lane -> lane l returns the sum over the warp's lanes of a[l]
+// (a 32 x 32 block with one row per lane, summed down its columns): five
+// exchange rounds, each lane keeping half of its columns -- a fixed tree, so
+// the same bits on every call.  a is clobbered.
+__device__ __forceinline__ float warp_column_sums(float (&a)[32], int lane) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < off; ++i) {
+            const float send = upper ? a[i] : a[i + off];
+            const float keep = upper ? a[i + off] : a[i];
+            a[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    return a[0];
 }
 
 // ---------------------------------------------------------------------------
@@ -197,12 +216,23 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem], one elected thread.  KIND_TF32 selects
-// kind::tf32 (fp32 operands), otherwise kind::f16 (bf16 operands).
-template <bool KIND_TF32>
+// Operand kinds of tcgen05.mma: kind::f16 (bf16 operands), kind::tf32 (fp32
+// operands), kind::f8f6f4 (8-bit E4M3 operands).
+constexpr int kKindF16 = 0;
+constexpr int kKindTf32 = 1;
+constexpr int kKindF8 = 2;
+
+// D[tmem] (+)= A[smem] * B[smem], one elected thread.
+template <int KIND>
 __device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                      uint32_t idesc, uint32_t accumulate) {
-    if constexpr (KIND_TF32) {
+    if constexpr (KIND == kKindF8) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    } else if constexpr (KIND == kKindTf32) {
         asm volatile(
             "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
@@ -306,10 +336,16 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 }
 
 // D (M = 256 over the pair) (+)= A * B; issued by one thread of the leader CTA.
-template <bool KIND_TF32>
+template <int KIND>
 __device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
-    if constexpr (KIND_TF32) {
+    if constexpr (KIND == kKindF8) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    } else if constexpr (KIND == kKindTf32) {
         asm volatile(
             "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
@@ -353,17 +389,18 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo_
     return d;
 }
 
-// Instruction descriptor for tcgen05.mma kind::f16 / kind::tf32 with fp32
-// accumulation, M = m_rows (128 for one CTA, 256 for a CTA pair), N = n_cols,
-// A K-major, B K- or MN-major.
-__host__ __device__ constexpr uint32_t umma_idesc(bool tf32, bool b_mn_major, uint32_t n_cols,
+// Instruction descriptor for tcgen05.mma (kind::f16 with bf16, kind::tf32,
+// kind::f8f6f4 with E4M3 operands) with fp32 accumulation, M = m_rows (128 for
+// one CTA, 256 for a CTA pair), N = n_cols, A K-major, B K- or MN-major.
+__host__ __device__ constexpr uint32_t umma_idesc(int kind, bool b_mn_major, uint32_t n_cols,
                                                   uint32_t m_rows = 128) {
-    return (1u << 4)                          // D format: f32
-           | ((tf32 ? 2u : 1u) << 7)          // A format: bf16 = 1, tf32 = 2
-           | ((tf32 ? 2u : 1u) << 10)         // B format
-           | ((b_mn_major ? 1u : 0u) << 16)   // B major-ness
-           | ((n_cols >> 3) << 17)            // N >> 3
-           | ((m_rows >> 4) << 24);           // M >> 4
+    // operand format codes: bf16 = 1 (kind::f16), tf32 = 2 (kind::tf32), E4M3 = 0 (kind::f8f6f4)
+    return (1u << 4)                                                          // D format: f32
+           | ((kind == kKindTf32 ? 2u : kind == kKindF8 ? 0u : 1u) << 7)     // A format
+           | ((kind == kKindTf32 ? 2u : kind == kKindF8 ? 0u : 1u) << 10)    // B format
+           | ((b_mn_major ? 1u : 0u) << 16)                                   // B major-ness
+           | ((n_cols >> 3) << 17)                                            // N >> 3
+           | ((m_rows >> 4) << 24);                                           // M >> 4
 }
 
 }  // namespace rmm

@@ -28,6 +28,7 @@
 // error word and returns.
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "rmm_device.cuh"
@@ -39,10 +40,26 @@ namespace {
 constexpr int kThreads = 192;  // 6 warps
 constexpr int kBM = 128;
 
+// The tensor-core operand kind of an input type, and the type the product is
+// stored in (E4M3 operands give a bf16 output).
+template <typename T>
+struct KindOf {
+    static constexpr int value = sizeof(T) == 4 ? kKindTf32 : sizeof(T) == 1 ? kKindF8 : kKindF16;
+};
+template <typename T>
+struct OutOf {
+    using type = T;
+};
+template <>
+struct OutOf<__nv_fp8_e4m3> {
+    using type = __nv_bfloat16;
+};
+
 template <typename T, int BMODE, int BN>
 struct Cfg {
     static constexpr int ES = sizeof(T);
     static constexpr bool TF32 = (ES == 4);
+    static constexpr int KIND = KindOf<T>::value;
     static constexpr bool B_MN = (BMODE != kBKMajor);
     static constexpr int BK = 128 / ES;        // one 128-byte swizzle row of K
     static constexpr int UK = 32 / ES;         // K per tcgen05.mma
@@ -197,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1) gather_gemm_kernel(const __grid_c
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = umma_idesc(C::TF32, C::B_MN, BN);
+            constexpr uint32_t idesc = umma_idesc(C::KIND, C::B_MN, BN);
             uint32_t it = 0, tcount = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
@@ -223,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1) gather_gemm_kernel(const __grid_c
                         const uint64_t adesc = sw128_desc(a_addr + kk * 32, 16, 1024);
                         const uint64_t bdesc = C::B_MN ? sw128_desc(b_addr + kk * C::UK * 128, C::GROUP_BYTES, 1024)
                                                        : sw128_desc(b_addr + kk * 32, 16, 1024);
-                        umma<C::TF32>(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        umma<C::KIND>(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     umma_commit(&empty[s]);
                 }
@@ -298,23 +315,26 @@ __global__ void __launch_bounds__(kThreads, 1) gather_gemm_kernel(const __grid_c
 // ----------------------------------------------------------------------------
 template <typename T, int BMODE, int BN>
 struct PairCfg {
+    using TO = typename OutOf<T>::type;               // stored output type
     static constexpr int ES = sizeof(T);
     static constexpr bool TF32 = (ES == 4);
+    static constexpr int KIND = KindOf<T>::value;
     static constexpr bool B_MN = (BMODE != kBKMajor);
-    static constexpr int BK = 128 / ES;
-    static constexpr int UK = 32 / ES;
+    static constexpr int BK = 128 / ES;               // one 128-byte swizzle row of K
+    static constexpr int UK = 32 / ES;                // K per tcgen05.mma (32 bytes)
     static constexpr int HALF_N = BN / 2;             // B columns held by one CTA
     static constexpr int A_BYTES = kBM * 128;         // 128 rows x 128 B
     static constexpr int B_BYTES = HALF_N * 128;      // BK rows x HALF_N (MN) or HALF_N rows x 128 B (K)
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES = 6;
     static constexpr int TMEM_COLS = 2 * BN;
-    static constexpr int GROUP_BYTES = BK * 128;
-    // epilogue: EPI_WARPS warps, two per TMEM lane quadrant for bf16 (each owns
-    // half of the tile's columns), with two staging buffers of 32 x 32 each
-    static constexpr int EPI_WARPS = (ES == 2) ? 8 : 4;
+    static constexpr int GROUP_BYTES = BK * 128;      // one 128-byte-wide column group of an MN-major B tile
+    static constexpr int GROUP_N = 128 / ES;          // B columns in one group
+    // epilogue: EPI_WARPS warps, two per TMEM lane quadrant for a bf16 output
+    // (each owns half of the tile's columns), with two staging buffers of 32 x 32 each
+    static constexpr int EPI_WARPS = (sizeof(TO) == 2) ? 8 : 4;
     static constexpr int NT = 32 * (2 + EPI_WARPS);
-    static constexpr int ROW_BYTES = 32 * ES;                 // 64 (bf16) or 128 (fp32)
+    static constexpr int ROW_BYTES = 32 * (int)sizeof(TO);    // 64 (bf16) or 128 (fp32)
     static constexpr int OUT_BUF = 32 * ROW_BYTES;
     static constexpr int OUT_BYTES = EPI_WARPS * 2 * OUT_BUF;
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + OUT_BYTES + 256;
@@ -488,11 +508,52 @@ __device__ __noinline__ uint32_t split_part_epilogue(const GemmParams& p, uint32
     return slot;
 }
 
+// ----------------------------------------------------------------------------
+// Producer-fused scoring (see GemmParams::emit_s2).
+// ----------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ float stored_value(float x) {
+    if constexpr (sizeof(T) == 2)
+        return __bfloat162float(__float2bfloat16_rn(x));
+    else
+        return x;
+}
+
+// Row group rg's sum for columns [col0, col0 + 32) (lane = column) goes to the
+// workspace; the warp that completes the chunk's row groups adds them in
+// row-group order into emit_s2 and resets the chunk's counter.
+__device__ __noinline__ void emit_scores_chunk(const GemmParams& p, float colsum, int h, int rg, int col0) {
+    const int lane = threadIdx.x & 31;
+    const int rgs = 8 * p.m_tiles;
+    const bool in = col0 + lane < p.m;
+    float* base = p.emit_partials + (int64_t)h * rgs * p.m + col0 + lane;
+    if (in) __stcg(base + (int64_t)rg * p.m, colsum);
+    __threadfence();
+    __syncwarp();
+    unsigned* cnt = p.emit_counters + (int64_t)h * p.n_tiles * 8 + col0 / 32;
+    unsigned done = 0;
+    if (lane == 0) done = atomicAdd(cnt, 1u);
+    done = __shfl_sync(0xffffffffu, done, 0);
+    if (done != (unsigned)(rgs - 1)) return;
+    if (lane == 0) atomicExch(cnt, 0u);  // ready for the next launch
+    __threadfence();                     // the other row groups' sums after their counts
+    if (in) {
+        float z = 0.f;
+        for (int g = 0; g < rgs; ++g) z += __ldcg(base + (int64_t)g * p.m);
+        p.emit_s2[(int64_t)h * p.m + col0 + lane] = z;
+    }
+}
+
 // K loops of at most this many k-blocks make every epilogue warp poll the
 // accumulator barrier itself.
 constexpr int kAllPollMaxKb = 16;
 
-template <typename T, int BMODE, int BN, bool SPLIT>
+// Optional parts of the CTA-pair kernel, compiled in only where a plan uses
+// them (the plain kernel keeps the hot loops of its first form).
+constexpr int kFeatEmit = 1;  // column scores of the stored output (GemmParams::emit_s2)
+constexpr int kFeatSkip = 2;  // k-blocks without a kept index skipped (GemmParams::kb_keep)
+
+template <typename T, int BMODE, int BN, bool SPLIT, int FEAT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN>::NT, 1)
     pair_gemm_kernel(const __grid_constant__ GemmParams p) {
     using C = PairCfg<T, BMODE, BN>;
@@ -553,9 +614,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
                 if (p.causal && n0 > m0 + 2 * kBM - 1) continue;
                 const int row_base = (h / p.group) * p.b_head_rows;
                 const int kb_hi = pair_kb_end<C::BK>(p, w, m0);
-                for (int kb = w.kb0; kb < kb_hi; ++kb, ++it) {
+                const uint8_t* keep = (FEAT & kFeatSkip) ? p.kb_keep + (int64_t)h * p.kb_keep_stride : nullptr;
+                for (int kb = w.kb0; kb < kb_hi; ++kb) {
+                    if constexpr (FEAT & kFeatSkip)
+                        if (kb != w.kb0 && !keep[kb]) continue;  // no kept index in this k-block
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
+                    ++it;
                     if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err, kErrTimeoutProducer)) {
                         ok = false;
                         break;
@@ -570,9 +635,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
                                          h / p.b_head_div);
                     } else {
 #pragma unroll
-                        for (int g = 0; g < C::HALF_N / 64; ++g)
+                        for (int g = 0; g < C::HALF_N / C::GROUP_N; ++g)
                             tma_load_2d_pair(sb + g * C::GROUP_BYTES, &p.map_b, bar,
-                                             n0 + (int)rank * C::HALF_N + 64 * g, row_base + kb * C::BK);
+                                             n0 + (int)rank * C::HALF_N + C::GROUP_N * g, row_base + kb * C::BK);
                     }
                 }
             }
@@ -580,7 +645,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (leader only)
         if (leader && lane == 0) {
-            constexpr uint32_t idesc = umma_idesc(C::TF32, C::B_MN, BN, 256);
+            constexpr uint32_t idesc = umma_idesc(C::KIND, C::B_MN, BN, 256);
             uint32_t it = 0, tcount = 0;
             bool ok = true;
             for (int u = cluster; u < units && ok; u += nclusters) {
@@ -595,9 +660,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
                 const int kb_hi = pair_kb_end<C::BK>(p, w, m0);
-                for (int kb = w.kb0; kb < kb_hi; ++kb, ++it) {
+                const uint8_t* keep = (FEAT & kFeatSkip) ? p.kb_keep + (int64_t)h * p.kb_keep_stride : nullptr;
+                for (int kb = w.kb0; kb < kb_hi; ++kb) {
+                    if constexpr (FEAT & kFeatSkip)
+                        if (kb != w.kb0 && !keep[kb]) continue;  // the producer skips it too
                     const int s = it % C::STAGES;
                     const uint32_t ph = (it / C::STAGES) & 1u;
+                    ++it;
                     if (!mbar_wait(&full[s], ph, abort_flag, p.err, kErrTimeoutMma)) {
                         ok = false;
                         break;
@@ -610,7 +679,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
                         const uint64_t adesc = sw128_desc(a_addr + kk * 32, 16, 1024);
                         const uint64_t bdesc = C::B_MN ? sw128_desc(b_addr + kk * C::UK * 128, C::GROUP_BYTES, 1024)
                                                        : sw128_desc(b_addr + kk * 32, 16, 1024);
-                        umma_pair<C::TF32>(d_tmem, adesc, bdesc, idesc, (kb != w.kb0 || kk != 0) ? 1u : 0u);
+                        umma_pair<C::KIND>(d_tmem, adesc, bdesc, idesc, (kb != w.kb0 || kk != 0) ? 1u : 0u);
                     }
                     umma_commit_pair(&empty[s], 0x3);
                 }
@@ -641,7 +710,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
             uint8_t* buf = out + slot * C::OUT_BUF;
             if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
             __syncwarp();
-            stage_row<T>(buf, lane, v);
+            stage_row<typename C::TO>(buf, lane, v);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -676,7 +745,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
                 taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
             }
             if (SPLIT && row0 < p.n && w.part >= 0) {
-                slot = split_part_epilogue<T, BN, H>(p, taddr, w.t - whole, w.part, (int)rank, q, e, half, n0, row0,
+                slot = split_part_epilogue<typename C::TO, BN, H>(p, taddr, w.t - whole, w.part, (int)rank, q, e, half, n0, row0,
                                                      h, out, slot);
             } else if (row0 < p.n) {
                 bool inf_staged = false;
@@ -692,7 +761,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
                             for (int i = 0; i < 32; ++i) v[i] = -__int_as_float(0x7f800000);
                             if (lane == 0) bulk_wait_group_read<0>();
                             __syncwarp();
-                            stage_row<T>(buf, lane, v);
+                            stage_row<typename C::TO>(buf, lane, v);
                             fence_proxy_async_smem();
                             __syncwarp();
                             inf_staged = true;
@@ -713,8 +782,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
                         v[i] = (p.causal && col0 + i > row) ? -__int_as_float(0x7f800000) : x;
                     }
                     emit(v, col0, row0, h);
+                    if constexpr (FEAT & kFeatEmit) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float y = stored_value<typename C::TO>(v[i]);
+                            v[i] = row < p.n ? y * y : 0.f;
+                        }
+                        emit_scores_chunk(p, warp_column_sums(v, lane), h, (mt * 2 + (int)rank) * 4 + q, col0);
+                    }
                 }
                 if (skip && inf_staged) slot ^= 1u;  // the -inf buffer may still be read: use the other one next
+            } else if ((FEAT & kFeatEmit) && !skip) {
+                // no rows of this warp's slice exist: its row group adds zeros
+#pragma unroll 1
+                for (int ch = half; ch < BN / 32; ch += H) {
+                    const int col0 = n0 + ch * 32;
+                    if (col0 >= p.m) break;
+                    emit_scores_chunk(p, 0.f, h, (mt * 2 + (int)rank) * 4 + q, col0);
+                }
             }
             if (!skip) {
                 tc_fence_before();
@@ -736,10 +821,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<T, BMODE, BN
     }
 }
 
-template <typename T, int BMODE, int BN>
-cudaError_t launch_pair(const GemmParams& p, int num_sms, cudaStream_t s) {
+template <typename T, int BMODE, int BN, bool SPLIT, int FEAT>
+cudaError_t launch_pair_inst(const GemmParams& p, int num_sms, cudaStream_t s) {
     using C = PairCfg<T, BMODE, BN>;
-    auto kern = p.split_tiles > 0 ? pair_gemm_kernel<T, BMODE, BN, true> : pair_gemm_kernel<T, BMODE, BN, false>;
+    auto kern = pair_gemm_kernel<T, BMODE, BN, SPLIT, FEAT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
     if (e != cudaSuccess) return e;
     const int total = p.heads * p.m_tiles * p.n_tiles;
@@ -747,6 +832,24 @@ cudaError_t launch_pair(const GemmParams& p, int num_sms, cudaStream_t s) {
     const int clusters = units < num_sms / 2 ? units : num_sms / 2;
     if (clusters <= 0) return cudaSuccess;
     return launch_pdl(kern, dim3(2 * clusters), dim3(C::NT), C::SMEM, s, p);
+}
+
+// The instantiation a launch needs: split tail or not, emission (never with a
+// split tail) and block skipping (bf16 row tiles only) as the plan set them.
+template <typename T, int BMODE, int BN>
+cudaError_t launch_pair(const GemmParams& p, int num_sms, cudaStream_t s) {
+    const bool split = p.split_tiles > 0, emit = p.emit_s2 != nullptr, skip = p.kb_keep != nullptr;
+    if (emit && split) return cudaErrorInvalidValue;
+    if constexpr (BMODE == kBRows) {
+        if (skip && emit) return launch_pair_inst<T, BMODE, BN, false, kFeatEmit | kFeatSkip>(p, num_sms, s);
+        if (skip) return split ? launch_pair_inst<T, BMODE, BN, true, kFeatSkip>(p, num_sms, s)
+                               : launch_pair_inst<T, BMODE, BN, false, kFeatSkip>(p, num_sms, s);
+    } else {
+        if (skip) return cudaErrorInvalidValue;
+    }
+    if (emit) return launch_pair_inst<T, BMODE, BN, false, kFeatEmit>(p, num_sms, s);
+    return split ? launch_pair_inst<T, BMODE, BN, true, 0>(p, num_sms, s)
+                 : launch_pair_inst<T, BMODE, BN, false, 0>(p, num_sms, s);
 }
 
 template <typename T, int BMODE, int BN>
@@ -785,6 +888,8 @@ void pair_split_tail(int64_t tiles, int64_t num_kb, int clusters, int* split_til
 }
 
 size_t gemm_smem_bytes(int dtype, int bn, bool pair) {
+    if (dtype == 2)
+        return bn == 256 ? PairCfg<__nv_fp8_e4m3, kBRows, 256>::SMEM : PairCfg<__nv_fp8_e4m3, kBRows, 128>::SMEM;
     if (pair) {
         if (dtype == 1) return bn == 256 ? PairCfg<float, kBKMajor, 256>::SMEM : PairCfg<float, kBKMajor, 128>::SMEM;
         return bn == 256 ? PairCfg<__nv_bfloat16, kBRows, 256>::SMEM : PairCfg<__nv_bfloat16, kBRows, 128>::SMEM;
@@ -794,6 +899,11 @@ size_t gemm_smem_bytes(int dtype, int bn, bool pair) {
 }
 
 cudaError_t launch_gemm(const GemmParams& p, const GemmLaunch& l, cudaStream_t s) {
+    if (l.dtype == 2) {  // E4M3 operands: CTA pairs, B as rows (MN-major)
+        if (!l.pair || l.b_mode != kBRows) return cudaErrorInvalidValue;
+        return l.bn == 256 ? launch_pair<__nv_fp8_e4m3, kBRows, 256>(p, l.num_sms, s)
+                           : launch_pair<__nv_fp8_e4m3, kBRows, 128>(p, l.num_sms, s);
+    }
     if (l.pair) {
         if (l.dtype == 1) {
             if (l.b_mode != kBKMajor) return cudaErrorInvalidValue;

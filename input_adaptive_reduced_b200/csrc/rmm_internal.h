@@ -148,7 +148,9 @@ cudaError_t launch_pack_ab(const PackArgs& a, const PackArgs& b, cudaStream_t s)
 // else 0, for t < rows_out (rows t >= a.d are zero); a.rows = columns of B.
 // Used for attention PV, where the product is bound by reading P and a
 // zero-masked V gives the same sum over I without a copy of P's columns.
-cudaError_t launch_mask_rows(const PackArgs& a, int64_t rows_out, cudaStream_t s);
+// block_any (or nullptr): [heads][ceil(rows_out / 64)] bytes, 1 where the
+// 64-row block holds a kept row.
+cudaError_t launch_mask_rows(const PackArgs& a, int64_t rows_out, cudaStream_t s, uint8_t* block_any = nullptr);
 
 // ---------------------------------------------------------------- GEMM
 // How the B operand reaches shared memory (see rmm_gemm.cu).
@@ -185,6 +187,22 @@ struct __align__(64) GemmParams {
     int32_t split_tiles, split_f;
     float* split_partials;
     unsigned* split_counters;
+    // CTA-pair kernel, producer-fused scoring (no split tail): when emit_s2 is
+    // set, every epilogue warp squares its 32 x 32 block of stored outputs and
+    // sums each column over its 32 rows into emit_partials[h][row group][m]
+    // (row group = 32-row slice of the output); emit_counters[h][column chunk]
+    // counts the row groups done, and the warp that completes a chunk adds the
+    // row groups in order into emit_s2[h][m] and resets the counter.
+    float* emit_s2;
+    float* emit_partials;
+    unsigned* emit_counters;
+    // CTA-pair kernel, K axis on a masked operand (attention PV with V's
+    // unkept rows zeroed): kb_keep[h * kb_keep_stride + kb] == 0 says that
+    // k-block kb of head h holds no kept index, so its products are zero and
+    // the K loop skips it (the first k-block of a unit always runs, so that
+    // every accumulator is written).
+    const uint8_t* kb_keep;
+    int32_t kb_keep_stride;
 };
 
 struct GemmLaunch {
@@ -202,6 +220,7 @@ size_t gemm_smem_bytes(int dtype, int bn, bool pair);
 // the last wave is full or too short to split).
 void pair_split_tail(int64_t tiles, int64_t num_kb, int clusters, int* split_tiles, int* split_f);
 constexpr int kSplitCounterWarps = 8;  // counters per CTA per split tile (epilogue warps)
+
 
 // ---------------------------------------------------------------- decode step
 // Attention with group * n <= 8 query vectors per KV head (rmm_decode.cu).
@@ -262,7 +281,8 @@ struct rmm_plan {
     rmm_problem p;
     int64_t k;
     int64_t ldp;        // row stride of the packed operands (k rounded up to 8)
-    int es;             // element size
+    int es;             // element size of A and B
+    int es_out;         // element size of Y (2 for E4M3 operands: a bf16 output)
     int group;          // heads / kv_heads
     bool need_select;   // scores + TopK on each call
     bool fused_select;  // one-kernel selection
@@ -286,4 +306,11 @@ struct rmm_plan {
     bool decode_select; // decode QK: the features are selected inside the product kernel
     int dec_tokens, dec_parts;          // pv: tokens per CTA, token ranges per KV head
     size_t off_dec_cnt, off_dec_mask, off_dec_part;  // pv: counters (header), membership words, partials
+    size_t off_kb_keep;                               // masked PV: per-head 64-token blocks holding a kept token
+    bool given_scores;  // RMM_FLAG_GIVEN_SCORES: I = TopK of the caller's scores (no score pass)
+    bool emit_scores;   // RMM_FLAG_EMIT_SCORES: column scores of Y (epilogue, or a score pass over Y)
+    size_t off_emit_cnt, off_emit_part;               // epilogue form: counters (header), row-group sums
+    int emit_nsplit;                                  // score-pass form over Y: its row splits,
+    int64_t emit_rows_per_split;
+    size_t off_emit_ycnt, off_emit_ypart;             // its counters (header) and partials
 };

@@ -8,6 +8,7 @@
 // with TMA.  Used for A in every mode and for K in the QK mode.
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "rmm_internal.h"
@@ -56,7 +57,9 @@ __device__ __forceinline__ void pack_block(const T* __restrict__ src, int64_t ro
         for (int q = 0; q < 4; ++q) {
             if (q >= nq) break;
             T* o = dh + (r + q) * ld_dst + t0;
-            if constexpr (sizeof(T) == 2) {
+            if constexpr (sizeof(T) == 1) {
+                *reinterpret_cast<uint2*>(o) = *reinterpret_cast<const uint2*>(vals[q]);
+            } else if constexpr (sizeof(T) == 2) {
                 *reinterpret_cast<uint4*>(o) = *reinterpret_cast<const uint4*>(vals[q]);
             } else {
                 reinterpret_cast<uint4*>(o)[0] = reinterpret_cast<const uint4*>(vals[q])[0];
@@ -202,7 +205,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) mask_rows_kernel(
     const T* __restrict__ src, int64_t d, int64_t cols, int64_t ld_src, int64_t stride_src, int group,
     const int32_t* __restrict__ I, int64_t I_stride, int64_t k, T* __restrict__ dst, int64_t ld_dst,
-    int64_t stride_dst, int64_t rows_out) {
+    int64_t stride_dst, int64_t rows_out, uint8_t* __restrict__ block_any) {
     pdl_wait();
     pdl_trigger();
     constexpr int V = 16 / sizeof(T);
@@ -219,6 +222,9 @@ __global__ void __launch_bounds__(256) mask_rows_kernel(
         if (j >= r0 && j < r0 + kMaskRows && j < d) keep[j - r0] = 1;
     }
     __syncthreads();
+    // whether any row of this block is kept (the product skips blocks with none)
+    const int any = __syncthreads_or(threadIdx.x < kMaskRows ? keep[threadIdx.x] : 0);
+    if (block_any && threadIdx.x == 0) block_any[(int64_t)h * gridDim.x + blockIdx.x] = any ? 1 : 0;
     const int cpr = (int)(cols / V);
     const int64_t left = rows_out - r0;
     const int nrows = left < kMaskRows ? (int)left : kMaskRows;
@@ -268,7 +274,9 @@ __global__ void __launch_bounds__(256) pack_narrow_kernel(
             vals[v] = j >= 0 ? srow[j] : T(0.f);
         }
         T* o = dh + (r0 + r) * ld_dst + 8 * c;
-        if constexpr (sizeof(T) == 2) {
+        if constexpr (sizeof(T) == 1) {
+            *reinterpret_cast<uint2*>(o) = *reinterpret_cast<const uint2*>(vals);
+        } else if constexpr (sizeof(T) == 2) {
             *reinterpret_cast<uint4*>(o) = *reinterpret_cast<const uint4*>(vals);
         } else {
             reinterpret_cast<uint4*>(o)[0] = reinterpret_cast<const uint4*>(vals)[0];
@@ -333,6 +341,10 @@ cudaError_t launch_mask_columns(const PackArgs& a, cudaStream_t s) {
 cudaError_t launch_pack_rows(const PackArgs& a, cudaStream_t s) {
     if (a.k == 0 || a.rows == 0) return cudaSuccess;
     dim3 grid((unsigned)((a.k + kRowsPerCta - 1) / kRowsPerCta), (unsigned)a.heads);
+    if (a.dtype == 2)
+        return launch_pdl(pack_rows_kernel<__nv_fp8_e4m3>, grid, dim3(256), 0, s, (const __nv_fp8_e4m3*)a.src, a.d,
+                          a.rows, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k, (__nv_fp8_e4m3*)a.dst,
+                          a.ld_dst, a.stride_dst);
     if (a.dtype == 1)
         return launch_pdl(pack_rows_kernel<float>, grid, dim3(256), 0, s, (const float*)a.src, a.d, a.rows, a.ld_src,
                           a.stride_src, a.group, a.I, a.I_stride, a.k, (float*)a.dst, a.ld_dst, a.stride_dst);
@@ -341,7 +353,7 @@ cudaError_t launch_pack_rows(const PackArgs& a, cudaStream_t s) {
                       a.ld_dst, a.stride_dst);
 }
 
-bool pack_ab_one_launch(int dtype, int64_t ld_a) { return dtype == 0 && ld_a > kNarrowMax; }
+bool pack_ab_one_launch(int dtype, int64_t ld_a) { return (dtype == 0 || dtype == 2) && ld_a > kNarrowMax; }
 
 cudaError_t launch_pack_ab(const PackArgs& a, const PackArgs& b, cudaStream_t s) {
     if (!pack_ab_one_launch(a.dtype, a.ld_dst) || b.dtype != a.dtype) return cudaErrorInvalidValue;
@@ -353,20 +365,23 @@ cudaError_t launch_pack_ab(const PackArgs& a, const PackArgs& b, cudaStream_t s)
     const int64_t total = n_a + n_b;
     if (total == 0) return cudaSuccess;
     if (total > 0x7fffffff) return cudaErrorInvalidValue;
+    if (a.dtype == 2)
+        return launch_pdl(pack_ab_kernel<__nv_fp8_e4m3>, dim3((unsigned)total), dim3(256), 0, s, a, b, a_x, a_y,
+                          n_a, b_x);
     return launch_pdl(pack_ab_kernel<__nv_bfloat16>, dim3((unsigned)total), dim3(256), 0, s, a, b, a_x, a_y, n_a,
                       b_x);
 }
 
-cudaError_t launch_mask_rows(const PackArgs& a, int64_t rows_out, cudaStream_t s) {
+cudaError_t launch_mask_rows(const PackArgs& a, int64_t rows_out, cudaStream_t s, uint8_t* block_any) {
     dim3 grid((unsigned)((rows_out + kMaskRows - 1) / kMaskRows), (unsigned)a.heads);
     if (grid.x == 0 || a.rows == 0) return cudaSuccess;
     if (a.dtype == 1)
         return launch_pdl(mask_rows_kernel<float>, grid, dim3(256), 0, s, (const float*)a.src, a.d, a.rows, a.ld_src,
                           a.stride_src, a.group, a.I, a.I_stride, a.k, (float*)a.dst, a.ld_dst, a.stride_dst,
-                          rows_out);
+                          rows_out, block_any);
     return launch_pdl(mask_rows_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, (const __nv_bfloat16*)a.src, a.d,
                       a.rows, a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k, (__nv_bfloat16*)a.dst,
-                      a.ld_dst, a.stride_dst, rows_out);
+                      a.ld_dst, a.stride_dst, rows_out, block_any);
 }
 
 cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s) {
@@ -383,9 +398,13 @@ cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_pack(const PackArgs& a, cudaStream_t s) {
+    using F8 = __nv_fp8_e4m3;
     if (a.ld_dst <= kNarrowMax) {
         dim3 g((unsigned)((a.rows + kNarrowRows - 1) / kNarrowRows), (unsigned)a.heads);
         if (g.x == 0) return cudaSuccess;
+        if (a.dtype == 2)
+            return launch_pdl(pack_narrow_kernel<F8>, g, dim3(256), 0, s, (const F8*)a.src, a.rows, a.d, a.ld_src,
+                              a.stride_src, a.group, a.I, a.I_stride, a.k, (F8*)a.dst, a.ld_dst, a.stride_dst);
         if (a.dtype == 1)
             return launch_pdl(pack_narrow_kernel<float>, g, dim3(256), 0, s, (const float*)a.src, a.rows, a.d,
                               a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k, (float*)a.dst, a.ld_dst,
@@ -397,6 +416,9 @@ cudaError_t launch_pack(const PackArgs& a, cudaStream_t s) {
     dim3 grid((unsigned)((a.ld_dst + 8 * kPackThreads - 1) / (8 * kPackThreads)),
               (unsigned)((a.rows + kPackRows - 1) / kPackRows), (unsigned)a.heads);
     if (grid.y == 0) return cudaSuccess;
+    if (a.dtype == 2)
+        return launch_pdl(pack_kernel<F8>, grid, dim3(kPackThreads), 0, s, (const F8*)a.src, a.rows, a.d, a.ld_src,
+                          a.stride_src, a.group, a.I, a.I_stride, a.k, (F8*)a.dst, a.ld_dst, a.stride_dst);
     if (a.dtype == 1)
         return launch_pdl(pack_kernel<float>, grid, dim3(kPackThreads), 0, s, (const float*)a.src, a.rows, a.d,
                           a.ld_src, a.stride_src, a.group, a.I, a.I_stride, a.k, (float*)a.dst, a.ld_dst,

@@ -12,6 +12,8 @@
 // lower index is kept, and I is written in ascending order.
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "rmm_internal.h"
@@ -31,6 +33,24 @@ struct Vec16<__nv_bfloat16> {
         for (int i = 0; i < 4; ++i) {
             x[2 * i] = __uint_as_float(w[i] << 16);
             x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+};
+template <>
+struct Vec16<__nv_fp8_e4m3> {  // 8-bit E4M3 codes, decoded exactly (the low-bit form)
+    static constexpr int N = 16;
+    __device__ static void load(const __nv_fp8_e4m3* p, float (&x)[16]) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __half2 lo(__nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] & 0xffffu), __NV_E4M3));
+            const __half2 hi(__nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] >> 16), __NV_E4M3));
+            const float2 a = __half22float2(lo), b = __half22float2(hi);
+            x[4 * i] = a.x;
+            x[4 * i + 1] = a.y;
+            x[4 * i + 2] = b.x;
+            x[4 * i + 3] = b.y;
         }
     }
 };
@@ -667,8 +687,12 @@ size_t normselect_smem_bytes(int64_t d, int dtype) {
 
 cudaError_t launch_colnorm(const SelectArgs& a, cudaStream_t s) {
     if (a.nsplit < 1 || a.nsplit > kMaxSplit) return cudaErrorInvalidValue;
-    const int V = a.dtype == 1 ? 4 : 8;
+    const int V = a.dtype == 1 ? 4 : a.dtype == 2 ? 16 : 8;  // elements per 16-byte load
     dim3 grid((unsigned)((a.d + 32 * V - 1) / (32 * V)), (unsigned)a.nsplit, (unsigned)a.heads);
+    if (a.dtype == 2)
+        return launch_pdl(colnorm_kernel<__nv_fp8_e4m3>, grid, dim3(32 * kColWarps), 0, s,
+                          (const __nv_fp8_e4m3*)a.A, a.n, a.d, a.lda, a.stride_a, a.rows_per_split, a.nsplit,
+                          a.partials, a.counters, a.scores, a.causal_rows);
     if (a.dtype == 1)
         return launch_pdl(colnorm_kernel<float>, grid, dim3(32 * kColWarps), 0, s, (const float*)a.A, a.n, a.d,
                           a.lda, a.stride_a, a.rows_per_split, a.nsplit, a.partials, a.counters, a.scores,

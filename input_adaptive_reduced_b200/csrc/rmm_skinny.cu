@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(const __grid_cons
                 for (int kk = 0; kk < kSkBK / 16; ++kk) {
                     const uint64_t mdesc = sw128_desc(g_addr + kk * 16 * 128, kSkGroupBytes, 1024);
                     const uint64_t ndesc = sw128_desc(a_addr + kk * 32, 16, 1024);
-                    umma<false>(tmem_base, mdesc, ndesc, idesc, (kb > kb_beg || kk > 0) ? 1u : 0u);
+                    umma<kKindF16>(tmem_base, mdesc, ndesc, idesc, (kb > kb_beg || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(&empty[s]);
             }

@@ -302,6 +302,40 @@ def test_deterministic(rmm):
     assert torch.equal(I1, I2) and torch.equal(Y1, Y2)
 
 
+@pytest.mark.parametrize("n,d,m,rho", [(260, 4096, 520, 0.7), (256, 1024, 512, 0.3), (1100, 8192, 2056, 0.6)])
+def test_linear_back_to_back(rmm, n, d, m, rho):
+    """Two different inputs run back to back on one plan and workspace with no
+    host synchronisation in between (the workspace's counters are returned
+    to zero by the kernels), each matching the oracle; shapes with ragged
+    row / column tiles, a grid smaller than one wave, and a split tail."""
+    k = oracle.retained_count(rho, d)
+    dev = torch.device("cuda")
+    ins = []
+    for seed in (61, 62):
+        (A, B), _ = gap.enforce_boundary_gaps(lambda g: W.mlp_up(seed, n=n, d=d, m=m, col_gain=g),
+                                              lambda x: gap.scores_2d(x[0]), [k])
+        ins.append((A, B))
+    p = rmm.rmm_problem_init(rmm.RMM_LINEAR, rmm.RMM_BF16, n, d, m)
+    p.rho = rho
+    plan = rmm.Plan(p)
+    ws = rmm.workspace_for(plan)
+    outs = []
+    for A, B in ins:
+        Y = torch.empty((n, m), dtype=torch.bfloat16, device=dev)
+        I = torch.empty(plan.k, dtype=torch.int32, device=dev)
+        rmm.rmm_matmul(plan, A.to(dev), B.to(dev), Y, I, ws)
+        outs.append((Y, I))
+    torch.cuda.synchronize()
+    rmm.check_workspaces()
+    rows = list(range(0, n, 7))
+    for (A, B), (Y, I) in zip(ins, outs):
+        I_ref, _ = oracle.select(A, rho=rho)
+        assert_indices_equal(I, I_ref)
+        A64, B64 = oracle.as_f64(A), oracle.as_f64(B)
+        assert_product_close(Y[rows], oracle.reduced_product(A64, B64, I_ref, rows),
+                             np.abs(A64[rows][:, I_ref]), np.abs(B64[I_ref]))
+
+
 def _split_parts(tiles, num_kb):
     """Parts per tile of the CTA-pair kernel's split tail on this GPU (1 = none):
     the last wave's tiles are cut into f <= 4 K-parts that still fit one wave,

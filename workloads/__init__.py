@@ -20,6 +20,8 @@ exp(N(0,1))):
                  V [H_kv][n][d_v] = N(0,1)
   linear_70b     bf16 B in {8192x28672, 28672x8192, 8192x10240} = N(0, 0.014);
                  A as mlp_up (d = 8192) or as mlp_down (d = 28672)
+  quantize_e4m3  per-tensor 8-bit E4M3 codes (scale = amax / 448) of any of the
+                 above, for the low-bit form
   attn_decode    one decode step per sequence: q [B*H][n][d_h] and the K cache
                  [B*H_kv][t][d_h] as attn_qk; V cache [B*H_kv][t][d_v] = N(0,1);
                  P [B*H][n][t] = row softmax of N(0,2) logits (as attn_pv),
@@ -36,7 +38,7 @@ import torch
 
 __all__ = [
     "gen", "linear_small", "mlp_up", "mlp_down", "attn_qk", "attn_pv", "attn_decode", "linear_70b",
-    "duplicate_columns", "LLAMA8B_MLP", "LLAMA70B_LINEAR",
+    "duplicate_columns", "quantize_e4m3", "LLAMA8B_MLP", "LLAMA70B_LINEAR",
 ]
 
 LLAMA8B_MLP = {"up": (4096, 14336), "down": (14336, 4096)}
@@ -176,6 +178,17 @@ def attn_decode(seed: int, t: int, batch: int = 1, n: int = 1, heads: int = 32, 
         gain = torch.as_tensor(p_gain, dtype=torch.float64).to(device)
         P = (P.double() * gain[:, None, :]).float()
     return q.to(dtype).contiguous(), K.to(dtype).contiguous(), V.to(dtype).contiguous(), P.to(dtype).contiguous()
+
+
+def quantize_e4m3(x: torch.Tensor):
+    """Per-tensor 8-bit E4M3 codes of x and their scale: scale = amax / 448
+    (the largest E4M3 magnitude), codes = round-to-nearest(x / scale) as
+    torch's float8_e4m3fn conversion gives them.  Returns (codes, scale);
+    x ~ codes * scale.  Input preparation for the low-bit form only."""
+    xf = x.float()
+    amax = float(xf.abs().max())
+    scale = amax / 448.0 if amax > 0 else 1.0
+    return (xf / scale).to(torch.float8_e4m3fn).contiguous(), scale
 
 
 def duplicate_columns(A: torch.Tensor, pairs) -> torch.Tensor:

@@ -244,8 +244,10 @@ RMM_API rmm_status rmm_matmul_ex(const rmm_plan* plan, const void* A, const void
    multiples of 8 elements, lds and ldp >= t.  workspace: device memory of
    rmm_softmax_workspace_size(heads, n, t) bytes, 256-byte aligned, zeroed
    once (cudaMemsetAsync) before its first use; the kernel leaves its
-   counters at zero.  Errors: RMM_ERR_INVALID_ARG / RMM_ERR_UNSUPPORTED /
-   RMM_ERR_WORKSPACE before any launch. */
+   counters at zero, and if it gives up waiting for a row of S to arrive in
+   shared memory (about two seconds) it writes a nonzero code into the
+   workspace's first word.  Errors: RMM_ERR_INVALID_ARG / RMM_ERR_UNSUPPORTED /
+   RMM_ERR_WORKSPACE before any launch, RMM_ERR_CUDA if the launch fails. */
 RMM_API size_t rmm_softmax_workspace_size(int64_t heads, int64_t n, int64_t t);
 RMM_API rmm_status rmm_softmax_scores(const void* S, void* P, float* s2, int64_t heads, int64_t n, int64_t t,
                                       int64_t lds, int64_t stride_s, int64_t ldp, int64_t stride_p, uint32_t flags,

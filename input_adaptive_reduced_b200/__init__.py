@@ -366,10 +366,17 @@ def workspace_for(plan: Plan, device=None, stream=None):
 def check_workspaces():
     """Synchronise and read the error word of every workspace this module
     allocated; raise RmmError(RMM_ERR_TIMEOUT) if a kernel gave up on a wait."""
+    import torch
     with _cache_lock:
         items = [(p, ws) for p in list(_ws_plans) for ws in list(p._ws.values())]
+        raw = [ws for key, ws in _plans.items() if key[0] in ("softmax", "attention")]
     for plan, ws in items:
         _check(rmm_workspace_status(plan, ws), "kernel wait")
+    if raw:
+        torch.cuda.synchronize()
+    for ws in raw:  # the softmax and attention workspaces keep their error word in the first 4 bytes
+        if int(ws[:4].view(torch.int32).item()) != 0:
+            raise RmmError(RMM_ERR_TIMEOUT, "kernel wait")
 
 
 def _k_fields(p: rmm_problem, rho, k):

@@ -71,9 +71,12 @@ struct __align__(64) AttnParams {
 template <int MODE>
 struct AttnCfg {
     static constexpr bool OUT = MODE == kOutput;
+    // K (and V) stages: the score-only passes keep four K blocks in flight; the
+    // output pass, whose stages also hold V and which needs two P tiles, two
+    static constexpr int STAGES = OUT ? 2 : 4;
     static constexpr int KV_BYTES = OUT ? 2 * TILE : TILE;  // K (and V) of one key block
     static constexpr int STAT_BYTES = MODE == kRowStats ? 2 * 4 * BQ * 4 : 0;  // per-quarter (m, l) of each row
-    static constexpr size_t SMEM = 1024 + TILE + 2 * (size_t)KV_BYTES + (OUT ? 2 * TILE : 0) + STAT_BYTES + 256;
+    static constexpr size_t SMEM = 1024 + TILE + STAGES * (size_t)KV_BYTES + (OUT ? 2 * TILE : 0) + STAT_BYTES + 256;
     static constexpr uint32_t TMEM_COLS = OUT ? 512 : 256;  // two S buffers (+ O)
 };
 
@@ -85,22 +88,12 @@ __device__ __forceinline__ void attn_block(const AttnParams& p, int& h, int& qb)
     qb = p.causal ? p.q_blocks - 1 - r : r;
 }
 
-// Whether key block kb takes part for query block qb: inside the causal
-// range, and in the output pass only if one of its tokens is kept.
-template <int MODE>
-__device__ __forceinline__ bool key_block_used(const AttnParams& p, int h, int qb, int kb) {
-    if (p.causal && kb > qb) return false;
-    if constexpr (MODE == kOutput) {
-        const uint32_t* w = p.tok_mask + (int64_t)h * p.mask_words;
-        uint32_t any = 0;
-#pragma unroll
-        for (int i = 0; i < BKEY / 32; ++i) {
-            const int64_t wi = (int64_t)kb * (BKEY / 32) + i;
-            if (wi < p.mask_words) any |= __ldg(w + wi);
-        }
-        return any != 0;
-    }
-    return true;
+constexpr int kMaxKeyBlocks = (int)(kMaxSelectD / BKEY);  // key blocks of the longest sequence
+
+// Output pass: whether key block kb holds a kept token (bit kb of used_bits,
+// filled from the token mask when the CTA starts).
+__device__ __forceinline__ bool block_used(const uint32_t* used_bits, int kb) {
+    return (used_bits[kb >> 5] >> (kb & 31)) & 1u;
 }
 
 template <int MODE>
@@ -109,27 +102,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;
-    uint8_t* sKV = sQ + TILE;                         // 2 stages: K tile (then V tile)
-    uint8_t* sP = sKV + 2 * C::KV_BYTES;              // 2 P tiles (output pass)
+    uint8_t* sKV = sQ + TILE;                         // STAGES stages: K tile (then V tile)
+    uint8_t* sP = sKV + C::STAGES * C::KV_BYTES;      // 2 P tiles (output pass)
     float* stat = reinterpret_cast<float*>(sP + (C::OUT ? 2 * TILE : 0));  // [2][4][BQ] (row statistics)
     uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stat) + C::STAT_BYTES);
     uint64_t* q_full = bars;
-    uint64_t* kv_full = bars + 1;
-    uint64_t* kv_empty = bars + 3;
-    uint64_t* s_full = bars + 5;
-    uint64_t* s_empty = bars + 7;
-    uint64_t* p_full = bars + 9;
-    uint64_t* p_empty = bars + 11;
-    uint64_t* o_full = bars + 13;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
+    uint64_t* kv_full = bars + 1;                 // [STAGES]
+    uint64_t* kv_empty = kv_full + C::STAGES;     // [STAGES]
+    uint64_t* s_full = kv_empty + C::STAGES;      // [2]
+    uint64_t* s_empty = s_full + 2;
+    uint64_t* p_full = s_empty + 2;
+    uint64_t* p_empty = p_full + 2;
+    uint64_t* o_full = p_empty + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(o_full + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
             mbar_init(&s_empty[s], kRowWarps);  // one arrival per row warp
             mbar_init(&p_full[s], kRowWarps);
@@ -158,6 +153,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
     const int g = h / p.group;
     const int q0 = qb * BQ;
     const int kb_end = p.causal ? min(qb + 1, p.k_blocks) : p.k_blocks;
+    __shared__ uint32_t used_bits[(kMaxKeyBlocks + 31) / 32];
+    if constexpr (C::OUT) {
+        // which key blocks hold a kept token (the token mask is written by the
+        // selection that runs before this pass)
+        const uint32_t* w = p.tok_mask + (int64_t)h * p.mask_words;
+        for (int kb0 = warp * 32; kb0 < kb_end; kb0 += kThreads) {
+            const int kb = kb0 + lane;
+            uint32_t any = 0;
+            if (kb < kb_end) {
+#pragma unroll
+                for (int i = 0; i < BKEY / 32; ++i) {
+                    const int64_t wi = (int64_t)kb * (BKEY / 32) + i;
+                    if (wi < p.mask_words) any |= __ldg(w + wi);
+                }
+            }
+            const uint32_t bits = __ballot_sync(0xffffffffu, any != 0u);
+            if (lane == 0) used_bits[kb0 >> 5] = bits;
+        }
+        __syncthreads();
+    }
+    auto used = [&](int kb) { return !C::OUT || block_used(used_bits, kb); };
 
     if (warp == 0) {
         // ---------------------------------------------------------------- loads
@@ -167,9 +183,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
             tma_load_3d(sQ + ATOM, &p.map_q, q_full, 64, q0, h);
             uint32_t it = 0;
             for (int kb = 0; kb < kb_end; ++kb) {
-                if (!key_block_used<MODE>(p, h, qb, kb)) continue;
-                const int s = it & 1;
-                const uint32_t ph = (it >> 1) & 1u;
+                if (!used(kb)) continue;
+                const int s = it % C::STAGES;
+                const uint32_t ph = (it / C::STAGES) & 1u;
                 ++it;
                 if (!mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, p.err, kErrTimeoutProducer)) break;
                 uint8_t* dst = sKV + s * C::KV_BYTES;
@@ -194,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
                 if (!mbar_wait(&p_full[pb], (j >> 1) & 1u, abort_flag, p.err, kErrTimeoutMma)) return false;
                 tc_fence_after();
                 const uint32_t p_addr = smem_u32(sP + pb * TILE);
-                const uint32_t v_addr = smem_u32(sKV + pb * C::KV_BYTES + TILE);
+                const uint32_t v_addr = smem_u32(sKV + (j % C::STAGES) * C::KV_BYTES + TILE);
 #pragma unroll
                 for (int kk = 0; kk < BKEY / 16; ++kk) {
                     const uint64_t adesc = sw128_desc(p_addr + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
@@ -202,30 +218,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
                     umma<kKindF16>(tmem_base + 256, adesc, bdesc, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(&p_empty[pb]);
-                umma_commit(&kv_empty[pb]);
+                umma_commit(&kv_empty[j % C::STAGES]);
                 return true;
             };
             bool ok = mbar_wait(q_full, 0u, abort_flag, p.err, kErrTimeoutMma);
             uint32_t it = 0;
             for (int kb = 0; kb < kb_end && ok; ++kb) {
-                if (!key_block_used<MODE>(p, h, qb, kb)) continue;
-                const int s = it & 1;
-                const uint32_t ph = (it >> 1) & 1u;
+                if (!used(kb)) continue;
+                const int s = it % C::STAGES;                 // K (and V) stage
+                const uint32_t ph = (it / C::STAGES) & 1u;
+                const int sb = it & 1;                        // S buffer
+                const uint32_t sph = (it >> 1) & 1u;
                 if (!mbar_wait(&kv_full[s], ph, abort_flag, p.err, kErrTimeoutMma) ||
-                    !mbar_wait(&s_empty[s], ph ^ 1u, abort_flag, p.err, kErrTimeoutMma)) {
+                    !mbar_wait(&s_empty[sb], sph ^ 1u, abort_flag, p.err, kErrTimeoutMma)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t k_addr = smem_u32(sKV + s * C::KV_BYTES);
-                const uint32_t d_tmem = tmem_base + s * BKEY;
+                const uint32_t d_tmem = tmem_base + sb * BKEY;
 #pragma unroll
                 for (int kk = 0; kk < DH / 16; ++kk) {
                     const uint64_t adesc = sw128_desc(q_addr + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
                     const uint64_t bdesc = sw128_desc(k_addr + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
                     umma<kKindF16>(d_tmem, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&s_full[s]);
+                umma_commit(&s_full[sb]);
                 if constexpr (C::OUT) {
                     if (it > 0 && !pv(it - 1)) ok = false;
                 } else {
@@ -246,18 +264,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
         const int row = q0 + r_loc;
         const bool row_ok = row < p.n;
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-        // rows past n: m = 0 and 1/l = 0, so that every weight is 2^-inf * 0 = 0
-        float m = MODE == kRowStats ? -INFINITY : 0.f, l = 0.f, inv_l = 0.f;
+        // Every weight is 2^(x - b) with x = scale * score and b = m + log2(l)
+        // the row's base (one exp per weight, no division); rows past n and
+        // rows without a key get b = +inf, so that all their weights are 0.
+        float m = -INFINITY, l = 0.f, b = INFINITY;
         if (MODE != kRowStats && row_ok) {
             m = p.row_m[(int64_t)h * p.n + row];
             l = p.row_l[(int64_t)h * p.n + row];
-            inv_l = l > 0.f ? 1.0f / l : 0.f;
+            if (l > 0.f) b = m + log2f(l);
         }
+        const float scale = p.scale_log2;
         const uint32_t* mask_h = p.tok_mask ? p.tok_mask + (int64_t)h * p.mask_words : nullptr;
+        // output pass: lane j holds this warp's mask word of key block 32 * keep_base + j
+        uint32_t keep_reg = 0u;
+        int keep_base = -1;
         uint32_t it = 0;
         bool ok = true;
         for (int kb = 0; kb < kb_end && ok; ++kb) {
-            if (!key_block_used<MODE>(p, h, qb, kb)) continue;
+            if (!used(kb)) continue;
             const int sb = it & 1;
             const uint32_t ph = (it >> 1) & 1u;
             ++it;
@@ -280,22 +304,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
             uint32_t raw[32];
             tmem_ld_32x32b_x32(tmem_base + lane_base + sb * BKEY + cq * 32, raw);
             tmem_ld_wait();
+            // the scores are in registers: this S buffer may be overwritten
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[sb]);
+            // x = scale * score, -inf where masked (one uniform test per chunk)
             float x[32];
+            if (__all_sync(0xffffffffu, all_in)) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const bool valid = all_in || (!none_in && k0 + i < p.n && (!p.causal || k0 + i <= row));
-                x[i] = valid ? __uint_as_float(raw[i]) * p.scale_log2 : -INFINITY;
+                for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(raw[i]) * scale;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const bool valid = !none_in && k0 + i < p.n && (!p.causal || k0 + i <= row);
+                    x[i] = valid ? __uint_as_float(raw[i]) * scale : -INFINITY;
+                }
             }
             if constexpr (MODE == kRowStats) {
                 if (!none_in) {
-                    float mc = -INFINITY;
+                    float mc[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) mc = fmaxf(mc, x[i]);
-                    const float mn = fmaxf(m, mc);
-                    float acc = l * exp2f(m - mn);
+                    for (int i = 4; i < 32; ++i) mc[i & 3] = fmaxf(mc[i & 3], x[i]);
+                    const float mn = fmaxf(m, fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])));
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) acc += exp2f(x[i] - mn);  // 2^-inf = 0
-                    l = acc;
+                    for (int i = 0; i < 32; ++i) acc[i & 3] += fast_exp2(x[i] - mn);  // 2^-inf = 0
+                    l = fmaf(l, fast_exp2(m - mn), (acc[0] + acc[1]) + (acc[2] + acc[3]));
                     m = mn;
                 }
             } else if constexpr (MODE == kColScores) {
@@ -303,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
                 if (__any_sync(0xffffffffu, !none_in)) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const float pr = exp2f(x[i] - m) * inv_l;  // 0 where masked
+                        const float pr = fast_exp2(x[i] - b);  // 0 where masked
                         x[i] = pr * pr;
                     }
                     z = warp_column_sums(x, lane);  // this warp's 32 rows, summed per key
@@ -312,28 +346,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
                 if (key < p.n) p.col_part[((int64_t)h * p.q_blocks * 4 + qb * 4 + quad) * p.n + key] = z;
             } else {
                 // P masked to the kept tokens, rounded to bf16, into the swizzled P tile
-                const int64_t wi = (int64_t)k0 >> 5;
-                const uint32_t keep_bits = (!none_in && wi < p.mask_words) ? __ldg(mask_h + wi) : 0u;
+                if ((kb >> 5) != keep_base) {  // the same for every lane
+                    keep_base = kb >> 5;
+                    const int64_t wi = (int64_t)(keep_base * 32 + lane) * (BKEY / 32) + cq;
+                    keep_reg = wi < p.mask_words ? __ldg(mask_h + wi) : 0u;
+                }
+                const uint32_t keep_bits = __shfl_sync(0xffffffffu, keep_reg, kb & 31);
                 uint8_t* prow = sP + sb * TILE + (cq >> 1) * ATOM + r_loc * 128;
 #pragma unroll
                 for (int gi = 0; gi < 4; ++gi) {
-                    uint32_t w[4];
+                    uint32_t w[4] = {0u, 0u, 0u, 0u};
+                    if (keep_bits != 0u) {  // the same for every lane: a chunk without a kept token stays 0
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i0 = gi * 8 + 2 * e;
-                        const float p0 = ((keep_bits >> i0) & 1u) ? exp2f(x[i0] - m) * inv_l : 0.f;
-                        const float p1 = ((keep_bits >> (i0 + 1)) & 1u) ? exp2f(x[i0 + 1] - m) * inv_l : 0.f;
-                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-                        w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                        for (int e = 0; e < 4; ++e) {
+                            const int i0 = gi * 8 + 2 * e;
+                            const float p0 = ((keep_bits >> i0) & 1u) ? fast_exp2(x[i0] - b) : 0.f;
+                            const float p1 = ((keep_bits >> (i0 + 1)) & 1u) ? fast_exp2(x[i0 + 1] - b) : 0.f;
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+                            w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                        }
                     }
                     const int gran = (cq & 1) * 4 + gi;
                     *reinterpret_cast<uint4*>(prow + ((gran ^ (r_loc & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
-            // this S buffer may be overwritten
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[sb]);
             if constexpr (C::OUT) {
                 fence_proxy_async_smem();  // the P tile's generic stores before the MMA reads it
                 __syncwarp();
@@ -354,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const float mj = stat[j * BQ + r_loc];
-                    if (mj > -INFINITY) lr += stat[4 * BQ + j * BQ + r_loc] * exp2f(mj - mr);
+                    if (mj > -INFINITY) lr += stat[4 * BQ + j * BQ + r_loc] * fast_exp2(mj - mr);
                 }
                 p.row_m[(int64_t)h * p.n + row] = mr;
                 p.row_l[(int64_t)h * p.n + row] = lr;

@@ -93,6 +93,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// 2^x on the special-function unit (PTX ex2.approx.ftz.f32): one instruction,
+// a few ulp of relative error, results below 2^-126 flushed to 0, 2^-inf = 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // a[i] of every lane -> lane l returns the sum over the warp's lanes of a[l]
 // (a 32 x 32 block with one row per lane, summed down its columns): five
 // exchange rounds, each lane keeping half of its columns -- a fixed tree, so

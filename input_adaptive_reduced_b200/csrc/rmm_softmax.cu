@@ -9,19 +9,25 @@
 // its rows into per-column sums, so the PV op can take them as given scores
 // (RMM_FLAG_GIVEN_SCORES) and skip its score pass.
 //
-// Grid (row blocks of kRows rows, heads), 256 threads.  Thread x owns the
-// 16-byte column groups x, x + 256, ... of every row; a CTA walks its rows in
-// batches (several rows in flight), finds each row's maximum and exponential
-// sum by block reductions, writes P and keeps the squares of the rounded
-// weights in registers (its columns, its rows in row order).  The CTA's column
-// sums go to the workspace; the last CTA of the head adds the row blocks' sums
-// in block order (the same bits on every call) and resets the head's counter.
+// Grid (row blocks of kRows rows, heads), 256 threads, two CTAs per SM.  The
+// op is bound by moving S in and P out, so the rows of S stream into shared
+// memory by bulk copies (cp.async.bulk, kStages stages of R rows; under the
+// causal mask only the first ceil8(i + 1) entries of row i) while the CTA
+// works on earlier rows.  Thread x owns the 16-byte column groups x, x + 256,
+// ... of every row.  Per batch of R rows: the row maxima (warp shuffles, then
+// the 8 warps' maxima in warp order), the exponentials and the row sums (the
+// same two steps), then P and the squares of the stored weights, which the
+// thread keeps in registers (its columns, its rows in row order).  The CTA's
+// column sums go to the workspace; the last CTA of the head adds the row
+// blocks' sums in block order (the same bits on every call) and resets the
+// head's counter.
 #include <cmath>
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "rmm.h"
+#include "rmm_device.cuh"
 #include "rmm_internal.h"
 
 namespace rmm {
@@ -29,130 +35,174 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kRows = 128;  // rows per CTA
+constexpr int kRows = 128;           // rows per CTA
+constexpr int kStages = 4;           // row batches in flight
+constexpr int kStageElems = 8192;    // bf16 entries per stage (16 KB)
+constexpr size_t kSmem = (size_t)kStages * kStageElems * 2;
+constexpr size_t kHeader = 256;      // workspace: error word, then the counters
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-__device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
 
-// E columns per thread per row (t <= kThreads * E), B rows per batch.
-template <int E, int B>
-__global__ void __launch_bounds__(kThreads) softmax_scores_kernel(
+// E columns per thread per row (t <= kThreads * E); R rows per stage.
+template <int E>
+__global__ void __launch_bounds__(kThreads, 2) softmax_scores_kernel(
     const __nv_bfloat16* __restrict__ S, __nv_bfloat16* __restrict__ P, float* __restrict__ s2,
-    float* __restrict__ partials, unsigned* __restrict__ counters, int n, int t, int64_t lds, int64_t stride_s,
-    int64_t ldp, int64_t stride_p, int causal, int row_blocks) {
-    constexpr int V = E / 8;  // 16-byte groups per thread per row
-    __shared__ float red[B][kWarps];
+    float* __restrict__ partials, unsigned* __restrict__ counters, int* err, int n, int t, int64_t lds,
+    int64_t stride_s, int64_t ldp, int64_t stride_p, int causal, int row_blocks) {
+    constexpr int V = E / 8;                       // 16-byte groups per thread per row
+    constexpr int W = kThreads * E;                // entries per staged row
+    constexpr int R = kStageElems / W;             // rows per stage
+    static_assert(R >= 1, "a stage holds at least one row");
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    uint16_t* stage = reinterpret_cast<uint16_t*>(smem_raw);
+    __shared__ uint64_t full[kStages];
+    __shared__ float red_m[2][R][kWarps], red_l[2][R][kWarps];
     __shared__ int last_cta;
-    pdl_wait();
-    pdl_trigger();
+    __shared__ int abort_flag;
     const int h = blockIdx.y, rb = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint16_t* Sh = reinterpret_cast<const uint16_t*>(S) + (int64_t)h * stride_s;
     uint16_t* Ph = reinterpret_cast<uint16_t*>(P) + (int64_t)h * stride_p;
-    const float ninf = -__int_as_float(0x7f800000);
-    constexpr float kLog2e = 1.4426950408889634f;  // scores are taken in base 2: e^x = 2^(x log2 e)
+    constexpr float kLog2e = 1.4426950408889634f;  // e^x = 2^(x log2 e)
+    const int r0 = rb * kRows, r1 = min(n, r0 + kRows);
+    const int batches = (r1 - r0 + R - 1) / R;
+    // entries of row i that are read: all t, or under the causal mask the
+    // 16-byte groups up to the diagonal
+    auto row_len = [&](int row) { return causal ? min(t, (row + 8) & ~7) : t; };
+    auto issue = [&](int j) {
+        const int st = j % kStages;
+        uint32_t bytes = 0;
+        for (int b = 0; b < R; ++b) {
+            const int row = r0 + j * R + b;
+            if (row < r1) bytes += 2u * (uint32_t)row_len(row);
+        }
+        mbar_arrive_expect_tx(&full[st], bytes);
+        for (int b = 0; b < R; ++b) {
+            const int row = r0 + j * R + b;
+            if (row < r1)
+                bulk_load(stage + ((size_t)st * R + b) * W, Sh + (int64_t)row * lds, 2u * row_len(row), &full[st]);
+        }
+    };
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) mbar_init(&full[i], 1);
+        abort_flag = 0;
+        mbar_fence_init();
+    }
+    __syncthreads();
+    pdl_wait();
+    pdl_trigger();
+    if (tid == 0)
+        for (int j = 0; j < min(kStages, batches); ++j) issue(j);
     float acc[E];
 #pragma unroll
     for (int i = 0; i < E; ++i) acc[i] = 0.f;
-    const int r0 = rb * kRows, r1 = min(n, r0 + kRows);
 #pragma unroll 1
-    for (int r = r0; r < r1; r += B) {
-        float x[B][E];
-        float mx[B];
-        bool vin[B][V];  // the 16-byte group holds an entry that is read (not masked)
+    for (int j = 0; j < batches; ++j) {
+        const int st = j % kStages, par = j & 1;
+        const bool got = mbar_wait(&full[st], (uint32_t)(j / kStages) & 1u, &abort_flag, err, kErrTimeoutEpilogue);
+        // this thread's scores (-inf where masked) and their maximum per row
+        float x[R][E];
+        int len[R];
 #pragma unroll
-        for (int b = 0; b < B; ++b) {
-            const int row = r + b;
-            mx[b] = ninf;
+        for (int b = 0; b < R; ++b) {
+            const int row = r0 + j * R + b;
+            len[b] = row < r1 ? row_len(row) : 0;
+            const uint16_t* src = stage + ((size_t)st * R + b) * W;
+            float mx = -INFINITY;
 #pragma unroll
             for (int v = 0; v < V; ++v) {
                 const int c0 = 8 * (tid + kThreads * v);
-                const bool in = row < r1 && c0 < t && (!causal || c0 <= row);
-                vin[b][v] = in;
-                uint4 q = make_uint4(0u, 0u, 0u, 0u);
-                if (in) q = __ldcs(reinterpret_cast<const uint4*>(Sh + (int64_t)row * lds + c0));
-                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-                const bool whole = !causal || c0 + 7 <= row;  // no entry of the group past the diagonal
+                if (c0 < len[b]) {
+                    const uint4 q = *reinterpret_cast<const uint4*>(src + c0);
+                    const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const bool live = in && (whole || c0 + j <= row);
-                    const float y = live ? bf16_bits_to_float((w[j >> 1] >> (16 * (j & 1))) & 0xffffu) * kLog2e
-                                         : ninf;
-                    x[b][8 * v + j] = y;
-                    mx[b] = fmaxf(mx[b], y);
-                }
-            }
-        }
-        // row maxima
+                    for (int i = 0; i < 8; ++i)
+                        x[b][8 * v + i] = __uint_as_float((i & 1) ? (wd[i >> 1] & 0xffff0000u) : (wd[i >> 1] << 16));
+                    if (causal && c0 + 7 > row) {  // the group on the diagonal
 #pragma unroll
-        for (int b = 0; b < B; ++b) {
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) mx[b] = fmaxf(mx[b], __shfl_xor_sync(0xffffffffu, mx[b], o));
-            if (lane == 0) red[b][warp] = mx[b];
-        }
-        __syncthreads();
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-            float m = red[b][0];
-#pragma unroll
-            for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[b][w]);
-            mx[b] = m;
-        }
-        __syncthreads();
-        // exponentials and row sums
-        float sum[B];
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-            sum[b] = 0.f;
-            const bool finite_row = mx[b] > ninf;  // a row without a finite entry is written as zeros
-#pragma unroll
-            for (int v = 0; v < V; ++v) {
-                if (finite_row && vin[b][v]) {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float e = exp2f(x[b][8 * v + j] - mx[b]);  // 2^-inf = 0 where masked
-                        x[b][8 * v + j] = e;
-                        sum[b] += e;
+                        for (int i = 0; i < 8; ++i)
+                            if (c0 + i > row) x[b][8 * v + i] = -INFINITY;
                     }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) x[b][8 * v + j] = 0.f;
+                    for (int i = 0; i < 8; ++i) x[b][8 * v + i] = -INFINITY;
                 }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx = fmaxf(mx, x[b][8 * v + i]);
             }
 #pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) sum[b] += __shfl_xor_sync(0xffffffffu, sum[b], o);
-            if (lane == 0) red[b][warp] = sum[b];
+            for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (lane == 0) red_m[par][b][warp] = mx;
+        }
+        // every thread has read the stage: it may be refilled
+        if (!__syncthreads_and(got)) break;
+        if (tid == 0 && j + kStages < batches) {
+            fence_proxy_async_smem();
+            issue(j + kStages);
+        }
+        // exponentials relative to the row maximum, and the row sums
+#pragma unroll
+        for (int b = 0; b < R; ++b) {
+            float mx = red_m[par][b][0];
+#pragma unroll
+            for (int w = 1; w < kWarps; ++w) mx = fmaxf(mx, red_m[par][b][w]);
+            // a row without a finite entry gets base +inf: all its weights are 0
+            const float base = mx == -INFINITY ? INFINITY : mx * kLog2e;
+            float sm[2] = {0.f, 0.f};
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                const int c0 = 8 * (tid + kThreads * v);
+                if (c0 < len[b]) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float e = fast_exp2(fmaf(x[b][8 * v + i], kLog2e, -base));  // 2^-inf = 0 where masked
+                        x[b][8 * v + i] = e;
+                        sm[i & 1] += e;
+                    }
+                }
+            }
+            float sum = sm[0] + sm[1];
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            if (lane == 0) red_l[par][b][warp] = sum;
         }
         __syncthreads();
+        // P = the exponentials over the row sum, rounded to bf16; the squares of
+        // the stored weights
 #pragma unroll
-        for (int b = 0; b < B; ++b) {
-            float z = 0.f;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) z += red[b][w];
-            sum[b] = z;
-        }
-        __syncthreads();
-        // store P; add the squares of the stored weights
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-            const int row = r + b;
+        for (int b = 0; b < R; ++b) {
+            const int row = r0 + j * R + b;
             if (row >= r1) break;
-            const float inv = sum[b] > 0.f ? 1.0f / sum[b] : 0.f;
+            float sum = red_l[par][b][0];
+#pragma unroll
+            for (int w = 1; w < kWarps; ++w) sum += red_l[par][b][w];
+            const float inv = sum > 0.f ? 1.0f / sum : 0.f;
 #pragma unroll
             for (int v = 0; v < V; ++v) {
                 const int c0 = 8 * (tid + kThreads * v);
                 if (c0 >= t) continue;
-                uint32_t w[4];
+                uint4 out = make_uint4(0u, 0u, 0u, 0u);  // past the causal range: 0
+                if (c0 < len[b]) {
+                    uint32_t wv[4];
 #pragma unroll
-                for (int j = 0; j < 8; j += 2) {
-                    const __nv_bfloat162 p2 = __floats2bfloat162_rn(x[b][8 * v + j] * inv, x[b][8 * v + j + 1] * inv);
-                    const float2 f = __bfloat1622float2(p2);
-                    acc[8 * v + j] += f.x * f.x;
-                    acc[8 * v + j + 1] += f.y * f.y;
-                    w[j >> 1] = *reinterpret_cast<const uint32_t*>(&p2);
+                    for (int i = 0; i < 8; i += 2) {
+                        const __nv_bfloat162 p2 = __floats2bfloat162_rn(x[b][8 * v + i] * inv, x[b][8 * v + i + 1] * inv);
+                        wv[i >> 1] = *reinterpret_cast<const uint32_t*>(&p2);
+                        const float lo = __uint_as_float(wv[i >> 1] << 16), hi = __uint_as_float(wv[i >> 1] & 0xffff0000u);
+                        acc[8 * v + i] = fmaf(lo, lo, acc[8 * v + i]);
+                        acc[8 * v + i + 1] = fmaf(hi, hi, acc[8 * v + i + 1]);
+                    }
+                    out = make_uint4(wv[0], wv[1], wv[2], wv[3]);
                 }
-                *reinterpret_cast<uint4*>(Ph + (int64_t)row * ldp + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4*>(Ph + (int64_t)row * ldp + c0) = out;
             }
         }
     }
@@ -181,13 +231,16 @@ __global__ void __launch_bounds__(kThreads) softmax_scores_kernel(
     if (tid == 0) counters[h] = 0u;
 }
 
-template <int E, int B>
-cudaError_t launch_softmax(const void* S, void* P, float* s2, float* partials, unsigned* counters, int64_t heads,
-                           int64_t n, int64_t t, int64_t lds, int64_t stride_s, int64_t ldp, int64_t stride_p,
-                           int causal, int row_blocks, cudaStream_t s) {
-    return launch_pdl(softmax_scores_kernel<E, B>, dim3((unsigned)row_blocks, (unsigned)heads), dim3(kThreads), 0, s,
+template <int E>
+cudaError_t launch_softmax(const void* S, void* P, float* s2, float* partials, unsigned* counters, int* err,
+                           int64_t heads, int64_t n, int64_t t, int64_t lds, int64_t stride_s, int64_t ldp,
+                           int64_t stride_p, int causal, int row_blocks, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(softmax_scores_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(softmax_scores_kernel<E>, dim3((unsigned)row_blocks, (unsigned)heads), dim3(kThreads), kSmem, s,
                       static_cast<const __nv_bfloat16*>(S), static_cast<__nv_bfloat16*>(P), s2, partials, counters,
-                      (int)n, (int)t, lds, stride_s, ldp, stride_p, causal, row_blocks);
+                      err, (int)n, (int)t, lds, stride_s, ldp, stride_p, causal, row_blocks);
 }
 
 }  // namespace
@@ -198,7 +251,7 @@ extern "C" {
 size_t rmm_softmax_workspace_size(int64_t heads, int64_t n, int64_t t) {
     if (heads < 1 || n < 1 || t < 1) return 0;
     const int64_t row_blocks = (n + rmm::kRows - 1) / rmm::kRows;
-    return rmm::align256(static_cast<size_t>(heads) * sizeof(unsigned)) +
+    return rmm::kHeader + rmm::align256(static_cast<size_t>(heads) * sizeof(unsigned)) +
            rmm::align256(static_cast<size_t>(heads) * row_blocks * t * sizeof(float));
 }
 
@@ -219,21 +272,22 @@ rmm_status rmm_softmax_scores(const void* S, void* P, float* s2, int64_t heads, 
     const size_t need = rmm_softmax_workspace_size(heads, n, t);
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return RMM_ERR_WORKSPACE;
     const int row_blocks = static_cast<int>((n + rmm::kRows - 1) / rmm::kRows);
-    unsigned* counters = static_cast<unsigned*>(ws);
-    float* partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+    int* err = static_cast<int*>(ws);
+    unsigned* counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + rmm::kHeader);
+    float* partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + rmm::kHeader +
                                                rmm::align256(static_cast<size_t>(heads) * sizeof(unsigned)));
     const int causal = (flags & RMM_FLAG_CAUSAL) ? 1 : 0;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (t <= 2048)
-        e = rmm::launch_softmax<8, 4>(S, P, s2, partials, counters, heads, n, t, lds, stride_s, ldp, stride_p, causal,
-                                      row_blocks, s);
+        e = rmm::launch_softmax<8>(S, P, s2, partials, counters, err, heads, n, t, lds, stride_s, ldp, stride_p, causal,
+                                   row_blocks, s);
     else if (t <= 4096)
-        e = rmm::launch_softmax<16, 4>(S, P, s2, partials, counters, heads, n, t, lds, stride_s, ldp, stride_p, causal,
-                                       row_blocks, s);
+        e = rmm::launch_softmax<16>(S, P, s2, partials, counters, err, heads, n, t, lds, stride_s, ldp, stride_p,
+                                    causal, row_blocks, s);
     else
-        e = rmm::launch_softmax<32, 2>(S, P, s2, partials, counters, heads, n, t, lds, stride_s, ldp, stride_p, causal,
-                                       row_blocks, s);
+        e = rmm::launch_softmax<32>(S, P, s2, partials, counters, err, heads, n, t, lds, stride_s, ldp, stride_p,
+                                    causal, row_blocks, s);
     return e == cudaSuccess ? RMM_OK : RMM_ERR_CUDA;
 }
 

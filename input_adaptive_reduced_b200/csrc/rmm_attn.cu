@@ -19,11 +19,14 @@
 // all d_h with exact zeros), as the library's QK op does.
 //
 // One CTA computes 128 query rows of one head: warp 0 loads by TMA (Q once,
-// then K and V blocks of 128 keys, two stages), warp 1 issues tcgen05.mma
-// (S = Q K^T into one of two TMEM buffers; O += P V into a third), and 16
-// row warps, four per TMEM lane quadrant, each own 32 rows x 32 keys of every
-// block (one row per thread): they read their S chunk from TMEM and write P
-// into a swizzled shared tile for the PV product.  Every wait is bounded.
+// then K (and V) blocks of 128 keys, two or three stages), warp 1 issues
+// tcgen05.mma (S = Q K^T into one of two TMEM buffers; O += P V into a
+// third), and the row warps, a quarter of them per TMEM lane quadrant, each
+// own 32 rows x 32 or 64 keys of every block (one row per thread): they read
+// their S chunks from TMEM and, in the output pass, write P as bf16 pairs back
+// into TMEM, where the PV product takes it as its A operand.  The score-only
+// passes fit two CTAs on an SM (8 row warps), the output pass one (16 row
+// warps).  Every wait is bounded.
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -47,9 +50,9 @@ constexpr int BQ = 128;    // query rows per CTA
 constexpr int BKEY = 128;  // keys per block
 constexpr int DH = 128;    // head dimension of Q and K
 constexpr int DV = 128;    // value dimension
-constexpr int kRowWarps = 16;                 // 4 per TMEM lane quadrant, 32 keys each
-constexpr int kThreads = 32 * (2 + kRowWarps);
 constexpr int ATOM = 128 * 128;  // one 64-column swizzle atom of 128 rows (bytes)
+constexpr uint32_t kColO = 256;  // output pass: O accumulator columns
+constexpr uint32_t kColP = 384;  // output pass: two P buffers of BKEY / 2 columns (bf16 pairs)
 constexpr int TILE = 2 * ATOM;   // a 128 x 128 bf16 operand tile
 
 struct __align__(64) AttnParams {
@@ -71,13 +74,23 @@ struct __align__(64) AttnParams {
 template <int MODE>
 struct AttnCfg {
     static constexpr bool OUT = MODE == kOutput;
-    // K (and V) stages: the score-only passes keep four K blocks in flight; the
-    // output pass, whose stages also hold V and which needs two P tiles, two
-    static constexpr int STAGES = OUT ? 2 : 4;
+    // Row warps: RW / 4 per TMEM lane quadrant, each owning CH 32-key chunks of
+    // every key block.  The score-only passes run 8 (64 keys each) with two K
+    // stages, so that two CTAs share an SM; the output pass, whose stages also
+    // hold V and which needs two P tiles, runs 16 (32 keys each), one CTA per SM.
+    static constexpr int RW = OUT ? 16 : 8;
+    static constexpr int CQ = RW / 4;      // key groups per block
+    static constexpr int CH = 4 / CQ;      // 32-key chunks per warp and block
+    static constexpr int NT = 32 * (2 + RW);
+    static constexpr int MINB = OUT ? 1 : 2;  // CTAs per SM
+    static constexpr int STAGES = OUT ? 3 : 2;
     static constexpr int KV_BYTES = OUT ? 2 * TILE : TILE;  // K (and V) of one key block
-    static constexpr int STAT_BYTES = MODE == kRowStats ? 2 * 4 * BQ * 4 : 0;  // per-quarter (m, l) of each row
-    static constexpr size_t SMEM = 1024 + TILE + STAGES * (size_t)KV_BYTES + (OUT ? 2 * TILE : 0) + STAT_BYTES + 256;
-    static constexpr uint32_t TMEM_COLS = OUT ? 512 : 256;  // two S buffers (+ O)
+    static constexpr int STAT_BYTES = MODE == kRowStats ? 2 * CQ * BQ * 4 : 0;  // per-group (m, l) of each row
+    static constexpr size_t SMEM = 1024 + TILE + STAGES * (size_t)KV_BYTES + STAT_BYTES + 256;
+    // TMEM columns: two S buffers [0, 256); output pass: O [256, 384) and two
+    // bf16 P buffers [384, 512), 64 columns each
+    static constexpr uint32_t TMEM_COLS = OUT ? 512 : 256;
+    static_assert(!OUT || CH == 1, "the output pass keeps one mask word per warp and block");
 };
 
 // Query block of CTA b: the longest causal key ranges first.
@@ -97,14 +110,13 @@ __device__ __forceinline__ bool block_used(const uint32_t* used_bits, int kb) {
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(AttnCfg<MODE>::NT, AttnCfg<MODE>::MINB) attn_pass_kernel(const __grid_constant__ AttnParams p) {
     using C = AttnCfg<MODE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;
     uint8_t* sKV = sQ + TILE;                         // STAGES stages: K tile (then V tile)
-    uint8_t* sP = sKV + C::STAGES * C::KV_BYTES;      // 2 P tiles (output pass)
-    float* stat = reinterpret_cast<float*>(sP + (C::OUT ? 2 * TILE : 0));  // [2][4][BQ] (row statistics)
+    float* stat = reinterpret_cast<float*>(sKV + C::STAGES * C::KV_BYTES);  // [2][CQ][BQ] (row statistics)
     uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stat) + C::STAT_BYTES);
     uint64_t* q_full = bars;
     uint64_t* kv_full = bars + 1;                 // [STAGES]
@@ -126,8 +138,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
-            mbar_init(&s_empty[s], kRowWarps);  // one arrival per row warp
-            mbar_init(&p_full[s], kRowWarps);
+            mbar_init(&s_empty[s], C::RW);  // one arrival per row warp
+            mbar_init(&p_full[s], C::RW);
             mbar_init(&p_empty[s], 1);
         }
         mbar_init(o_full, 1);
@@ -158,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
         // which key blocks hold a kept token (the token mask is written by the
         // selection that runs before this pass)
         const uint32_t* w = p.tok_mask + (int64_t)h * p.mask_words;
-        for (int kb0 = warp * 32; kb0 < kb_end; kb0 += kThreads) {
+        for (int kb0 = warp * 32; kb0 < kb_end; kb0 += C::NT) {
             const int kb = kb0 + lane;
             uint32_t any = 0;
             if (kb < kb_end) {
@@ -204,18 +216,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
             constexpr uint32_t idesc_s = umma_idesc(kKindF16, false, BKEY, 128);  // S = Q K^T
             constexpr uint32_t idesc_o = umma_idesc(kKindF16, true, DV, 128);     // O += P V (V MN-major)
             const uint32_t q_addr = smem_u32(sQ);
-            // O += P_j V_j for the j-th used block (P tile j % 2, K/V stage j % 2)
+            // O += P_j V_j for the j-th used block (P buffer j % 2 in TMEM, K/V stage j % STAGES)
             auto pv = [&](uint32_t j) -> bool {
                 const int pb = j & 1;
                 if (!mbar_wait(&p_full[pb], (j >> 1) & 1u, abort_flag, p.err, kErrTimeoutMma)) return false;
                 tc_fence_after();
-                const uint32_t p_addr = smem_u32(sP + pb * TILE);
+                const uint32_t p_tmem = tmem_base + kColP + pb * (BKEY / 2);
                 const uint32_t v_addr = smem_u32(sKV + (j % C::STAGES) * C::KV_BYTES + TILE);
 #pragma unroll
                 for (int kk = 0; kk < BKEY / 16; ++kk) {
-                    const uint64_t adesc = sw128_desc(p_addr + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
                     const uint64_t bdesc = sw128_desc(v_addr + kk * 16 * 128, ATOM, 1024);
-                    umma<kKindF16>(tmem_base + 256, adesc, bdesc, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_ts(tmem_base + kColO, p_tmem + kk * 8, bdesc, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(&p_empty[pb]);
                 umma_commit(&kv_empty[j % C::STAGES]);
@@ -259,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
     } else {
         // ---------------------------------------------------------------- rows
         const int quad = warp & 3;         // TMEM lane quadrant: rows quad*32 .. +32
-        const int cq = (warp - 2) >> 2;    // key quarter: keys cq*32 .. +32 of every block
+        const int cq = (warp - 2) >> 2;    // key group: chunks cq*CH .. +CH of every block
         const int r_loc = quad * 32 + lane;
         const int row = q0 + r_loc;
         const bool row_ok = row < p.n;
@@ -278,36 +289,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
         // output pass: lane j holds this warp's mask word of key block 32 * keep_base + j
         uint32_t keep_reg = 0u;
         int keep_base = -1;
-        uint32_t it = 0;
-        bool ok = true;
-        for (int kb = 0; kb < kb_end && ok; ++kb) {
-            if (!used(kb)) continue;
-            const int sb = it & 1;
-            const uint32_t ph = (it >> 1) & 1u;
-            ++it;
-            if (!mbar_wait(&s_full[sb], ph, abort_flag, p.err, kErrTimeoutEpilogue)) {
-                ok = false;
-                break;
-            }
-            if constexpr (C::OUT) {
-                if (!mbar_wait(&p_empty[sb], ph ^ 1u, abort_flag, p.err, kErrTimeoutEpilogue)) {
-                    ok = false;
-                    break;
-                }
-            }
-            tc_fence_after();
-            const int k0 = kb * BKEY + cq * 32;  // this warp's first key
+        // One 32-key chunk (chunk cc of key block kb, in buffer sb) of this row.
+        auto chunk = [&](int kb, int cc, int sb, const uint32_t (&raw)[32]) {
+            const int k0 = kb * BKEY + cc * 32;  // the chunk's first key
             // which of the 32 keys of this row count: all, none, or some (the
             // diagonal block and the last block)
             const bool all_in = row_ok && k0 + 31 < p.n && (!p.causal || k0 + 31 <= row);
             const bool none_in = !row_ok || k0 >= p.n || (p.causal && k0 > row);
-            uint32_t raw[32];
-            tmem_ld_32x32b_x32(tmem_base + lane_base + sb * BKEY + cq * 32, raw);
-            tmem_ld_wait();
-            // the scores are in registers: this S buffer may be overwritten
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[sb]);
             // x = scale * score, -inf where masked (one uniform test per chunk)
             float x[32];
             if (__all_sync(0xffffffffu, all_in)) {
@@ -348,49 +336,77 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
                 // P masked to the kept tokens, rounded to bf16, into the swizzled P tile
                 if ((kb >> 5) != keep_base) {  // the same for every lane
                     keep_base = kb >> 5;
-                    const int64_t wi = (int64_t)(keep_base * 32 + lane) * (BKEY / 32) + cq;
+                    const int64_t wi = (int64_t)(keep_base * 32 + lane) * (BKEY / 32) + cc;
                     keep_reg = wi < p.mask_words ? __ldg(mask_h + wi) : 0u;
                 }
                 const uint32_t keep_bits = __shfl_sync(0xffffffffu, keep_reg, kb & 31);
-                uint8_t* prow = sP + sb * TILE + (cq >> 1) * ATOM + r_loc * 128;
+                uint32_t w[16];
 #pragma unroll
-                for (int gi = 0; gi < 4; ++gi) {
-                    uint32_t w[4] = {0u, 0u, 0u, 0u};
-                    if (keep_bits != 0u) {  // the same for every lane: a chunk without a kept token stays 0
+                for (int e = 0; e < 16; ++e) w[e] = 0u;
+                if (keep_bits != 0u) {  // the same for every lane: a chunk without a kept token stays 0
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i0 = gi * 8 + 2 * e;
-                            const float p0 = ((keep_bits >> i0) & 1u) ? fast_exp2(x[i0] - b) : 0.f;
-                            const float p1 = ((keep_bits >> (i0 + 1)) & 1u) ? fast_exp2(x[i0 + 1] - b) : 0.f;
-                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-                            w[e] = *reinterpret_cast<const uint32_t*>(&b2);
-                        }
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = ((keep_bits >> (2 * e)) & 1u) ? fast_exp2(x[2 * e] - b) : 0.f;
+                        const float p1 = ((keep_bits >> (2 * e + 1)) & 1u) ? fast_exp2(x[2 * e + 1] - b) : 0.f;
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+                        w[e] = *reinterpret_cast<const uint32_t*>(&b2);
                     }
-                    const int gran = (cq & 1) * 4 + gi;
-                    *reinterpret_cast<uint4*>(prow + ((gran ^ (r_loc & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
+                // keys 2e, 2e + 1 of the chunk -> one 32-bit column of this row's lane
+                tmem_st_32x32b_x16(tmem_base + lane_base + kColP + sb * (BKEY / 2) + cc * 16, w);
+            }
+        };
+        uint32_t it = 0;
+        bool ok = true;
+        for (int kb = 0; kb < kb_end && ok; ++kb) {
+            if (!used(kb)) continue;
+            const int sb = it & 1;
+            const uint32_t ph = (it >> 1) & 1u;
+            ++it;
+            if (!mbar_wait(&s_full[sb], ph, abort_flag, p.err, kErrTimeoutEpilogue)) {
+                ok = false;
+                break;
             }
             if constexpr (C::OUT) {
-                fence_proxy_async_smem();  // the P tile's generic stores before the MMA reads it
+                if (!mbar_wait(&p_empty[sb], ph ^ 1u, abort_flag, p.err, kErrTimeoutEpilogue)) {
+                    ok = false;
+                    break;
+                }
+            }
+            tc_fence_after();
+            uint32_t raw[C::CH][32];
+#pragma unroll
+            for (int c = 0; c < C::CH; ++c)
+                tmem_ld_32x32b_x32(tmem_base + lane_base + sb * BKEY + (cq * C::CH + c) * 32, raw[c]);
+            tmem_ld_wait();
+            // the scores are in registers: this S buffer may be overwritten
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[sb]);
+#pragma unroll
+            for (int c = 0; c < C::CH; ++c) chunk(kb, cq * C::CH + c, sb, raw[c]);
+            if constexpr (C::OUT) {
+                tmem_st_wait();  // this warp's P columns are written before the MMA reads them
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_full[sb]);
             }
         }
         if constexpr (MODE == kRowStats) {
-            // the four key quarters' (m, l) of each row, combined in quarter order;
+            // the key groups' (m, l) of each row, combined in group order;
             // every row warp reaches this barrier once, whether or not a wait gave up
             stat[cq * BQ + r_loc] = m;
-            stat[4 * BQ + cq * BQ + r_loc] = l;
-            asm volatile("bar.sync 1, %0;" ::"n"(32 * kRowWarps) : "memory");
+            stat[C::CQ * BQ + cq * BQ + r_loc] = l;
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * C::RW) : "memory");
             if (cq == 0 && row_ok) {
                 float mr = stat[r_loc];
 #pragma unroll
-                for (int j = 1; j < 4; ++j) mr = fmaxf(mr, stat[j * BQ + r_loc]);
+                for (int j = 1; j < C::CQ; ++j) mr = fmaxf(mr, stat[j * BQ + r_loc]);
                 float lr = 0.f;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < C::CQ; ++j) {
                     const float mj = stat[j * BQ + r_loc];
-                    if (mj > -INFINITY) lr += stat[4 * BQ + j * BQ + r_loc] * fast_exp2(mj - mr);
+                    if (mj > -INFINITY) lr += stat[C::CQ * BQ + j * BQ + r_loc] * fast_exp2(mj - mr);
                 }
                 p.row_m[(int64_t)h * p.n + row] = mr;
                 p.row_l[(int64_t)h * p.n + row] = lr;
@@ -403,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_pass_kernel(const __grid_con
             tc_fence_after();
             uint32_t raw[32];
             if (have && ok) {
-                tmem_ld_32x32b_x32(tmem_base + lane_base + 256 + cq * 32, raw);
+                tmem_ld_32x32b_x32(tmem_base + lane_base + kColO + cq * 32, raw);
                 tmem_ld_wait();
             } else {
 #pragma unroll
@@ -485,7 +501,7 @@ cudaError_t launch_pass(const AttnParams& p, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(attn_pass_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::SMEM);
     if (e != cudaSuccess) return e;
-    return launch_pdl(attn_pass_kernel<MODE>, dim3((unsigned)(p.q_blocks * p.heads)), dim3(kThreads), C::SMEM, s, p);
+    return launch_pdl(attn_pass_kernel<MODE>, dim3((unsigned)(p.q_blocks * p.heads)), dim3(C::NT), C::SMEM, s, p);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }

@@ -242,12 +242,13 @@ RMM_API rmm_status rmm_matmul_ex(const rmm_plan* plan, const void* A, const void
    for c > i (those entries are not read; P is written as 0 there).  Every
    row needs a finite entry.  Sizes: t a multiple of 8, t <= 8192; strides
    multiples of 8 elements, lds and ldp >= t.  workspace: device memory of
-   rmm_softmax_workspace_size(heads, n, t) bytes, 256-byte aligned, zeroed
-   once (cudaMemsetAsync) before its first use; the kernel leaves its
-   counters at zero, and if it gives up waiting for a row of S to arrive in
-   shared memory (about two seconds) it writes a nonzero code into the
-   workspace's first word.  Errors: RMM_ERR_INVALID_ARG / RMM_ERR_UNSUPPORTED /
-   RMM_ERR_WORKSPACE before any launch, RMM_ERR_CUDA if the launch fails. */
+   rmm_softmax_workspace_size(heads, n, t) bytes, 256-byte aligned, its
+   first word (an error word) zeroed once (cudaMemsetAsync) before its first
+   use: if the kernel gives up waiting for a row of S to arrive in shared
+   memory (about two seconds) it writes a nonzero code there.  Two launches:
+   the weights with per-row-block column sums, then their sum in block order.
+   Errors: RMM_ERR_INVALID_ARG / RMM_ERR_UNSUPPORTED / RMM_ERR_WORKSPACE
+   before any launch, RMM_ERR_CUDA if a launch fails. */
 RMM_API size_t rmm_softmax_workspace_size(int64_t heads, int64_t n, int64_t t);
 RMM_API rmm_status rmm_softmax_scores(const void* S, void* P, float* s2, int64_t heads, int64_t n, int64_t t,
                                       int64_t lds, int64_t stride_s, int64_t ldp, int64_t stride_p, uint32_t flags,

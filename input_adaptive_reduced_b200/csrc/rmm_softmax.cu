@@ -9,7 +9,8 @@
 // its rows into per-column sums, so the PV op can take them as given scores
 // (RMM_FLAG_GIVEN_SCORES) and skip its score pass.
 //
-// Grid (row blocks of kRows rows, heads), 256 threads, two CTAs per SM.  The
+// Grid (row blocks of rows_per_cta rows, heads), 256 threads, three CTAs per
+// SM.  The
 // op is bound by moving S in and P out, so the rows of S stream into shared
 // memory by bulk copies (cp.async.bulk, kStages stages of R rows; under the
 // causal mask only the first ceil8(i + 1) entries of row i) while the CTA
@@ -18,9 +19,9 @@
 // the 8 warps' maxima in warp order), the exponentials and the row sums (the
 // same two steps), then P and the squares of the stored weights, which the
 // thread keeps in registers (its columns, its rows in row order).  The CTA's
-// column sums go to the workspace; the last CTA of the head adds the row
-// blocks' sums in block order (the same bits on every call) and resets the
-// head's counter.
+// column sums go to the workspace, and a second kernel (one thread per
+// column) adds the row blocks' sums in block order: the same bits on every
+// call.
 #include <cmath>
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -35,13 +36,23 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kRows = 128;           // rows per CTA
+constexpr int kMaxRows = 128;        // rows per CTA, fewer when the grid would be small
+constexpr int kMinCtas = 512;        // about three CTAs per SM of a 148-SM part
 constexpr int kStages = 4;           // row batches in flight
 constexpr int kStageElems = 8192;    // bf16 entries per stage (16 KB)
 constexpr size_t kSmem = (size_t)kStages * kStageElems * 2;
-constexpr size_t kHeader = 256;      // workspace: error word, then the counters
+constexpr size_t kHeader = 256;      // workspace: error word, then the column partials
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Rows per CTA: 128, halved (down to 16) while the grid has fewer than
+// kMinCtas CTAs.  A function of the sizes alone, so that the workspace size
+// and the launch agree.
+int64_t rows_per_cta(int64_t heads, int64_t n) {
+    int64_t r = kMaxRows;
+    while (r > 16 && heads * ((n + r - 1) / r) < kMinCtas) r /= 2;
+    return r;
+}
 
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
     asm volatile(
@@ -53,10 +64,10 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
 
 // E columns per thread per row (t <= kThreads * E); R rows per stage.
 template <int E>
-__global__ void __launch_bounds__(kThreads, 2) softmax_scores_kernel(
-    const __nv_bfloat16* __restrict__ S, __nv_bfloat16* __restrict__ P, float* __restrict__ s2,
-    float* __restrict__ partials, unsigned* __restrict__ counters, int* err, int n, int t, int64_t lds,
-    int64_t stride_s, int64_t ldp, int64_t stride_p, int causal, int row_blocks) {
+__global__ void __launch_bounds__(kThreads, 3) softmax_scores_kernel(
+    const __nv_bfloat16* __restrict__ S, __nv_bfloat16* __restrict__ P,
+    float* __restrict__ partials, int* err, int n, int t, int64_t lds,
+    int64_t stride_s, int64_t ldp, int64_t stride_p, int causal, int row_blocks, int rows) {
     constexpr int V = E / 8;                       // 16-byte groups per thread per row
     constexpr int W = kThreads * E;                // entries per staged row
     constexpr int R = kStageElems / W;             // rows per stage
@@ -65,14 +76,13 @@ __global__ void __launch_bounds__(kThreads, 2) softmax_scores_kernel(
     uint16_t* stage = reinterpret_cast<uint16_t*>(smem_raw);
     __shared__ uint64_t full[kStages];
     __shared__ float red_m[2][R][kWarps], red_l[2][R][kWarps];
-    __shared__ int last_cta;
     __shared__ int abort_flag;
     const int h = blockIdx.y, rb = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint16_t* Sh = reinterpret_cast<const uint16_t*>(S) + (int64_t)h * stride_s;
     uint16_t* Ph = reinterpret_cast<uint16_t*>(P) + (int64_t)h * stride_p;
     constexpr float kLog2e = 1.4426950408889634f;  // e^x = 2^(x log2 e)
-    const int r0 = rb * kRows, r1 = min(n, r0 + kRows);
+    const int r0 = rb * rows, r1 = min(n, r0 + rows);
     const int batches = (r1 - r0 + R - 1) / R;
     // entries of row i that are read: all t, or under the causal mask the
     // 16-byte groups up to the diagonal
@@ -206,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 2) softmax_scores_kernel(
             }
         }
     }
-    // this CTA's column sums, then the head's last CTA adds them in block order
+    // this CTA's column sums
     float* part = partials + ((int64_t)h * row_blocks + rb) * t;
 #pragma unroll
     for (int v = 0; v < V; ++v) {
@@ -216,31 +226,42 @@ __global__ void __launch_bounds__(kThreads, 2) softmax_scores_kernel(
         __stcg(dst, make_float4(acc[8 * v], acc[8 * v + 1], acc[8 * v + 2], acc[8 * v + 3]));
         __stcg(dst + 1, make_float4(acc[8 * v + 4], acc[8 * v + 5], acc[8 * v + 6], acc[8 * v + 7]));
     }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) last_cta = atomicAdd(counters + h, 1u) == (unsigned)(row_blocks - 1) ? 1 : 0;
-    __syncthreads();
-    if (!last_cta) return;
-    __threadfence();
-    const float* ph = partials + (int64_t)h * row_blocks * t;
-    for (int c = tid; c < t; c += kThreads) {
-        float z = 0.f;
-        for (int j = 0; j < row_blocks; ++j) z += __ldcg(ph + (int64_t)j * t + c);
-        s2[(int64_t)h * t + c] = z;
+}
+
+// s2[h][c] = the row blocks' column sums added in block order (16 loads in
+// flight per thread).
+__global__ void __launch_bounds__(256) softmax_scores_reduce_kernel(const float* __restrict__ partials,
+                                                                    float* __restrict__ s2, int t, int row_blocks) {
+    pdl_wait();
+    pdl_trigger();
+    const int h = blockIdx.y;
+    const int c = blockIdx.x * 256 + threadIdx.x;
+    if (c >= t) return;
+    const float* pc = partials + (int64_t)h * row_blocks * t + c;
+    float z = 0.f;
+    for (int b = 0; b < row_blocks; b += 16) {
+        float v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) v[u] = b + u < row_blocks ? __ldcg(pc + (int64_t)(b + u) * t) : 0.f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) z += v[u];  // the terms past the last block are +0
     }
-    if (tid == 0) counters[h] = 0u;
+    s2[(int64_t)h * t + c] = z;
 }
 
 template <int E>
-cudaError_t launch_softmax(const void* S, void* P, float* s2, float* partials, unsigned* counters, int* err,
-                           int64_t heads, int64_t n, int64_t t, int64_t lds, int64_t stride_s, int64_t ldp,
-                           int64_t stride_p, int causal, int row_blocks, cudaStream_t s) {
+cudaError_t launch_softmax(const void* S, void* P, float* s2, float* partials, int* err, int64_t heads, int64_t n,
+                           int64_t t, int64_t lds, int64_t stride_s, int64_t ldp, int64_t stride_p, int causal,
+                           int row_blocks, int rows, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(softmax_scores_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(softmax_scores_kernel<E>, dim3((unsigned)row_blocks, (unsigned)heads), dim3(kThreads), kSmem, s,
-                      static_cast<const __nv_bfloat16*>(S), static_cast<__nv_bfloat16*>(P), s2, partials, counters,
-                      err, (int)n, (int)t, lds, stride_s, ldp, stride_p, causal, row_blocks);
+    e = launch_pdl(softmax_scores_kernel<E>, dim3((unsigned)row_blocks, (unsigned)heads), dim3(kThreads), kSmem, s,
+                   static_cast<const __nv_bfloat16*>(S), static_cast<__nv_bfloat16*>(P), partials, err, (int)n,
+                   (int)t, lds, stride_s, ldp, stride_p, causal, row_blocks, rows);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(softmax_scores_reduce_kernel, dim3((unsigned)((t + 255) / 256), (unsigned)heads), dim3(256), 0,
+                      s, (const float*)partials, s2, (int)t, row_blocks);
 }
 
 }  // namespace
@@ -250,9 +271,9 @@ extern "C" {
 
 size_t rmm_softmax_workspace_size(int64_t heads, int64_t n, int64_t t) {
     if (heads < 1 || n < 1 || t < 1) return 0;
-    const int64_t row_blocks = (n + rmm::kRows - 1) / rmm::kRows;
-    return rmm::kHeader + rmm::align256(static_cast<size_t>(heads) * sizeof(unsigned)) +
-           rmm::align256(static_cast<size_t>(heads) * row_blocks * t * sizeof(float));
+    const int64_t rows = rmm::rows_per_cta(heads, n);
+    const int64_t row_blocks = (n + rows - 1) / rows;
+    return rmm::kHeader + rmm::align256(static_cast<size_t>(heads) * row_blocks * t * sizeof(float));
 }
 
 rmm_status rmm_softmax_scores(const void* S, void* P, float* s2, int64_t heads, int64_t n, int64_t t, int64_t lds,
@@ -271,23 +292,22 @@ rmm_status rmm_softmax_scores(const void* S, void* P, float* s2, int64_t heads, 
     if (t > 8192 || heads > 65535 || n > (int64_t(1) << 30)) return RMM_ERR_UNSUPPORTED;
     const size_t need = rmm_softmax_workspace_size(heads, n, t);
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return RMM_ERR_WORKSPACE;
-    const int row_blocks = static_cast<int>((n + rmm::kRows - 1) / rmm::kRows);
+    const int rows = static_cast<int>(rmm::rows_per_cta(heads, n));
+    const int row_blocks = static_cast<int>((n + rows - 1) / rows);
     int* err = static_cast<int*>(ws);
-    unsigned* counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + rmm::kHeader);
-    float* partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + rmm::kHeader +
-                                               rmm::align256(static_cast<size_t>(heads) * sizeof(unsigned)));
+    float* partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + rmm::kHeader);
     const int causal = (flags & RMM_FLAG_CAUSAL) ? 1 : 0;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (t <= 2048)
-        e = rmm::launch_softmax<8>(S, P, s2, partials, counters, err, heads, n, t, lds, stride_s, ldp, stride_p, causal,
-                                   row_blocks, s);
+        e = rmm::launch_softmax<8>(S, P, s2, partials, err, heads, n, t, lds, stride_s, ldp, stride_p, causal,
+                                   row_blocks, rows, s);
     else if (t <= 4096)
-        e = rmm::launch_softmax<16>(S, P, s2, partials, counters, err, heads, n, t, lds, stride_s, ldp, stride_p,
-                                    causal, row_blocks, s);
+        e = rmm::launch_softmax<16>(S, P, s2, partials, err, heads, n, t, lds, stride_s, ldp, stride_p,
+                                    causal, row_blocks, rows, s);
     else
-        e = rmm::launch_softmax<32>(S, P, s2, partials, counters, err, heads, n, t, lds, stride_s, ldp, stride_p,
-                                    causal, row_blocks, s);
+        e = rmm::launch_softmax<32>(S, P, s2, partials, err, heads, n, t, lds, stride_s, ldp, stride_p,
+                                    causal, row_blocks, rows, s);
     return e == cudaSuccess ? RMM_OK : RMM_ERR_CUDA;
 }
 

@@ -268,8 +268,10 @@ rmm_status run_product(const rmm_plan* plan, const void* A, const void* B, void*
             // I_inout the one-row select writes no index list
             const bool words_only =
                 plan->decode && p.mode == RMM_PV && plan->select16 && !plan->select_small && !I_inout && !s2_in;
-            st = run_select(plan, A, words_only ? nullptr : I, nullptr, ws, stream, s2_in);
-            if (st != RMM_OK) return st;
+            if (!plan->qk_cluster) {  // (else selected together with the masked copy of Q, below)
+                st = run_select(plan, A, words_only ? nullptr : I, nullptr, ws, stream, s2_in);
+                if (st != RMM_OK) return st;
+            }
         }
     }
     if (p.n == 0 || p.m == 0) return RMM_OK;
@@ -445,7 +447,24 @@ rmm_status run_product(const rmm_plan* plan, const void* A, const void* B, void*
         pm.ld_dst = p.d;
         pm.stride_dst = p.n * p.d;
         pm.heads = static_cast<int>(p.heads);
-        if (rmm::launch_mask_columns(pm, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        if (plan->qk_cluster) {
+            rmm::QkMaskArgs qa{};
+            qa.Q = A;
+            qa.n = p.n;
+            qa.d = p.d;
+            qa.ldq = p.lda;
+            qa.stride_q = p.stride_a;
+            qa.heads = static_cast<int>(p.heads);
+            qa.k = k;
+            qa.I = I;
+            qa.Qm = pm.dst;
+            qa.ldm = pm.ld_dst;
+            qa.stride_m = pm.stride_dst;
+            qa.cluster = plan->qk_cluster;
+            if (rmm::launch_qk_select_mask(qa, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        } else if (rmm::launch_mask_columns(pm, stream) != cudaSuccess) {
+            return RMM_ERR_CUDA;
+        }
         if (!encode_kmajor_map(&gp.map_a, es, pm.dst, p.d, p.n, p.heads, p.d, p.n * p.d, box_k, 128))
             return RMM_ERR_CUDA;
         gp.k = static_cast<int32_t>(p.d);
@@ -617,7 +636,7 @@ int32_t launches_per_call(const rmm_plan* plan) {
     const bool given = (p.flags & RMM_FLAG_USE_GIVEN_INDICES) != 0;
     const bool identity = !given && plan->k == p.d;
     int32_t n = 0;
-    if (!given && !identity && !plan->decode_select)
+    if (!given && !identity && !plan->decode_select && !plan->qk_cluster)  // (QK: with the masked Q below)
         n += (plan->given_scores || plan->fused_select || plan->select16 || plan->select_small) ? 1 : 2;
     if (plan->emit_scores && p.m > 0 && p.n > 0 && !product_on_pairs(plan)) n += 1;  // score pass over Y
     if (p.n == 0 || p.m == 0) return n;
@@ -728,6 +747,11 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     // one bf16 row per head: a counting select over the magnitude bits
     plan->select16 = p->n == 1 && p->dtype == RMM_BF16 && p->d % 8 == 0 && p->d <= 65535;
     plan->select_small = rmm::select_small_fits(p->n, p->d);
+    // QK with a selected I: the scores, the TopK and the masked copy of Q in one launch
+    plan->qk_cluster = p->mode == RMM_QK && plan->need_select && !plan->given_scores && !plan->decode &&
+                               p->n >= 1 && p->m >= 1 && rmm::qk_select_mask_fits(p->dtype, p->d)
+                           ? rmm::qk_select_cluster(p->heads, p->n, sms)
+                           : 0;
     // Row splits for the score pass: enough CTAs to keep HBM busy (about two
     // per SM), at most 16 partials per column, at least 64 rows each.
     const int vec = 16 / plan->es;

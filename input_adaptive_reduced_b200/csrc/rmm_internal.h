@@ -133,6 +133,27 @@ cudaError_t launch_pack(const PackArgs& a, cudaStream_t s);
 // source's shape; used for attention scores, where the product is bound by
 // its output and a zero-masked operand gives the same sum over I).
 cudaError_t launch_mask_columns(const PackArgs& a, cudaStream_t s);
+
+// QK feature selection and the masked copy of Q in one launch (bf16,
+// d <= 256 and a multiple of 8): a cluster of `cluster` CTAs per query head
+// sums the squares of Q's features over its rows, the cluster's first CTA
+// adds the CTAs' sums in rank order through distributed shared memory, takes
+// the TopK (ties to the lower feature), writes I and hands the kept-feature
+// words to the cluster; every CTA then writes its rows of Q with the unkept
+// features zeroed.
+struct QkMaskArgs {
+    const void* Q;          // [heads][n][ldq] bf16
+    int64_t n, d, ldq, stride_q;
+    int heads;
+    int64_t k;
+    int32_t* I;             // [heads][k] out, ascending
+    void* Qm;               // [heads][n][ldm] bf16 out
+    int64_t ldm, stride_m;
+    int cluster;            // CTAs per head: 1, 2, 4 or 8
+};
+bool qk_select_mask_fits(int dtype, int64_t d);
+int qk_select_cluster(int64_t heads, int64_t n, int sms);
+cudaError_t launch_qk_select_mask(const QkMaskArgs& a, cudaStream_t s);
 // dst[h][c][t] = src[h / group][I[h][t]][c]: gathered rows written K-major
 // (rows = number of source columns c; I == nullptr means I[t] = t).
 cudaError_t launch_pack_rows_transposed(const PackArgs& a, cudaStream_t s);
@@ -304,6 +325,7 @@ struct rmm_plan {
     size_t off_split_cnt, off_split;    // its counters (in the header) and fp32 partials
     bool decode;        // bf16 attention with group * n <= 8 query vectors per KV head (rmm_decode.cu)
     bool decode_select; // decode QK: the features are selected inside the product kernel
+    int qk_cluster;     // QK, bf16, d <= 256: selection and masked Q in one cluster launch (CTAs per head), else 0
     int dec_tokens, dec_parts;          // pv: tokens per CTA, token ranges per KV head
     size_t off_dec_cnt, off_dec_mask, off_dec_part;  // pv: counters (header), membership words, partials
     size_t off_kb_keep;                               // masked PV: per-head 64-token blocks holding a kept token

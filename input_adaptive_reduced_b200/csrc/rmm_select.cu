@@ -16,6 +16,7 @@
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
+#include "rmm_device.cuh"
 #include "rmm_internal.h"
 
 namespace rmm {
@@ -475,6 +476,150 @@ __global__ void __launch_bounds__(32 * kSmallWarps) select_small_kernel(const T*
     }
 }
 
+// ------------------------------------------------------------------ QK select + mask
+// One launch for the QK op's feature selection and its masked copy of Q
+// (d <= 256): grid (cluster, heads), a cluster of C CTAs per query head, CTA
+// c owning rows [c R, (c + 1) R).  Thread t sums the squares of the 8
+// features of 16-byte column group t mod (d / 8) over rows t div (d / 8),
+// + G, ... in row order (G row groups); the row groups are added in order
+// in shared memory; the cluster's first CTA adds the C CTAs' sums in rank
+// order through distributed shared memory (the same order for every call),
+// one warp takes the TopK with warp_topk_bits, writes I and stores the
+// kept-feature words into every CTA of the cluster; after a second cluster
+// barrier each CTA writes its rows of Q with the unkept features set to +0.
+constexpr int kQkThreads = 256;
+
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+// (ordered after the cluster barrier by the barrier's own "memory" clobber)
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t cluster_addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr));
+    return v;
+}
+
+__device__ __forceinline__ void st_dsmem_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+template <int J>  // d <= 32 J
+__global__ void __launch_bounds__(kQkThreads, 1) qk_select_mask_kernel(
+    const __nv_bfloat16* __restrict__ Q, int64_t n, int64_t d, int64_t ldq, int64_t stride_q, int64_t k,
+    int32_t* __restrict__ I, __nv_bfloat16* __restrict__ Qm, int64_t ldm, int64_t stride_m, int64_t rows_per_cta) {
+    __shared__ float red[kQkThreads * 8];  // [row group][feature]
+    __shared__ float part[32 * J];         // this CTA's feature sums
+    __shared__ uint32_t keepw[J];          // kept-feature words, from the cluster's first CTA
+    pdl_wait();
+    pdl_trigger();
+    const uint32_t rank = cluster_ctarank(), csize = cluster_nctarank();
+    const int h = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cg = (int)(d / 8);           // 16-byte column groups per row
+    const int groups = kQkThreads / cg;    // row groups
+    const int c = tid % cg, g = tid / cg;
+    const int64_t r0 = (int64_t)rank * rows_per_cta;
+    const int64_t r1 = min(n, r0 + rows_per_cta);
+    const __nv_bfloat16* Qh = Q + (int64_t)h * stride_q;
+    float acc[8];
+#pragma unroll
+    for (int v = 0; v < 8; ++v) acc[v] = 0.f;
+    if (g < groups) {
+        const __nv_bfloat16* base = Qh + c * 8;
+        int64_t r = r0 + g;
+        for (; r + 7 * groups < r1; r += 8 * groups) {  // eight rows in flight, added in row order
+            uint4 q[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) q[u] = __ldg(reinterpret_cast<const uint4*>(base + (r + u * groups) * ldq));
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const float x = __uint_as_float((v & 1) ? (w[v >> 1] & 0xffff0000u) : (w[v >> 1] << 16));
+                    acc[v] = fmaf(x, x, acc[v]);
+                }
+            }
+        }
+        for (; r < r1; r += groups) {
+            const uint4 q = __ldg(reinterpret_cast<const uint4*>(base + r * ldq));
+            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const float x = __uint_as_float((v & 1) ? (w[v >> 1] & 0xffff0000u) : (w[v >> 1] << 16));
+                acc[v] = fmaf(x, x, acc[v]);
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < 8; ++v) red[g * d + c * 8 + v] = acc[v];
+    }
+    __syncthreads();
+    for (int f = tid; f < d; f += kQkThreads) {
+        float sum = red[f];
+        for (int gg = 1; gg < groups; ++gg) sum += red[gg * d + f];
+        part[f] = sum;
+    }
+    cluster_sync_all();  // every CTA's sums are complete and visible to the cluster
+    if (rank == 0 && warp == 0) {
+        uint32_t key[J];
+        bool valid[J];
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int f = lane + 32 * j;
+            valid[j] = f < d;
+            float sum = 0.f;
+            if (valid[j]) {
+                // the C sums loaded together, then added in rank order
+                const uint32_t a = smem_u32(&part[f]);
+                float v[8];
+#pragma unroll
+                for (int cr = 0; cr < 8; ++cr) v[cr] = cr < (int)csize ? ld_dsmem_f32(mapa_shared(a, (uint32_t)cr)) : 0.f;
+#pragma unroll
+                for (int cr = 0; cr < 8; ++cr) sum += v[cr];  // +0 past the cluster's size
+            }
+            key[j] = __float_as_uint(sum);
+        }
+        const uint32_t kept_bits = warp_topk_bits<J>(key, valid, (uint32_t)k, lane);
+        int32_t* Ih = I + (int64_t)h * k;
+        uint32_t before = 0;
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const bool kept = (kept_bits >> j) & 1u;
+            const unsigned b = __ballot_sync(0xffffffffu, kept);
+            if (kept) Ih[before + __popc(b & ((1u << lane) - 1u))] = lane + 32 * j;
+            before += __popc(b);
+            if (lane < (int)csize) st_dsmem_u32(mapa_shared(smem_u32(&keepw[j]), (uint32_t)lane), b);
+        }
+    }
+    cluster_sync_all();  // the kept-feature words are in every CTA of the cluster
+    if (g >= groups) return;
+    // this thread's column group, as in the sums: the AND masks of its 8 features
+    const uint32_t bits = (keepw[c >> 2] >> ((c & 3) * 8)) & 0xffu;  // features 8 c .. 8 c + 7
+    uint32_t am[4];
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+        am[v] = ((bits >> (2 * v)) & 1u ? 0x0000ffffu : 0u) | ((bits >> (2 * v + 1)) & 1u ? 0xffff0000u : 0u);
+    const __nv_bfloat16* src = Qh + c * 8;
+    __nv_bfloat16* dst = Qm + (int64_t)h * stride_m + c * 8;
+    int64_t r = r0 + g;
+    for (; r + 3 * groups < r1; r += 4 * groups) {  // four rows in flight
+        uint4 q[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) q[u] = __ldg(reinterpret_cast<const uint4*>(src + (r + u * groups) * ldq));
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(dst + (r + u * groups) * ldm) =
+                make_uint4(q[u].x & am[0], q[u].y & am[1], q[u].z & am[2], q[u].w & am[3]);
+    }
+    for (; r < r1; r += groups) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(src + r * ldq));
+        *reinterpret_cast<uint4*>(dst + r * ldm) = make_uint4(q.x & am[0], q.y & am[1], q.z & am[2], q.w & am[3]);
+    }
+}
+
 // ------------------------------------------------------------------ one row
 // n = 1, bf16: column j's score is a_j^2, exact in fp32, so two scores are
 // equal exactly when |a_j| are, and they order as |a_j| does, i.e. as the 15
@@ -760,6 +905,46 @@ cudaError_t launch_select16(const SelectArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     return launch_pdl(select16_kernel, dim3(a.heads), dim3(kSel16Threads), smem, s, (const __nv_bfloat16*)a.A, a.d,
                       a.stride_a, a.k, a.I, a.s2, a.mask, a.mask_words);
+}
+
+bool qk_select_mask_fits(int dtype, int64_t d) { return dtype == 0 && d >= 8 && d <= 256 && d % 8 == 0; }
+
+// CTAs per head: about two CTAs per SM over all heads, at least 16 rows each,
+// at most 8 (the portable cluster size).
+int qk_select_cluster(int64_t heads, int64_t n, int sms) {
+    int c = 1;
+    while (c < 8 && heads * c < 2LL * sms && n / (2 * c) >= 16) c *= 2;
+    return c;
+}
+
+template <int J>
+cudaError_t launch_qk_select_mask_j(const QkMaskArgs& a, cudaStream_t s) {
+    const int64_t rows = (a.n + a.cluster - 1) / a.cluster;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)a.cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)a.cluster, (unsigned)a.heads);
+    cfg.blockDim = dim3(kQkThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, qk_select_mask_kernel<J>, (const __nv_bfloat16*)a.Q, a.n, a.d, a.ldq, a.stride_q,
+                              a.k, a.I, (__nv_bfloat16*)a.Qm, a.ldm, a.stride_m, rows);
+}
+
+cudaError_t launch_qk_select_mask(const QkMaskArgs& a, cudaStream_t s) {
+    if (!qk_select_mask_fits(0, a.d) || a.k < 1 || a.k > a.d || a.n < 1 || a.heads < 1 || a.heads > 65535 ||
+        (a.cluster != 1 && a.cluster != 2 && a.cluster != 4 && a.cluster != 8))
+        return cudaErrorInvalidValue;
+    if (a.d <= 64) return launch_qk_select_mask_j<2>(a, s);
+    if (a.d <= 128) return launch_qk_select_mask_j<4>(a, s);
+    return launch_qk_select_mask_j<8>(a, s);
 }
 
 cudaError_t launch_identity(int32_t* I, int64_t k, int heads, cudaStream_t s) {

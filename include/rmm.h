@@ -321,9 +321,9 @@ RMM_API size_t rmm_attention_workspace_size(const rmm_attn_problem* p);
    [heads][n][d_v]: bf16 device memory, 16-byte aligned.  I_out ([heads][k_d])
    and T_out ([heads][k_t]) receive the index sets when not NULL.  workspace:
    device memory of rmm_attention_workspace_size(p) bytes, 256-byte aligned,
-   zeroed once (cudaMemsetAsync) before its first use; the kernels return its
-   counters to zero, and a kernel that gives up on a wait (about two seconds)
-   writes a nonzero code into its first word.  Asynchronous on `stream`.
+   its first word (an error word) zeroed once (cudaMemsetAsync) before its
+   first use: a kernel that gives up on a wait (about two seconds) writes a
+   nonzero code there.  Asynchronous on `stream`.
    Errors: RMM_ERR_INVALID_ARG / RMM_ERR_UNSUPPORTED / RMM_ERR_WORKSPACE before
    any launch, RMM_ERR_CUDA if a launch fails. */
 RMM_API rmm_status rmm_attention(const rmm_attn_problem* p, const void* Q, const void* K, const void* V, void* O,

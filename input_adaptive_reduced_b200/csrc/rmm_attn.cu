@@ -15,8 +15,9 @@
 //              kernel adds the slices in order, and TopK picks T_h;
 //   kOutput    O = sum over the key blocks holding a kept token of
 //              (P masked to T_h, rounded to bf16) V, on the tensor cores.
-// Masked features are zeroed in a copy of Q (the contraction then runs over
-// all d_h with exact zeros), as the library's QK op does.
+// The feature selection and the copy of Q with the unkept features zeroed
+// come from one cluster launch, as in the library's QK op (the contraction
+// then runs over all d_h with exact zeros).
 //
 // One CTA computes 128 query rows of one head: warp 0 loads by TMA (Q once,
 // then K (and V) blocks of 128 keys, two or three stages), warp 1 issues
@@ -517,38 +518,18 @@ int64_t retained(double rho, int64_t d) {
 // Workspace layout of one problem (offsets in bytes, 256-aligned).
 struct AttnLayout {
     int64_t kd, kt, q_blocks, mask_words;
-    int nsplit;
-    int64_t rows_per_split;
-    bool fused_select;
-    size_t err, cnt, part, scores, I, T, qm, rm, rl, cpart, a2, mask, total;
+    size_t err, I, T, qm, rm, rl, cpart, a2, mask, total;
 };
 
-AttnLayout attn_layout(const rmm_attn_problem* p, int sms) {
+AttnLayout attn_layout(const rmm_attn_problem* p) {
     AttnLayout L{};
     L.kd = retained(p->rho_d, p->d_h);
     L.kt = retained(p->rho_t, p->n);
     L.q_blocks = (p->n + BQ - 1) / BQ;
     L.mask_words = (p->n + 31) / 32;
-    L.fused_select = p->n * p->d_h * 2 <= (int64_t(128) << 10);
-    int64_t ns = (2LL * sms + p->heads - 1) / p->heads;
-    const int64_t mx = (p->n + 63) / 64;
-    if (ns > mx) ns = mx;
-    if (ns > 16) ns = 16;
-    if (ns < 1) ns = 1;
-    int64_t rps = (p->n + ns - 1) / ns;
-    rps = (rps + 7) / 8 * 8;
-    if (rps < 8) rps = 8;
-    L.nsplit = static_cast<int>((p->n + rps - 1) / rps);
-    L.rows_per_split = rps;
     size_t off = 0;
     L.err = off;  // error word: a kernel that gave up on a wait records its code
     off += 256;
-    L.cnt = off;  // score-pass counters of the feature selection (zero between calls)
-    off += align256(static_cast<size_t>(p->heads) * sizeof(unsigned));
-    L.part = off;
-    off += align256(static_cast<size_t>(p->heads) * L.nsplit * p->d_h * sizeof(float));
-    L.scores = off;
-    off += align256(static_cast<size_t>(p->heads) * p->d_h * sizeof(float));
     L.I = off;
     off += align256(static_cast<size_t>(p->heads) * L.kd * sizeof(int32_t));
     L.T = off;
@@ -606,8 +587,7 @@ extern "C" {
 
 size_t rmm_attention_workspace_size(const rmm_attn_problem* p) {
     if (rmm::validate_attn(p) != RMM_OK) return 0;
-    const int sms = rmm::device_sms();
-    return rmm::attn_layout(p, sms > 0 ? sms : 148).total;
+    return rmm::attn_layout(p).total;
 }
 
 rmm_status rmm_attention(const rmm_attn_problem* p, const void* Q, const void* K, const void* V, void* O,
@@ -623,7 +603,7 @@ rmm_status rmm_attention(const rmm_attn_problem* p, const void* Q, const void* K
         return RMM_ERR_INVALID_ARG;
     const int sms = device_sms();
     if (sms <= 0) return RMM_ERR_CUDA;
-    const AttnLayout L = attn_layout(p, sms);
+    const AttnLayout L = attn_layout(p);
     if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return RMM_ERR_WORKSPACE;
     uint8_t* w = static_cast<uint8_t*>(ws);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -632,54 +612,37 @@ rmm_status rmm_attention(const rmm_attn_problem* p, const void* Q, const void* K
     int32_t* I = I_out ? I_out : reinterpret_cast<int32_t*>(w + L.I);
     int32_t* T = T_out ? T_out : reinterpret_cast<int32_t*>(w + L.T);
 
-    // 1. features: I_h = TopK of Q_h's column norms
-    SelectArgs sa{};
-    sa.A = Q;
-    sa.dtype = RMM_BF16;
-    sa.n = n;
-    sa.d = p->d_h;
-    sa.lda = p->ldq;
-    sa.stride_a = p->stride_q;
-    sa.heads = H;
-    sa.k = L.kd;
-    sa.I = I;
+    // 1. features: I_h = TopK of Q_h's column norms, and 2. Q with the unkept
+    // features zeroed, in one cluster launch (every feature kept: Q as it is)
     cudaError_t e;
+    const __nv_bfloat16* Qs = static_cast<const __nv_bfloat16*>(Q);
+    int64_t ldqs = p->ldq, stride_qs = p->stride_q;
     if (L.kd == p->d_h) {
         e = launch_identity(I, L.kd, H, s);
-    } else if (L.fused_select) {
-        e = launch_normselect(sa, s);
     } else {
-        sa.partials = reinterpret_cast<float*>(w + L.part);
-        sa.counters = reinterpret_cast<unsigned*>(w + L.cnt);
-        sa.scores = reinterpret_cast<float*>(w + L.scores);
-        sa.nsplit = L.nsplit;
-        sa.rows_per_split = L.rows_per_split;
-        e = launch_colnorm(sa, s);
-        if (e == cudaSuccess) e = launch_topk(sa, s);
+        QkMaskArgs qa{};
+        qa.Q = Q;
+        qa.n = n;
+        qa.d = p->d_h;
+        qa.ldq = p->ldq;
+        qa.stride_q = p->stride_q;
+        qa.heads = H;
+        qa.k = L.kd;
+        qa.I = I;
+        qa.Qm = w + L.qm;
+        qa.ldm = p->d_h;
+        qa.stride_m = n * p->d_h;
+        qa.cluster = qk_select_cluster(H, n, sms);
+        e = launch_qk_select_mask(qa, s);
+        Qs = reinterpret_cast<const __nv_bfloat16*>(w + L.qm);
+        ldqs = p->d_h;
+        stride_qs = n * p->d_h;
     }
     if (e != cudaSuccess) return RMM_ERR_CUDA;
-    // 2. Q with the unkept features zeroed
-    __nv_bfloat16* Qm = reinterpret_cast<__nv_bfloat16*>(w + L.qm);
-    PackArgs pm{};
-    pm.src = Q;
-    pm.dtype = RMM_BF16;
-    pm.rows = n;
-    pm.d = p->d_h;
-    pm.ld_src = p->ldq;
-    pm.stride_src = p->stride_q;
-    pm.group = 1;
-    pm.I = I;
-    pm.I_stride = L.kd;
-    pm.k = L.kd;
-    pm.dst = Qm;
-    pm.ld_dst = p->d_h;
-    pm.stride_dst = n * p->d_h;
-    pm.heads = H;
-    if (launch_mask_columns(pm, s) != cudaSuccess) return RMM_ERR_CUDA;
 
     AttnParams ap;
     std::memset(&ap, 0, sizeof(ap));
-    if (!encode_map(&ap.map_q, Qm, p->d_h, n, H, p->d_h, n * p->d_h) ||
+    if (!encode_map(&ap.map_q, Qs, p->d_h, n, H, ldqs, stride_qs) ||
         !encode_map(&ap.map_k, K, p->d_h, n, p->kv_heads, p->ldk, p->stride_k) ||
         !encode_map(&ap.map_v, V, p->d_v, n, p->kv_heads, p->ldv, p->stride_v))
         return RMM_ERR_CUDA;

@@ -122,8 +122,8 @@ def test_exact_tie_per_head_features(rmm, n):
     duplicated over a dropped one (even heads above it, odd heads below it),
     through each selection path the heads take: n = 2 the decode QK kernel
     selects in-kernel, n = 4 the one-warp-per-head select (select() on
-    [heads, 4, 128]), n = 512 the one-CTA score+select, n = 1024 the score pass
-    and the radix select."""
+    [heads, 4, 128]), n = 512 and n = 1024 the QK op's cluster selection
+    (eight CTAs per head adding their column sums in rank order)."""
     H, Hkv, dh, rho = 8, 2, 128, 0.8
     k = oracle.retained_count(rho, dh)
     nk = max(n, 64)  # keys: a multiple of 8
@@ -487,6 +487,26 @@ def _qk_check(rmm, Q, K, rho, causal):
         g = oracle.kv_head_of(h, H, K.shape[0])
         assert_product_close(S[h], S_ref[h], np.abs(Q64[h][:, I_ref[h]]), np.abs(K64[g][:, I_ref[h]]).T,
                              alpha=alpha, mask=mask)
+
+
+@pytest.mark.parametrize("dh,n,H,Hkv,causal", [
+    (64, 1000, 8, 2, True),    # eight CTAs per head in the selection's cluster, 125 rows each
+    (96, 80, 4, 4, False),     # four CTAs; 12 column groups: 21 row groups, 4 idle threads
+    (256, 520, 2, 1, True),    # eight CTAs per head, eight 32-feature words
+    (128, 40, 64, 8, True),    # many heads, few rows: two CTAs per head
+    (128, 24, 8, 2, False),    # one CTA per head
+])
+def test_qk_cluster_selection(rmm, dh, n, H, Hkv, causal):
+    """The QK op's selection and masked copy of Q in one cluster launch (bf16,
+    d_h <= 256): I bit-exact and S against the oracle across head dims,
+    cluster sizes and ragged row ranges."""
+    rhos = (0.5, 0.8)
+    ks = [oracle.retained_count(r, dh) for r in rhos]
+    (Q, K), _ = gap.enforce_boundary_gaps(
+        lambda g: W.attn_qk(26, n=n, heads=H, kv_heads=Hkv, head_dim=dh, col_gain=g),
+        lambda x: gap.scores_per_head(x[0]), ks)
+    for rho in rhos:
+        _qk_check(rmm, Q, K, rho, causal)
 
 
 @pytest.mark.parametrize("causal", [True, False])

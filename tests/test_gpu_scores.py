@@ -111,7 +111,7 @@ def _causal_logits(seed, H, n, t, causal, device):
 
 
 @pytest.mark.parametrize("H,n,t,causal", [(4, 512, 512, True), (2, 300, 4096, False), (2, 64, 8192, False),
-                                          (3, 1000, 1000, True)])
+                                          (3, 1000, 1000, True), (2, 1100, 1536, True), (1, 2048, 2048, True)])
 def test_softmax_scores(rmm, H, n, t, causal):
     dev = torch.device("cuda")
     S = _causal_logits(74, H, n, t, causal, dev)

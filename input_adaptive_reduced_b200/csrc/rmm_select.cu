@@ -623,89 +623,119 @@ __global__ void __launch_bounds__(kQkThreads, 1) qk_select_mask_kernel(
 // ------------------------------------------------------------------ one row
 // n = 1, bf16: column j's score is a_j^2, exact in fp32, so two scores are
 // equal exactly when |a_j| are, and they order as |a_j| does, i.e. as the 15
-// low bits of a_j's bf16 encoding (for NaN and infinity too).  The TopK is then
-// a counting select over 32768 keys: one pass of 16-bit counts (d <= 65535) in
-// 64 KiB of shared memory, the threshold key T from the counts, and the
-// emission of the kept indices in order (ties at T: the lowest indices), the
-// row re-read from L2.  One 512-thread CTA per head; three fit on an SM.
-constexpr int kSel16Threads = 512;
-constexpr int kSel16Words = 16384;  // 32768 16-bit counts
+// low bits of a_j's bf16 encoding (for NaN and infinity too).  The TopK is
+// then a two-digit radix select over those keys: counts of the high 8 bits
+// find the bin holding the k-th largest key, counts of the low 7 bits among
+// that bin's keys find the key T itself, and the kept columns (above T, then
+// the lowest-indexed keys equal to T) are emitted in order.  A cluster of C
+// CTAs per head splits the row into C ranges of whole 256-key steps; the
+// CTAs add their counts in rank order through distributed shared memory
+// (every CTA finds the same T) and exchange their kept counts to place their
+// output.  256 threads, four CTAs per SM; each pass reads the CTA's range
+// again (from L2).
+constexpr int kRowThreads = 256;
+constexpr int kRowWarps = kRowThreads / 32;
 
-__global__ void __launch_bounds__(kSel16Threads, 3) select16_kernel(const __nv_bfloat16* __restrict__ A, int64_t d,
-                                                                 int64_t stride_a, int64_t k,
-                                                                 int32_t* __restrict__ I, float* __restrict__ s2,
-                                                                 uint32_t* __restrict__ mask, int64_t mask_words) {
+__device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t cluster_addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr));
+    return v;
+}
+
+__global__ void __launch_bounds__(kRowThreads, 4) select16_kernel(const __nv_bfloat16* __restrict__ A, int64_t d,
+                                                               int64_t stride_a, int64_t k,
+                                                               int32_t* __restrict__ I, float* __restrict__ s2,
+                                                               uint32_t* __restrict__ mask, int64_t mask_words,
+                                                               int64_t seg) {
+    __shared__ uint32_t hist[kRowWarps][256];  // per-warp counts; later each warp's staged indices
+    __shared__ uint32_t tot1[256], tot2[128];  // this CTA's counts: high 8 bits, then low 7 bits in the bin
+    __shared__ uint32_t scan_part[kRowWarps];
+    __shared__ uint32_t s_bin, s_above;
+    __shared__ uint32_t cta_cnt[2];            // this CTA's keys above T and equal to T
+    __shared__ uint32_t warp_gt[kRowWarps], warp_eq[kRowWarps], eq_before[kRowWarps], sel_before[kRowWarps];
     pdl_wait();
     pdl_trigger();
-    extern __shared__ uint32_t cnt[];  // count of key 2w in the low half of word w, of key 2w+1 in the high half
-    __shared__ uint32_t part[kSel16Threads / 32];
-    __shared__ uint32_t s_T, s_gt;
-    __shared__ uint32_t warp_gt[kSel16Threads / 32], warp_eq[kSel16Threads / 32];
-    __shared__ uint32_t eq_before[kSel16Threads / 32], sel_before[kSel16Threads / 32];
+    const uint32_t rank = cluster_ctarank(), C = cluster_nctarank();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int h = blockIdx.x;
+    const int h = blockIdx.y;
     const uint16_t* a = reinterpret_cast<const uint16_t*>(A + (int64_t)h * stride_a);
-    for (int w = tid; w < kSel16Words; w += kSel16Threads) cnt[w] = 0u;
-    __syncthreads();
-    // four 16-byte loads in flight per thread, then their 32 counts
+    const int64_t c0 = min(d, (int64_t)rank * seg), c1 = min(d, c0 + seg);  // this CTA's keys (multiples of 8)
     const uint4* a4 = reinterpret_cast<const uint4*>(a);
-    for (int64_t q0 = tid; q0 < d / 8; q0 += 4 * kSel16Threads) {
-        uint4 v[4];
+
+    // counts of bin_of(key) over the CTA's keys into the per-warp histograms
+    // (bin -1: not counted), then summed over the warps into tot[0, bins)
+    auto count = [&](int bins, uint32_t* tot, auto bin_of) {
+        for (int i = tid; i < kRowWarps * 256; i += kRowThreads) (&hist[0][0])[i] = 0u;
+        __syncthreads();
+        for (int64_t q0 = c0 / 8 + tid; q0 < c1 / 8; q0 += 4 * kRowThreads) {
+            uint4 v[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            v[u] = q0 + u * kSel16Threads < d / 8 ? __ldg(a4 + q0 + u * kSel16Threads) : make_uint4(0u, 0u, 0u, 0u);
+            for (int u = 0; u < 4; ++u)
+                v[u] = q0 + u * kRowThreads < c1 / 8 ? __ldg(a4 + q0 + u * kRowThreads) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            if (q0 + u * kSel16Threads >= d / 8) break;
-            const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            for (int u = 0; u < 4; ++u) {
+                if (q0 + u * kRowThreads >= c1 / 8) break;
+                const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const uint32_t k0 = w4[x] & 0x7fffu, k1 = (w4[x] >> 16) & 0x7fffu;
-                atomicAdd(&cnt[k0 >> 1], 1u << ((k0 & 1u) << 4));
-                atomicAdd(&cnt[k1 >> 1], 1u << ((k1 & 1u) << 4));
+                for (int x = 0; x < 8; ++x) {
+                    const int b = bin_of((w4[x >> 1] >> (16 * (x & 1))) & 0x7fffu);
+                    if (b >= 0) atomicAdd(&hist[warp][b], 1u);
+                }
             }
         }
-    }
-    __syncthreads();
-    // thread t owns the 64 keys [32768 - 64 (t + 1), 32768 - 64 t), counted from the top
-    const int w_hi = kSel16Words - 32 * tid;  // its words are [w_hi - 32, w_hi)
-    uint32_t c = 0;
-    for (int w = w_hi - 32; w < w_hi; ++w) c += (cnt[w] & 0xffffu) + (cnt[w] >> 16);
-    const uint32_t incl = warp_incl_scan(c, lane);
-    if (lane == 31) part[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        const uint32_t v = lane < kSel16Threads / 32 ? part[lane] : 0u;
-        const uint32_t pi = warp_incl_scan(v, lane);
-        if (lane < kSel16Threads / 32) part[lane] = pi - v;
-    }
-    __syncthreads();
-    const uint32_t before = part[warp] + incl - c;  // keys above this thread's range
-    if (before < (uint32_t)k && (uint32_t)k <= before + c) {
-        uint32_t run = before;
-        for (int key = 2 * w_hi - 1; key >= 2 * (w_hi - 32); --key) {
-            const uint32_t ck = (cnt[key >> 1] >> ((key & 1) << 4)) & 0xffffu;
-            if (run + ck >= (uint32_t)k) {
-                s_T = (uint32_t)key;
-                s_gt = run;
-                break;
-            }
-            run += ck;
+        __syncthreads();
+        for (int b = tid; b < bins; b += kRowThreads) {
+            uint32_t sum = 0;
+#pragma unroll
+            for (int w = 0; w < kRowWarps; ++w) sum += hist[w][b];
+            tot[b] = sum;
         }
-    }
-    __syncthreads();
-    const uint32_t T = s_T, r = (uint32_t)k - s_gt;  // keys equal to T that are kept
-    // the counts are no longer needed: each warp stages a step's kept indices
-    // in 256 words of their space and writes them out contiguously
-    int32_t* wbuf = reinterpret_cast<int32_t*>(cnt) + warp * 256;
-    // Emission.  Warp w owns a segment of whole 256-key steps; in a step lane l
-    // holds keys [8l, 8l + 8) of it from one 16-byte load (d is a multiple of
-    // 8, so a lane's keys are all in range or all out).  Per lane, bit x of
-    // g / e marks key x above / equal to T; warp prefix sums place them.
-    const int64_t steps = (d + 255) / 256;
-    const int64_t seg = (steps + kSel16Threads / 32 - 1) / (kSel16Threads / 32) * 256;
-    const int64_t beg = (int64_t)warp * seg;
-    const int64_t end = min(d, beg + seg);
+    };
+    // the cluster's count of bin b (thread t takes bin bins - 1 - t), the CTAs
+    // added in rank order; then the largest bin B with above0 + (keys in bins
+    // >= B) >= k: s_bin = B, s_above = above0 + keys in bins > B
+    auto find_bin = [&](int bins, const uint32_t* tot, uint32_t above0) {
+        const int b = bins - 1 - tid;
+        uint32_t g = 0;
+        if (tid < bins) {
+            const uint32_t addr = smem_u32(&tot[b]);
+            for (uint32_t cr = 0; cr < C; ++cr) g += ld_dsmem_u32(mapa_shared(addr, cr));
+        }
+        const uint32_t incl = warp_incl_scan(g, lane);
+        if (lane == 31) scan_part[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const uint32_t v = lane < kRowWarps ? scan_part[lane] : 0u;
+            const uint32_t pi = warp_incl_scan(v, lane);
+            if (lane < kRowWarps) scan_part[lane] = pi - v;
+        }
+        __syncthreads();
+        const uint32_t upto = above0 + scan_part[warp] + incl;  // keys in bins >= b
+        if (tid < bins && upto >= (uint32_t)k && upto - g < (uint32_t)k) {
+            s_bin = (uint32_t)b;
+            s_above = upto - g;
+        }
+        __syncthreads();
+    };
+
+    count(256, tot1, [](uint32_t key) { return (int)(key >> 7); });
+    cluster_sync_all();  // every CTA's high-digit counts are complete
+    find_bin(256, tot1, 0u);
+    const uint32_t B1 = s_bin, above1 = s_above;
+    count(128, tot2, [B1](uint32_t key) { return (key >> 7) == B1 ? (int)(key & 127u) : -1; });
+    cluster_sync_all();  // every CTA's low-digit counts are complete
+    find_bin(128, tot2, above1);
+    const uint32_t T = (B1 << 7) | s_bin, r = (uint32_t)k - s_above;  // the k-th largest key; its ties kept
+
+    // Emission.  Warp w owns a segment of whole 256-key steps of the CTA's
+    // range; in a step lane l holds keys [8l, 8l + 8) of it from one 16-byte
+    // load (d is a multiple of 8, so a lane's keys are all in range or all
+    // out).  Per lane, bit x of g / e marks key x above / equal to T; warp
+    // prefix sums place them, the earlier CTAs' totals place the CTA.
+    const int64_t steps = (c1 - c0 + 255) / 256;
+    const int64_t wseg = (steps + kRowWarps - 1) / kRowWarps * 256;
+    const int64_t beg = c0 + (int64_t)warp * wseg;
+    const int64_t end = min(c1, beg + wseg);
     auto bits_of = [&](const uint4& v, uint32_t& g, uint32_t& e) {
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
         g = 0u;
@@ -734,20 +764,40 @@ __global__ void __launch_bounds__(kSel16Threads, 3) select16_kernel(const __nv_b
         warp_eq[warp] = eq;
     }
     __syncthreads();
+    if (tid == 0) {
+        uint32_t g = 0, e = 0;
+        for (int w = 0; w < kRowWarps; ++w) {
+            g += warp_gt[w];
+            e += warp_eq[w];
+        }
+        cta_cnt[0] = g;
+        cta_cnt[1] = e;
+    }
+    cluster_sync_all();  // every CTA's kept counts are complete
     if (warp == 0) {
-        const uint32_t e = lane < kSel16Threads / 32 ? warp_eq[lane] : 0u;
-        const uint32_t g = lane < kSel16Threads / 32 ? warp_gt[lane] : 0u;
-        const uint32_t eb = warp_incl_scan(e, lane) - e;
-        const uint32_t take = eb >= r ? 0u : min(e, r - eb);
-        const uint32_t sel = g + take;
-        const uint32_t sb = warp_incl_scan(sel, lane) - sel;
-        if (lane < kSel16Threads / 32) {
-            eq_before[lane] = eb;
+        // the ties and the kept columns of the CTAs before this one, in rank order
+        const bool before = lane < (int)rank;
+        const uint32_t ga = before ? ld_dsmem_u32(mapa_shared(smem_u32(&cta_cnt[0]), (uint32_t)lane)) : 0u;
+        const uint32_t ea = before ? ld_dsmem_u32(mapa_shared(smem_u32(&cta_cnt[1]), (uint32_t)lane)) : 0u;
+        const uint32_t eb = warp_incl_scan(ea, lane) - ea;
+        const uint32_t take = eb >= r ? 0u : min(ea, r - eb);
+        const uint32_t eq_cta = __reduce_add_sync(0xffffffffu, ea);
+        const uint32_t sel_cta = __reduce_add_sync(0xffffffffu, ga + take);
+        // then this CTA's warps, in warp order
+        const uint32_t e = lane < kRowWarps ? warp_eq[lane] : 0u;
+        const uint32_t g = lane < kRowWarps ? warp_gt[lane] : 0u;
+        const uint32_t ewb = eq_cta + warp_incl_scan(e, lane) - e;
+        const uint32_t wtake = ewb >= r ? 0u : min(e, r - ewb);
+        const uint32_t sel = g + wtake;
+        const uint32_t sb = sel_cta + warp_incl_scan(sel, lane) - sel;
+        if (lane < kRowWarps) {
+            eq_before[lane] = ewb;
             sel_before[lane] = sb;
         }
     }
-    __syncthreads();
+    cluster_sync_all();  // no CTA reads another's counts after this: each may finish on its own
     uint32_t eq_run = eq_before[warp], sel_run = sel_before[warp];
+    int32_t* wbuf = reinterpret_cast<int32_t*>(hist[warp]);  // this warp's staged indices of a step
     int32_t* Ih = I ? I + (int64_t)h * k : nullptr;  // nullptr: only the membership words are wanted
     for (int64_t b0 = beg; b0 < end; b0 += 256) {
         const int64_t j = b0 + 8 * lane;
@@ -762,12 +812,12 @@ __global__ void __launch_bounds__(kSel16Threads, 3) select16_kernel(const __nv_b
         if (__any_sync(0xffffffffu, e != 0u)) {  // ties at T: the lowest indices are kept
             const uint32_t ec = __popc(e);
             const uint32_t ei = warp_incl_scan(ec, lane);
-            uint32_t rank = eq_run + ei - ec;
+            uint32_t rk = eq_run + ei - ec;
 #pragma unroll
             for (int x = 0; x < 8; ++x)
                 if ((e >> x) & 1u) {
-                    if (rank < r) sel |= 1u << x;
-                    ++rank;
+                    if (rk < r) sel |= 1u << x;
+                    ++rk;
                 }
             eq_run += __shfl_sync(0xffffffffu, ei, 31);
         }
@@ -899,12 +949,33 @@ cudaError_t launch_select_small(const SelectArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_select16(const SelectArgs& a, cudaStream_t s) {
-    if (a.dtype != 0 || a.n != 1 || a.d > 65535 || a.d % 8 != 0) return cudaErrorInvalidValue;
-    const size_t smem = (size_t)kSel16Words * 4;
-    cudaError_t e = cudaFuncSetAttribute(select16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(select16_kernel, dim3(a.heads), dim3(kSel16Threads), smem, s, (const __nv_bfloat16*)a.A, a.d,
-                      a.stride_a, a.k, a.I, a.s2, a.mask, a.mask_words);
+    if (a.dtype != 0 || a.n != 1 || a.d > 65535 || a.d % 8 != 0 || a.heads < 1 || a.heads > 65535)
+        return cudaErrorInvalidValue;
+    // CTAs per head: up to 8, while the heads leave room (about four CTAs per
+    // SM) and every CTA keeps at least 2048 keys
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess)
+        return cudaErrorInvalidValue;
+    int C = 1;
+    while (C < 8 && (int64_t)a.heads * 2 * C <= 4LL * sms && a.d / (2 * C) >= 2048) C *= 2;
+    const int64_t seg = ((a.d + C - 1) / C + 255) / 256 * 256;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)C;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)C, (unsigned)a.heads);
+    cfg.blockDim = dim3(kRowThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, select16_kernel, (const __nv_bfloat16*)a.A, (int64_t)a.d, (int64_t)a.stride_a,
+                              (int64_t)a.k, a.I, a.s2, a.mask, (int64_t)a.mask_words, seg);
 }
 
 bool qk_select_mask_fits(int dtype, int64_t d) { return dtype == 0 && d >= 8 && d <= 256 && d % 8 == 0; }

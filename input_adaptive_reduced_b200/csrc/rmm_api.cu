@@ -752,12 +752,14 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
                                p->n >= 1 && p->m >= 1 && rmm::qk_select_mask_fits(p->dtype, p->d)
                            ? rmm::qk_select_cluster(p->heads, p->n, sms)
                            : 0;
-    // Row splits for the score pass: enough CTAs to keep HBM busy (about two
-    // per SM), at most 16 partials per column, at least 64 rows each.
+    // Row splits for the score pass: as many CTAs as fit on the SMs at once
+    // (two per SM; one CTA more than that would run as a second wave of its
+    // own), at most 16 partials per column, at least 64 rows each.
     const int vec = 16 / plan->es;
     const int64_t colblocks = (p->d + 32 * vec - 1) / (32 * vec);
     const int64_t target = 2LL * sms;
-    int64_t nsplit = (target + colblocks * p->heads - 1) / (colblocks * p->heads);
+    int64_t nsplit = target / (colblocks * p->heads);
+    if (nsplit < 1) nsplit = 1;
     const int64_t max_split = (p->n + 63) / 64;
     if (nsplit > max_split) nsplit = max_split;
     // a causal P: splits of 512 rows, those above a column block end at once

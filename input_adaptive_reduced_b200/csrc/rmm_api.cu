@@ -847,8 +847,8 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     if (plan->emit_scores) {
         // epilogue form: row groups of 32 rows x m per head
         off += align256(static_cast<size_t>(p->heads) * 8 * ((p->n + 255) / 256) * p->m * sizeof(float));
-        // score-pass form: row splits as for a score pass over A
-        int64_t ens = (2LL * sms + y_colblocks * p->heads - 1) / (y_colblocks * p->heads);
+        // score-pass form: row splits as for a score pass over A (one wave)
+        int64_t ens = (2LL * sms) / (y_colblocks * p->heads);
         const int64_t emax = (p->n + 63) / 64;
         if (ens > emax) ens = emax;
         if (ens > 16) ens = 16;

@@ -154,3 +154,51 @@ def test_decode_full(rmm, rho):
     idx = torch.tensor(heads, device=dev)
     assert_heads_close(S[idx], np.stack(S_ref), aS, bS, alpha=alpha)
     assert_heads_close(O[idx], np.stack(O_ref), aO, bO)
+
+
+@pytest.mark.parametrize("n", [2048, 4096])
+def test_fused_attention_full(rmm, n):
+    """The fused RMM attention at the bench's attention point (32 query / 8 KV
+    heads, causal, rho_d = rho_t = 0.8): I bit-exact on every head; on three
+    heads the oracle's three steps in full, T bit-exact where the oracle's
+    token scores are separated at the boundary by more than the fp32 sums'
+    error (n 2^-24 relative) and otherwise differing only in tokens that close
+    to the k-th score, and O on sampled rows within the bound the op derives
+    for its bf16 weights."""
+    H, Hkv, dh, rho = 32, 8, 128, 0.8
+    kd, kt = oracle.retained_count(rho, dh), oracle.retained_count(rho, n)
+    (Q, K), _ = gap.enforce_boundary_gaps(
+        lambda g: W.attn_qk(106, n=n, col_gain=g), lambda x: gap.scores_per_head(x[0]), [kd])
+    V = torch.randn((Hkv, n, 128), generator=W.gen(107)).to(torch.bfloat16)
+    alpha = 1.0 / math.sqrt(dh)
+    dev = torch.device("cuda")
+    O, I, T = rmm.attention(Q.to(dev), K.to(dev), V.to(dev), rho, rho, causal=True, alpha=alpha,
+                            return_sets=True)
+    torch.cuda.synchronize()
+    rmm.check_workspaces()
+    I_all = np.stack([oracle.select(Q[h], k=kd)[0] for h in range(H)])
+    assert_indices_equal(I, I_all)
+    Tg = T.cpu().numpy()
+    rows = sample_rows(n, 5)
+    err = n * 2.0 ** -24
+    compared = 0
+    for h in (0, 13, 31):
+        g = oracle.kv_head_of(h, H, Hkv)
+        O_ref, I_ref, T_ref, P_ref = oracle.rmm_attention(Q[h:h + 1], K[g:g + 1], V[g:g + 1], rho, rho, alpha,
+                                                          True)
+        assert np.array_equal(I_ref[0], I_all[h])
+        a2 = (P_ref[0] ** 2).sum(axis=0)
+        if gap.boundary_gap(a2, kt) >= 2 * err:
+            assert np.array_equal(Tg[h], T_ref[0]), h
+        else:
+            kth = np.sort(a2)[::-1][kt - 1]
+            for t in np.setxor1d(Tg[h], T_ref[0]):
+                assert abs(a2[t] - kth) <= 4 * err * kth, (h, int(t))
+        if not np.array_equal(Tg[h], T_ref[0]):
+            continue  # the output is the oracle's only over the same token set
+        V64 = oracle.as_f64(V[g])
+        absP, absV = np.abs(P_ref[0][rows][:, T_ref[0]]), np.abs(V64[T_ref[0]])
+        fro = max(2e-3, 2.0 ** -8 * np.linalg.norm(absP @ absV) / max(np.linalg.norm(O_ref[0][rows]), 1e-300))
+        assert_product_close(O[h][rows], O_ref[0][rows], absP, absV, rel_fro=fro)
+        compared += 1
+    assert compared >= 1, "no sampled head kept the oracle's token set"

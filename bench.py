@@ -611,6 +611,32 @@ def run_sweep(args):
             out.write(line + "\n")
             out.flush()
 
+    # GPU time of 20 ops replayed from a CUDA graph, so that the host's launch
+    # cost is not what is timed (tiny and decode-sized ops)
+    gs = torch.cuda.Stream(dev)
+
+    def graph_lat(fn, reps=20):
+        with torch.cuda.stream(gs):
+            for _ in range(3):
+                fn()
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=gs):
+            for _ in range(reps):
+                fn()
+        best = float("inf")
+        for _ in range(5):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(gs)
+            with torch.cuda.stream(gs):
+                g.replay()
+            b.record(gs)
+            torch.cuda.synchronize(dev)
+            best = min(best, a.elapsed_time(b) / reps)
+        del g
+        return best
+
     def linear_points(cfg, name, A, B, rhos):
         n, d = A.shape
         m = B.shape[1]
@@ -624,9 +650,14 @@ def run_sweep(args):
             hbm = 2.0 * (n * d + k * m + n * m)  # A once, retained B rows once, Y
             bound = "tensor" if n >= 512 else "hbm"
             frac = (flops / (t * 1e-3) / 1e12) / peak_tf if bound == "tensor" else (hbm / (t * 1e-3) / 1e9) / peak_gbs
+            rec = {}
+            if cfg == 1:  # a few microseconds of GPU work: the op and cuBLAS replayed from graphs too
+                Y = torch.empty((n, m), dtype=A.dtype, device=dev)
+                rec = {"ms_gpu_graph": graph_lat(lambda: rmm.matmul(A, B, rho=rho, out=Y)),
+                       "ms_dense_gpu_graph": graph_lat(lambda: torch.matmul(A, B, out=Y))}
             emit({"config": cfg, "op": name, "n": n, "d": d, "m": m, "rho": rho, "k": k, "ms": t,
                   "useful_tflops": flops / (t * 1e-3) / 1e12, "gbs": hbm / (t * 1e-3) / 1e9,
-                  "bound": bound, "frac": frac, "ms_dense_cublas": t_dense})
+                  "bound": bound, "frac": frac, "ms_dense_cublas": t_dense, **rec})
 
     # 1: tiny fp32
     if want(1, "fp32", 64):
@@ -687,32 +718,7 @@ def run_sweep(args):
         del P, V, Vr
     # decode step: one query row per head against t cached tokens (Llama-3.1-8B
     # attention: 32 / 8 heads, d_h = d_v = 128, `batch` sequences); GPU time of
-    # 20 ops replayed from a CUDA graph, so that the host's launch cost is not
-    # what is timed
-    gs = torch.cuda.Stream(dev)
-
-    def graph_lat(fn, reps=20):
-        with torch.cuda.stream(gs):
-            for _ in range(3):
-                fn()
-        torch.cuda.synchronize(dev)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=gs):
-            for _ in range(reps):
-                fn()
-        best = float("inf")
-        for _ in range(5):
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(gs)
-            with torch.cuda.stream(gs):
-                g.replay()
-            b.record(gs)
-            torch.cuda.synchronize(dev)
-            best = min(best, a.elapsed_time(b) / reps)
-        del g
-        return best
-
+    # 20 ops replayed from a CUDA graph
     for batch, t in ((1, 4096), (8, 4096), (8, 32768), (16, 32768)):
         key = f"{batch}x{t}"
         if not (want("decode", "qk", key) or want("decode", "pv", key)):

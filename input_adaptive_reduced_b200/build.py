@@ -12,7 +12,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "librmm.so")
 SOURCES = ["rmm_api.cu", "rmm_select.cu", "rmm_pack.cu", "rmm_gemm.cu", "rmm_skinny.cu", "rmm_static.cu",
-           "rmm_selftest.cu", "rmm_decode.cu", "rmm_softmax.cu", "rmm_attn.cu"]
+           "rmm_selftest.cu", "rmm_decode.cu", "rmm_softmax.cu", "rmm_attn.cu",
+           "rmm_tiny.cu"]
 HEADERS = ["rmm_device.cuh", "rmm_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

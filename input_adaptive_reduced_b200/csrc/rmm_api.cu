@@ -256,6 +256,28 @@ rmm_status run_product(const rmm_plan* plan, const void* A, const void* B, void*
     const int es = plan->es;
     const int64_t k = plan->k;
 
+    if (plan->tiny) {  // scores, TopK and product in one launch
+        rmm::TinyArgs ta{};
+        ta.A = static_cast<const float*>(A);
+        ta.B = static_cast<const float*>(B);
+        ta.Y = static_cast<float*>(Y);
+        ta.I_out = given ? nullptr : I_inout;
+        ta.I_given = given ? I_inout : nullptr;
+        ta.n = static_cast<int>(p.n);
+        ta.d = static_cast<int>(p.d);
+        ta.m = static_cast<int>(p.m);
+        ta.k = static_cast<int>(k);
+        ta.lda = p.lda;
+        ta.ldb = p.ldb;
+        ta.ldy = p.ldy;
+        ta.alpha = p.alpha;
+        const bool traced = plan->product_start && plan->product_stop;
+        if (traced && cudaEventRecord(plan->product_start, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        if (rmm::launch_tiny(ta, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        if (traced && cudaEventRecord(plan->product_stop, stream) != cudaSuccess) return RMM_ERR_CUDA;
+        return RMM_OK;
+    }
+
     // ---- index set
     int32_t* I = I_inout ? I_inout : ws_at<int32_t>(ws, plan->off_I);
     const bool identity = !given && k == p.d;
@@ -636,6 +658,7 @@ int32_t launches_per_call(const rmm_plan* plan) {
     const bool given = (p.flags & RMM_FLAG_USE_GIVEN_INDICES) != 0;
     const bool identity = !given && plan->k == p.d;
     int32_t n = 0;
+    if (plan->tiny) return 1;  // scores, TopK and product in one launch
     if (!given && !identity && !plan->decode_select && !plan->qk_cluster)  // (QK: with the masked Q below)
         n += (plan->given_scores || plan->fused_select || plan->select16 || plan->select_small) ? 1 : 2;
     if (plan->emit_scores && p.m > 0 && p.n > 0 && !product_on_pairs(plan)) n += 1;  // score pass over Y
@@ -698,6 +721,8 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     // product with swapped operands instead of staging it.
     plan->skinny = p->mode == RMM_LINEAR && p->dtype == RMM_BF16 && p->heads == 1 && p->n >= 1 && p->n <= 64 &&
                    p->m >= 1;
+    plan->tiny = rmm::tiny_fits(*p, plan->k);
+    if (plan->tiny) plan->pack_b = false;
     if (plan->skinny) {
         plan->pack_b = false;
         plan->sk_np = rmm::skinny_pad(p->n);

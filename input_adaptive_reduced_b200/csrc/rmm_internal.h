@@ -7,6 +7,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "rmm.h"
+
 namespace rmm {
 
 // ---------------------------------------------------------------- launches
@@ -141,6 +143,23 @@ cudaError_t launch_mask_columns(const PackArgs& a, cudaStream_t s);
 // the TopK (ties to the lower feature), writes I and hands the kept-feature
 // words to the cluster; every CTA then writes its rows of Q with the unkept
 // features zeroed.
+// The whole op in one launch for tiny fp32 problems (LINEAR, one head,
+// n <= kTinyMaxRows, d <= 256, a selected or given index set): scores, TopK
+// and an fp32 FMA product.
+constexpr int kTinyMaxRows = 64;
+struct TinyArgs {
+    const float* A;
+    const float* B;
+    float* Y;
+    int32_t* I_out;          // [k] out, or nullptr
+    const int32_t* I_given;  // [k] in (RMM_FLAG_USE_GIVEN_INDICES), or nullptr
+    int n, d, m, k;
+    int64_t lda, ldb, ldy;
+    float alpha;
+};
+bool tiny_fits(const rmm_problem& p, int64_t k);  // k: the plan's index count
+cudaError_t launch_tiny(const TinyArgs& a, cudaStream_t s);
+
 struct QkMaskArgs {
     const void* Q;          // [heads][n][ldq] bf16
     int64_t n, d, ldq, stride_q;
@@ -319,6 +338,7 @@ struct rmm_plan {
     size_t header_bytes;  // zeroed by rmm_workspace_init: error word + colnorm counters
     cudaEvent_t product_start, product_stop;  // tracing hook, may be null
     bool skinny;        // n <= 64 bf16 LINEAR: swapped-operand split-K product
+    bool tiny;          // tiny fp32 LINEAR: the whole op in one launch (tiny_fits)
     int sk_np, sk_splits;
     bool pv_mask;       // bf16 PV with a selected T: V's unkept rows zeroed per query head, P read as stored
     int split_tiles, split_f;           // split tail of the CTA-pair product (0, 1: none)

@@ -43,12 +43,39 @@ def _linear_case(rmm, A, B, rho, rows=None):
 @pytest.mark.parametrize("rho", [0.25, 0.5, 1.0])
 @pytest.mark.parametrize("seed", [1, 2])
 def test_linear_fp32_tiny(rmm, rho, seed):
-    """64 x 256 x 256 fp32 (tf32 tensor cores), all sorted scores >= 1e-3 apart."""
+    """64 x 256 x 256 fp32 (the one-launch tiny kernel: scores, TopK and an fp32
+    FMA product), all sorted scores >= 1e-3 apart."""
     A, B = W.linear_small(seed)
     g = gap.all_gaps_gain(oracle.column_scores_sq(A))
     A, B = W.linear_small(seed, col_gain=g)
     assert gap.min_adjacent_gap(oracle.column_scores_sq(A)) >= 1e-3
     _linear_case(rmm, A, B, rho)
+
+
+@pytest.mark.parametrize("n,d,m,rho", [(1, 100, 72, 0.5), (17, 256, 300, 0.8), (64, 64, 4, 0.9),
+                                       (64, 252, 132, 0.3), (40, 4, 8, 0.5)])
+def test_tiny_fp32_shapes(rmm, n, d, m, rho):
+    """The one-launch fp32 kernel across its limits: one row, d up to 256 with
+    ragged 32-column words, one 16-byte group of output columns, several
+    32-column and 16-row CTAs, k = 2; then with a given index set, a scale and
+    a padded row stride of A."""
+    k = oracle.retained_count(rho, d)
+    (A, B), _ = gap.enforce_boundary_gaps(lambda g: W.linear_small(61, n=n, d=d, m=m, col_gain=g),
+                                          lambda x: gap.scores_2d(x[0]), [k])
+    p = rmm.rmm_problem_init(rmm.RMM_LINEAR, rmm.RMM_F32, n, d, m)
+    p.rho = rho
+    assert rmm.Plan(p).kernel_launches == 1
+    _linear_case(rmm, A, B, rho)
+    dev = torch.device("cuda")
+    I = torch.from_numpy(np.sort(np.random.default_rng(d).choice(d, size=k, replace=False)).astype(np.int32))
+    Apad = torch.zeros((n, d + 4), dtype=torch.float32)
+    Apad[:, :d] = A
+    Y = rmm.matmul(Apad.to(dev)[:, :d], B.to(dev), indices=I.to(dev), alpha=0.375)
+    torch.cuda.synchronize()
+    A64, B64 = oracle.as_f64(A), oracle.as_f64(B)
+    I64 = I.numpy()
+    assert_product_close(Y, 0.375 * oracle.reduced_product(A64, B64, I64), np.abs(A64[:, I64]), np.abs(B64[I64]),
+                         alpha=0.375)
 
 
 @pytest.mark.parametrize("direction", ["copy_up", "copy_down"])

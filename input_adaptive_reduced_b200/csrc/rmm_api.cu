@@ -769,7 +769,7 @@ rmm_status rmm_plan_create(rmm_plan** out, const rmm_problem* p, size_t* workspa
     const size_t head_bytes = static_cast<size_t>(p->n) * p->d * plan->es;
     plan->fused_select = p->dtype != RMM_FP8_E4M3 && head_bytes <= kFusedSelectBytes &&
                          rmm::normselect_smem_bytes(p->d, p->dtype) <= 180 * 1024;
-    // one bf16 row per head: a counting select over the magnitude bits
+    // one bf16 row per head: a radix select over the magnitude bits
     plan->select16 = p->n == 1 && p->dtype == RMM_BF16 && p->d % 8 == 0 && p->d <= 65535;
     plan->select_small = rmm::select_small_fits(p->n, p->d);
     // QK with a selected I: the scores, the TopK and the masked copy of Q in one launch

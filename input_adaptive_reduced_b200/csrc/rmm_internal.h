@@ -107,8 +107,9 @@ cudaError_t launch_normselect(const SelectArgs& a, cudaStream_t s);
 // d <= 256 columns, n <= 8 rows: one warp per head ranks the columns.
 bool select_small_fits(int64_t n, int64_t d);
 cudaError_t launch_select_small(const SelectArgs& a, cudaStream_t s);
-// n = 1 bf16 rows (d <= 65535, a multiple of 8): a counting select over the
-// 15 magnitude bits, the same I as the fp32 score path.
+// n = 1 bf16 rows (d <= 65535, a multiple of 8): a two-digit radix select over
+// the 15 magnitude bits on a cluster of CTAs per head, the same I as the fp32
+// score path.
 cudaError_t launch_select16(const SelectArgs& a, cudaStream_t s);
 // I[h][j] = j for j < k (k == d: every index kept).
 cudaError_t launch_identity(int32_t* I, int64_t k, int heads, cudaStream_t s);
@@ -326,7 +327,7 @@ struct rmm_plan {
     int group;          // heads / kv_heads
     bool need_select;   // scores + TopK on each call
     bool fused_select;  // one-kernel selection
-    bool select16;      // n = 1 bf16: the counting select over magnitude bits
+    bool select16;      // n = 1 bf16: the radix select over magnitude bits (a cluster per head)
     bool select_small;  // d <= 256, n <= 8: one warp per head ranks the columns
     int nsplit;
     int64_t rows_per_split;

@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kTinyThreads) tiny_rmm_kernel(const float* __r
     }
     cp_async_wait_all();
     __syncthreads();
-    if (I_given) {
+    if (I_given) {  // an index outside [0, d) (a caller's error) reads nothing and adds nothing
         for (int t = tid; t < k; t += kTinyThreads) sI[t] = __ldg(I_given + t);
     } else {
         // column scores: thread f sums column f in row order
@@ -87,15 +87,16 @@ __global__ void __launch_bounds__(kTinyThreads) tiny_rmm_kernel(const float* __r
     // 16-byte group is all inside or all past the last column)
     for (int e = tid; e < k * (kTinyCols / 4); e += kTinyThreads) {
         const int t = e >> 3, c = (e & 7) * 4;
-        const bool in = c0 + c < m;  // else the copy fills zeros
-        cp_async_16(smem_u32(sB + t * kTinyCols + c), B + (int64_t)sI[t] * ldb + (in ? c0 + c : 0), in ? 16u : 0u);
+        const bool in = c0 + c < m && sI[t] >= 0 && sI[t] < d;  // else the copy fills zeros
+        cp_async_16(smem_u32(sB + t * kTinyCols + c), in ? B + (int64_t)sI[t] * ldb + c0 + c : B, in ? 16u : 0u);
     }
     cp_async_wait_all();
     __syncthreads();
     // this CTA's rows of A[:, I], contiguous (k <= 256 floats a row)
     for (int e = tid; e < kTinyRows * k; e += kTinyThreads) {
         const int rl = e / k, t = e - rl * k;
-        sAk[rl * 32 * J + t] = r0 + rl < n ? sA[(r0 + rl) * d + sI[t]] : 0.f;
+        const int j = sI[t];
+        sAk[rl * 32 * J + t] = r0 + rl < n && j >= 0 && j < d ? sA[(r0 + rl) * d + j] : 0.f;
     }
     __syncthreads();
     // Y[r, c0 + 2 g .. + 1] = alpha sum_t A[r, I_t] B[I_t, c0 + 2 g .. + 1], t ascending

@@ -662,19 +662,26 @@ __global__ void __launch_bounds__(kRowThreads, 4) select16_kernel(const __nv_bfl
     const int64_t c0 = min(d, (int64_t)rank * seg), c1 = min(d, c0 + seg);  // this CTA's keys (multiples of 8)
     const uint4* a4 = reinterpret_cast<const uint4*>(a);
 
-    // counts of bin_of(key) over the CTA's keys into the per-warp histograms
-    // (bin -1: not counted), then summed over the warps into tot[0, bins)
+    // Warp w owns a segment of whole 256-key steps of the CTA's range, the
+    // same in every pass, so that its counts also place its output.
+    const int64_t steps = (c1 - c0 + 255) / 256;
+    const int64_t wseg = (steps + kRowWarps - 1) / kRowWarps * 256;
+    const int64_t beg = min(c1, c0 + (int64_t)warp * wseg);
+    const int64_t end = min(c1, beg + wseg);
+    // counts of bin_of(key) over the warp's keys into its histogram (bin -1:
+    // not counted; four 16-byte loads in flight per lane), then summed over
+    // the warps into tot[0, bins)
     auto count = [&](int bins, uint32_t* tot, auto bin_of) {
         for (int i = tid; i < kRowWarps * 256; i += kRowThreads) (&hist[0][0])[i] = 0u;
         __syncthreads();
-        for (int64_t q0 = c0 / 8 + tid; q0 < c1 / 8; q0 += 4 * kRowThreads) {
+        for (int64_t q0 = beg / 8 + lane; q0 < end / 8; q0 += 4 * 32) {
             uint4 v[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                v[u] = q0 + u * kRowThreads < c1 / 8 ? __ldg(a4 + q0 + u * kRowThreads) : make_uint4(0u, 0u, 0u, 0u);
+                v[u] = q0 + u * 32 < end / 8 ? __ldg(a4 + q0 + u * 32) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                if (q0 + u * kRowThreads >= c1 / 8) break;
+                if (q0 + u * 32 >= end / 8) break;
                 const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
                 for (int x = 0; x < 8; ++x) {
@@ -690,6 +697,12 @@ __global__ void __launch_bounds__(kRowThreads, 4) select16_kernel(const __nv_bfl
             for (int w = 0; w < kRowWarps; ++w) sum += hist[w][b];
             tot[b] = sum;
         }
+    };
+    // the warp's keys in bins above b0 (and, with eq, the count of bin b0)
+    auto warp_above = [&](int bins, uint32_t b0) {
+        uint32_t c = 0;
+        for (int b = lane; b < bins; b += 32) c += (uint32_t)b > b0 ? hist[warp][b] : 0u;
+        return __reduce_add_sync(0xffffffffu, c);
     };
     // the cluster's count of bin b (thread t takes bin bins - 1 - t), the CTAs
     // added in rank order; then the largest bin B with above0 + (keys in bins
@@ -722,20 +735,20 @@ __global__ void __launch_bounds__(kRowThreads, 4) select16_kernel(const __nv_bfl
     cluster_sync_all();  // every CTA's high-digit counts are complete
     find_bin(256, tot1, 0u);
     const uint32_t B1 = s_bin, above1 = s_above;
+    const uint32_t gt_hi = warp_above(256, B1);  // this warp's keys in higher bins
     count(128, tot2, [B1](uint32_t key) { return (key >> 7) == B1 ? (int)(key & 127u) : -1; });
     cluster_sync_all();  // every CTA's low-digit counts are complete
     find_bin(128, tot2, above1);
-    const uint32_t T = (B1 << 7) | s_bin, r = (uint32_t)k - s_above;  // the k-th largest key; its ties kept
+    const uint32_t B2 = s_bin;
+    const uint32_t T = (B1 << 7) | B2, r = (uint32_t)k - s_above;  // the k-th largest key; its ties kept
+    // this warp's keys above T and equal to T, from its histograms
+    const uint32_t gt_w = gt_hi + warp_above(128, B2), eq_w = hist[warp][B2];
 
-    // Emission.  Warp w owns a segment of whole 256-key steps of the CTA's
-    // range; in a step lane l holds keys [8l, 8l + 8) of it from one 16-byte
-    // load (d is a multiple of 8, so a lane's keys are all in range or all
-    // out).  Per lane, bit x of g / e marks key x above / equal to T; warp
-    // prefix sums place them, the earlier CTAs' totals place the CTA.
-    const int64_t steps = (c1 - c0 + 255) / 256;
-    const int64_t wseg = (steps + kRowWarps - 1) / kRowWarps * 256;
-    const int64_t beg = c0 + (int64_t)warp * wseg;
-    const int64_t end = min(c1, beg + wseg);
+    // Emission.  In a 256-key step of its segment lane l holds keys [8l, 8l + 8)
+    // from one 16-byte load (d is a multiple of 8, so a lane's keys are all in
+    // range or all out).  Per lane, bit x of g / e marks key x above / equal
+    // to T; warp prefix sums place them, the warps' and the earlier CTAs'
+    // totals place the warp.
     auto bits_of = [&](const uint4& v, uint32_t& g, uint32_t& e) {
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
         g = 0u;
@@ -747,21 +760,9 @@ __global__ void __launch_bounds__(kRowThreads, 4) select16_kernel(const __nv_bfl
             e |= (uint32_t)(k0 == T) << (2 * u) | (uint32_t)(k1 == T) << (2 * u + 1);
         }
     };
-    uint32_t gt = 0, eq = 0;
-    for (int64_t b0 = beg; b0 < end; b0 += 256) {
-        const int64_t j = b0 + 8 * lane;
-        if (j < end) {
-            uint32_t g, e;
-            bits_of(__ldg(reinterpret_cast<const uint4*>(a + j)), g, e);
-            gt += __popc(g);
-            eq += __popc(e);
-        }
-    }
-    gt = __reduce_add_sync(0xffffffffu, gt);
-    eq = __reduce_add_sync(0xffffffffu, eq);
     if (lane == 0) {
-        warp_gt[warp] = gt;
-        warp_eq[warp] = eq;
+        warp_gt[warp] = gt_w;
+        warp_eq[warp] = eq_w;
     }
     __syncthreads();
     if (tid == 0) {

@@ -52,14 +52,14 @@ constexpr int BKEY = 128;  // keys per block
 constexpr int DH = 128;    // head dimension of Q and K
 constexpr int DV = 128;    // value dimension
 constexpr int ATOM = 128 * 128;  // one 64-column swizzle atom of 128 rows (bytes)
-constexpr uint32_t kColO = 256;  // output pass: O accumulator columns
-constexpr uint32_t kColP = 384;  // output pass: two P buffers of BKEY / 2 columns (bf16 pairs)
+constexpr uint32_t kColO = 128;  // output pass: O accumulator columns (S and then P in [0, 128))
 constexpr int TILE = 2 * ATOM;   // a 128 x 128 bf16 operand tile
 
 struct __align__(64) AttnParams {
     CUtensorMap map_q;  // masked Q: {d_h, n, heads}, box {64, 128, 1}
-    CUtensorMap map_k;  // K: {d_h, n, kv_heads}, box {64, 128, 1}
-    CUtensorMap map_v;  // V: {d_v, n, kv_heads}, box {64, 128, 1}
+    CUtensorMap map_k;   // K: {d_h, n, kv_heads}, box {64, 128, 1} (score passes)
+    CUtensorMap map_kh;  // output pass: K with a {64, 64, 1} box (half a key block)
+    CUtensorMap map_vh;  // output pass: V {d_v, n, kv_heads} with a {64, 64, 1} box
     __nv_bfloat16* O;   // [heads][n][ldo]
     int64_t ldo, stride_o;
     float* row_m;       // [heads][n]: maximum of the row's scaled scores (base-2 units)
@@ -76,22 +76,26 @@ template <int MODE>
 struct AttnCfg {
     static constexpr bool OUT = MODE == kOutput;
     // Row warps: RW / 4 per TMEM lane quadrant, each owning CH 32-key chunks of
-    // every key block.  The score-only passes run 8 (64 keys each) with two K
-    // stages, so that two CTAs share an SM; the output pass, whose stages also
-    // hold V and which needs two P tiles, runs 16 (32 keys each), one CTA per SM.
-    static constexpr int RW = OUT ? 16 : 8;
+    // every key block.  Every pass runs 8 (64 keys each) and fits two CTAs on
+    // an SM.  The score-only passes keep two S buffers and two K stages.  The
+    // output pass keeps one S buffer, whose two 64-key halves (one per key
+    // group of row warps) run S -> P -> PV on their own barriers, P written over
+    // the scores it came from; K and V have one stage each, loaded and released
+    // by halves, so that one half's exponentials overlap the other half's
+    // products and the next block's scores.
+    static constexpr int RW = 8;
     static constexpr int CQ = RW / 4;      // key groups per block
     static constexpr int CH = 4 / CQ;      // 32-key chunks per warp and block
     static constexpr int NT = 32 * (2 + RW);
-    static constexpr int MINB = OUT ? 1 : 2;  // CTAs per SM
-    static constexpr int STAGES = OUT ? 3 : 2;
-    static constexpr int KV_BYTES = OUT ? 2 * TILE : TILE;  // K (and V) of one key block
+    static constexpr int MINB = 2;         // CTAs per SM
+    static constexpr int STAGES = OUT ? 1 : 2;  // K stages
+    static constexpr int V_BYTES = OUT ? TILE : 0;  // one V stage
     static constexpr int STAT_BYTES = MODE == kRowStats ? 2 * CQ * BQ * 4 : 0;  // per-group (m, l) of each row
-    static constexpr size_t SMEM = 1024 + TILE + STAGES * (size_t)KV_BYTES + STAT_BYTES + 256;
-    // TMEM columns: two S buffers [0, 256); output pass: O [256, 384) and two
-    // bf16 P buffers [384, 512), 64 columns each
-    static constexpr uint32_t TMEM_COLS = OUT ? 512 : 256;
-    static_assert(!OUT || CH == 1, "the output pass keeps one mask word per warp and block");
+    static constexpr size_t SMEM = 1024 + TILE + STAGES * (size_t)TILE + V_BYTES + STAT_BYTES + 256;
+    // TMEM columns: score passes two S buffers [0, 256); output pass one S
+    // buffer [0, 128), whose 32-key chunks take their bf16 P pairs in their
+    // first 16 columns, and O [128, 256)
+    static constexpr uint32_t TMEM_COLS = 256;
 };
 
 // Query block of CTA b: the longest causal key ranges first.
@@ -116,39 +120,48 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::NT, AttnCfg<MODE>::MINB) attn_p
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;
-    uint8_t* sKV = sQ + TILE;                         // STAGES stages: K tile (then V tile)
-    float* stat = reinterpret_cast<float*>(sKV + C::STAGES * C::KV_BYTES);  // [2][CQ][BQ] (row statistics)
+    uint8_t* sK = sQ + TILE;                          // STAGES K tiles
+    uint8_t* sV = sK + C::STAGES * TILE;              // output pass: one V tile
+    float* stat = reinterpret_cast<float*>(sV + C::V_BYTES);  // [2][CQ][BQ] (row statistics)
     uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stat) + C::STAT_BYTES);
+    // [2] each: score passes index K stages and S buffers by 2; the output pass
+    // indexes the halves of its one K stage, V stage and S buffer
     uint64_t* q_full = bars;
-    uint64_t* kv_full = bars + 1;                 // [STAGES]
-    uint64_t* kv_empty = kv_full + C::STAGES;     // [STAGES]
-    uint64_t* s_full = kv_empty + C::STAGES;      // [2]
-    uint64_t* s_empty = s_full + 2;
-    uint64_t* p_full = s_empty + 2;
-    uint64_t* p_empty = p_full + 2;
-    uint64_t* o_full = p_empty + 2;
+    uint64_t* k_full = bars + 1;
+    uint64_t* k_empty = bars + 3;
+    uint64_t* s_full = bars + 5;
+    uint64_t* s_empty = bars + 7;                 // output pass: the half's P has been read
+    uint64_t* p_full = bars + 9;                  // output pass: the half's P written
+    uint64_t* v_full = bars + 11;
+    uint64_t* v_empty = bars + 13;
+    uint64_t* o_full = bars + 15;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(o_full + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
-        }
         for (int s = 0; s < 2; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
             mbar_init(&s_full[s], 1);
-            mbar_init(&s_empty[s], C::RW);  // one arrival per row warp
-            mbar_init(&p_full[s], C::RW);
-            mbar_init(&p_empty[s], 1);
+            // score passes: one arrival per row warp once its scores are in
+            // registers; output pass: the MMA's commit after the half's PV product
+            mbar_init(&s_empty[s], C::OUT ? 1 : C::RW);
+            mbar_init(&p_full[s], C::RW / 2);  // the row warps of the half
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
         }
         mbar_init(o_full, 1);
         *abort_flag = 0;
         mbar_fence_init();
         tma_prefetch_map(&p.map_q);
-        tma_prefetch_map(&p.map_k);
-        if (C::OUT) tma_prefetch_map(&p.map_v);
+        if (C::OUT) {
+            tma_prefetch_map(&p.map_kh);
+            tma_prefetch_map(&p.map_vh);
+        } else {
+            tma_prefetch_map(&p.map_k);
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_holder, C::TMEM_COLS);
@@ -195,77 +208,138 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::NT, AttnCfg<MODE>::MINB) attn_p
             tma_load_3d(sQ, &p.map_q, q_full, 0, q0, h);
             tma_load_3d(sQ + ATOM, &p.map_q, q_full, 64, q0, h);
             uint32_t it = 0;
-            for (int kb = 0; kb < kb_end; ++kb) {
+            bool ok = true;
+            for (int kb = 0; kb < kb_end && ok; ++kb) {
                 if (!used(kb)) continue;
                 const int s = it % C::STAGES;
                 const uint32_t ph = (it / C::STAGES) & 1u;
-                ++it;
-                if (!mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag, p.err, kErrTimeoutProducer)) break;
-                uint8_t* dst = sKV + s * C::KV_BYTES;
-                mbar_arrive_expect_tx(&kv_full[s], C::KV_BYTES);
-                tma_load_3d(dst, &p.map_k, &kv_full[s], 0, kb * BKEY, g);
-                tma_load_3d(dst + ATOM, &p.map_k, &kv_full[s], 64, kb * BKEY, g);
                 if constexpr (C::OUT) {
-                    tma_load_3d(dst + TILE, &p.map_v, &kv_full[s], 0, kb * BKEY, g);
-                    tma_load_3d(dst + TILE + ATOM, &p.map_v, &kv_full[s], 64, kb * BKEY, g);
+                    // each half of K once the previous block's scores of that
+                    // half are done, then each half of V once the previous
+                    // block's PV product of that half has read it; a half is
+                    // rows hh * 64 .. +64 of both 64-column swizzle atoms
+                    for (int hh = 0; hh < 2 && ok; ++hh) {
+                        if (!mbar_wait(&k_empty[hh], ph ^ 1u, abort_flag, p.err, kErrTimeoutProducer)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&k_full[hh], TILE / 2);
+                        tma_load_3d(sK + hh * (ATOM / 2), &p.map_kh, &k_full[hh], 0, kb * BKEY + hh * 64, g);
+                        tma_load_3d(sK + ATOM + hh * (ATOM / 2), &p.map_kh, &k_full[hh], 64, kb * BKEY + hh * 64, g);
+                    }
+                    for (int hh = 0; hh < 2 && ok; ++hh) {
+                        if (!mbar_wait(&v_empty[hh], ph ^ 1u, abort_flag, p.err, kErrTimeoutProducer)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&v_full[hh], TILE / 2);
+                        tma_load_3d(sV + hh * (ATOM / 2), &p.map_vh, &v_full[hh], 0, kb * BKEY + hh * 64, g);
+                        tma_load_3d(sV + ATOM + hh * (ATOM / 2), &p.map_vh, &v_full[hh], 64, kb * BKEY + hh * 64, g);
+                    }
+                } else {
+                    if (!mbar_wait(&k_empty[s], ph ^ 1u, abort_flag, p.err, kErrTimeoutProducer)) break;
+                    uint8_t* dst = sK + s * TILE;
+                    mbar_arrive_expect_tx(&k_full[s], TILE);
+                    tma_load_3d(dst, &p.map_k, &k_full[s], 0, kb * BKEY, g);
+                    tma_load_3d(dst + ATOM, &p.map_k, &k_full[s], 64, kb * BKEY, g);
                 }
+                ++it;
             }
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_s = umma_idesc(kKindF16, false, BKEY, 128);  // S = Q K^T
-            constexpr uint32_t idesc_o = umma_idesc(kKindF16, true, DV, 128);     // O += P V (V MN-major)
+            constexpr uint32_t idesc_s = umma_idesc(kKindF16, false, BKEY, 128);      // S = Q K^T
+            constexpr uint32_t idesc_sh = umma_idesc(kKindF16, false, BKEY / 2, 128); // half of S
+            constexpr uint32_t idesc_o = umma_idesc(kKindF16, true, DV, 128);         // O += P V (V MN-major)
             const uint32_t q_addr = smem_u32(sQ);
-            // O += P_j V_j for the j-th used block (P buffer j % 2 in TMEM, K/V stage j % STAGES)
-            auto pv = [&](uint32_t j) -> bool {
-                const int pb = j & 1;
-                if (!mbar_wait(&p_full[pb], (j >> 1) & 1u, abort_flag, p.err, kErrTimeoutMma)) return false;
-                tc_fence_after();
-                const uint32_t p_tmem = tmem_base + kColP + pb * (BKEY / 2);
-                const uint32_t v_addr = smem_u32(sKV + (j % C::STAGES) * C::KV_BYTES + TILE);
-#pragma unroll
-                for (int kk = 0; kk < BKEY / 16; ++kk) {
-                    const uint64_t bdesc = sw128_desc(v_addr + kk * 16 * 128, ATOM, 1024);
-                    umma_ts(tmem_base + kColO, p_tmem + kk * 8, bdesc, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(&p_empty[pb]);
-                umma_commit(&kv_empty[j % C::STAGES]);
-                return true;
-            };
             bool ok = mbar_wait(q_full, 0u, abort_flag, p.err, kErrTimeoutMma);
-            uint32_t it = 0;
-            for (int kb = 0; kb < kb_end && ok; ++kb) {
-                if (!used(kb)) continue;
-                const int s = it % C::STAGES;                 // K (and V) stage
-                const uint32_t ph = (it / C::STAGES) & 1u;
-                const int sb = it & 1;                        // S buffer
-                const uint32_t sph = (it >> 1) & 1u;
-                if (!mbar_wait(&kv_full[s], ph, abort_flag, p.err, kErrTimeoutMma) ||
-                    !mbar_wait(&s_empty[sb], sph ^ 1u, abort_flag, p.err, kErrTimeoutMma)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t k_addr = smem_u32(sKV + s * C::KV_BYTES);
-                const uint32_t d_tmem = tmem_base + sb * BKEY;
-#pragma unroll
-                for (int kk = 0; kk < DH / 16; ++kk) {
-                    const uint64_t adesc = sw128_desc(q_addr + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bdesc = sw128_desc(k_addr + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
-                    umma<kKindF16>(d_tmem, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(&s_full[sb]);
-                if constexpr (C::OUT) {
-                    if (it > 0 && !pv(it - 1)) ok = false;
-                } else {
-                    umma_commit(&kv_empty[s]);  // K consumed by this block's scores
-                }
-                ++it;
-            }
             if constexpr (C::OUT) {
-                if (ok && it > 0) ok = pv(it - 1);
+                // S half hh of the j-th used block (key block kb) into TMEM
+                // columns hh * 64 .. +64, once K's half has landed and the
+                // previous block's PV product of that half has read its P
+                auto issue_s = [&](int kb, uint32_t j, int hh) -> bool {
+                    (void)kb;
+                    if (!mbar_wait(&k_full[hh], j & 1u, abort_flag, p.err, kErrTimeoutMma) ||
+                        !mbar_wait(&s_empty[hh], (j & 1u) ^ 1u, abort_flag, p.err, kErrTimeoutMma))
+                        return false;
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_u32(sK) + hh * (ATOM / 2);
+#pragma unroll
+                    for (int kk = 0; kk < DH / 16; ++kk) {
+                        const uint64_t adesc = sw128_desc(q_addr + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
+                        const uint64_t bdesc = sw128_desc(k_addr + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
+                        umma<kKindF16>(tmem_base + hh * (BKEY / 2), adesc, bdesc, idesc_sh, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&s_full[hh]);
+                    umma_commit(&k_empty[hh]);  // K's half consumed
+                    return true;
+                };
+                // O += P V over the half's 64 keys, once its row warps have
+                // written P over the scores and V's half has landed
+                auto issue_pv = [&](uint32_t j, int hh) -> bool {
+                    if (!mbar_wait(&p_full[hh], j & 1u, abort_flag, p.err, kErrTimeoutMma) ||
+                        !mbar_wait(&v_full[hh], j & 1u, abort_flag, p.err, kErrTimeoutMma))
+                        return false;
+                    tc_fence_after();
+                    const uint32_t v_addr = smem_u32(sV);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        // keys 16 kk .. +16: chunk kk / 2, its P columns (kk % 2) * 8 .. +8
+                        const int kk = hh * 4 + q;
+                        const uint64_t bdesc = sw128_desc(v_addr + kk * 16 * 128, ATOM, 1024);
+                        umma_ts(tmem_base + kColO, tmem_base + (kk >> 1) * 32 + (kk & 1) * 8, bdesc, idesc_o,
+                                (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&s_empty[hh]);  // the half's P read: it may take the next scores
+                    umma_commit(&v_empty[hh]);
+                    return true;
+                };
+                auto next_used = [&](int kb) {
+                    while (kb < kb_end && !used(kb)) ++kb;
+                    return kb;
+                };
+                // order: S(0, 0), S(0, 1), then per block j: PV(j, 0), S(j+1, 0),
+                // PV(j, 1), S(j+1, 1)
+                int kb = next_used(0);
+                uint32_t j = 0;
+                if (ok && kb < kb_end) ok = issue_s(kb, 0, 0) && issue_s(kb, 0, 1);
+                while (ok && kb < kb_end) {
+                    const int kn = next_used(kb + 1);
+                    ok = issue_pv(j, 0);
+                    if (ok && kn < kb_end) ok = issue_s(kn, j + 1, 0);
+                    if (ok) ok = issue_pv(j, 1);
+                    if (ok && kn < kb_end) ok = issue_s(kn, j + 1, 1);
+                    kb = kn;
+                    ++j;
+                }
                 umma_commit(o_full);
+            } else {
+                uint32_t it = 0;
+                for (int kb = 0; kb < kb_end && ok; ++kb) {
+                    if (!used(kb)) continue;
+                    const int s = it % C::STAGES;  // K stage
+                    const uint32_t ph = (it / C::STAGES) & 1u;
+                    const int sb = it & 1;         // S buffer
+                    const uint32_t sph = (it >> 1) & 1u;
+                    if (!mbar_wait(&k_full[s], ph, abort_flag, p.err, kErrTimeoutMma) ||
+                        !mbar_wait(&s_empty[sb], sph ^ 1u, abort_flag, p.err, kErrTimeoutMma)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_u32(sK + s * TILE);
+                    const uint32_t d_tmem = tmem_base + sb * BKEY;
+#pragma unroll
+                    for (int kk = 0; kk < DH / 16; ++kk) {
+                        const uint64_t adesc = sw128_desc(q_addr + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
+                        const uint64_t bdesc = sw128_desc(k_addr + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
+                        umma<kKindF16>(d_tmem, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&s_full[sb]);
+                    umma_commit(&k_empty[s]);  // K consumed by this block's scores
+                    ++it;
+                }
             }
         }
     } else {
@@ -287,8 +361,11 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::NT, AttnCfg<MODE>::MINB) attn_p
         }
         const float scale = p.scale_log2;
         const uint32_t* mask_h = p.tok_mask ? p.tok_mask + (int64_t)h * p.mask_words : nullptr;
-        // output pass: lane j holds this warp's mask word of key block 32 * keep_base + j
-        uint32_t keep_reg = 0u;
+        // output pass: lane j holds this warp's mask words (one per chunk) of key
+        // block 32 * keep_base + j
+        uint32_t keep_reg[C::CH];
+#pragma unroll
+        for (int c = 0; c < C::CH; ++c) keep_reg[c] = 0u;
         int keep_base = -1;
         // One 32-key chunk (chunk cc of key block kb, in buffer sb) of this row.
         auto chunk = [&](int kb, int cc, int sb, const uint32_t (&raw)[32]) {
@@ -297,20 +374,35 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::NT, AttnCfg<MODE>::MINB) attn_p
             // diagonal block and the last block)
             const bool all_in = row_ok && k0 + 31 < p.n && (!p.causal || k0 + 31 <= row);
             const bool none_in = !row_ok || k0 >= p.n || (p.causal && k0 > row);
-            // x = scale * score, -inf where masked (one uniform test per chunk)
-            float x[32];
-            if (__all_sync(0xffffffffu, all_in)) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(raw[i]) * scale;
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const bool valid = !none_in && k0 + i < p.n && (!p.causal || k0 + i <= row);
-                    x[i] = valid ? __uint_as_float(raw[i]) * scale : -INFINITY;
-                }
-            }
+            // one uniform test per chunk: every key counts, or some are masked
+            const bool uniform = __all_sync(0xffffffffu, all_in);
+            auto valid = [&](int i) { return !none_in && k0 + i < p.n && (!p.causal || k0 + i <= row); };
+            auto sc = [&](int i) { return __uint_as_float(raw[i]); };
             if constexpr (MODE == kRowStats) {
-                if (!none_in) {
+                if (uniform) {
+                    // the largest scaled score is the scale times the largest
+                    // (or, for a negative scale, the smallest) raw score: rounding
+                    // keeps the order; each weight is then one fma and one ex2
+                    float mc[4] = {sc(0), sc(1), sc(2), sc(3)};
+                    if (scale >= 0.f) {
+#pragma unroll
+                        for (int i = 4; i < 32; ++i) mc[i & 3] = fmaxf(mc[i & 3], sc(i));
+                        mc[0] = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+                    } else {
+#pragma unroll
+                        for (int i = 4; i < 32; ++i) mc[i & 3] = fminf(mc[i & 3], sc(i));
+                        mc[0] = fminf(fminf(mc[0], mc[1]), fminf(mc[2], mc[3]));
+                    }
+                    const float mn = fmaxf(m, mc[0] * scale);
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[i & 3] += fast_exp2(fmaf(sc(i), scale, -mn));
+                    l = fmaf(l, fast_exp2(m - mn), (acc[0] + acc[1]) + (acc[2] + acc[3]));
+                    m = mn;
+                } else if (!none_in) {
+                    float x[32];  // x = scale * score, -inf where masked
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] = valid(i) ? sc(i) * scale : -INFINITY;
                     float mc[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
                     for (int i = 4; i < 32; ++i) mc[i & 3] = fmaxf(mc[i & 3], x[i]);
@@ -324,55 +416,73 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::NT, AttnCfg<MODE>::MINB) attn_p
             } else if constexpr (MODE == kColScores) {
                 float z = 0.f;
                 if (__any_sync(0xffffffffu, !none_in)) {
+                    // P^2 = 2^(2 (x - b)) in one fma and one ex2; 0 where masked
+                    const float s2 = 2.f * scale, nb2 = -2.f * b;
+                    float q[32];
+                    if (uniform) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float pr = fast_exp2(x[i] - b);  // 0 where masked
-                        x[i] = pr * pr;
+                        for (int i = 0; i < 32; ++i) q[i] = fast_exp2(fmaf(sc(i), s2, nb2));
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) q[i] = fast_exp2(valid(i) ? fmaf(sc(i), s2, nb2) : -INFINITY);
                     }
-                    z = warp_column_sums(x, lane);  // this warp's 32 rows, summed per key
+                    z = warp_column_sums(q, lane);  // this warp's 32 rows, summed per key
                 }
                 const int key = k0 + lane;
                 if (key < p.n) p.col_part[((int64_t)h * p.q_blocks * 4 + qb * 4 + quad) * p.n + key] = z;
             } else {
-                // P masked to the kept tokens, rounded to bf16, into the swizzled P tile
+                // P masked to the kept tokens, rounded to bf16, written over the
+                // chunk's first 16 score columns (in registers by now)
                 if ((kb >> 5) != keep_base) {  // the same for every lane
                     keep_base = kb >> 5;
-                    const int64_t wi = (int64_t)(keep_base * 32 + lane) * (BKEY / 32) + cc;
-                    keep_reg = wi < p.mask_words ? __ldg(mask_h + wi) : 0u;
+#pragma unroll
+                    for (int c = 0; c < C::CH; ++c) {
+                        const int64_t wi = (int64_t)(keep_base * 32 + lane) * (BKEY / 32) + cq * C::CH + c;
+                        keep_reg[c] = wi < p.mask_words ? __ldg(mask_h + wi) : 0u;
+                    }
                 }
-                const uint32_t keep_bits = __shfl_sync(0xffffffffu, keep_reg, kb & 31);
+                const uint32_t keep_bits = __shfl_sync(0xffffffffu, keep_reg[cc - cq * C::CH], kb & 31);
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) w[e] = 0u;
                 if (keep_bits != 0u) {  // the same for every lane: a chunk without a kept token stays 0
+                    // bit i: key k0 + i is kept and inside this row's causal range
+                    const int lim = none_in ? 0 : min(32, min(p.n, p.causal ? row + 1 : p.n) - k0);
+                    const uint32_t live = keep_bits & (lim >= 32 ? 0xffffffffu : ((1u << lim) - 1u));
+                    // each weight is 2^(x - b), x - b in one fma
+                    if (__all_sync(0xffffffffu, live == 0xffffffffu)) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float p0 = ((keep_bits >> (2 * e)) & 1u) ? fast_exp2(x[2 * e] - b) : 0.f;
-                        const float p1 = ((keep_bits >> (2 * e + 1)) & 1u) ? fast_exp2(x[2 * e + 1] - b) : 0.f;
-                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-                        w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                        for (int e = 0; e < 16; ++e) {
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(fast_exp2(fmaf(sc(2 * e), scale, -b)),
+                                                                            fast_exp2(fmaf(sc(2 * e + 1), scale, -b)));
+                            w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const float p0 = ((live >> (2 * e)) & 1u) ? fast_exp2(fmaf(sc(2 * e), scale, -b)) : 0.f;
+                            const float p1 =
+                                ((live >> (2 * e + 1)) & 1u) ? fast_exp2(fmaf(sc(2 * e + 1), scale, -b)) : 0.f;
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+                            w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                        }
                     }
                 }
                 // keys 2e, 2e + 1 of the chunk -> one 32-bit column of this row's lane
-                tmem_st_32x32b_x16(tmem_base + lane_base + kColP + sb * (BKEY / 2) + cc * 16, w);
+                tmem_st_32x32b_x16(tmem_base + lane_base + cc * 32, w);
             }
         };
         uint32_t it = 0;
         bool ok = true;
         for (int kb = 0; kb < kb_end && ok; ++kb) {
             if (!used(kb)) continue;
-            const int sb = it & 1;
-            const uint32_t ph = (it >> 1) & 1u;
+            // S buffer (the output pass has one, and waits for its key group's half)
+            const int sb = C::OUT ? 0 : (int)(it & 1u);
+            const uint32_t ph = C::OUT ? (it & 1u) : ((it >> 1) & 1u);
             ++it;
-            if (!mbar_wait(&s_full[sb], ph, abort_flag, p.err, kErrTimeoutEpilogue)) {
+            if (!mbar_wait(&s_full[C::OUT ? cq : sb], ph, abort_flag, p.err, kErrTimeoutEpilogue)) {
                 ok = false;
                 break;
-            }
-            if constexpr (C::OUT) {
-                if (!mbar_wait(&p_empty[sb], ph ^ 1u, abort_flag, p.err, kErrTimeoutEpilogue)) {
-                    ok = false;
-                    break;
-                }
             }
             tc_fence_after();
             uint32_t raw[C::CH][32];
@@ -380,17 +490,19 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::NT, AttnCfg<MODE>::MINB) attn_p
             for (int c = 0; c < C::CH; ++c)
                 tmem_ld_32x32b_x32(tmem_base + lane_base + sb * BKEY + (cq * C::CH + c) * 32, raw[c]);
             tmem_ld_wait();
-            // the scores are in registers: this S buffer may be overwritten
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[sb]);
+            if constexpr (!C::OUT) {
+                // the scores are in registers: this S buffer may be overwritten
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_empty[sb]);
+            }
 #pragma unroll
             for (int c = 0; c < C::CH; ++c) chunk(kb, cq * C::CH + c, sb, raw[c]);
             if constexpr (C::OUT) {
                 tmem_st_wait();  // this warp's P columns are written before the MMA reads them
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[sb]);
+                if (lane == 0) mbar_arrive(&p_full[cq]);
             }
         }
         if constexpr (MODE == kRowStats) {
@@ -414,29 +526,33 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::NT, AttnCfg<MODE>::MINB) attn_p
             }
         }
         if constexpr (C::OUT) {
-            __nv_bfloat16* orow = p.O + (int64_t)h * p.stride_o + (int64_t)row * p.ldo + cq * 32;
             const bool have = ok && it > 0;
             if (have && !mbar_wait(o_full, 0u, abort_flag, p.err, kErrTimeoutEpilogue)) ok = false;
             tc_fence_after();
-            uint32_t raw[32];
-            if (have && ok) {
-                tmem_ld_32x32b_x32(tmem_base + lane_base + kColO + cq * 32, raw);
-                tmem_ld_wait();
-            } else {
+#pragma unroll 1
+            for (int c = 0; c < C::CH; ++c) {
+                const int col = (cq * C::CH + c) * 32;  // this warp's output columns col .. +32
+                uint32_t raw[32];
+                if (have && ok) {
+                    tmem_ld_32x32b_x32(tmem_base + lane_base + kColO + col, raw);
+                    tmem_ld_wait();
+                } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) raw[i] = 0u;  // no kept token in this row's range
-            }
-            if (row_ok) {
+                    for (int i = 0; i < 32; ++i) raw[i] = 0u;  // no kept token in this row's range
+                }
+                if (row_ok) {
+                    __nv_bfloat16* orow = p.O + (int64_t)h * p.stride_o + (int64_t)row * p.ldo + col;
 #pragma unroll
-                for (int gi = 0; gi < 4; ++gi) {
-                    uint32_t w[4];
+                    for (int gi = 0; gi < 4; ++gi) {
+                        uint32_t w[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(raw[gi * 8 + 2 * e]),
-                                                                        __uint_as_float(raw[gi * 8 + 2 * e + 1]));
-                        w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                        for (int e = 0; e < 4; ++e) {
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(raw[gi * 8 + 2 * e]),
+                                                                            __uint_as_float(raw[gi * 8 + 2 * e + 1]));
+                            w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                        }
+                        *reinterpret_cast<uint4*>(orow + gi * 8) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
-                    *reinterpret_cast<uint4*>(orow + gi * 8) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
         }
@@ -481,15 +597,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
     return fn;
 }
 
-// 3-D bf16 map {cols, rows, heads} with a {64, 128, 1} box and 128-byte swizzle.
+// 3-D bf16 map {cols, rows, heads} with a {64, box_rows, 1} box and 128-byte swizzle.
 bool encode_map(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int64_t heads, int64_t ld,
-                int64_t stride_h) {
+                int64_t stride_h, uint32_t box_rows = 128) {
     auto enc = encoder();
     if (!enc) return false;
     uint64_t head_bytes = heads > 1 ? static_cast<uint64_t>(stride_h) * 2 : static_cast<uint64_t>(ld) * 2 * rows;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(heads)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * 2, head_bytes};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -644,7 +760,8 @@ rmm_status rmm_attention(const rmm_attn_problem* p, const void* Q, const void* K
     std::memset(&ap, 0, sizeof(ap));
     if (!encode_map(&ap.map_q, Qs, p->d_h, n, H, ldqs, stride_qs) ||
         !encode_map(&ap.map_k, K, p->d_h, n, p->kv_heads, p->ldk, p->stride_k) ||
-        !encode_map(&ap.map_v, V, p->d_v, n, p->kv_heads, p->ldv, p->stride_v))
+        !encode_map(&ap.map_kh, K, p->d_h, n, p->kv_heads, p->ldk, p->stride_k, 64) ||
+        !encode_map(&ap.map_vh, V, p->d_v, n, p->kv_heads, p->ldv, p->stride_v, 64))
         return RMM_ERR_CUDA;
     ap.O = static_cast<__nv_bfloat16*>(O);
     ap.ldo = p->ldo;

@@ -20,14 +20,15 @@
 // then runs over all d_h with exact zeros).
 //
 // One CTA computes 128 query rows of one head: warp 0 loads by TMA (Q once,
-// then K (and V) blocks of 128 keys, two or three stages), warp 1 issues
-// tcgen05.mma (S = Q K^T into one of two TMEM buffers; O += P V into a
-// third), and the row warps, a quarter of them per TMEM lane quadrant, each
-// own 32 rows x 32 or 64 keys of every block (one row per thread): they read
-// their S chunks from TMEM and, in the output pass, write P as bf16 pairs back
-// into TMEM, where the PV product takes it as its A operand.  The score-only
-// passes fit two CTAs on an SM (8 row warps), the output pass one (16 row
-// warps).  Every wait is bounded.
+// then K (and V) blocks of 128 keys), warp 1 issues tcgen05.mma, and 8 row
+// warps, two per TMEM lane quadrant, each own 32 rows x 64 keys of every block
+// (one row per thread).  The score passes put S = Q K^T into one of two TMEM
+// buffers while the row warps read the other.  The output pass keeps one S
+// buffer in two 64-key halves, one per key group of row warps: a half's row
+// warps read their scores and write P as bf16 pairs over them, and the PV
+// product (O in TMEM) takes that P as its A operand, while the other half is
+// being scored or exponentiated.  Every pass fits two CTAs on an SM.  Every
+// wait is bounded.
 #include <cmath>
 #include <cstdint>
 #include <cstring>

@@ -256,11 +256,10 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::NT, AttnCfg<MODE>::MINB) attn_p
             const uint32_t q_addr = smem_u32(sQ);
             bool ok = mbar_wait(q_full, 0u, abort_flag, p.err, kErrTimeoutMma);
             if constexpr (C::OUT) {
-                // S half hh of the j-th used block (key block kb) into TMEM
-                // columns hh * 64 .. +64, once K's half has landed and the
-                // previous block's PV product of that half has read its P
-                auto issue_s = [&](int kb, uint32_t j, int hh) -> bool {
-                    (void)kb;
+                // S half hh of the j-th used key block into TMEM columns
+                // hh * 64 .. +64, once K's half has landed and the previous
+                // block's PV product of that half has read its P
+                auto issue_s = [&](uint32_t j, int hh) -> bool {
                     if (!mbar_wait(&k_full[hh], j & 1u, abort_flag, p.err, kErrTimeoutMma) ||
                         !mbar_wait(&s_empty[hh], (j & 1u) ^ 1u, abort_flag, p.err, kErrTimeoutMma))
                         return false;
@@ -304,13 +303,13 @@ __global__ void __launch_bounds__(AttnCfg<MODE>::NT, AttnCfg<MODE>::MINB) attn_p
                 // PV(j, 1), S(j+1, 1)
                 int kb = next_used(0);
                 uint32_t j = 0;
-                if (ok && kb < kb_end) ok = issue_s(kb, 0, 0) && issue_s(kb, 0, 1);
+                if (ok && kb < kb_end) ok = issue_s(0, 0) && issue_s(0, 1);
                 while (ok && kb < kb_end) {
                     const int kn = next_used(kb + 1);
                     ok = issue_pv(j, 0);
-                    if (ok && kn < kb_end) ok = issue_s(kn, j + 1, 0);
+                    if (ok && kn < kb_end) ok = issue_s(j + 1, 0);
                     if (ok) ok = issue_pv(j, 1);
-                    if (ok && kn < kb_end) ok = issue_s(kn, j + 1, 1);
+                    if (ok && kn < kb_end) ok = issue_s(j + 1, 1);
                     kb = kn;
                     ++j;
                 }

@@ -176,6 +176,18 @@ def oracle_sample(inputs64, rho: float, rows: int):
     return time.perf_counter() - t0, flops
 
 
+def oracle_timed(inputs64, rho: float, rows: int, min_seconds: float, max_reps: int = 100):
+    """Repeat oracle_sample until at least `min_seconds` of CPU work (at least
+    once, at most `max_reps` times).  Returns (seconds, useful flops, repetitions)."""
+    t, f, reps = 0.0, 0.0, 0
+    while reps < max(1, max_reps) and (reps == 0 or t < min_seconds):
+        ti, fi = oracle_sample(inputs64, rho, rows)
+        t += ti
+        f += fi
+        reps += 1
+    return t, f, reps
+
+
 def cpu_inputs(n_rows: int, seed: int):
     import workloads as W
     import oracle
@@ -435,10 +447,10 @@ def run_rmm(args):
     if rank == 0 and world == 1 and not args.no_cpu:
         rows = args.cpu_rows
         inputs64 = cpu_inputs(n, seed=1)
-        t, f = oracle_sample(inputs64, rho, rows)
+        t, f, reps = oracle_timed(inputs64, rho, rows, args.cpu_seconds)
         cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cores_used(), "kind": "oracle",
-               "sample": f"full selection of both ops and {rows} of {n} output rows of each product, "
-                         f"fp64 C with OpenMP over rows; {t:.1f} s"}
+               "sample": f"{reps} x (full selection of both ops and {rows} of {n} output rows of each "
+                         f"product), fp64 C with OpenMP over rows; {t:.1f} s"}
 
     launches = sum(e["rmm"]["plan"].kernel_launches for e in ops.values()) * args.steps
     if rank == 0:
@@ -836,6 +848,8 @@ def main(argv=None):
     ap.add_argument("--n", type=int, default=4096)
     ap.add_argument("--rho", type=float, default=0.8)
     ap.add_argument("--cpu-rows", type=int, default=64)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="repeat the CPU oracle sample until this much CPU time has been timed")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-extra-points", action="store_true",

@@ -117,3 +117,23 @@ def test_metric_counts_the_methods_k():
     for d in (128, 256, 4096, 8192, 14336, 28672, 32768):
         for rho in (0.25, 0.5, 0.6, 0.7, 0.8, 0.9, 1.0):
             assert bench.retained(rho, d) == oracle.retained_count(rho, d), (rho, d)
+
+
+def test_cpu_baseline_repeats_the_sample_until_its_time_budget(monkeypatch):
+    """The RMM arm's cpu_baseline times the oracle sample repeatedly until the
+    requested CPU time is reached (at least once, at most max_reps times), and
+    reports the flops and seconds of all repetitions together."""
+    import bench
+    clock = {"t": 0.0}
+
+    def fake_sample(inputs64, rho, rows):
+        clock["t"] += 0.3
+        return 0.3, 2.0 * rows
+
+    monkeypatch.setattr(bench, "oracle_sample", fake_sample)
+    t, f, reps = bench.oracle_timed(None, 0.8, 64, min_seconds=1.0)
+    assert reps == 4 and abs(t - 1.2) < 1e-9 and f == 4 * 128.0
+    t, f, reps = bench.oracle_timed(None, 0.8, 64, min_seconds=0.0)
+    assert reps == 1 and f == 128.0
+    t, f, reps = bench.oracle_timed(None, 0.8, 64, min_seconds=100.0, max_reps=5)
+    assert reps == 5

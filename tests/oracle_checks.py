@@ -284,9 +284,10 @@ def check_e4m3_decoding(impl):
 def check_attention(impl, seed=19):
     """RMM attention [§3.3 "Attention"]: with every feature and token kept it is
     softmax(alpha Q K^T + M) V per head with grouped-query K/V (scipy's softmax,
-    a library routine); with tokens dropped the error of O_h obeys
-    Proposition 1 (Eq. 12) for the product P_h V_g, and T_h is the TopK of
-    P_h's column norms."""
+    a library routine); with features and tokens dropped, I_h holds Q_h's
+    largest column norms, P_h is scipy's row softmax of the scores over I_h
+    alone, the error of O_h obeys Proposition 1 (Eq. 12) for the product
+    P_h V_g, and T_h is the TopK of P_h's column norms."""
     import scipy.special
     rng = _rng(seed)
     H, Hkv, n, dh, dv = 4, 2, 12, 8, 6
@@ -303,8 +304,17 @@ def check_attention(impl, seed=19):
         assert np.allclose(O[h], ref, rtol=1e-12, atol=1e-14), h
     O, I, T, P = impl.rmm_attention(Q, K, V, 0.5, 0.5, alpha, True)
     kt = impl.retained_count(0.5, n)
+    kd = impl.retained_count(0.5, dh)
     for h in range(H):
         g = h // (H // Hkv)
+        # the features are Q_h's top column norms (brute force over all subsets
+        # of size kd would pick the same set: the norms here are distinct), and
+        # P_h is the row softmax of the scores over those features only
+        q2 = (Q[h] ** 2).sum(axis=0)
+        assert np.array_equal(np.sort(I[h]), np.sort(np.argsort(-q2, kind="stable")[:kd])), h
+        feats = np.sort(I[h])
+        logits = np.where(mask, -np.inf, alpha * Q[h][:, feats] @ K[g][:, feats].T)
+        assert np.allclose(P[h], scipy.special.softmax(logits, axis=1), rtol=1e-12, atol=1e-15), h
         s2 = (P[h] ** 2).sum(axis=0)
         assert np.array_equal(T[h], impl.topk_indices(s2, kt))
         full = P[h] @ V[g]

@@ -149,6 +149,28 @@ def _attention_unscaled(Q, K, V, rho_d, rho_t, alpha, causal=True):
     return oracle.rmm_attention(Q, K, V, rho_d, rho_t, 1.0, causal)
 
 
+def _attention_features_from_keys(Q, K, V, rho_d, rho_t, alpha, causal=True):
+    """Feature set chosen from the column norms of the head's K instead of Q."""
+    Q, K, V = oracle.as_f64(Q), oracle.as_f64(K), oracle.as_f64(V)
+    H, Hkv, n = Q.shape[0], K.shape[0], Q.shape[1]
+    kd = oracle.retained_count(rho_d, Q.shape[2])
+    I = np.stack([oracle.topk_indices(oracle.column_scores_sq(K[h // (H // Hkv)]), kd) for h in range(H)])
+    mask = np.triu(np.ones((n, K.shape[1]), dtype=bool), 1) if causal else np.zeros((n, K.shape[1]), dtype=bool)
+    S = np.stack([np.where(mask, -np.inf, alpha * Q[h][:, I[h]] @ K[h // (H // Hkv)][:, I[h]].T) for h in range(H)])
+    P = oracle.softmax_rows(S)
+    kt = oracle.retained_count(rho_t, P.shape[2])
+    T = np.stack([oracle.select(P[h], k=kt)[0] for h in range(H)])
+    O = np.stack([oracle.reduced_product(P[h], V[h // (H // Hkv)], T[h]) for h in range(H)])
+    return O, I, T, P
+
+
+def _attention_scores_over_all_features(Q, K, V, rho_d, rho_t, alpha, causal=True):
+    """I reported, but the scores taken over every feature of Q and K."""
+    _, I, _, _ = oracle.rmm_attention(Q, K, V, rho_d, rho_t, alpha, causal)
+    O, _, T, P = oracle.rmm_attention(Q, K, V, 1.0, rho_t, alpha, causal)
+    return O, I, T, P
+
+
 def _count_floor(rho, d):
     return max(1, int(math.floor(rho * d)))
 
@@ -177,6 +199,8 @@ MUTANTS = {
     "e4m3_subnormals_flushed": _mutant(decode_e4m3=_e4m3_no_subnormals),
     "attention_tokens_from_scores": _mutant(rmm_attention=_attention_tokens_from_scores),
     "attention_without_scale": _mutant(rmm_attention=_attention_unscaled),
+    "attention_features_from_keys": _mutant(rmm_attention=_attention_features_from_keys),
+    "attention_scores_over_all_features": _mutant(rmm_attention=_attention_scores_over_all_features),
 }
 
 

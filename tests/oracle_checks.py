@@ -230,6 +230,44 @@ def check_grouped_heads(impl, seed=17):
         np.testing.assert_allclose(O[h], P[h] @ V[g], rtol=1e-12, atol=1e-12)
 
 
+def _best_subset(norms_sq, k):
+    """The k-subset with the largest sum of squared norms, by enumeration."""
+    best = max(itertools.combinations(range(len(norms_sq)), k), key=lambda c: sum(norms_sq[j] for j in c))
+    return np.array(best)
+
+
+def check_grouped_heads_reduced(impl, seed=20):
+    """§3.3 "Attention" below rho = 1, per head with grouped-query K/V: the QK
+    form keeps the features of Q_h (not of K_g) whose column norms are largest
+    (enumeration over every feature subset), the PV form keeps the tokens of
+    P_h whose column norms are largest (enumeration over every token subset),
+    and each result's error against the dense product obeys Proposition 1
+    (Eq. 12): ||X Y - X_I Y_I||_F <= sum over dropped j of ||X_:j|| ||Y_j:||."""
+    rng = _rng(seed)
+    H, Hkv, n, t, dh = 4, 2, 5, 8, 6
+    # Q's feature norms are ordered against K's, so the two choices differ
+    Q = rng.standard_normal((H, n, dh)) * np.geomspace(4.0, 0.25, dh)
+    K = rng.standard_normal((Hkv, t, dh)) * np.geomspace(0.25, 4.0, dh)
+    P = rng.random((H, n, t)) * np.geomspace(3.0, 0.3, t)
+    V = rng.standard_normal((Hkv, t, dh)) * np.geomspace(0.3, 3.0, t)[:, None]
+    alpha = 0.5
+    S, I = impl.rmm_qk(Q, K, 0.5, alpha, causal=False)
+    O, T = impl.rmm_pv(P, V, 0.5)
+    kd, kt = impl.retained_count(0.5, dh), impl.retained_count(0.5, t)
+    for h in range(H):
+        g = h // (H // Hkv)
+        qn = (Q[h] ** 2).sum(axis=0)
+        assert np.array_equal(np.sort(I[h]), _best_subset(qn, kd)), h
+        dropped = np.setdiff1d(np.arange(dh), I[h])
+        bound = alpha * sum(np.sqrt(qn[j]) * np.linalg.norm(K[g][:, j]) for j in dropped)
+        assert np.linalg.norm(alpha * Q[h] @ K[g].T - S[h]) <= bound * (1 + 1e-12) + 1e-15, h
+        pn = (P[h] ** 2).sum(axis=0)
+        assert np.array_equal(np.sort(T[h]), _best_subset(pn, kt)), h
+        dropped = np.setdiff1d(np.arange(t), T[h])
+        bound = sum(np.sqrt(pn[j]) * np.linalg.norm(V[g][j]) for j in dropped)
+        assert np.linalg.norm(P[h] @ V[g] - O[h]) <= bound * (1 + 1e-12) + 1e-15, h
+
+
 def check_softmax(impl, seed=18):
     """P = softmax(S + M) over the key axis of each row [§3.3 "Attention"]:
     a constant row gives 1/t; two keys give the logistic function of their
@@ -334,6 +372,7 @@ ALL_CHECKS = [
     check_invariants,
     check_one_row_ties,
     check_grouped_heads,
+    check_grouped_heads_reduced,
     check_softmax,
     check_e4m3_decoding,
     check_attention,

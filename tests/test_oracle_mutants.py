@@ -98,6 +98,26 @@ def _pv_interleaved(P, V, rho, heads=None, rows=None):
     return O, T
 
 
+def _qk_features_from_keys(Q, K, rho, alpha, causal=True, heads=None, rows=None):
+    """Each query head's features chosen by its K head's column norms."""
+    Q, K = oracle.as_f64(Q), oracle.as_f64(K)
+    H, Hkv = Q.shape[0], K.shape[0]
+    k = oracle.retained_count(rho, Q.shape[2])
+    I = np.stack([oracle.select(K[h // (H // Hkv)], k=k)[0] for h in range(H)])
+    S = np.stack([oracle.reduced_scores(Q[h], K[h // (H // Hkv)], I[h], alpha, causal) for h in range(H)])
+    return S, I
+
+
+def _pv_tokens_by_value_norms(P, V, rho, heads=None, rows=None):
+    """Each head's tokens chosen by the row norms of V instead of P's column norms."""
+    P, V = oracle.as_f64(P), oracle.as_f64(V)
+    H, Hkv = P.shape[0], V.shape[0]
+    k = oracle.retained_count(rho, P.shape[2])
+    T = np.stack([oracle.topk_indices((V[h // (H // Hkv)] ** 2).sum(axis=1), k) for h in range(H)])
+    O = np.stack([oracle.reduced_product(P[h], V[h // (H // Hkv)], T[h]) for h in range(H)])
+    return O, T
+
+
 def _softmax_no_max_shift(S):
     with np.errstate(over="ignore", invalid="ignore"):
         E = np.exp(oracle.as_f64(S))
@@ -191,6 +211,8 @@ MUTANTS = {
     "k_floor_not_ceil": _mutant(retained_count=_count_floor),
     "k_no_rounding_snap": _mutant(retained_count=_count_no_snap),
     "gqa_heads_interleaved": _mutant(rmm_qk=_qk_interleaved, rmm_pv=_pv_interleaved),
+    "qk_features_from_keys": _mutant(rmm_qk=_qk_features_from_keys),
+    "pv_tokens_by_value_norms": _mutant(rmm_pv=_pv_tokens_by_value_norms),
     "softmax_without_max_shift": _mutant(softmax_rows=_softmax_no_max_shift),
     "softmax_over_the_query_axis": _mutant(softmax_rows=_softmax_over_columns),
     "softmax_mask_as_zero_logit": _mutant(softmax_rows=_softmax_mask_as_zero_logit),

@@ -268,6 +268,22 @@ def check_grouped_heads_reduced(impl, seed=20):
         assert np.linalg.norm(P[h] @ V[g] - O[h]) <= bound * (1 + 1e-12) + 1e-15, h
 
 
+def check_row_subsets(impl, seed=21):
+    """The sampled-row forms used at full size give exactly the rows of the full
+    result (whose values the other checks pin): the reduced product's rows, and
+    the causal scores' rows with each row's own position deciding its mask."""
+    rng = _rng(seed)
+    A, B = rng.standard_normal((9, 12)), rng.standard_normal((12, 7))
+    I = np.array([1, 2, 5, 7, 8, 11], dtype=np.int32)
+    rows = [8, 0, 4, 3]
+    assert np.array_equal(impl.reduced_product(A, B, I, rows=rows), impl.reduced_product(A, B, I)[rows])
+    Q, K = rng.standard_normal((9, 8)), rng.standard_normal((11, 8))
+    Iq = np.array([0, 3, 4, 6], dtype=np.int32)
+    full = impl.reduced_scores(Q, K, Iq, 0.25, True)
+    assert np.array_equal(impl.reduced_scores(Q, K, Iq, 0.25, True, rows=[5, 2, 8]), full[[5, 2, 8]])
+    assert np.isneginf(full[2, 3]) and np.isfinite(full[2, 2]), "key t > row i is masked"
+
+
 def check_softmax(impl, seed=18):
     """P = softmax(S + M) over the key axis of each row [§3.3 "Attention"]:
     a constant row gives 1/t; two keys give the logistic function of their
@@ -373,6 +389,7 @@ ALL_CHECKS = [
     check_one_row_ties,
     check_grouped_heads,
     check_grouped_heads_reduced,
+    check_row_subsets,
     check_softmax,
     check_e4m3_decoding,
     check_attention,

@@ -20,6 +20,7 @@ def _mutant(**overrides):
         column_scores_sq=oracle.column_scores_sq,
         topk_indices=oracle.topk_indices,
         reduced_product=oracle.reduced_product,
+        reduced_scores=oracle.reduced_scores,
         rmm_qk=oracle.rmm_qk,
         rmm_pv=oracle.rmm_pv,
         softmax_rows=oracle.softmax_rows,
@@ -118,6 +119,25 @@ def _pv_tokens_by_value_norms(P, V, rho, heads=None, rows=None):
     return O, T
 
 
+def _scores_rows_masked_by_position_in_sample(Q, K, I, alpha, causal, rows=None):
+    """Sampled rows masked by their position in the sample, not their own row."""
+    if rows is None:
+        return oracle.reduced_scores(Q, K, I, alpha, causal)
+    Q, K = oracle.as_f64(Q), oracle.as_f64(K)
+    I = np.asarray(I)
+    S = alpha * Q[np.asarray(rows)][:, I] @ K[:, I].T
+    if causal:
+        S = np.where(np.arange(K.shape[0])[None, :] > np.arange(len(rows))[:, None], -np.inf, S)
+    return S
+
+
+def _product_rows_from_the_top(A, B, I, rows=None):
+    """Sampled rows taken as the first len(rows) rows."""
+    if rows is None:
+        return oracle.reduced_product(A, B, I)
+    return oracle.reduced_product(A, B, I)[: len(rows)]
+
+
 def _softmax_no_max_shift(S):
     with np.errstate(over="ignore", invalid="ignore"):
         E = np.exp(oracle.as_f64(S))
@@ -212,6 +232,8 @@ MUTANTS = {
     "k_no_rounding_snap": _mutant(retained_count=_count_no_snap),
     "gqa_heads_interleaved": _mutant(rmm_qk=_qk_interleaved, rmm_pv=_pv_interleaved),
     "qk_features_from_keys": _mutant(rmm_qk=_qk_features_from_keys),
+    "sampled_score_rows_masked_by_sample_position": _mutant(reduced_scores=_scores_rows_masked_by_position_in_sample),
+    "sampled_product_rows_from_the_top": _mutant(reduced_product=_product_rows_from_the_top),
     "pv_tokens_by_value_norms": _mutant(rmm_pv=_pv_tokens_by_value_norms),
     "softmax_without_max_shift": _mutant(softmax_rows=_softmax_no_max_shift),
     "softmax_over_the_query_axis": _mutant(softmax_rows=_softmax_over_columns),

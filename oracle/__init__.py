@@ -13,14 +13,19 @@ calls it.  Every function pins to the paper as follows (tests/test_oracle_pins.p
   column_scores_sq    -- n=1 closed form, 2^p scaling, exact small-integer sums
   topk_indices        -- brute force over all subsets (Theorem 1 / Eq. 18)
   reduced_product     -- rho=1 equals numpy's dense product; Prop. 1 / Cor. 1 /
-                         Eq. 17 bounds; equality in the rank-one construction
-  reduced_scores      -- rho=1 equals alpha*Q K^T; causal entries are -inf
-  rmm_qk / rmm_pv     -- per-head bounds and rho=1 dense special cases
+                         Eq. 17 bounds; equality in the rank-one construction;
+                         sampled rows equal the full result's rows
+  reduced_scores      -- rho=1 equals alpha*Q K^T; causal entries are -inf;
+                         sampled rows masked by their own position
+  rmm_qk / rmm_pv     -- rho=1 dense special cases; below rho = 1 the sets are
+                         the largest column norms of Q (QK) and P (PV) by
+                         enumeration over every subset, within Proposition 1
   decode_e4m3         -- hand-worked codes (golden file) and every code against
                          torch's float8_e4m3fn conversion
-  rmm_attention       -- rho = 1 equals scipy's softmax attention; the token step
-                         obeys Proposition 1 on P V; its sets are the TopK of
-                         the oracle's own column norms
+  rmm_attention       -- rho = 1 equals scipy's softmax attention; I is Q's
+                         largest column norms and P scipy's softmax over I
+                         alone; the token step obeys Proposition 1 on P V; its
+                         sets are the TopK of the oracle's own column norms
   softmax_rows        -- closed forms (uniform row, two-key logistic), masked
                          entries exactly 0, rows sum to 1 and not columns,
                          per-row shift invariance, large logits stay finite
